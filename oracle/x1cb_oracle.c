@@ -1,0 +1,283 @@
+/*
+ * Plain CPU oracle for the fused INT8 bottleneck convolutions.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library calls this file: only the
+ * tests, the smoke check and the benchmark's CPU-baseline leg load it.  It
+ * shares no code, header, table or helper with the CUDA path; it has its own
+ * layout index arithmetic and its own requantisation.  Everything is written
+ * as the plain definition, slow and obvious, with 64-bit intermediates.
+ *
+ * What it computes (per output pixel (b,h,w) and output channel o):
+ *
+ *   acc = sum_{r,s,i} X[b, h+r-pad, w+s-pad, i] * Wt[o, i, r, s]
+ *         (taps that fall outside the image contribute 0)
+ *   t   = (acc + bias[o]) * m[o] + (residual ? R[b,h,w,o] * m_r : 0) + 2^(S-1)
+ *   y   = floor(t / 2^S)
+ *   out = min(max(y, 0), 127)
+ *
+ * Sources:
+ *  - Inspur MLPerf v2.0 ResNet50 convolution-merge article
+ *    (news.cnblogs.com/n/719672), section 2.2: Conv3 is followed by Bn, then
+ *    the Shortcut Sum with the block input and a Relu; Conv1 and Conv2 are each
+ *    followed by Bn and Relu.  Section 3.4: Bn+Sum+Relu is applied to every
+ *    Conv3 result before the write-back.  Section 3.1: data, weight and output
+ *    are int8.
+ *  - The requantisation rule above (folded BN as an int32 bias and an int32
+ *    per-channel multiplier, residual multiplier m_r, round-half-up through
+ *    +2^(S-1), arithmetic right shift by S, ReLU and saturation to [0,127]) is
+ *    this library's statement of the fused op; the pages name the steps but
+ *    print no formula.
+ *  - Section 3.1 of the same article defines the layouts: activations
+ *    [B, C/32, H, W, 32] (NC/32HW32) and 1x1 weights [O1, I1, O2, I2] with
+ *    O2 = 128 and I2 = 32.  The 3x3 weight layout [O1, R, S, I1, O2, I2] is
+ *    this library's extension (the pages give none).
+ *  - Didi Cloud IFX DAWNBench article (blog.csdn.net/didi_cloud), section on
+ *    inference optimisation: CONV+BN+RELU as one fused unit (the 3x3 stage).
+ *
+ * Domain: 1 <= S <= 60, fan-in R*R*Ic <= 36864, so every intermediate fits in
+ * int64 with room to spare.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* floor(t / 2^S), written with C's truncating division so that nothing relies
+ * on the implementation-defined right shift of a negative value. */
+static int64_t floor_div_pow2(int64_t t, int S)
+{
+    int64_t d = (int64_t)1 << S;
+    int64_t q = t / d;
+    if (t % d != 0 && t < 0)
+        q -= 1;
+    return q;
+}
+
+/* One output element of the epilogue: BN (bias, multiplier), optional
+ * shortcut Sum, rounding shift, ReLU and saturation to int8. */
+int8_t x1o_requant(int64_t acc, int32_t bias, int32_t m, int has_res, int32_t r,
+                   int32_t m_r, int S)
+{
+    int64_t t = (acc + (int64_t)bias) * (int64_t)m;
+    if (has_res)
+        t += (int64_t)r * (int64_t)m_r;
+    t += (int64_t)1 << (S - 1);
+    int64_t y = floor_div_pow2(t, S);
+    if (y < 0)
+        y = 0;
+    if (y > 127)
+        y = 127;
+    return (int8_t)y;
+}
+
+/* ---- layouts (section 3.1 of the Inspur article) ------------------------- */
+
+/* NC/32HW32: element (b, c, h, w) of a [B, C/32, H, W, 32] tensor. */
+static size_t nc32_index(int64_t b, int64_t c, int64_t h, int64_t w, int64_t C, int64_t H,
+                         int64_t W)
+{
+    return (size_t)((((b * (C / 32) + c / 32) * H + h) * W + w) * 32 + c % 32);
+}
+
+/* NHWC: element (b, h, w, c). */
+static size_t nhwc_index(int64_t b, int64_t h, int64_t w, int64_t c, int64_t H, int64_t W,
+                         int64_t C)
+{
+    return (size_t)(((b * H + h) * W + w) * C + c);
+}
+
+/* Blocked weight [O1, R, S, I1, O2=128, I2=32]: element (o, i, r, s).  For
+ * R = S = 1 this is the article's [O1, I1, O2, I2]. */
+static size_t wblk_index(int64_t o, int64_t i, int64_t r, int64_t s, int64_t Ic, int64_t R)
+{
+    int64_t I1 = Ic / 32;
+    return (size_t)((((((o / 128) * R + r) * R + s) * I1 + i / 32) * 128 + o % 128) * 32 +
+                    i % 32);
+}
+
+/* OIHW (PyTorch convolution weight order): element (o, i, r, s). */
+static size_t oihw_index(int64_t o, int64_t i, int64_t r, int64_t s, int64_t Ic, int64_t R)
+{
+    return (size_t)(((o * Ic + i) * R + r) * R + s);
+}
+
+void x1o_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C)
+{
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h)
+            for (int64_t w = 0; w < W; ++w)
+                for (int64_t c = 0; c < C; ++c)
+                    nc32[nc32_index(b, c, h, w, C, H, W)] = nhwc[nhwc_index(b, h, w, c, H, W, C)];
+}
+
+void x1o_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C)
+{
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h)
+            for (int64_t w = 0; w < W; ++w)
+                for (int64_t c = 0; c < C; ++c)
+                    nhwc[nhwc_index(b, h, w, c, H, W, C)] = nc32[nc32_index(b, c, h, w, C, H, W)];
+}
+
+void x1o_pack_weight(const int8_t *oihw, int8_t *blk, int Oc, int Ic, int R)
+{
+    for (int64_t o = 0; o < Oc; ++o)
+        for (int64_t i = 0; i < Ic; ++i)
+            for (int64_t r = 0; r < R; ++r)
+                for (int64_t s = 0; s < R; ++s)
+                    blk[wblk_index(o, i, r, s, Ic, R)] = oihw[oihw_index(o, i, r, s, Ic, R)];
+}
+
+void x1o_unpack_weight(const int8_t *blk, int8_t *oihw, int Oc, int Ic, int R)
+{
+    for (int64_t o = 0; o < Oc; ++o)
+        for (int64_t i = 0; i < Ic; ++i)
+            for (int64_t r = 0; r < R; ++r)
+                for (int64_t s = 0; s < R; ++s)
+                    oihw[oihw_index(o, i, r, s, Ic, R)] = blk[wblk_index(o, i, r, s, Ic, R)];
+}
+
+/* ---- the fused convolution ---------------------------------------------- */
+
+/* All Oc outputs of one pixel.  x is NHWC, wt is OIHW, r (may be NULL) and
+ * the result row are indexed by channel. */
+static void conv_pixel(const int8_t *x, const int8_t *wt, const int32_t *bias, const int32_t *m,
+                       int S, const int8_t *r_row, int32_t m_r, int8_t *out_row, int64_t b,
+                       int64_t h, int64_t w, int H, int W, int Ic, int Oc, int R, int pad)
+{
+    for (int64_t o = 0; o < Oc; ++o) {
+        int64_t acc = 0;
+        for (int64_t rr = 0; rr < R; ++rr) {
+            int64_t hi = h + rr - pad;
+            if (hi < 0 || hi >= H)
+                continue;
+            for (int64_t ss = 0; ss < R; ++ss) {
+                int64_t wi = w + ss - pad;
+                if (wi < 0 || wi >= W)
+                    continue;
+                const int8_t *xp = x + nhwc_index(b, hi, wi, 0, H, W, Ic);
+                for (int64_t i = 0; i < Ic; ++i)
+                    acc += (int64_t)xp[i] * (int64_t)wt[oihw_index(o, i, rr, ss, Ic, R)];
+            }
+        }
+        out_row[o] = x1o_requant(acc, bias[o], m[o], r_row != NULL, r_row ? r_row[o] : 0, m_r, S);
+    }
+}
+
+/* Full-tensor fused convolution, stride 1, zero padding `pad`, output H x W.
+ * x: [B,H,W,Ic] NHWC.  wt: [Oc,Ic,R,R].  r: [B,H,W,Oc] or NULL.
+ * out: [B,H,W,Oc]. */
+void x1o_conv(const int8_t *x, const int8_t *wt, const int32_t *bias, const int32_t *m, int S,
+              const int8_t *r, int32_t m_r, int8_t *out, int B, int H, int W, int Ic, int Oc,
+              int R, int pad)
+{
+    int64_t rows = (int64_t)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < rows; ++bh) {
+        int64_t b = bh / H, h = bh % H;
+        for (int64_t w = 0; w < W; ++w) {
+            size_t p = nhwc_index(b, h, w, 0, H, W, Oc);
+            conv_pixel(x, wt, bias, m, S, r ? r + p : NULL, m_r, out + p, b, h, w, H, W, Ic, Oc,
+                       R, pad);
+        }
+    }
+}
+
+/* The same convolution evaluated only at `n` chosen pixels.  pix[k] is the
+ * flattened index (b*H + h)*W + w; out_rows is [n, Oc]. */
+void x1o_conv_pixels(const int8_t *x, const int8_t *wt, const int32_t *bias, const int32_t *m,
+                     int S, const int8_t *r, int32_t m_r, const int64_t *pix, int64_t n,
+                     int8_t *out_rows, int B, int H, int W, int Ic, int Oc, int R, int pad)
+{
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t k = 0; k < n; ++k) {
+        int64_t p = pix[k];
+        int64_t b = p / ((int64_t)H * W), h = (p / W) % H, w = p % W;
+        conv_pixel(x, wt, bias, m, S, r ? r + (size_t)p * Oc : NULL, m_r,
+                   out_rows + (size_t)k * Oc, b, h, w, H, W, Ic, Oc, R, pad);
+    }
+}
+
+/* Res3.x bottleneck block (section 2.2 of the Inspur article): conv1 1x1
+ * Cin->Cmid +Bn+Relu, conv2 3x3 pad 1 Cmid->Cmid +Bn+Relu, conv3 1x1
+ * Cmid->Cin +Bn + Sum with the block input + Relu.  All three stages use the
+ * same shift S; only conv3 has the residual term. */
+void x1o_bottleneck(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                    const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                    const int32_t *b3, const int32_t *m3, int32_t m_r, int S, int8_t *out, int B,
+                    int H, int W, int Cin, int Cmid)
+{
+    size_t mid = (size_t)B * H * W * Cmid;
+    int8_t *y1 = (int8_t *)malloc(mid);
+    int8_t *y2 = (int8_t *)malloc(mid);
+    x1o_conv(x, w1, b1, m1, S, NULL, 0, y1, B, H, W, Cin, Cmid, 1, 0);
+    x1o_conv(y1, w2, b2, m2, S, NULL, 0, y2, B, H, W, Cmid, Cmid, 3, 1);
+    x1o_conv(y2, w3, b3, m3, S, x, m_r, out, B, H, W, Cmid, Cin, 1, 0);
+    free(y1);
+    free(y2);
+}
+
+/* The block evaluated only at `n` chosen output pixels: conv1 is evaluated on
+ * the 3x3 neighbourhood the pixel's conv2 needs, then conv2 and conv3 at the
+ * pixel itself.  out_rows is [n, Cin]. */
+void x1o_bottleneck_pixels(const int8_t *x, const int8_t *w1, const int32_t *b1,
+                           const int32_t *m1, const int8_t *w2, const int32_t *b2,
+                           const int32_t *m2, const int8_t *w3, const int32_t *b3,
+                           const int32_t *m3, int32_t m_r, int S, const int64_t *pix, int64_t n,
+                           int8_t *out_rows, int B, int H, int W, int Cin, int Cmid)
+{
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t k = 0; k < n; ++k) {
+        int64_t p = pix[k];
+        int64_t b = p / ((int64_t)H * W), h = (p / W) % H, w = p % W;
+        /* conv1 outputs on a 3x3 window stored as a tiny NHWC image. */
+        int8_t *win = (int8_t *)calloc((size_t)9 * Cmid, 1);
+        int8_t *y2 = (int8_t *)malloc((size_t)Cmid);
+        for (int64_t dr = 0; dr < 3; ++dr)
+            for (int64_t ds = 0; ds < 3; ++ds) {
+                int64_t hh = h + dr - 1, ww = w + ds - 1;
+                if (hh < 0 || hh >= H || ww < 0 || ww >= W)
+                    continue; /* zero padding of conv2's input */
+                conv_pixel(x, w1, b1, m1, S, NULL, 0, win + (dr * 3 + ds) * Cmid, b, hh, ww, H,
+                           W, Cin, Cmid, 1, 0);
+            }
+        /* conv2 at the window centre.  Out-of-image taps were left at zero,
+         * which is exactly the zero padding, so the window is treated as a
+         * 3x3 image with no further padding. */
+        for (int64_t o = 0; o < Cmid; ++o) {
+            int64_t acc = 0;
+            for (int64_t rr = 0; rr < 3; ++rr)
+                for (int64_t ss = 0; ss < 3; ++ss)
+                    for (int64_t i = 0; i < Cmid; ++i)
+                        acc += (int64_t)win[(rr * 3 + ss) * Cmid + i] *
+                               (int64_t)w2[oihw_index(o, i, rr, ss, Cmid, 3)];
+            y2[o] = x1o_requant(acc, b2[o], m2[o], 0, 0, 0, S);
+        }
+        /* conv3 at the pixel with the block input as the shortcut. */
+        const int8_t *r_row = x + (size_t)p * Cin;
+        for (int64_t o = 0; o < Cin; ++o) {
+            int64_t acc = 0;
+            for (int64_t i = 0; i < Cmid; ++i)
+                acc += (int64_t)y2[i] * (int64_t)w3[oihw_index(o, i, 0, 0, Cmid, 1)];
+            out_rows[(size_t)k * Cin + o] = x1o_requant(acc, b3[o], m3[o], 1, r_row[o], m_r, S);
+        }
+        free(win);
+        free(y2);
+    }
+}
+
+int x1o_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
