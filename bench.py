@@ -1,0 +1,423 @@
+"""Benchmark of the fused INT8 Conv3 + BN + shortcut Sum + ReLU (Res3.2, 1x1
+128 -> 512, 28x28) on B200, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--impl x1cb|reference]
+
+One step = one pass of the fused op over one batch (config 3: B=2048).
+Timing: CUDA events on the launching stream around exactly K launches,
+bracketed by a barrier and a device synchronise on both sides; the max over
+ranks.  Inputs (1.85 GB per step at B=2048) are larger than the 126 MB L2,
+so no flush is needed.  With N > 1 every rank runs its own batch (weak
+scaling, batches are independent; no collective on the data path).
+
+Prints one JSON line (rank 0).  The oracle (plain C on the host cores) is
+timed on a bounded sample as the CPU baseline; ``--impl reference`` times it
+as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from x1_conv_bn_b200 import synth  # noqa: E402
+
+METRIC = "fused int8 conv TOPS and HBM GB/s (% of roofline) at Res3.2 Conv3, B=2048"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="3", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="x1cb", choices=["x1cb", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target length of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---- small helpers (also exercised by the CPU tests) ---------------------------------
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def aggregate(per_rank_ms, units_per_rank):
+    """Whole-job throughput: units over all ranks / slowest rank's time."""
+    t = max(per_rank_ms)
+    return units_per_rank * len(per_rank_ms) / (t * 1e-3), t
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's value (all ranks take part; a no-op for one rank)."""
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return base + 7919 * rank
+
+
+def workload_units(cfg):
+    s = synth.CONFIGS[cfg]
+    return s.ops(), s.bytes_moved()
+
+
+def launches_per_step(cfg):
+    return 3 if isinstance(synth.CONFIGS[cfg], synth.BlockShape) else 1
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def read_traffic(profile_name, src_sha):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != src_sha:
+        return None
+    return float(m.group(1))
+
+
+def kernel_source_sha():
+    import hashlib
+
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "x1_conv_bn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:12]
+
+
+# ---- inputs on the device -----------------------------------------------------------
+
+def device_inputs(cfg, dev, seed):
+    import x1_conv_bn_b200 as X
+
+    s = synth.CONFIGS[cfg]
+    if isinstance(s, synth.BlockShape):
+        inp = synth.block_inputs(s, seed, device=dev)
+        x = X.x1cb_pack_act(inp.x)
+        ws = [X.x1cb_pack_weight(w) for w in inp.w]
+        ws_bytes = X.bottleneck_i8_workspace_size(s.B, s.H, s.W, s.Cmid)
+        work = torch.empty(ws_bytes, dtype=torch.int8, device=dev)
+        out = torch.empty_like(x)
+        del inp.x
+
+        def call(x_=None, out_=None, stream=None):
+            X.bottleneck_i8(x if x_ is None else x_, ws[0], inp.bias[0], inp.m[0], ws[1],
+                            inp.bias[1], inp.m[1], ws[2], inp.bias[2], inp.m[2], inp.m_r, inp.S,
+                            out=out if out_ is None else out_, workspace=work, stream=stream)
+
+        return call, {"x": x}, out
+    inp = synth.conv_inputs(s, seed, device=dev)
+    x = X.x1cb_pack_act(inp.x)
+    w = X.x1cb_pack_weight(inp.w)
+    r = X.x1cb_pack_act(inp.r)
+    del inp.x, inp.r
+    out = torch.empty((s.B, s.Oc // 32, s.H, s.W, 32), dtype=torch.int8, device=dev)
+
+    def call(x_=None, r_=None, out_=None, stream=None):
+        X.conv1x1_bn_add_relu_i8(x if x_ is None else x_, w, inp.bias, inp.m, inp.m_r, inp.S,
+                                 r if r_ is None else r_, out=out if out_ is None else out_,
+                                 stream=stream)
+
+    return call, {"x": x, "r": r}, out
+
+
+# ---- CPU oracle (baseline / reference arm) ---------------------------------------------
+
+class OracleSample:
+    """The oracle, as it stands, evaluated on a bounded sample of the workload:
+    the first n output pixels (all channels) of the batch, with n calibrated so
+    that one evaluation takes about `seconds` on the host cores."""
+
+    def __init__(self, cfg, seconds, seed=7):
+        from oracle import oracle as O
+
+        self.O = O
+        self.cfg = cfg
+        self.s = synth.CONFIGS[cfg]
+        self.cores = O.set_threads(0)
+        s = self.s
+        self.hw = s.H * s.W
+        self._make(1, seed)
+        t = self._run(self.hw)
+        per_px = t / self.hw
+        n = int(max(1, min(s.B * self.hw, seconds / max(per_px, 1e-9))))
+        imgs = (n + self.hw - 1) // self.hw
+        if imgs > 1:
+            self._make(imgs, seed)
+        self.n = n
+        self.imgs = imgs
+
+    def _make(self, imgs, seed):
+        s = self.s
+        if isinstance(s, synth.BlockShape):
+            self.inp = synth.block_inputs(synth.BlockShape(imgs, s.H, s.W, s.Cin, s.Cmid), seed)
+        else:
+            self.inp = synth.conv_inputs(
+                synth.ConvShape(imgs, s.H, s.W, s.Ic, s.Oc, s.R, s.has_res), seed)
+
+    def _run(self, n):
+        inp, O = self.inp, self.O
+        pix = torch.arange(n, dtype=torch.int64)
+        t0 = time.perf_counter()
+        if isinstance(self.s, synth.BlockShape):
+            O.bottleneck_pixels(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S, pix)
+        else:
+            O.conv_pixels(inp.x, inp.w, inp.bias, inp.m, inp.S, pix, inp.r, inp.m_r)
+        return time.perf_counter() - t0
+
+    def ops(self):
+        return synth.CONFIGS[self.cfg].ops() * self.n / (self.s.B * self.hw)
+
+    def time(self):
+        """(ops per second, seconds) of one evaluation of the sample."""
+        dt = self._run(self.n)
+        return self.ops() / dt, dt
+
+    def describe(self):
+        return (f"first {self.n} output pixels (all channels) of the {self.s.B}-image batch, "
+                f"i.e. {self.n / (self.s.B * self.hw):.2e} of the workload; oracle with int64 "
+                f"intermediates on {self.cores} host threads")
+
+
+# ---- main ------------------------------------------------------------------------------
+
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = a.config
+    s = synth.CONFIGS[cfg]
+    ops, nbytes = workload_units(cfg)
+    cfg_json = {"workload": synth.WORKLOAD_NAMES[cfg],
+                "shape": {k: getattr(s, k) for k in s.__dataclass_fields__},
+                "layout": "NC/32HW32 activations, blocked [O1,I1,O2,I2] weights",
+                "l2": "inputs larger than L2 (no flush): %.2f GB per step vs 126 MB" % (nbytes / 1e9),
+                "parallelism": f"replicas x{a.gpus} (independent batches)"}
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        per_step = min(5.0, max(0.05, 90.0 / max(1, a.steps + a.warmup)))
+        smp = OracleSample(cfg, per_step)
+        vals = []
+        for i in range(a.warmup + a.steps):
+            v, dt = smp.time()
+            if i >= a.warmup:
+                vals.append((v, dt))
+        v = smp.ops() * len(vals) / sum(dt for _, dt in vals) / 1e12
+        ms = 1e3 * sum(dt for _, dt in vals) / len(vals)
+        line = {"metric": METRIC, "value": v, "unit": "TOPS", "impl": "reference",
+                "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "int64", "data": "synthetic", "config": cfg_json,
+                "cpu_baseline": {"value": v, "unit": "TOPS", "cores": smp.cores,
+                                 "kind": "oracle", "sample": smp.describe() + ", per step"},
+                "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import x1_conv_bn_b200 as X
+    from x1_conv_bn_b200 import _build
+
+    if not os.path.exists(X.LIB_PATH):
+        _build.build()
+    X.lib()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    call, ins, out = device_inputs(cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank))
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, a.warmup)):
+            call(stream=stream)
+    torch.cuda.synchronize()
+    st, bits = X.x1cb_last_device_error(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {bits:#x} during warm-up")
+
+    # ---- timed region (device time, CUDA events on the launching stream) ----
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(a.steps):
+                call(stream=stream)
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    ms_step = e0.elapsed_time(e1) / a.steps
+    st, bits = X.x1cb_last_device_error(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {bits:#x} in the timed region")
+    ms_max = max_over_ranks(ms_step, dist, dev)
+    value_ops, _ = aggregate([ms_max] * world, ops)
+    tops = value_ops / 1e12
+
+    # ---- end to end through the API with host buffers ----
+    e2e = None
+    if not a.no_e2e:
+        host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in ins.items()}
+        for k in ins:
+            host_in[k].copy_(ins[k])
+        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dev_in = {k: torch.empty_like(v) for k, v in ins.items()}
+        dev_out = torch.empty_like(out)
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for k in dev_in:
+                dev_in[k].copy_(host_in[k], non_blocking=True)
+            if "r" in dev_in:
+                call(x_=dev_in["x"], r_=dev_in["r"], out_=dev_out, stream=stream)
+            else:
+                call(x_=dev_in["x"], out_=dev_out, stream=stream)
+            host_out.copy_(dev_out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(a.e2e_steps):
+                e2e_step()
+            e1.record(stream)
+        e1.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / a.e2e_steps, dist, dev)
+        e2e_ops, _ = aggregate([e2e_ms] * world, ops)
+        e2e = {"value": e2e_ops / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "how": "pinned host -> device copies, fused op, device -> pinned host, per step"}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    hbm, _, peak_kind = peaks()
+    launches = launches_per_step(cfg)
+    gbs = nbytes / (ms_max * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+            "frac": gbs / hbm, "peak_source": peak_kind + " (hbm_gbs)",
+            "traffic": read_traffic(f"conv1x1_res32_b{s.B}.md" if launches == 1 else
+                                    f"bottleneck_b{s.B}.md", kernel_source_sha()),
+            "algorithmic_bytes_per_launch": nbytes if launches == 1 else None,
+            "kernel": "conv_bn_act_kernel<true>" if launches == 1 else "3 launches"}
+    line = {"metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": cfg_json, "hbm_gbs": gbs, "roofline": roof,
+            "gpu_launches": a.steps * launches, "clocks": clk.summary(), "e2e": e2e}
+    if world == 1 and not a.no_cpu_baseline:
+        smp = OracleSample(cfg, a.cpu_seconds)
+        v, dt = smp.time()
+        line["cpu_baseline"] = {"value": v / 1e12, "unit": "TOPS", "cores": smp.cores,
+                                "kind": "oracle", "sample": smp.describe(), "seconds": dt}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * x1cb: fused INT8 ResNet bottleneck convolutions for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only; no CUDA or framework types appear in
+ * the signatures (a stream is passed as `void *`, the value of a
+ * cudaStream_t; NULL means the legacy default stream).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layouts (Inspur MLPerf v2.0 ResNet50 convolution-merge article,
+ * news.cnblogs.com/n/719672, section 3.1):
+ *   activations  NC/32HW32 = [B, C/32, H, W, 32] int8: element (b, c, h, w) at
+ *                (((b*C/32 + c/32)*H + h)*W + w)*32 + c%32.
+ *   1x1 weights  [O1, I1, O2, I2] = [Oc/128, Ic/32, 128, 32] int8: element
+ *                (o, i) at (((o/128)*Ic/32 + i/32)*128 + o%128)*32 + i%32.
+ *   3x3 weights  [O1, R, S, I1, O2, I2] = [Oc/128, 3, 3, Ic/32, 128, 32] int8
+ *                (this library's extension of the same blocking; the pages
+ *                give no 3x3 layout).
+ *   bias, m      [Oc] int32 each (folded BN: per-channel bias and fixed-point
+ *                multiplier).
+ * Requantisation of every output element (the article names Bn, Sum and Relu
+ * after Conv3 in sections 2.2 and 3.4 and int8 data in section 3.1; this is
+ * the exact integer rule the library implements):
+ *   t   = (acc + bias[o]) * m[o] + r * m_r + 2^(S-1)   (64-bit, exact)
+ *   out = min(max(t >> S, 0), 127)                      (>> = floor division)
+ * where acc is the exact int32 sum of x*w over the receptive field and the
+ * r*m_r term is present only when a residual tensor is passed.
+ *
+ * Memory: every pointer is DEVICE memory owned by the caller, 16-byte
+ * aligned.  Inputs and outputs must not overlap.  The library never
+ * allocates device memory in any call.
+ * Execution: every call only enqueues work on `stream` and returns after the
+ * argument checks and the launch; results are ready when the stream is
+ * synchronised.  A bounded-wait timeout inside a kernel (which never happens
+ * in normal operation) is recorded in a sticky device status word, read with
+ * x1cb_last_device_error().
+ * Limits: stride 1; 1 <= S <= 60; Ic and Oc multiples of 32 and 128 with
+ * Ic <= 4096; the weights of 128 output channels (R*R*Ic*128 bytes) must fit
+ * in shared memory (Ic <= 1280 for 1x1 with a residual, Ic <= 128 for 3x3);
+ * requires an sm_100 device.
+ * Errors: a negative X1CB_ERR_* status; nothing is launched in that case.
+ */
+#ifndef X1CB_H
+#define X1CB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define X1CB_OK 0
+#define X1CB_ERR_NULL (-1)      /* a required pointer is NULL */
+#define X1CB_ERR_SHAPE (-2)     /* a size or parameter is outside the limits above */
+#define X1CB_ERR_ALIGN (-3)     /* a pointer is not 16-byte aligned */
+#define X1CB_ERR_ARCH (-4)      /* no sm_100 device is current */
+#define X1CB_ERR_CUDA (-5)      /* a CUDA runtime/driver call failed */
+#define X1CB_ERR_TIMEOUT (-6)   /* a kernel gave up a bounded wait */
+#define X1CB_ERR_WORKSPACE (-7) /* workspace missing or too small */
+#define X1CB_ERR_OVERLAP (-8)   /* an output overlaps an input */
+
+/*
+ * Fused 1x1 Conv3 + folded BN + shortcut Sum + ReLU + int8 requantisation
+ * (the merged Conv3+Bn+Sum+Relu kernel of the Inspur article, sections 2.2,
+ * 3.3 and 3.4: the 1x1 convolution is the GEMM out[M,N] = x[M,K].w[N,K]^T
+ * with M = B*H*W, N = Oc, K = Ic, and Bn+Sum+Relu is applied to the
+ * accumulator before the single write-back).
+ *   x    [B, Ic/32, H, W, 32]   input activations (read)
+ *   w    [Oc/128, Ic/32, 128, 32] blocked weights (read)
+ *   bias [Oc], m [Oc]           folded BN (read)
+ *   m_r, S                      residual multiplier and shift
+ *   r    [B, Oc/32, H, W, 32]   shortcut (read); may be NULL for no Sum term
+ *   out  [B, Oc/32, H, W, 32]   result (written)
+ * Returns X1CB_OK or a negative X1CB_ERR_*.
+ */
+int conv1x1_bn_add_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
+                           const int32_t *m, int32_t m_r, int32_t S, const int8_t *r,
+                           int8_t *out, int B, int H, int W, int Ic, int Oc, void *stream);
+
+/*
+ * Fused 3x3 convolution (stride 1, zero padding `pad`, which must be 1) +
+ * folded BN + ReLU + int8 requantisation, no shortcut (Conv2 of the Res3.x
+ * block, Inspur article section 2.2; the CONV+BN+RELU fusion of the Didi
+ * Cloud IFX DAWNBench article, inference-optimisation section).
+ *   x [B, Ic/32, H, W, 32]; w [Oc/128, 3, 3, Ic/32, 128, 32];
+ *   bias, m [Oc]; out [B, Oc/32, H, W, 32].
+ */
+int conv3x3_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
+                       int32_t S, int8_t *out, int B, int H, int W, int Ic, int Oc, int pad,
+                       void *stream);
+
+/* Bytes of device workspace bottleneck_i8 needs: two [B, Cmid/32, H, W, 32]
+ * intermediates. */
+size_t bottleneck_i8_workspace_size(int B, int H, int W, int Cmid);
+
+/*
+ * Res3.x bottleneck block (Inspur article section 2.2): conv1 1x1 Cin->Cmid
+ * +BN+ReLU, conv2 3x3 pad 1 Cmid->Cmid +BN+ReLU, conv3 1x1 Cmid->Cin +BN +
+ * Sum with the block input + ReLU.  Three launches on `stream`, no host
+ * synchronisation between them.
+ *   x   [B, Cin/32, H, W, 32] block input, also the shortcut (read)
+ *   w1  [Cmid/128, Cin/32, 128, 32]; w2 [Cmid/128, 3, 3, Cmid/32, 128, 32];
+ *   w3  [Cin/128, Cmid/32, 128, 32]; b*, m* [Cmid], [Cmid], [Cin]
+ *   m_r, S                 residual multiplier of conv3; S is shared by all
+ *   out [B, Cin/32, H, W, 32] (written)
+ *   workspace              caller-owned device memory of at least
+ *                          bottleneck_i8_workspace_size() bytes
+ */
+int bottleneck_i8(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                  const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                  const int32_t *b3, const int32_t *m3, int32_t m_r, int32_t S, int8_t *out,
+                  void *workspace, size_t ws_bytes, int B, int H, int W, int Cin, int Cmid,
+                  void *stream);
+
+/* Layout conversions on the device (offline steps of the article's section
+ * 3.1).  nhwc [B, H, W, C] <-> nc32 [B, C/32, H, W, 32]; C % 32 == 0. */
+int x1cb_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, void *stream);
+int x1cb_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C, void *stream);
+
+/* oihw [Oc, Ic, R, R] (the usual convolution weight order) -> blocked
+ * [Oc/128, R, R, Ic/32, 128, 32]; R in {1, 3}. */
+int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *x1cb_status_string(int status);
+
+/* Synchronises the current device, then returns X1CB_ERR_TIMEOUT if any
+ * kernel since the last clear gave up a bounded wait, else X1CB_OK (or
+ * X1CB_ERR_CUDA if the device cannot be read).  The raw bits go to *bits
+ * when bits is not NULL.  clear != 0 resets the word. */
+int x1cb_last_device_error(unsigned int *bits, int clear);
+
+/* Limit of every in-kernel wait, in nanoseconds (default 2 s; 0 restores the
+ * default).  Applies to launches made after the call. */
+void x1cb_set_wait_limit_ns(unsigned long long ns);
+
+/* Test hook: mode 1 makes the next launches' MMA warp wait on a barrier that
+ * nothing arrives on, so the bounded-wait path runs out and reports
+ * X1CB_ERR_TIMEOUT without hanging; mode 0 restores normal operation. */
+void x1cb_debug_inject(int mode);
+
+/* Describes the launch plan chosen for a convolution shape into buf (a
+ * short text), for tests and benchmarks.  Returns X1CB_OK or an error. */
+int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, char *buf,
+                       size_t len);
+
+/* Library version, e.g. "x1cb 0.1.0 sm_100a". */
+const char *x1cb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* X1CB_H */

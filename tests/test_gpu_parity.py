@@ -1,0 +1,311 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Integer arithmetic has a unique result, so every comparison is bit-exact.
+Inputs come from the seeded generators in x1_conv_bn_b200.synth; the GPU side
+packs them with its own pack kernels, the oracle computes from the logical
+NHWC/OIHW tensors with its own code, and the packed GPU output is compared
+with the oracle output packed by the oracle.
+"""
+import pytest
+import torch
+
+import x1_conv_bn_b200 as X
+from x1_conv_bn_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from x1_conv_bn_b200 import _build
+
+    _build.build()
+    X.lib()
+    X.x1cb_debug_inject(0)
+    X.x1cb_set_wait_limit_ns(0)
+    st, bits = X.x1cb_last_device_error(clear=True)
+
+
+def _gpu_conv(inp: synth.ConvInputs):
+    s = inp.shape
+    x = X.x1cb_pack_act(inp.x.to(DEV).contiguous())
+    w = X.x1cb_pack_weight(inp.w.to(DEV).contiguous())
+    bias, m = inp.bias.to(DEV), inp.m.to(DEV)
+    if s.R == 1:
+        r = X.x1cb_pack_act(inp.r.to(DEV).contiguous()) if inp.r is not None else None
+        out = X.conv1x1_bn_add_relu_i8(x, w, bias, m, inp.m_r, inp.S, r)
+    else:
+        assert inp.r is None
+        out = X.conv3x3_bn_relu_i8(x, w, bias, m, inp.S)
+    torch.cuda.synchronize()
+    st, bits = X.x1cb_last_device_error(clear=True)
+    assert st == 0, bits
+    return out.cpu()
+
+
+def _oracle_conv(oracle, inp):
+    return oracle.conv(inp.x, inp.w, inp.bias, inp.m, inp.S, inp.r, inp.m_r)
+
+
+def _assert_spread(ref):
+    # the case exercises the arithmetic, not only the clamps
+    frac0 = (ref == 0).float().mean().item()
+    assert frac0 < 0.95 and (ref == 127).float().mean().item() < 0.95
+
+
+# ---- layout kernels -----------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 32), (2, 5, 7, 96), (3, 28, 28, 128), (1, 3, 130, 64)])
+def test_pack_unpack_act(oracle, shape):
+    g = torch.Generator().manual_seed(1)
+    x = torch.randint(-128, 128, shape, generator=g, dtype=torch.int8)
+    got = X.x1cb_pack_act(x.to(DEV)).cpu()
+    assert torch.equal(got, oracle.pack_act(x))
+    back = X.x1cb_unpack_act(X.x1cb_pack_act(x.to(DEV))).cpu()
+    assert torch.equal(back, x)
+
+
+@pytest.mark.parametrize("shape", [(128, 32, 1), (512, 128, 1), (256, 64, 3), (128, 128, 3)])
+def test_pack_weight(oracle, shape):
+    Oc, Ic, R = shape
+    g = torch.Generator().manual_seed(2)
+    w = torch.randint(-128, 128, (Oc, Ic, R, R), generator=g, dtype=torch.int8)
+    got = X.x1cb_pack_weight(w.to(DEV)).cpu()
+    assert torch.equal(got, oracle.pack_weight(w))
+
+
+# ---- fused 1x1 ------------------------------------------------------------------
+
+SMALL_1X1 = [
+    # B, H, W, Ic, Oc   (several tiles, ragged pixel and batch tails)
+    (1, 1, 1, 32, 128),
+    (1, 28, 28, 128, 512),
+    (3, 28, 28, 128, 512),
+    (9, 28, 28, 128, 512),
+    (2, 7, 9, 64, 256),
+    (5, 14, 14, 256, 1024),
+    (7, 7, 7, 512, 2048),
+    (3, 56, 56, 64, 256),
+    (2, 3, 5, 1024, 128),
+    (17, 2, 3, 32, 384),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL_1X1, ids=[str(s) for s in SMALL_1X1])
+@pytest.mark.parametrize("has_res", [True, False], ids=["res", "nores"])
+def test_conv1x1_parity(oracle, shape, has_res):
+    s = synth.ConvShape(*shape, R=1, has_res=has_res)
+    inp = synth.conv_inputs(s, seed=hash(shape) & 0xFFFF)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref), (got != ref).sum().item()
+    _assert_spread(ref)
+
+
+@pytest.mark.parametrize("S", [12, 24, 31, 40])
+def test_conv1x1_full_int8_range(oracle, S):
+    """x, w, r over [-128, 127], negative multipliers, wide bias, several shifts."""
+    s = synth.ConvShape(4, 9, 13, 96, 256, 1, True)
+    inp = synth.full_range_conv_inputs(s, 90 + S, S=S)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref), (got != ref).sum().item()
+
+
+def test_conv1x1_hand_cases(oracle):
+    """The golden requantisation cases through the full kernel: channel o gets
+    acc = a_o (x = (a, 0, ...), w = 1 on channel 0), bias, m and residual of case o."""
+    from tests.test_oracle_pins import HAND
+
+    cases = [c for c in HAND if abs(c[0]) <= 127 and c[5] == 24]
+    Oc = 128
+    Ic = 32
+    x = torch.zeros(1, 1, 1, Ic, dtype=torch.int8)
+    w = torch.zeros(Oc, Ic, 1, 1, dtype=torch.int8)
+    bias = torch.zeros(Oc, dtype=torch.int32)
+    m = torch.zeros(Oc, dtype=torch.int32)
+    r = torch.zeros(1, 1, 1, Oc, dtype=torch.int8)
+    # one pixel: x[0] = 1 so acc_o = w[o, 0]
+    x[0, 0, 0, 0] = 1
+    exp = []
+    m_r = 1 << 23
+    for acc, b, mm, rr, mr, S, e in cases:
+        if rr is not None and mr != m_r:
+            continue
+        w[len(exp), 0, 0, 0] = acc
+        bias[len(exp)] = b
+        m[len(exp)] = mm
+        r[0, 0, 0, len(exp)] = 0 if rr is None else rr
+        exp.append(e)
+    n = len(exp)
+    inp = synth.ConvInputs(synth.ConvShape(1, 1, 1, Ic, Oc, 1, True), x, w, bias, m, r, m_r, 24)
+    got = X.x1cb_unpack_act(_gpu_conv(inp).to(DEV)).cpu()
+    assert got.reshape(-1)[:n].tolist() == exp
+    assert torch.equal(got, _oracle_conv(oracle, inp))
+
+
+# ---- fused 3x3 ------------------------------------------------------------------
+
+SMALL_3X3 = [
+    (1, 1, 1, 32, 128),
+    (2, 28, 28, 128, 128),
+    (3, 5, 7, 64, 256),
+    (1, 3, 130, 32, 128),
+    (11, 6, 6, 128, 128),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL_3X3, ids=[str(s) for s in SMALL_3X3])
+def test_conv3x3_parity(oracle, shape):
+    s = synth.ConvShape(*shape, R=3, has_res=False)
+    inp = synth.conv_inputs(s, seed=hash(shape) & 0xFFFF)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref), (got != ref).sum().item()
+
+
+def test_conv3x3_full_int8_range(oracle):
+    s = synth.ConvShape(2, 9, 11, 64, 128, 3, False)
+    inp = synth.full_range_conv_inputs(s, 7, S=33)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref)
+
+
+def test_centre_tap_3x3_equals_1x1():
+    s = synth.ConvShape(3, 10, 12, 64, 128, 1, False)
+    inp = synth.conv_inputs(s, 5)
+    w3 = torch.zeros(128, 64, 3, 3, dtype=torch.int8)
+    w3[:, :, 1, 1] = inp.w[:, :, 0, 0]
+    a = _gpu_conv(inp)
+    inp3 = synth.ConvInputs(synth.ConvShape(3, 10, 12, 64, 128, 3, False), inp.x, w3, inp.bias,
+                            inp.m, None, 0, inp.S)
+    assert torch.equal(a, _gpu_conv(inp3))
+
+
+# ---- bottleneck block -------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(2, 28, 28, 512, 128), (1, 6, 5, 256, 128), (3, 9, 4, 384, 128)])
+def test_bottleneck_parity(oracle, shape):
+    s = synth.BlockShape(*shape)
+    inp = synth.block_inputs(s, seed=31)
+    ref = oracle.pack_act(oracle.bottleneck(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S))
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    ws = [X.x1cb_pack_weight(w.to(DEV)) for w in inp.w]
+    bs = [b.to(DEV) for b in inp.bias]
+    ms = [m.to(DEV) for m in inp.m]
+    out = X.bottleneck_i8(x, ws[0], bs[0], ms[0], ws[1], bs[1], ms[1], ws[2], bs[2], ms[2],
+                          inp.m_r, inp.S)
+    torch.cuda.synchronize()
+    assert torch.equal(out.cpu(), ref)
+    _assert_spread(ref)
+
+
+# ---- full-size workloads, sampled --------------------------------------------------
+
+def _sample_pixels(B, H, W, n, seed):
+    g = torch.Generator().manual_seed(seed)
+    P = B * H * W
+    pix = torch.randint(0, P, (n,), generator=g)
+    edges = torch.tensor([0, W - 1, (H - 1) * W, H * W - 1, P - 1, P - H * W, P // 2])
+    return torch.unique(torch.cat([pix, edges.clamp(0, P - 1)]))
+
+
+def _gather_nc32(t_nc32_cpu, pix, H, W):
+    """Rows [n, C] of a packed [B, C/32, H, W, 32] tensor at flattened pixels."""
+    B, C1 = t_nc32_cpu.shape[:2]
+    flat = t_nc32_cpu.permute(0, 2, 3, 1, 4).reshape(B * H * W, C1 * 32)
+    return flat[pix]
+
+
+@pytest.mark.parametrize("cfg", ["1", "2", "3", "4a", "4b", "4c"])
+def test_full_size_1x1_sampled(oracle, cfg):
+    s = synth.CONFIGS[cfg]
+    inp = synth.conv_inputs(s, synth.CONFIG_SEEDS[cfg])
+    got = _gpu_conv(inp)
+    pix = _sample_pixels(s.B, s.H, s.W, 1500, 7)
+    ref = oracle.conv_pixels(inp.x, inp.w, inp.bias, inp.m, inp.S, pix, inp.r, inp.m_r)
+    assert torch.equal(_gather_nc32(got, pix, s.H, s.W), ref)
+    _assert_spread(ref)
+
+
+def test_full_size_block_sampled(oracle):
+    s = synth.CONFIGS["5"]
+    inp = synth.block_inputs(s, synth.CONFIG_SEEDS["5"])
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    ws = [X.x1cb_pack_weight(w.to(DEV)) for w in inp.w]
+    bs = [b.to(DEV) for b in inp.bias]
+    ms = [m.to(DEV) for m in inp.m]
+    out = X.bottleneck_i8(x, ws[0], bs[0], ms[0], ws[1], bs[1], ms[1], ws[2], bs[2], ms[2],
+                          inp.m_r, inp.S)
+    torch.cuda.synchronize()
+    pix = _sample_pixels(s.B, s.H, s.W, 400, 8)
+    ref = oracle.bottleneck_pixels(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S, pix)
+    assert torch.equal(_gather_nc32(out.cpu(), pix, s.H, s.W), ref)
+    _assert_spread(ref)
+
+
+# ---- safety properties ----------------------------------------------------------------
+
+def test_guard_bands_untouched():
+    s = synth.ConvShape(3, 7, 9, 64, 256, 1, True)
+    inp = synth.conv_inputs(s, 3)
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    w = X.x1cb_pack_weight(inp.w.to(DEV))
+    r = X.x1cb_pack_act(inp.r.to(DEV))
+    n = s.pixels * s.Oc
+    pad = 4096
+    buf = torch.full((n + 2 * pad,), 0x5A, dtype=torch.int8, device=DEV)
+    out = buf[pad:pad + n].view(s.B, s.Oc // 32, s.H, s.W, 32)
+    X.conv1x1_bn_add_relu_i8(x, w, inp.bias.to(DEV), inp.m.to(DEV), inp.m_r, inp.S, r, out=out)
+    torch.cuda.synchronize()
+    assert (buf[:pad] == 0x5A).all() and (buf[pad + n:] == 0x5A).all()
+
+
+def test_repeatable_and_stream_ordered(oracle):
+    s = synth.ConvShape(16, 28, 28, 128, 512, 1, True)
+    inp = synth.conv_inputs(s, 12)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        a = _gpu_conv(inp)
+        b = _gpu_conv(inp)
+    assert torch.equal(a, b)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(oracle):
+    """A wait that nothing satisfies (test hook) runs out after 50 ms; the
+    kernel returns, the status word says timeout, and the next call is exact."""
+    s = synth.ConvShape(4, 28, 28, 128, 512, 1, True)
+    inp = synth.conv_inputs(s, 44)
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    w = X.x1cb_pack_weight(inp.w.to(DEV))
+    r = X.x1cb_pack_act(inp.r.to(DEV))
+    bias, m = inp.bias.to(DEV), inp.m.to(DEV)
+    X.x1cb_last_device_error(clear=True)
+    try:
+        X.x1cb_set_wait_limit_ns(50_000_000)
+        X.x1cb_debug_inject(1)
+        X.conv1x1_bn_add_relu_i8(x, w, bias, m, inp.m_r, inp.S, r)
+        st, bits = X.x1cb_last_device_error(clear=True)
+    finally:
+        X.x1cb_debug_inject(0)
+        X.x1cb_set_wait_limit_ns(0)
+    assert st == X.X1CB_ERR_TIMEOUT
+    assert bits & 2  # the MMA warp's wait ran out
+    assert not bits & 8  # every copy in flight landed before exit
+    out = X.conv1x1_bn_add_relu_i8(x, w, bias, m, inp.m_r, inp.S, r)
+    torch.cuda.synchronize()
+    assert X.x1cb_last_device_error(clear=True)[0] == 0
+    assert torch.equal(out.cpu(), oracle.pack_act(_oracle_conv(oracle, inp)))
+
+
+def test_empty_batch_is_noop():
+    x = torch.empty((0, 4, 28, 28, 32), dtype=torch.int8, device=DEV)
+    w = torch.zeros((4, 4, 128, 32), dtype=torch.int8, device=DEV)
+    b = torch.zeros(512, dtype=torch.int32, device=DEV)
+    out = X.conv1x1_bn_add_relu_i8(x, w, b, b, 0, 24, None)
+    assert out.shape == (0, 16, 28, 28, 32)

@@ -1,0 +1,317 @@
+// The C ABI of include/x1cb.h: argument checks, launch plans (cached per
+// shape), and the three-stage bottleneck chain.  All compute is in the
+// kernels of x1cb_conv.cu and x1cb_pack.cu.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "x1cb_internal.h"
+
+namespace x1cb {
+namespace {
+
+std::atomic<unsigned long long> g_wait_limit_ns{0};
+std::atomic<int> g_inject{0};
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
+struct DevInfo {
+    int ok = 0;  // 1 = sm_100, -1 = not
+    int sms = 0;
+};
+
+int device_info(int &sms)
+{
+    static std::mutex mu;
+    static DevInfo info[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return X1CB_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (info[dev].ok == 0) {
+        int major = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return X1CB_ERR_CUDA;
+        info[dev].ok = (major == 10) ? 1 : -1;
+        info[dev].sms = n;
+    }
+    if (info[dev].ok != 1)
+        return X1CB_ERR_ARCH;
+    sms = info[dev].sms;
+    return X1CB_OK;
+}
+
+// Small cache of launch plans keyed by shape (the tile search is not free and
+// a B=1 call is latency-bound).
+struct PlanKey {
+    int B, H, W, Ic, Oc, R, has_res, sms;
+    bool operator==(const PlanKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
+};
+
+int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
+             int m_r, int sms)
+{
+    static std::mutex mu;
+    static PlanKey keys[32];
+    static ConvPlan plans[32];
+    static int used = 0, next = 0;
+    PlanKey k;
+    std::memset(&k, 0, sizeof(k));
+    k = PlanKey{B, H, W, Ic, Oc, R, has_res, sms};
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < used; ++i)
+            if (keys[i] == k) {
+                p = plans[i];
+                goto found;
+            }
+    }
+    if (int e = plan_conv(p, B, H, W, Ic, Oc, R, has_res, S, m_r, sms))
+        return e;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        keys[next] = k;
+        plans[next] = p;
+        next = (next + 1) % 32;
+        if (used < 32)
+            ++used;
+    }
+found:
+    p.S = S;
+    p.m_r = m_r;
+    p.inject = g_inject.load();
+    const unsigned long long lim = g_wait_limit_ns.load();
+    p.wait_limit_ns = lim ? lim : kDefaultWaitNs;
+    return X1CB_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb)
+{
+    if (!a || !b || na == 0 || nb == 0)
+        return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Checks shared by the convolution entry points.
+int check_conv_shape(int B, int H, int W, int Ic, int Oc, int S)
+{
+    if (B < 0 || H < 0 || W < 0)
+        return X1CB_ERR_SHAPE;
+    if (Ic < 32 || Ic % 32 || Ic > 4096 || Oc < 128 || Oc % 128 || Oc > 65536)
+        return X1CB_ERR_SHAPE;
+    if (S < 1 || S > 60)
+        return X1CB_ERR_SHAPE;
+    if (static_cast<long long>(H) * W > INT_MAX / 2)
+        return X1CB_ERR_SHAPE;
+    // every tensor byte offset must stay far below 2^40 (TMA stride limit)
+    const long long px = static_cast<long long>(B) * H * W;
+    if (px * (Ic > Oc ? Ic : Oc) >= (1LL << 40))
+        return X1CB_ERR_SHAPE;
+    return X1CB_OK;
+}
+
+int conv_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
+                int32_t m_r, int32_t S, const int8_t *r, int8_t *out, int B, int H, int W, int Ic,
+                int Oc, int R, void *stream)
+{
+    if (int e = check_conv_shape(B, H, W, Ic, Oc, S))
+        return e;
+    const size_t px = static_cast<size_t>(B) * H * W;
+    if (px == 0)
+        return X1CB_OK;  // empty batch or image: nothing to do (pointers may be NULL)
+    if (!x || !w || !bias || !m || !out)
+        return X1CB_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out) || (r && !aligned16(r)) ||
+        (reinterpret_cast<uintptr_t>(bias) & 3u) || (reinterpret_cast<uintptr_t>(m) & 3u))
+        return X1CB_ERR_ALIGN;
+    const size_t out_bytes = px * Oc;
+    if (overlap(out, out_bytes, x, px * Ic) || overlap(out, out_bytes, r, r ? px * Oc : 0) ||
+        overlap(out, out_bytes, w, static_cast<size_t>(Oc) * Ic * R * R) ||
+        overlap(out, out_bytes, bias, Oc * 4u) || overlap(out, out_bytes, m, Oc * 4u))
+        return X1CB_ERR_OVERLAP;
+    int sms = 0;
+    if (int e = device_info(sms))
+        return e;
+    ConvPlan p;
+    if (int e = get_plan(p, B, H, W, Ic, Oc, R, r != nullptr, S, m_r, sms))
+        return e;
+    return launch_conv(p, x, w, bias, m, r, out, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace x1cb
+
+using namespace x1cb;
+
+extern "C" {
+
+int conv1x1_bn_add_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
+                           const int32_t *m, int32_t m_r, int32_t S, const int8_t *r,
+                           int8_t *out, int B, int H, int W, int Ic, int Oc, void *stream)
+{
+    return conv_common(x, w, bias, m, m_r, S, r, out, B, H, W, Ic, Oc, 1, stream);
+}
+
+int conv3x3_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
+                       int32_t S, int8_t *out, int B, int H, int W, int Ic, int Oc, int pad,
+                       void *stream)
+{
+    if (pad != 1)
+        return X1CB_ERR_SHAPE;
+    return conv_common(x, w, bias, m, 0, S, nullptr, out, B, H, W, Ic, Oc, 3, stream);
+}
+
+size_t bottleneck_i8_workspace_size(int B, int H, int W, int Cmid)
+{
+    if (B < 0 || H < 0 || W < 0 || Cmid < 0)
+        return 0;
+    const size_t mid = static_cast<size_t>(B) * H * W * Cmid;
+    return 2 * ((mid + 255) & ~static_cast<size_t>(255));
+}
+
+int bottleneck_i8(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                  const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                  const int32_t *b3, const int32_t *m3, int32_t m_r, int32_t S, int8_t *out,
+                  void *workspace, size_t ws_bytes, int B, int H, int W, int Cin, int Cmid,
+                  void *stream)
+{
+    if (int e = check_conv_shape(B, H, W, Cin, Cmid, S))
+        return e;
+    if (int e = check_conv_shape(B, H, W, Cmid, Cin, S))
+        return e;
+    if (static_cast<size_t>(B) * H * W == 0)
+        return X1CB_OK;
+    if (!x || !w1 || !b1 || !m1 || !w2 || !b2 || !m2 || !w3 || !b3 || !m3 || !out)
+        return X1CB_ERR_NULL;
+    const size_t need = bottleneck_i8_workspace_size(B, H, W, Cmid);
+    if (need > 0 && (!workspace || ws_bytes < need))
+        return X1CB_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace))
+        return X1CB_ERR_ALIGN;
+    const size_t px = static_cast<size_t>(B) * H * W;
+    if (overlap(out, px * Cin, x, px * Cin) || overlap(workspace, need, x, px * Cin) ||
+        overlap(workspace, need, out, px * Cin))
+        return X1CB_ERR_OVERLAP;
+    if (px == 0)
+        return X1CB_OK;
+    int8_t *y1 = static_cast<int8_t *>(workspace);
+    int8_t *y2 = y1 + need / 2;
+    if (int e = conv_common(x, w1, b1, m1, 0, S, nullptr, y1, B, H, W, Cin, Cmid, 1, stream))
+        return e;
+    if (int e = conv_common(y1, w2, b2, m2, 0, S, nullptr, y2, B, H, W, Cmid, Cmid, 3, stream))
+        return e;
+    return conv_common(y2, w3, b3, m3, m_r, S, x, out, B, H, W, Cmid, Cin, 1, stream);
+}
+
+int x1cb_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, void *stream)
+{
+    if (B < 0 || H < 0 || W < 0 || C < 32 || C % 32)
+        return X1CB_ERR_SHAPE;
+    if (static_cast<size_t>(B) * H * W == 0)
+        return X1CB_OK;
+    if (!nhwc || !nc32)
+        return X1CB_ERR_NULL;
+    if (!aligned16(nhwc) || !aligned16(nc32))
+        return X1CB_ERR_ALIGN;
+    const size_t n = static_cast<size_t>(B) * H * W * C;
+    if (overlap(nhwc, n, nc32, n))
+        return X1CB_ERR_OVERLAP;
+    return launch_pack_act(nhwc, nc32, B, H, W, C, static_cast<cudaStream_t>(stream));
+}
+
+int x1cb_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C, void *stream)
+{
+    if (B < 0 || H < 0 || W < 0 || C < 32 || C % 32)
+        return X1CB_ERR_SHAPE;
+    if (static_cast<size_t>(B) * H * W == 0)
+        return X1CB_OK;
+    if (!nhwc || !nc32)
+        return X1CB_ERR_NULL;
+    if (!aligned16(nhwc) || !aligned16(nc32))
+        return X1CB_ERR_ALIGN;
+    const size_t n = static_cast<size_t>(B) * H * W * C;
+    if (overlap(nhwc, n, nc32, n))
+        return X1CB_ERR_OVERLAP;
+    return launch_unpack_act(nc32, nhwc, B, H, W, C, static_cast<cudaStream_t>(stream));
+}
+
+int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R, void *stream)
+{
+    if (!oihw || !blocked)
+        return X1CB_ERR_NULL;
+    if (Oc < 128 || Oc % 128 || Ic < 32 || Ic % 32 || (R != 1 && R != 3))
+        return X1CB_ERR_SHAPE;
+    const size_t n = static_cast<size_t>(Oc) * Ic * R * R;
+    if (overlap(oihw, n, blocked, n))
+        return X1CB_ERR_OVERLAP;
+    return launch_pack_weight(oihw, blocked, Oc, Ic, R, static_cast<cudaStream_t>(stream));
+}
+
+const char *x1cb_status_string(int s)
+{
+    switch (s) {
+    case X1CB_OK: return "ok";
+    case X1CB_ERR_NULL: return "null pointer";
+    case X1CB_ERR_SHAPE: return "unsupported shape or parameter";
+    case X1CB_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case X1CB_ERR_ARCH: return "no sm_100 device";
+    case X1CB_ERR_CUDA: return "CUDA call failed";
+    case X1CB_ERR_TIMEOUT: return "kernel wait timed out";
+    case X1CB_ERR_WORKSPACE: return "workspace missing or too small";
+    case X1CB_ERR_OVERLAP: return "output overlaps an input";
+    default: return "unknown status";
+    }
+}
+
+int x1cb_last_device_error(unsigned int *bits, int clear)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return X1CB_ERR_CUDA;
+    const unsigned int v = read_and_clear_dev_status(clear != 0);
+    if (cudaGetLastError() != cudaSuccess)
+        return X1CB_ERR_CUDA;
+    if (bits)
+        *bits = v;
+    return v ? X1CB_ERR_TIMEOUT : X1CB_OK;
+}
+
+void x1cb_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns); }
+
+void x1cb_debug_inject(int mode) { g_inject.store(mode); }
+
+int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, char *buf,
+                       size_t len)
+{
+    if (!buf || len == 0)
+        return X1CB_ERR_NULL;
+    if (int e = check_conv_shape(B, H, W, Ic, Oc, 24))
+        return e;
+    if (R != 1 && R != 3)
+        return X1CB_ERR_SHAPE;
+    if (static_cast<long long>(B) * H * W == 0)
+        return X1CB_ERR_SHAPE;
+    int sms = 148;
+    if (device_info(sms) != X1CB_OK)
+        sms = 148;  // describe for a B200 when no device is present
+    ConvPlan p;
+    if (int e = plan_conv(p, B, H, W, Ic, Oc, R, has_res, 24, 0, sms))
+        return e;
+    std::snprintf(buf, len,
+                  "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
+                  "a_stages=%d r_stages=%d smem=%d grid=%d",
+                  p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
+                  p.kb_per_tile, p.a_stages, p.r_stages, p.smem_bytes, p.grid);
+    return X1CB_OK;
+}
+
+const char *x1cb_version(void) { return "x1cb 0.1.0 sm_100a"; }
+
+}  // extern "C"

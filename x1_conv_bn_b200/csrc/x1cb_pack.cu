@@ -1,0 +1,119 @@
+// Layout conversions (Inspur MLPerf ResNet50 convolution-merge article,
+// news.cnblogs.com/n/719672, section 3.1): NHWC <-> NC/32HW32 activations and
+// OIHW -> blocked [O1, R, S, I1, O2=128, I2=32] weights.  These are the
+// article's offline preparation steps; they move 32-byte channel chunks with
+// 16-byte vector accesses.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "x1cb_internal.h"
+
+namespace x1cb {
+namespace {
+
+// One thread per (image, channel block, pixel): consecutive threads take
+// consecutive pixels of one channel block, so the NC/32HW32 side is fully
+// contiguous and the NHWC side reads whole 32-byte sectors.
+__global__ void pack_act_kernel(const int8_t *__restrict__ nhwc, int8_t *__restrict__ nc32,
+                                long long B, long long HW, long long C)
+{
+    const long long C1 = C / 32;
+    const long long n = B * C1 * HW;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long hw = i % HW;
+        const long long c1 = (i / HW) % C1;
+        const long long b = i / (HW * C1);
+        const uint4 *src = reinterpret_cast<const uint4 *>(nhwc + (b * HW + hw) * C + c1 * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(nc32 + i * 32);
+        const uint4 a = src[0], c = src[1];
+        dst[0] = a;
+        dst[1] = c;
+    }
+}
+
+__global__ void unpack_act_kernel(const int8_t *__restrict__ nc32, int8_t *__restrict__ nhwc,
+                                  long long B, long long HW, long long C)
+{
+    const long long C1 = C / 32;
+    const long long n = B * C1 * HW;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long hw = i % HW;
+        const long long c1 = (i / HW) % C1;
+        const long long b = i / (HW * C1);
+        const uint4 *src = reinterpret_cast<const uint4 *>(nc32 + i * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(nhwc + (b * HW + hw) * C + c1 * 32);
+        const uint4 a = src[0], c = src[1];
+        dst[0] = a;
+        dst[1] = c;
+    }
+}
+
+// One thread per destination byte (weights are small).
+__global__ void pack_weight_kernel(const int8_t *__restrict__ oihw, int8_t *__restrict__ blk,
+                                   int Oc, int Ic, int R)
+{
+    const long long n = static_cast<long long>(Oc) * Ic * R * R;
+    const int I1 = Ic / 32;
+    for (long long d = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; d < n;
+         d += static_cast<long long>(gridDim.x) * blockDim.x) {
+        // d = ((((ob*R + r)*R + s)*I1 + i1)*128 + o2)*32 + i2
+        long long t = d;
+        const int i2 = static_cast<int>(t % 32);
+        t /= 32;
+        const int o2 = static_cast<int>(t % 128);
+        t /= 128;
+        const int i1 = static_cast<int>(t % I1);
+        t /= I1;
+        const int s = static_cast<int>(t % R);
+        t /= R;
+        const int r = static_cast<int>(t % R);
+        const int ob = static_cast<int>(t / R);
+        const long long o = static_cast<long long>(ob) * 128 + o2;
+        const long long i = static_cast<long long>(i1) * 32 + i2;
+        blk[d] = oihw[((o * Ic + i) * R + r) * R + s];
+    }
+}
+
+int grid_for(long long n, int threads)
+{
+    long long g = (n + threads - 1) / threads;
+    if (g > 148LL * 64)
+        g = 148LL * 64;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+int launch_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, cudaStream_t s)
+{
+    const long long n = static_cast<long long>(B) * H * W * (C / 32);
+    if (n == 0)
+        return X1CB_OK;
+    pack_act_kernel<<<grid_for(n, 256), 256, 0, s>>>(nhwc, nc32, B, static_cast<long long>(H) * W,
+                                                      C);
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+int launch_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C, cudaStream_t s)
+{
+    const long long n = static_cast<long long>(B) * H * W * (C / 32);
+    if (n == 0)
+        return X1CB_OK;
+    unpack_act_kernel<<<grid_for(n, 256), 256, 0, s>>>(nc32, nhwc, B,
+                                                        static_cast<long long>(H) * W, C);
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+int launch_pack_weight(const int8_t *oihw, int8_t *blk, int Oc, int Ic, int R, cudaStream_t s)
+{
+    const long long n = static_cast<long long>(Oc) * Ic * R * R;
+    if (n == 0)
+        return X1CB_OK;
+    pack_weight_kernel<<<grid_for(n, 256), 256, 0, s>>>(oihw, blk, Oc, Ic, R);
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+}  // namespace x1cb

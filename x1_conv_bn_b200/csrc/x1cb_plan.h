@@ -1,0 +1,51 @@
+// Launch plan of the fused implicit-GEMM convolution: geometry, tiling,
+// shared-memory carve-up.  Computed on the host, passed to the kernel by value.
+#pragma once
+#include <cstdint>
+
+namespace x1cb {
+
+constexpr int kThreads = 384;       // 12 warps: 4 control/producer + 8 epilogue
+constexpr int kEpiWarp0 = 4;        // first epilogue warp
+constexpr int kEpiWarps = 8;
+constexpr int kTileRows = 128;      // MMA M
+constexpr int kKBlock = 32;         // int8 channels per K block (one MMA K step)
+constexpr int kASlotBytes = kTileRows * kKBlock;  // 4 KB per A ring slot
+constexpr int kRChunks = 4;         // 32-channel chunks per residual stage
+constexpr int kRSlotBytes = kRChunks * kTileRows * 32;  // 16 KB
+constexpr int kTmemCols = 512;
+constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
+
+// Status bits of the device status word.
+constexpr unsigned kDevTimeoutProducer = 1u;
+constexpr unsigned kDevTimeoutMma = 2u;
+constexpr unsigned kDevTimeoutEpilogue = 4u;
+constexpr unsigned kDevDrainFailed = 8u;
+
+struct ConvPlan {
+    // problem
+    int B, H, W, Ic, Oc, R, pad;
+    int C1, O1;       // Ic/32, Oc/32
+    int Wp, Hp;       // spatial dims seen by the tensor maps (1x1: H*W and 1)
+    int has_res;
+    int S;
+    int m_r;
+    // M tile: tw x th pixels of tg images (rows = tw*th*tg <= 128)
+    int tw, th, tg, rows;
+    int nTw, nTh, nTg;
+    int num_m_tiles;
+    // N split: each CTA keeps NC output channels' weights resident
+    int NC, n_groups, nmma, n_subs;
+    int kb_per_tile;  // R*R*C1
+    // rings
+    int a_stages, r_stages;
+    // shared memory offsets from the 1024-aligned base
+    int off_w, off_a, off_r, off_cc, off_cm, off_bar, off_misc;
+    int smem_bytes;  // including alignment slack
+    // control
+    int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
+    unsigned long long wait_limit_ns;
+    int grid;
+};
+
+}  // namespace x1cb
