@@ -113,6 +113,33 @@ int bottleneck_i8(const int8_t *x, const int8_t *w1, const int32_t *b1, const in
                   void *workspace, size_t ws_bytes, int B, int H, int W, int Cin, int Cmid,
                   void *stream);
 
+/*
+ * bottleneck_i8 for callers that cannot allocate device memory.  The pages
+ * have no counterpart to this entry point; it exists for callers with no way
+ * to pass a workspace, such as an inference engine's plugin whose execution
+ * step must not allocate (allocation can synchronise the device or fail under
+ * memory pressure mid-request) or a runtime that fixes all device memory at
+ * start-up.  Same arguments and result as bottleneck_i8 without the
+ * workspace: the two intermediates live in a 32 MiB array built into the
+ * library (a file-scope __device__ array held by every GPU that loads the
+ * library until the process exits).  No allocator is called.
+ *   Limit: bottleneck_i8_workspace_size(B, H, W, Cmid) <= 32 MiB (for the
+ *   Res3.2 block, 28x28 with Cmid = 128: B <= 167); larger problems return
+ *   X1CB_ERR_WORKSPACE before anything is launched.
+ *   The first call with a given device current looks up the array's device
+ *   address (cudaGetSymbolAddress) and caches it; make that first call before
+ *   any stream capture.
+ *   Every call uses the same array, so calls that overlap on the GPU (other
+ *   streams, other threads) race with each other: serialise them.  Nothing in
+ *   the array needs to start at zero; its contents after a call are those of
+ *   that call's intermediates.
+ */
+int bottleneck_i8_noalloc(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                          const int8_t *w2, const int32_t *b2, const int32_t *m2,
+                          const int8_t *w3, const int32_t *b3, const int32_t *m3, int32_t m_r,
+                          int32_t S, int8_t *out, int B, int H, int W, int Cin, int Cmid,
+                          void *stream);
+
 /* Layout conversions on the device (offline steps of the article's section
  * 3.1).  nhwc [B, H, W, C] <-> nc32 [B, C/32, H, W, 32]; C % 32 == 0. */
 int x1cb_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, void *stream);

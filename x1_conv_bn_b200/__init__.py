@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
         L.bottleneck_i8_workspace_size.argtypes = [i, i, i, i]
         L.bottleneck_i8_workspace_size.restype = sz
         L.bottleneck_i8.argtypes = [vp] * 10 + [i32, i32, vp, vp, sz, i, i, i, i, i, vp]
+        L.bottleneck_i8_noalloc.argtypes = [vp] * 10 + [i32, i32, vp, i, i, i, i, i, vp]
         L.x1cb_pack_act.argtypes = [vp, vp, i, i, i, i, vp]
         L.x1cb_unpack_act.argtypes = [vp, vp, i, i, i, i, vp]
         L.x1cb_pack_weight.argtypes = [vp, vp, i, i, i, vp]
@@ -159,6 +160,26 @@ def bottleneck_i8(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r: int, S: int, out=N
         _dev(workspace, torch.int8, "workspace"), workspace.numel(), B, H, W, Cin, Cmid,
         _stream(stream))
     _check(st, "bottleneck_i8")
+    return out
+
+
+def bottleneck_i8_noalloc(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r: int, S: int, out=None,
+                          stream=None):
+    """bottleneck_i8 without a workspace argument, for callers that cannot
+    allocate device memory: the library keeps the two intermediates in a
+    built-in 32 MiB device array (problems that need more are rejected).
+    Calls share that array, so calls that overlap on the GPU race."""
+    B, Cin, H, W = _act_shape(x, "x")
+    Cmid = b1.numel()
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib().bottleneck_i8_noalloc(
+        _dev(x, torch.int8, "x"), _dev(w1, torch.int8, "w1"), _dev(b1, torch.int32, "b1"),
+        _dev(m1, torch.int32, "m1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
+        _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(b3, torch.int32, "b3"),
+        _dev(m3, torch.int32, "m3"), int(m_r), int(S), _dev(out, torch.int8, "out"),
+        B, H, W, Cin, Cmid, _stream(stream))
+    _check(st, "bottleneck_i8_noalloc")
     return out
 
 
