@@ -16,9 +16,12 @@
 //                  the activation tiles (one 128-row x 32-byte K block per slot)
 //      warp 1      MMA issuer: tcgen05.mma.kind::i8 into TMEM (int32), owner
 //                  of the TMEM allocation
-//      warp 2      TMA producer: shortcut (residual) tiles, far ahead of use
-//      warps 4-11  epilogue: tcgen05.ld, exact int64 requantisation, 16-byte
-//                  stores of NC/32HW32 output straight from registers
+//      warp 2      TMA producer of the I/O stages: each 16 KB stage receives a
+//                  shortcut tile (128 pixels x 128 channels) long before use
+//      warp 3      TMA store of finished I/O stages
+//      warps 4-11  epilogue: tcgen05.ld, exact requantisation; each result
+//                  byte overwrites the shortcut byte of the same (pixel,
+//                  channel) in the stage, which warp 3 then stores whole
 //  * a tile is 128 GEMM rows = tw x th pixels of tg images, chosen per shape
 //    so that whole TMA boxes cover the image (16 px x 8 images for 28x28 1x1)
 //  * TMEM holds 512 int32 columns; the accumulator ring lets the MMA of the
@@ -54,14 +57,18 @@ struct Bars {
     __device__ uint32_t never() const { return at(2); }
     __device__ uint32_t a_full(int s) const { return at(3 + s); }
     __device__ uint32_t a_empty(int s) const { return at(3 + a_stages + s); }
-    __device__ uint32_t r_full(int s) const { return at(3 + 2 * a_stages + s); }
-    __device__ uint32_t r_empty(int s) const { return at(3 + 2 * a_stages + r_stages + s); }
-    __device__ uint32_t acc_full(int s) const { return at(3 + 2 * a_stages + 2 * r_stages + s); }
+    // I/O stage s: io_full = shortcut landed (or stage free when there is no
+    // shortcut), out_ready = every epilogue warp wrote its results,
+    // io_empty = the store of the stage has read it.
+    __device__ uint32_t io_full(int s) const { return at(3 + 2 * a_stages + s); }
+    __device__ uint32_t out_ready(int s) const { return at(3 + 2 * a_stages + r_stages + s); }
+    __device__ uint32_t io_empty(int s) const { return at(3 + 2 * a_stages + 2 * r_stages + s); }
+    __device__ uint32_t acc_full(int s) const { return at(3 + 2 * a_stages + 3 * r_stages + s); }
     __device__ uint32_t acc_empty(int s) const
     {
-        return at(3 + 2 * a_stages + 2 * r_stages + 4 + s);
+        return at(3 + 2 * a_stages + 3 * r_stages + 4 + s);
     }
-    static int count(int a, int r) { return 3 + 2 * a + 2 * r + 8; }
+    static int count(int a, int r) { return 3 + 2 * a + 3 * r + 8; }
 };
 
 __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, int &h0, int &b0)
@@ -74,17 +81,18 @@ __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, 
     b0 = ig * p.tg;
 }
 
-// Requantise 32 accumulators of one pixel (channels n0..n0+31 of this CTA's
-// group) and pack them as 32 int8 bytes.
+// Generic exact requantisation of 32 accumulators of one pixel (channels
+// n0..n0+31 of this CTA's group), packed as 32 int8 bytes:
+//   t = acc*m + C (+ r*m_r),  C = bias*m + 2^(S-1),  y = clamp(t >> S, 0, 127).
 template <bool kRes>
-__device__ __forceinline__ void requant32(const uint32_t (&v)[32], const int32_t *cm,
-                                          const long long *cC, const uint32_t (&rw)[8],
-                                          int m_r, int S, uint32_t (&ow)[8])
+__device__ __forceinline__ void requant32(const uint32_t *v, const int32_t *cm,
+                                          const long long *cC, const uint32_t *rw, int m_r,
+                                          int S, uint32_t *ow)
 {
 #pragma unroll
     for (int q = 0; q < 8; ++q)
         ow[q] = 0u;
-#pragma unroll
+#pragma unroll 8
     for (int k = 0; k < 32; ++k) {
         long long t = static_cast<long long>(static_cast<int>(v[k])) * cm[k] + cC[k];
         if (kRes) {
@@ -97,11 +105,234 @@ __device__ __forceinline__ void requant32(const uint32_t (&v)[32], const int32_t
     }
 }
 
+// Exact fast form of the same requantisation, used when the CTA's constants
+// allow it (checked in the prologue).  With s = 32 - S >= 0 every term is
+// pre-scaled by 2^s: m' = m*2^s, C' = bias*m' + 2^31, and the residual term
+// becomes (r*2^(8*k8)) * (m_r*2^(s - 8*k8)).  Then
+//     t' = acc*m' + C' + r*m_r*2^s = t * 2^s,
+// so floor(t / 2^S) = floor(t' / 2^32) is exactly the high word of t' (no
+// shift, no 64-bit compare).  All three products fit their 32-bit operands and
+// the sum stays below 2^63 (prologue check), so nothing is approximated.
+// Processes n4 groups of 4 channels.
+template <bool kRes, int kGroups>
+__device__ __forceinline__ void requant_fast(const uint32_t *v, const int32_t *cm,
+                                             const long long *cC, const uint32_t *rw, int mr2,
+                                             const uint32_t (&rsel)[4], uint32_t *ow)
+{
+    const int4 *m4 = reinterpret_cast<const int4 *>(cm);
+    const longlong2 *c2 = reinterpret_cast<const longlong2 *>(cC);
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q)
+        ow[q] = requant4_fast<kRes>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], m4[q],
+                                    c2[2 * q], c2[2 * q + 1], kRes ? rw[q] : 0u, rsel, mr2);
+}
+
+// Exact all-32-bit form, used when the shortcut multiplier is a multiple of
+// 2^(S-1) (m_r = k * 2^(S-1)) and the CTA's constants allow it.  With
+// s = 33 - S >= 0 and m' = m * 2^s, every term of t * 2^s except the product
+// is a multiple of 2^32:
+//     t * 2^s = (acc + bias) * m' + 2^32 * (1 + r*k),
+// so y2 = floor(t * 2^s / 2^32) = hi32((acc + bias) * m') + 1 + r*k exactly
+// (mad.hi), and floor(t / 2^S) = floor(y2 / 2); clamping y2 to [0, 255]
+// before halving gives the [0, 127] clamp.  No 64-bit arithmetic.
+template <bool kRes, int kGroups>
+__device__ __forceinline__ void requant_hi32(const uint32_t *v, const int32_t *cm,
+                                             const int32_t *cb, const uint32_t *rw, int k,
+                                             const uint32_t (&rsel)[4], uint32_t *ow)
+{
+    const int4 *m4 = reinterpret_cast<const int4 *>(cm);
+    const int4 *b4 = reinterpret_cast<const int4 *>(cb);
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q)
+        ow[q] = requant4_hi32<kRes>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], m4[q],
+                                    b4[q], kRes ? rw[q] : 0u, rsel, k);
+}
+
+// Layer-wide conditions of the all-32-bit form (per channel: hi32_ok).
+__device__ __forceinline__ bool hi32_layer_ok(int m_r, int S, bool res)
+{
+    if (S < 2 || S > 33)
+        return false;
+    if (!res)
+        return true;
+    const long long q = 1ll << (S - 1);
+    if (static_cast<long long>(m_r) % q != 0)
+        return false;
+    const long long k = static_cast<long long>(m_r) / q;
+    return k >= -(1ll << 23) && k <= (1ll << 23);
+}
+
+// Per-channel conditions: m * 2^(33-S) fits int32, and acc + bias cannot
+// overflow int32 (|acc| <= K * 2^14).
+__device__ __forceinline__ bool hi32_ok(long long m, long long bias, int S, int K)
+{
+    if (S < 2 || S > 33)
+        return false;
+    const long long mp = m * (1ll << (33 - S));
+    if (mp < INT_MIN || mp > INT_MAX)
+        return false;
+    return (bias < 0 ? -bias : bias) + static_cast<long long>(K) * 16384 < (1ll << 31);
+}
+
+// Whether the fast form is exact for output channel o of a layer of fan-in K
+// (every |x|, |w| <= 128, so |acc| <= K * 2^14).
+__device__ __forceinline__ bool fast_form_ok(long long m, long long bias, int m_r, int S, int K,
+                                             bool res)
+{
+    if (S > 32)
+        return false;
+    const int sh = 32 - S;
+    const long long mp = m * (1ll << sh);
+    if (mp < INT_MIN || mp > INT_MAX)
+        return false;
+    double bound = static_cast<double>(K) * 16384.0 * fabs(static_cast<double>(mp)) +
+                   fabs(static_cast<double>(bias) * static_cast<double>(mp)) + 2147483648.0;
+    if (res) {
+        const int k8 = sh / 8 < 3 ? sh / 8 : 3;
+        const long long mr2 = static_cast<long long>(m_r) * (1ll << (sh - 8 * k8));
+        if (mr2 < INT_MIN || mr2 > INT_MAX)
+            return false;
+        bound += 128.0 * fabs(static_cast<double>(m_r)) * static_cast<double>(1ll << sh);
+    }
+    return bound < 4.0e18;  // < 2^62 with margin for the double rounding
+}
+
+// Epilogue of one warp.  For every tile of this CTA and every accumulator
+// slot it reads its 32 TMEM lanes (= 32 pixels of the tile), two adjacent
+// 32-channel chunks per I/O stage, requantises them (with the shortcut bytes
+// of the stage) and writes the 32-byte results back into the stage in place.
+struct EpiCtx {
+    const ConvPlan *p;
+    Bars bars;
+    WaitCtl ctl;
+    uint32_t tmem_base;
+    uint8_t *io;
+    const int32_t *cm;
+    const long long *cC;
+    int group, mt_first, mt_step;
+};
+
+// kMode: 2 = all-32-bit form, 1 = 64-bit fast form, 0 = generic.
+template <bool kRes, int kMode>
+__device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int lane)
+{
+    static_assert(kEpiWarps == 8, "two warps per lane quarter, two chunks each per stage");
+    const ConvPlan &p = *cx.p;
+    const int q = warp & 3;                    // TMEM lane quarter this warp may access
+    const int c0 = 2 * ((warp - kEpiWarp0) >> 2);  // first of the two chunks it takes per stage
+    const int row = q * 32 + lane;             // GEMM row = pixel of the tile
+    const int plane_t = p.tw * p.th;
+    const int xi = row % p.tw;
+    const int yi = (row / p.tw) % p.th;
+    const int gi = row / plane_t;
+    const bool in_box = row < p.rows;
+    // This row's 32 bytes inside chunk 0 of an I/O stage ([tg][4][th][tw][32]);
+    // rows outside the box read row 0's bytes and write nothing.
+    const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
+    const int chunk_stride = plane_t * 32;
+    const int n_slots = kTmemCols / p.nmma;
+    const int chunks_per_sub = p.nmma / 32;
+    const int stages_per_sub = chunks_per_sub / kRChunks;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    // Shortcut operands.  64-bit fast form: r*2^(8*k8) by one byte permute and
+    // m_r*2^(s-8*k8).  All-32-bit form: the sign-extended byte (k8 = 0) and
+    // k = m_r / 2^(S-1).
+    const int sh = 32 - p.S;
+    const int k8 = kMode == 2 ? 0 : (sh < 0 ? 0 : (sh / 8 < 3 ? sh / 8 : 3));
+    const int mr2 =
+        kMode == 1 ? static_cast<int>(static_cast<long long>(p.m_r) * (1ll << (sh - 8 * k8)))
+                   : (kMode == 2 ? static_cast<int>(static_cast<long long>(p.m_r) /
+                                                    (1ll << (p.S - 1)))
+                                 : 0);
+    uint32_t rsel[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        uint32_t sel = 0;
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t nib = i < k8 ? 4u : (i == k8 ? static_cast<uint32_t>(b) : 8u | b);
+            sel |= nib << (4 * i);
+        }
+        rsel[b] = sel;
+    }
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int st = 0;
+    uint32_t st_phase = 0;
+    for (int mt = cx.mt_first; mt < p.num_m_tiles; mt += cx.mt_step) {
+        for (int j = 0; j < p.n_subs; ++j) {
+            // Every lane waits; the vote keeps the decision warp-uniform so the
+            // .sync.aligned TMEM loads below always run converged.
+            if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.acc_full(acc), acc_phase, cx.ctl,
+                                                   kDevTimeoutEpilogue)))
+                return;
+            tc_fence_after();
+            const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
+            for (int rl = 0; rl < stages_per_sub; ++rl) {
+                if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.io_full(st), st_phase, cx.ctl,
+                                                       kDevTimeoutEpilogue)))
+                    return;
+                uint8_t *stage = cx.io + st * kRSlotBytes + row_off;
+                const int cs = rl * kRChunks + c0;         // chunk within the TMEM slot
+                const int gch = j * chunks_per_sub + cs;   // chunk within the CTA's channels
+                uint32_t v[64];
+                __syncwarp();
+                tmem_ld_32x32b_x64_sync(tbase + static_cast<uint32_t>(cs * 32), v);
+                uint4 *p0 = reinterpret_cast<uint4 *>(stage + c0 * chunk_stride);
+                uint4 *p1 = reinterpret_cast<uint4 *>(stage + (c0 + 1) * chunk_stride);
+                uint32_t rw[16];
+                if (kRes) {
+                    const uint4 ra = p0[0], rb = p0[1], rc = p1[0], rd = p1[1];
+                    rw[0] = ra.x; rw[1] = ra.y; rw[2] = ra.z; rw[3] = ra.w;
+                    rw[4] = rb.x; rw[5] = rb.y; rw[6] = rb.z; rw[7] = rb.w;
+                    rw[8] = rc.x; rw[9] = rc.y; rw[10] = rc.z; rw[11] = rc.w;
+                    rw[12] = rd.x; rw[13] = rd.y; rw[14] = rd.z; rw[15] = rd.w;
+                }
+                uint32_t ow[16];
+                if (kMode == 2) {
+                    requant_hi32<kRes, 16>(v, cx.cm + gch * 32,
+                                           reinterpret_cast<const int32_t *>(cx.cC) + gch * 32,
+                                           rw, mr2, rsel, ow);
+                } else if (kMode == 1) {
+                    requant_fast<kRes, 16>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2, rsel, ow);
+                } else {
+                    requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
+                    requant32<kRes>(v + 32, cx.cm + gch * 32 + 32, cx.cC + gch * 32 + 32, rw + 8,
+                                    p.m_r, p.S, ow + 8);
+                }
+                if (in_box) {
+                    p0[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    p0[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                    p1[0] = make_uint4(ow[8], ow[9], ow[10], ow[11]);
+                    p1[1] = make_uint4(ow[12], ow[13], ow[14], ow[15]);
+                }
+                // Results must be visible to the TMA store (async proxy).
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(cx.bars.out_ready(st));
+                if (++st == p.r_stages) {
+                    st = 0;
+                    st_phase ^= 1u;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(cx.bars.acc_empty(acc));
+            if (++acc == n_slots) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+}
+
 template <bool kRes>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_bn_act_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmW,
-                       const __grid_constant__ CUtensorMap tmR, int8_t *__restrict__ out,
+                       const __grid_constant__ CUtensorMap tmR,
+                       const __grid_constant__ CUtensorMap tmO,
                        const int32_t *__restrict__ bias, const int32_t *__restrict__ mult,
                        const ConvPlan p)
 {
@@ -123,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int group = blockIdx.x % p.n_groups;
     const int mt_first = blockIdx.x / p.n_groups;
     const int mt_step = gridDim.x / p.n_groups;
+    const int stages_per_tile = p.NC / (32 * kRChunks);
 
     // ---- set-up ---------------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -135,8 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bars.a_empty(s), 1);
         }
         for (int s = 0; s < p.r_stages; ++s) {
-            mbar_init(bars.r_full(s), 1);
-            mbar_init(bars.r_empty(s), kEpiWarps);
+            mbar_init(bars.io_full(s), 1);
+            mbar_init(bars.out_ready(s), kEpiWarps);
+            mbar_init(bars.io_empty(s), 1);
         }
         for (int s = 0; s < 4; ++s) {
             mbar_init(bars.acc_full(s), 1);
@@ -147,16 +380,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmO);
         if (kRes)
             tma_prefetch_desc(&tmR);
     }
-    // Folded-BN constants of this CTA's channels: C = bias*m + 2^(S-1), so
-    // that t = acc*m + C (+ r*m_r) needs one wide multiply-add per term.
+    // Folded-BN constants of this CTA's channels.  Generic form:
+    // C = bias*m + 2^(S-1), so that t = acc*m + C (+ r*m_r) is one wide
+    // multiply-add per term.  Fast form (when exact for every channel of the
+    // CTA): m' = m*2^(32-S), C' = bias*m' + 2^31 (see requant_fast).
+    // All-32-bit form (see requant_hi32): m'' = m*2^(33-S) and bias as int32.
+    const int K = p.kb_per_tile * kKBlock;
+    bool my_fast = true, my_hi = true;
+    for (int n = threadIdx.x; n < p.NC; n += blockDim.x) {
+        const int o = group * p.NC + n;
+        my_fast = my_fast && fast_form_ok(mult[o], bias[o], p.m_r, p.S, K, kRes);
+        my_hi = my_hi && hi32_ok(mult[o], bias[o], p.S, K);
+    }
+    const bool all_fast = __syncthreads_and(my_fast ? 1 : 0) != 0;
+    const bool all_hi = __syncthreads_and(my_hi ? 1 : 0) != 0 && hi32_layer_ok(p.m_r, p.S, kRes);
+    const int mode = all_hi ? 2 : (all_fast ? 1 : 0);
+    int32_t *cb = reinterpret_cast<int32_t *>(cC);  // bias, in the all-32-bit form
     for (int n = threadIdx.x; n < p.NC; n += blockDim.x) {
         const int o = group * p.NC + n;
         const long long mm = mult[o];
-        cm[n] = static_cast<int32_t>(mm);
-        cC[n] = static_cast<long long>(bias[o]) * mm + (1ll << (p.S - 1));
+        if (mode == 2) {
+            cm[n] = static_cast<int32_t>(mm * (1ll << (33 - p.S)));
+            cb[n] = bias[o];
+        } else if (mode == 1) {
+            const long long mp = mm * (1ll << (32 - p.S));
+            cm[n] = static_cast<int32_t>(mp);
+            cC[n] = static_cast<long long>(bias[o]) * mp + (1ll << 31);
+        } else {
+            cm[n] = static_cast<int32_t>(mm);
+            cC[n] = static_cast<long long>(bias[o]) * mm + (1ll << (p.S - 1));
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -178,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             group * (p.NC / 128));
             const uint32_t abytes = static_cast<uint32_t>(p.rows * 32);
             const uint32_t sa = sbase + p.off_a;
+            const uint64_t pol = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
@@ -193,8 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes);
-                    tma_load_5d(sa + stage * kASlotBytes, &tmA, bars.a_full(stage), 0,
-                                w0 + ds - p.pad, h0 + dr - p.pad, c1, b0);
+                    tma_load_5d_hint(sa + stage * kASlotBytes, &tmA, bars.a_full(stage), 0,
+                                     w0 + ds - p.pad, h0 + dr - p.pad, c1, b0, pol);
                     ++issued;
                     if (++stage == p.a_stages) {
                         stage = 0;
@@ -215,11 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ---- producer: shortcut tiles (issued as early as the ring allows) ------
-        if (kRes && lane == 0) {
+        // ---- producer of I/O stages: shortcut tiles, issued as early as the ring
+        // allows; without a shortcut it only hands out free stages ----------------
+        if (lane == 0) {
             const uint32_t rbytes = static_cast<uint32_t>(kRChunks * p.rows * 32);
-            const uint32_t sr = sbase + p.off_r;
-            const int stages_per_tile = p.NC / (32 * kRChunks);
+            const uint32_t sio = sbase + p.off_r;
+            const uint64_t pol = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
@@ -228,14 +487,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int w0, h0, b0;
                 tile_origin(p, mt, w0, h0, b0);
                 for (int rs = 0; rs < stages_per_tile; ++rs) {
-                    if (!mbar_wait(bars.r_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
+                    if (!mbar_wait(bars.io_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(bars.r_full(stage), rbytes);
-                    tma_load_5d(sr + stage * kRSlotBytes, &tmR, bars.r_full(stage), 0, w0, h0,
-                                group * (p.NC / 32) + rs * kRChunks, b0);
-                    ++issued;
+                    if (kRes) {
+                        mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
+                        const int o1 = group * (p.NC / 32) + rs * kRChunks;
+                        if (p.io_wide)
+                            tma_load_4d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
+                                             w0 * 4, h0, o1, b0, pol);
+                        else
+                            tma_load_5d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
+                                             0, w0, h0, o1, b0, pol);
+                        ++issued;
+                    } else {
+                        mbar_arrive(bars.io_full(stage));
+                    }
                     if (++stage == p.r_stages) {
                         stage = 0;
                         phase ^= 1u;
@@ -246,9 +514,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (long long i = issued - last; i < issued; ++i) {
                 const int s = static_cast<int>(i % p.r_stages);
                 const uint32_t ph = static_cast<uint32_t>((i / p.r_stages) & 1);
-                if (!mbar_drain(bars.r_full(s), ph, drain_ns))
+                if (!mbar_drain(bars.io_full(s), ph, drain_ns))
                     atomicOr(&g_dev_status, kDevDrainFailed);
             }
+        }
+        __syncwarp();
+    } else if (warp == 3) {
+        // ---- TMA store of finished I/O stages ----------------------------------------
+        // After issuing the store of stage i it waits until the store of stage
+        // i-1 has read its shared memory, then hands stage i-1 back.
+        if (lane == 0) {
+            const uint32_t sio = sbase + p.off_r;
+            const uint64_t pol = policy_evict_first();
+            int stage = 0, prev = -1;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
+                int w0, h0, b0;
+                tile_origin(p, mt, w0, h0, b0);
+                for (int rs = 0; rs < stages_per_tile; ++rs) {
+                    if (!mbar_wait(bars.out_ready(stage), phase, ctl, kDevTimeoutProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const int o1 = group * (p.NC / 32) + rs * kRChunks;
+                    if (p.io_wide)
+                        tma_store_4d_hint(&tmO, sio + stage * kRSlotBytes, w0 * 4, h0, o1, b0, pol);
+                    else
+                        tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0, h0, o1, b0, pol);
+                    bulk_commit();
+                    if (prev >= 0) {
+                        bulk_wait_read<1>();
+                        mbar_arrive(bars.io_empty(prev));
+                    }
+                    prev = stage;
+                    if (++stage == p.r_stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // Every store must have finished (read and written) before exit.
+            bulk_wait_all();
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -313,104 +620,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 atomicOr(&g_dev_status, kDevDrainFailed);
         }
         __syncwarp();
-    } else if (warp >= kEpiWarp0) {
+    } else {
         // ---- epilogue ---------------------------------------------------------------
-        const int q = warp & 3;           // TMEM lane quarter this warp may access
-        const int half = (warp - kEpiWarp0) >> 2;  // which chunks of a stage
-        const int row = q * 32 + lane;    // GEMM row = pixel of the tile
-        const int plane_t = p.tw * p.th;
-        const int xi = row % p.tw;
-        const int yi = (row / p.tw) % p.th;
-        const int gi = row / plane_t;
-        const bool in_box = row < p.rows;
-        const long long HWp = static_cast<long long>(p.Hp) * p.Wp;
-        const int n_slots = kTmemCols / p.nmma;
-        const int stages_per_sub = p.nmma / (32 * kRChunks);
-        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        const uint8_t *sr = smem + p.off_r;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        int r_stage = 0;
-        uint32_t r_phase = 0;
-        bool ok = true;
-        for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
-            int w0, h0, b0;
-            tile_origin(p, mt, w0, h0, b0);
-            const int b = b0 + gi, hh = h0 + yi, ww = w0 + xi;
-            const bool valid = in_box && b < p.B && hh < p.Hp && ww < p.Wp;
-            const long long pix_off =
-                (static_cast<long long>(b) * p.O1 * HWp + static_cast<long long>(hh) * p.Wp + ww) *
-                32;
-            for (int j = 0; ok && j < p.n_subs; ++j) {
-                // Every lane waits; the vote keeps the warp's decision uniform so
-                // that the .sync.aligned TMEM loads below always run converged.
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(bars.acc_full(acc), acc_phase, ctl, kDevTimeoutEpilogue))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                for (int rl = 0; rl < stages_per_sub; ++rl) {
-                    if (kRes && !__all_sync(0xffffffffu, mbar_wait(bars.r_full(r_stage), r_phase,
-                                                                   ctl, kDevTimeoutEpilogue))) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll 1
-                    for (int c = half; c < kRChunks; c += 2) {
-                        const int cs = rl * kRChunks + c;           // chunk within the sub
-                        const int gch = j * (p.nmma / 32) + cs;     // chunk within the group
-                        uint32_t v[32];
-                        __syncwarp();
-                        tmem_ld_32x32b_x32(tmem_base + lane_addr +
-                                               static_cast<uint32_t>(acc * p.nmma + cs * 32),
-                                           v);
-                        tmem_wait_ld(v);
-                        if (valid) {
-                            uint32_t rw[8];
-                            if (kRes) {
-                                const uint4 *rp = reinterpret_cast<const uint4 *>(
-                                    sr + r_stage * kRSlotBytes +
-                                    ((gi * kRChunks + c) * plane_t + yi * p.tw + xi) * 32);
-                                const uint4 ra = rp[0], rb = rp[1];
-                                rw[0] = ra.x; rw[1] = ra.y; rw[2] = ra.z; rw[3] = ra.w;
-                                rw[4] = rb.x; rw[5] = rb.y; rw[6] = rb.z; rw[7] = rb.w;
-                            } else {
-#pragma unroll
-                                for (int k = 0; k < 8; ++k)
-                                    rw[k] = 0u;
-                            }
-                            uint32_t ow[8];
-                            requant32<kRes>(v, cm + gch * 32, cC + gch * 32, rw, p.m_r, p.S, ow);
-                            const int o1 = group * (p.NC / 32) + gch;
-                            uint4 *op = reinterpret_cast<uint4 *>(
-                                out + pix_off + static_cast<long long>(o1) * HWp * 32);
-                            op[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                            op[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-                        }
-                    }
-                    if (kRes) {
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(bars.r_empty(r_stage));
-                        if (++r_stage == p.r_stages) {
-                            r_stage = 0;
-                            r_phase ^= 1u;
-                        }
-                    }
-                }
-                if (!ok)
-                    break;
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(bars.acc_empty(acc));
-                if (++acc == n_slots) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
-            }
-        }
+        const EpiCtx cx{&p, bars, ctl, tmem_base, smem + p.off_r, cm, cC,
+                        group, mt_first, mt_step};
+        if (mode == 2)
+            epilogue_warp<kRes, 2>(cx, warp, lane);
+        else if (mode == 1)
+            epilogue_warp<kRes, 1>(cx, warp, lane);
+        else
+            epilogue_warp<kRes, 0>(cx, warp, lane);
         __syncwarp();
     }
 
@@ -440,7 +659,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode()
 }
 
 int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
-               const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz)
+               const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8)
 {
     auto fn = get_encode();
     if (!fn)
@@ -455,7 +675,7 @@ int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
     }
     for (int i = 0; i < rank - 1; ++i)
         s[i] = strides_bytes[i];
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank),
+    CUresult r = fn(m, dtype, static_cast<cuuint32_t>(rank),
                     const_cast<void *>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? X1CB_OK : X1CB_ERR_CUDA;
@@ -532,7 +752,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     p.num_m_tiles = static_cast<int>(mtiles);
     p.kb_per_tile = R * R * p.C1;
 
-    const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 8) * 8 + 64;
+    const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 12) * 8 + 64;
     int chosen = 0;
     long long chosen_work = -1;
     for (int NC = std::min(Oc, 512); NC >= 128; NC -= 128) {
@@ -541,7 +761,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
         const int nmma = NC >= 256 ? 256 : 128;
         const int n_subs = NC / nmma;
         const int a_min = n_subs > 1 ? p.kb_per_tile + 2 : 4;
-        const int r_min = has_res ? 4 : 0;
+        const int r_min = has_res ? 4 : 2;
         const long long need = static_cast<long long>(p.kb_per_tile) * NC * 32 + NC * 12 +
                                a_min * kASlotBytes + r_min * kRSlotBytes + fixed;
         if (need > kSmemLimit || a_min > 48)
@@ -566,15 +786,14 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     const int rem = kSmemLimit - fixed - wbytes - p.NC * 12;
     // Split what is left between the two rings: the activation ring first gets
     // a tile's K blocks plus a few (capped), the shortcut ring the rest.
-    const int a_want = std::max(a_min, std::min(p.kb_per_tile + 4, 12));
-    if (has_res) {
-        p.r_stages = std::max(4, std::min(8, (rem - a_want * kASlotBytes) / kRSlotBytes));
-        p.a_stages = std::max(a_min, std::min(48, (rem - p.r_stages * kRSlotBytes) / kASlotBytes));
-    } else {
-        p.r_stages = 0;
-        p.a_stages = std::max(a_min, std::min(48, rem / kASlotBytes));
-    }
+    const int a_want = std::max(a_min, std::min(p.kb_per_tile + 2, 8));
+    // I/O stages carry the shortcut in and the result out; without a shortcut
+    // they only stage results for the TMA store, so fewer are needed.
+    const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 6;
+    p.r_stages = std::max(r_lo, std::min(r_hi, (rem - a_want * kASlotBytes) / kRSlotBytes));
+    p.a_stages = std::max(a_min, std::min(48, (rem - p.r_stages * kRSlotBytes) / kASlotBytes));
 
+    p.io_wide = p.tw * 4 <= 256 ? 1 : 0;  // TMA box dimensions are at most 256 elements
     p.off_w = 0;
     p.off_a = p.off_w + wbytes;
     p.off_r = p.off_a + p.a_stages * kASlotBytes;
@@ -599,7 +818,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
 int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32_t *bias,
                 const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream)
 {
-    CUtensorMap tmA, tmW, tmR;
+    CUtensorMap tmA, tmW, tmR, tmO;
     // Activations: dims (32 ch, Wp, Hp, C1, B); box (32, tw, th, 1, tg).
     {
         const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.C1,
@@ -618,18 +837,41 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         if (int e = encode_map(&tmW, w, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }
-    if (p.has_res) {
-        // Shortcut: dims (32, Wp, Hp, O1, B); box (32, tw, th, 4, tg), no swizzle.
+    // Shortcut and output, no swizzle: one box is one I/O stage [tg][4][th][tw][32].
+    // Wide form: the same bytes as 8-byte elements, dims (4*Wp, Hp, O1, B) and
+    // box (4*tw, th, 4, tg), so a box row is one contiguous run of tw*32 bytes.
+    if (p.io_wide) {
+        const uint64_t dims[4] = {(uint64_t)p.Wp * 4, (uint64_t)p.Hp, (uint64_t)p.O1,
+                                  (uint64_t)p.B};
+        const uint64_t str[3] = {(uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
+                                 (uint64_t)p.O1 * p.Hp * p.Wp * 32};
+        const uint32_t box[4] = {(uint32_t)p.tw * 4, (uint32_t)p.th, (uint32_t)kRChunks,
+                                 (uint32_t)p.tg};
+        if (int e = encode_map(&tmO, out, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+            return e;
+        if (p.has_res) {
+            if (int e = encode_map(&tmR, r, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                   CU_TENSOR_MAP_DATA_TYPE_UINT64))
+                return e;
+        } else {
+            tmR = tmO;  // unused
+        }
+    } else {
         const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.O1,
                                   (uint64_t)p.B};
         const uint64_t str[4] = {32, (uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
                                  (uint64_t)p.O1 * p.Hp * p.Wp * 32};
         const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)p.th, (uint32_t)kRChunks,
                                  (uint32_t)p.tg};
-        if (int e = encode_map(&tmR, r, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+        if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return e;
-    } else {
-        tmR = tmA;  // unused
+        if (p.has_res) {
+            if (int e = encode_map(&tmR, r, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+                return e;
+        } else {
+            tmR = tmO;  // unused
+        }
     }
     auto kern = p.has_res ? conv_bn_act_kernel<true> : conv_bn_act_kernel<false>;
     static bool attr_set[2] = {false, false};
@@ -639,7 +881,7 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
             return X1CB_ERR_CUDA;
         attr_set[p.has_res] = true;
     }
-    kern<<<p.grid, kThreads, p.smem_bytes, stream>>>(tmA, tmW, tmR, out, bias, mult, p);
+    kern<<<p.grid, kThreads, p.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, bias, mult, p);
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 

@@ -5,9 +5,10 @@
 
 namespace x1cb {
 
-constexpr int kThreads = 384;       // 12 warps: 4 control/producer + 8 epilogue
-constexpr int kEpiWarp0 = 4;        // first epilogue warp
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarp0 = 4;        // warps 0-3: producers, MMA issuer, store
+constexpr int kEpiWarps = 8;        // 2 per TMEM lane quarter
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+static_assert(kEpiWarp0 % 4 == 0 && kEpiWarps % 4 == 0, "roles must be whole warpgroups");
 constexpr int kTileRows = 128;      // MMA M
 constexpr int kKBlock = 32;         // int8 channels per K block (one MMA K step)
 constexpr int kASlotBytes = kTileRows * kKBlock;  // 4 KB per A ring slot
@@ -42,6 +43,7 @@ struct ConvPlan {
     // shared memory offsets from the 1024-aligned base
     int off_w, off_a, off_r, off_cc, off_cm, off_bar, off_misc;
     int smem_bytes;  // including alignment slack
+    int io_wide;  // shortcut/output maps use 8-byte elements (box rows of tw*32 bytes)
     // control
     int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
     unsigned long long wait_limit_ns;

@@ -126,6 +126,235 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *m, 
         : "memory");
 }
 
+// Tiled tensor stores from shared memory complete in bulk groups.  Every
+// coordinate must be >= 0; elements outside the tensor are not written.
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until every committed bulk group has completed (writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Byte permute (prmt.b32, default mode): each selector nibble picks one of
+// the 8 bytes of {b, a}; a set high bit in the nibble replicates that byte's
+// sign bit instead of copying it.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Four outputs of the exact fast requantisation (see requant32_fast):
+//   t_e = acc_e * m_e + c_e  (+ rs_e * mr2, rs_e = shortcut byte e permuted by rsel_e)
+//   y_e = max(min(hi32(t_e), 127), 0), four bytes packed into one word.
+#ifndef X1CB_PACK_PRMT
+// byte packing by multiply-adds (runs on the FMA pipe, which has headroom)
+#define PACK4                                          \
+    "mad.lo.u32 p, y1, 256, y0;\n\t"                 \
+    "mad.lo.u32 y2, y3, 256, y2;\n\t"                \
+    "mad.lo.u32 %0, y2, 65536, p;\n\t"
+#else
+#define PACK4                                          \
+    "prmt.b32 p, y0, y1, 0x0040;\n\t"                \
+    "prmt.b32 y2, y2, y3, 0x0040;\n\t"               \
+    "prmt.b32 %0, p, y2, 0x5410;\n\t"
+#endif
+template <bool kRes>
+__device__ __forceinline__ uint32_t requant4_fast(uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, int4 m, longlong2 c01,
+                                                  longlong2 c23, uint32_t rword,
+                                                  const uint32_t (&rsel)[4], int mr2)
+{
+    uint32_t d;
+    if (kRes) {
+        asm("{\n\t"
+            ".reg .b64 t0, t1, t2, t3;\n\t"
+            ".reg .b32 r0, r1, r2, r3, l0, l1, l2, l3, y0, y1, y2, y3, p;\n\t"
+            "mad.wide.s32 t0, %1, %5, %9;\n\t"
+            "mad.wide.s32 t1, %2, %6, %10;\n\t"
+            "mad.wide.s32 t2, %3, %7, %11;\n\t"
+            "mad.wide.s32 t3, %4, %8, %12;\n\t"
+            "prmt.b32 r0, %13, 0, %14;\n\t"
+            "prmt.b32 r1, %13, 0, %15;\n\t"
+            "prmt.b32 r2, %13, 0, %16;\n\t"
+            "prmt.b32 r3, %13, 0, %17;\n\t"
+            "mad.wide.s32 t0, r0, %18, t0;\n\t"
+            "mad.wide.s32 t1, r1, %18, t1;\n\t"
+            "mad.wide.s32 t2, r2, %18, t2;\n\t"
+            "mad.wide.s32 t3, r3, %18, t3;\n\t"
+            "mov.b64 {l0, y0}, t0;\n\t"
+            "mov.b64 {l1, y1}, t1;\n\t"
+            "mov.b64 {l2, y2}, t2;\n\t"
+            "mov.b64 {l3, y3}, t3;\n\t"
+            "min.relu.s32 y0, y0, 127;\n\t"
+            "min.relu.s32 y1, y1, 127;\n\t"
+            "min.relu.s32 y2, y2, 127;\n\t"
+            "min.relu.s32 y3, y3, 127;\n\t"
+            PACK4
+            "}"
+            : "=r"(d)
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
+              "l"(c01.x), "l"(c01.y), "l"(c23.x), "l"(c23.y), "r"(rword), "r"(rsel[0]),
+              "r"(rsel[1]), "r"(rsel[2]), "r"(rsel[3]), "r"(mr2));
+    } else {
+        asm("{\n\t"
+            ".reg .b64 t0, t1, t2, t3;\n\t"
+            ".reg .b32 l0, l1, l2, l3, y0, y1, y2, y3, p;\n\t"
+            "mad.wide.s32 t0, %1, %5, %9;\n\t"
+            "mad.wide.s32 t1, %2, %6, %10;\n\t"
+            "mad.wide.s32 t2, %3, %7, %11;\n\t"
+            "mad.wide.s32 t3, %4, %8, %12;\n\t"
+            "mov.b64 {l0, y0}, t0;\n\t"
+            "mov.b64 {l1, y1}, t1;\n\t"
+            "mov.b64 {l2, y2}, t2;\n\t"
+            "mov.b64 {l3, y3}, t3;\n\t"
+            "min.relu.s32 y0, y0, 127;\n\t"
+            "min.relu.s32 y1, y1, 127;\n\t"
+            "min.relu.s32 y2, y2, 127;\n\t"
+            "min.relu.s32 y3, y3, 127;\n\t"
+            PACK4
+            "}"
+            : "=r"(d)
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
+              "l"(c01.x), "l"(c01.y), "l"(c23.x), "l"(c23.y));
+    }
+    return d;
+}
+
+// Four outputs of the exact all-32-bit form (see requant_hi32):
+//   y2_e = hi32((acc_e + bias_e) * m_e) + 1 (+ r_e * k),  r_e = shortcut byte e
+//   out_e = min(max(y2_e, 0), 255) >> 1, four bytes packed into one word.
+template <bool kRes>
+__device__ __forceinline__ uint32_t requant4_hi32(uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, int4 m, int4 b, uint32_t rword,
+                                                  const uint32_t (&rsel)[4], int k)
+{
+    uint32_t d;
+    if (kRes) {
+        asm("{\n\t"
+            ".reg .b32 u0, u1, u2, u3, r0, r1, r2, r3, y0, y1, y2, y3, p, q;\n\t"
+            "add.s32 u0, %1, %9;\n\t"
+            "add.s32 u1, %2, %10;\n\t"
+            "add.s32 u2, %3, %11;\n\t"
+            "add.s32 u3, %4, %12;\n\t"
+            "prmt.b32 r0, %13, 0, %14;\n\t"
+            "prmt.b32 r1, %13, 0, %15;\n\t"
+            "prmt.b32 r2, %13, 0, %16;\n\t"
+            "prmt.b32 r3, %13, 0, %17;\n\t"
+            "mad.lo.s32 r0, r0, %18, 1;\n\t"
+            "mad.lo.s32 r1, r1, %18, 1;\n\t"
+            "mad.lo.s32 r2, r2, %18, 1;\n\t"
+            "mad.lo.s32 r3, r3, %18, 1;\n\t"
+            "mad.hi.s32 y0, u0, %5, r0;\n\t"
+            "mad.hi.s32 y1, u1, %6, r1;\n\t"
+            "mad.hi.s32 y2, u2, %7, r2;\n\t"
+            "mad.hi.s32 y3, u3, %8, r3;\n\t"
+            "min.relu.s32 y0, y0, 255;\n\t"
+            "min.relu.s32 y1, y1, 255;\n\t"
+            "min.relu.s32 y2, y2, 255;\n\t"
+            "min.relu.s32 y3, y3, 255;\n\t"
+            "mad.lo.u32 p, y1, 256, y0;\n\t"
+            "mad.lo.u32 q, y3, 256, y2;\n\t"
+            "mad.lo.u32 p, q, 65536, p;\n\t"
+            "shr.b32 p, p, 1;\n\t"
+            "and.b32 %0, p, 0x7f7f7f7f;\n\t"
+            "}"
+            : "=r"(d)
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
+              "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(rword), "r"(rsel[0]), "r"(rsel[1]),
+              "r"(rsel[2]), "r"(rsel[3]), "r"(k));
+    } else {
+        asm("{\n\t"
+            ".reg .b32 u0, u1, u2, u3, y0, y1, y2, y3, p, q;\n\t"
+            "add.s32 u0, %1, %9;\n\t"
+            "add.s32 u1, %2, %10;\n\t"
+            "add.s32 u2, %3, %11;\n\t"
+            "add.s32 u3, %4, %12;\n\t"
+            "mad.hi.s32 y0, u0, %5, 1;\n\t"
+            "mad.hi.s32 y1, u1, %6, 1;\n\t"
+            "mad.hi.s32 y2, u2, %7, 1;\n\t"
+            "mad.hi.s32 y3, u3, %8, 1;\n\t"
+            "min.relu.s32 y0, y0, 255;\n\t"
+            "min.relu.s32 y1, y1, 255;\n\t"
+            "min.relu.s32 y2, y2, 255;\n\t"
+            "min.relu.s32 y3, y3, 255;\n\t"
+            "mad.lo.u32 p, y1, 256, y0;\n\t"
+            "mad.lo.u32 q, y3, 256, y2;\n\t"
+            "mad.lo.u32 p, q, 65536, p;\n\t"
+            "shr.b32 p, p, 1;\n\t"
+            "and.b32 %0, p, 0x7f7f7f7f;\n\t"
+            "}"
+            : "=r"(d)
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
+              "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
+    }
+    return d;
+}
+
+// L2 policy for data read or written once: evict it first.
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                                 int c0, int c1, int c2, int c3, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "l"(pol)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_5d_hint(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                                 int c0, int c1, int c2, int c3, int c4,
+                                                 uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(c4), "l"(pol)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_4d_hint(const CUtensorMap *m, uint32_t src, int c0,
+                                                  int c1, int c2, int c3, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group.L2::cache_hint"
+        " [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(reinterpret_cast<uint64_t>(m)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(pol)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_5d_hint(const CUtensorMap *m, uint32_t src, int c0,
+                                                  int c1, int c2, int c3, int c4, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group.L2::cache_hint"
+        " [%0, {%2, %3, %4, %5, %6}], [%1], %7;" ::"l"(reinterpret_cast<uint64_t>(m)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "l"(pol)
+        : "memory");
+}
+
 // ---- tcgen05: TMEM, MMA, loads -----------------------------------------------
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
@@ -215,6 +444,44 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)
           "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
           "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
           "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// tcgen05.ld of 32 columns followed by its wait in one statement, so the
+// registers are defined only once the data has arrived.
+__device__ __forceinline__ void tmem_ld_32x32b_x32_sync(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// 32 lanes x 64 consecutive columns (two 32-channel chunks), load and wait.
+__device__ __forceinline__ void tmem_ld_32x32b_x64_sync(uint32_t taddr, uint32_t (&v)[64])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+          "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]),
+          "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]),
+          "=r"(v[48]), "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+          "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]), "=r"(v[63])
         : "r"(taddr)
         : "memory");
 }
