@@ -11,7 +11,7 @@
 //
 // How it computes it is designed for B200 rather than taken from the
 // article's A100 kernel:
-//  * one persistent CTA per SM, 12 warps, warp-specialised:
+//  * one persistent CTA per SM, 20 warps, warp-specialised:
 //      warp 0      TMA producer: weights (once, resident in shared memory) and
 //                  the activation tiles (one 128-row x 32-byte K block per slot)
 //      warp 1      MMA issuer: tcgen05.mma.kind::i8 into TMEM (int32), owner
@@ -19,7 +19,7 @@
 //      warp 2      TMA producer of the I/O stages: each 16 KB stage receives a
 //                  shortcut tile (128 pixels x 128 channels) long before use
 //      warp 3      TMA store of finished I/O stages
-//      warps 4-11  epilogue: tcgen05.ld, exact requantisation; each result
+//      warps 4-19  epilogue: tcgen05.ld, exact requantisation; each result
 //                  byte overwrites the shortcut byte of the same (pixel,
 //                  channel) in the stage, which warp 3 then stores whole
 //  * a tile is 128 GEMM rows = tw x th pixels of tg images, chosen per shape
@@ -216,11 +216,13 @@ struct EpiCtx {
 template <bool kRes, int kMode>
 __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int lane)
 {
-    static_assert(kEpiWarps == 8, "two warps per lane quarter, two chunks each per stage");
+    constexpr int kPerQuarter = kEpiWarps / 4;           // warps sharing a TMEM lane quarter
+    constexpr int kCPW = kRChunks / kPerQuarter;          // adjacent chunks per warp per stage
+    static_assert(kCPW == 1 || kCPW == 2, "one or two 32-channel chunks per warp and stage");
     const ConvPlan &p = *cx.p;
-    const int q = warp & 3;                    // TMEM lane quarter this warp may access
-    const int c0 = 2 * ((warp - kEpiWarp0) >> 2);  // first of the two chunks it takes per stage
-    const int row = q * 32 + lane;             // GEMM row = pixel of the tile
+    const int q = warp & 3;                               // TMEM lane quarter this warp may access
+    const int c0 = kCPW * ((warp - kEpiWarp0) >> 2);      // first chunk it takes per stage
+    const int row = q * 32 + lane;                        // GEMM row = pixel of the tile
     const int plane_t = p.tw * p.th;
     const int xi = row % p.tw;
     const int yi = (row / p.tw) % p.th;
@@ -274,36 +276,49 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                 uint8_t *stage = cx.io + st * kRSlotBytes + row_off;
                 const int cs = rl * kRChunks + c0;         // chunk within the TMEM slot
                 const int gch = j * chunks_per_sub + cs;   // chunk within the CTA's channels
-                uint32_t v[64];
+                uint32_t v[32 * kCPW];
                 __syncwarp();
-                tmem_ld_32x32b_x64_sync(tbase + static_cast<uint32_t>(cs * 32), v);
-                uint4 *p0 = reinterpret_cast<uint4 *>(stage + c0 * chunk_stride);
-                uint4 *p1 = reinterpret_cast<uint4 *>(stage + (c0 + 1) * chunk_stride);
-                uint32_t rw[16];
+                if (kCPW == 2)
+                    tmem_ld_32x32b_x64_sync(tbase + static_cast<uint32_t>(cs * 32),
+                                            *reinterpret_cast<uint32_t(*)[64]>(v));
+                else
+                    tmem_ld_32x32b_x32_sync(tbase + static_cast<uint32_t>(cs * 32),
+                                            *reinterpret_cast<uint32_t(*)[32]>(v));
+                uint4 *pc[kCPW];
+#pragma unroll
+                for (int i = 0; i < kCPW; ++i)
+                    pc[i] = reinterpret_cast<uint4 *>(stage + (c0 + i) * chunk_stride);
+                uint32_t rw[8 * kCPW];
                 if (kRes) {
-                    const uint4 ra = p0[0], rb = p0[1], rc = p1[0], rd = p1[1];
-                    rw[0] = ra.x; rw[1] = ra.y; rw[2] = ra.z; rw[3] = ra.w;
-                    rw[4] = rb.x; rw[5] = rb.y; rw[6] = rb.z; rw[7] = rb.w;
-                    rw[8] = rc.x; rw[9] = rc.y; rw[10] = rc.z; rw[11] = rc.w;
-                    rw[12] = rd.x; rw[13] = rd.y; rw[14] = rd.z; rw[15] = rd.w;
+#pragma unroll
+                    for (int i = 0; i < kCPW; ++i) {
+                        const uint4 ra = pc[i][0], rb = pc[i][1];
+                        rw[8 * i + 0] = ra.x; rw[8 * i + 1] = ra.y; rw[8 * i + 2] = ra.z;
+                        rw[8 * i + 3] = ra.w; rw[8 * i + 4] = rb.x; rw[8 * i + 5] = rb.y;
+                        rw[8 * i + 6] = rb.z; rw[8 * i + 7] = rb.w;
+                    }
                 }
-                uint32_t ow[16];
+                uint32_t ow[8 * kCPW];
                 if (kMode == 2) {
-                    requant_hi32<kRes, 16>(v, cx.cm + gch * 32,
-                                           reinterpret_cast<const int32_t *>(cx.cC) + gch * 32,
-                                           rw, mr2, rsel, ow);
+                    requant_hi32<kRes, 8 * kCPW>(v, cx.cm + gch * 32,
+                                                 reinterpret_cast<const int32_t *>(cx.cC) + gch * 32,
+                                                 rw, mr2, rsel, ow);
                 } else if (kMode == 1) {
-                    requant_fast<kRes, 16>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2, rsel, ow);
+                    requant_fast<kRes, 8 * kCPW>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2,
+                                                 rsel, ow);
                 } else {
-                    requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
-                    requant32<kRes>(v + 32, cx.cm + gch * 32 + 32, cx.cC + gch * 32 + 32, rw + 8,
-                                    p.m_r, p.S, ow + 8);
+#pragma unroll
+                    for (int i = 0; i < kCPW; ++i)
+                        requant32<kRes>(v + 32 * i, cx.cm + gch * 32 + 32 * i,
+                                        cx.cC + gch * 32 + 32 * i, rw + 8 * i, p.m_r, p.S,
+                                        ow + 8 * i);
                 }
                 if (in_box) {
-                    p0[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    p0[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-                    p1[0] = make_uint4(ow[8], ow[9], ow[10], ow[11]);
-                    p1[1] = make_uint4(ow[12], ow[13], ow[14], ow[15]);
+#pragma unroll
+                    for (int i = 0; i < kCPW; ++i) {
+                        pc[i][0] = make_uint4(ow[8 * i + 0], ow[8 * i + 1], ow[8 * i + 2], ow[8 * i + 3]);
+                        pc[i][1] = make_uint4(ow[8 * i + 4], ow[8 * i + 5], ow[8 * i + 6], ow[8 * i + 7]);
+                    }
                 }
                 // Results must be visible to the TMA store (async proxy).
                 fence_proxy_async_smem();

@@ -6,7 +6,7 @@
 namespace x1cb {
 
 constexpr int kEpiWarp0 = 4;        // warps 0-3: producers, MMA issuer, store
-constexpr int kEpiWarps = 8;        // 2 per TMEM lane quarter
+constexpr int kEpiWarps = 16;       // 4 per TMEM lane quarter
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 static_assert(kEpiWarp0 % 4 == 0 && kEpiWarps % 4 == 0, "roles must be whole warpgroups");
 constexpr int kTileRows = 128;      // MMA M
