@@ -148,6 +148,34 @@ def test_conv1x1_hand_cases(oracle):
     assert torch.equal(got, _oracle_conv(oracle, inp))
 
 
+def test_conv1x1_bias_too_large_to_fold(oracle):
+    """Biases beyond the range the MMA can fold (|bias| > 2^18) take the
+    all-32-bit form with the bias added in the epilogue."""
+    s = synth.ConvShape(3, 14, 14, 128, 256, 1, True)
+    inp = synth.conv_inputs(s, 71)
+    g = torch.Generator().manual_seed(72)
+    inp.bias = torch.randint(-(1 << 20), (1 << 20) + 1, (s.Oc,), generator=g, dtype=torch.int32)
+    inp.bias[0] = (1 << 18) + 1
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref)
+    assert 0.05 < (ref == 0).float().mean().item() < 0.95
+
+
+def test_conv1x1_mixed_epilogue_forms_across_ctas(oracle):
+    """B=1 splits the 512 output channels over 4 CTA groups; group 1 gets a
+    bias too large to fold, group 2 a multiplier too large for the 32-bit
+    forms, group 3 stays in the folded form: every CTA picks its own exact form."""
+    s = synth.CONFIGS["1"]
+    inp = synth.conv_inputs(s, 73)
+    inp.bias[128:256] = inp.bias[128:256] * 64  # |bias| up to 2^20: no fold
+    inp.m[256:384] = inp.m[256:384] * 4096      # m * 2^9 beyond int32: 64-bit form
+    assert "groups=4" in X.x1cb_describe_plan(1, 28, 28, 128, 512, 1, 1)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref)
+
+
 # ---- fused 3x3 ------------------------------------------------------------------
 
 SMALL_3X3 = [

@@ -135,7 +135,7 @@ __device__ __forceinline__ void requant_fast(const uint32_t *v, const int32_t *c
 // so y2 = floor(t * 2^s / 2^32) = hi32((acc + bias) * m') + 1 + r*k exactly
 // (mad.hi), and floor(t / 2^S) = floor(y2 / 2); clamping y2 to [0, 255]
 // before halving gives the [0, 127] clamp.  No 64-bit arithmetic.
-template <bool kRes, int kGroups>
+template <bool kRes, bool kAddBias, int kGroups>
 __device__ __forceinline__ void requant_hi32(const uint32_t *v, const int32_t *cm,
                                              const int32_t *cb, const uint32_t *rw, int k,
                                              const uint32_t (&rsel)[4], uint32_t *ow)
@@ -144,8 +144,45 @@ __device__ __forceinline__ void requant_hi32(const uint32_t *v, const int32_t *c
     const int4 *b4 = reinterpret_cast<const int4 *>(cb);
 #pragma unroll
     for (int q = 0; q < kGroups; ++q)
-        ow[q] = requant4_hi32<kRes>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], m4[q],
-                                    b4[q], kRes ? rw[q] : 0u, rsel, k);
+        ow[q] = requant4_hi32<kRes, kAddBias>(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                              v[4 * q + 3], m4[q],
+                                              kAddBias ? b4[q] : make_int4(0, 0, 0, 0),
+                                              kRes ? rw[q] : 0u, rsel, k);
+}
+
+// Bias folded into the MMA: one extra K step of 32 columns adds
+//   sum_c A[c] * D_n[c] = bias[n]
+// to every row of the accumulator, with the constant A row
+//   [1, 127 x 15, 1, 127 x 15]
+// and per-channel int8 digits D_n: D_n[0] = bias mod 127 (centred), the other
+// 30 digits (columns 1-15, 17-31) carry (bias - D_n[0]) / 127 in steps of at
+// most 127 in magnitude, D_n[16] = 0.  Exact for |bias| <= 30*127*127 + 63;
+// used for |bias| <= 2^18.  Because the two 16-byte halves of the A row are
+// equal, the sum does not depend on which half of a 32-byte row the 32-byte
+// swizzle presents first, so both tiles are written without swizzling.
+constexpr int kBiasFoldMax = 1 << 18;
+
+__device__ __forceinline__ void bias_digits(int bias, uint32_t (&w)[8])
+{
+    int8_t d[32];
+    const int d0 = ((bias + 63) % 127 + 127) % 127 - 63;  // bias mod 127 in [-63, 63]
+    int D = (bias - d0) / 127;
+    d[0] = static_cast<int8_t>(d0);
+    d[16] = 0;
+#pragma unroll
+    for (int c = 1; c < 32; ++c) {
+        if (c == 16)
+            continue;
+        const int step = D > 127 ? 127 : (D < -127 ? -127 : D);
+        d[c] = static_cast<int8_t>(step);
+        D -= step;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        w[i] = static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i])) |
+               static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i + 1])) << 8 |
+               static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i + 2])) << 16 |
+               static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i + 3])) << 24;
 }
 
 // Layer-wide conditions of the all-32-bit form (per channel: hi32_ok).
@@ -212,7 +249,8 @@ struct EpiCtx {
     int group, mt_first, mt_step;
 };
 
-// kMode: 2 = all-32-bit form, 1 = 64-bit fast form, 0 = generic.
+// kMode: 3 = all-32-bit form with the bias folded into the MMA, 2 = all-32-bit
+// form, 1 = 64-bit fast form, 0 = generic.
 template <bool kRes, int kMode>
 __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int lane)
 {
@@ -240,10 +278,10 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     // m_r*2^(s-8*k8).  All-32-bit form: the sign-extended byte (k8 = 0) and
     // k = m_r / 2^(S-1).
     const int sh = 32 - p.S;
-    const int k8 = kMode == 2 ? 0 : (sh < 0 ? 0 : (sh / 8 < 3 ? sh / 8 : 3));
+    const int k8 = kMode >= 2 ? 0 : (sh < 0 ? 0 : (sh / 8 < 3 ? sh / 8 : 3));
     const int mr2 =
         kMode == 1 ? static_cast<int>(static_cast<long long>(p.m_r) * (1ll << (sh - 8 * k8)))
-                   : (kMode == 2 ? static_cast<int>(static_cast<long long>(p.m_r) /
+                   : (kMode >= 2 ? static_cast<int>(static_cast<long long>(p.m_r) /
                                                     (1ll << (p.S - 1)))
                                  : 0);
     uint32_t rsel[4];
@@ -299,10 +337,10 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                     }
                 }
                 uint32_t ow[8 * kCPW];
-                if (kMode == 2) {
-                    requant_hi32<kRes, 8 * kCPW>(v, cx.cm + gch * 32,
-                                                 reinterpret_cast<const int32_t *>(cx.cC) + gch * 32,
-                                                 rw, mr2, rsel, ow);
+                if (kMode >= 2) {
+                    requant_hi32<kRes, kMode == 2, 8 * kCPW>(
+                        v, cx.cm + gch * 32, reinterpret_cast<const int32_t *>(cx.cC) + gch * 32,
+                        rw, mr2, rsel, ow);
                 } else if (kMode == 1) {
                     requant_fast<kRes, 8 * kCPW>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2,
                                                  rsel, ow);
@@ -411,14 +449,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         my_fast = my_fast && fast_form_ok(mult[o], bias[o], p.m_r, p.S, K, kRes);
         my_hi = my_hi && hi32_ok(mult[o], bias[o], p.S, K);
     }
+    bool my_fold = p.fold_room != 0;
+    for (int n = threadIdx.x; n < p.NC; n += blockDim.x) {
+        const int b = bias[group * p.NC + n];
+        my_fold = my_fold && b <= kBiasFoldMax && b >= -kBiasFoldMax;
+    }
     const bool all_fast = __syncthreads_and(my_fast ? 1 : 0) != 0;
     const bool all_hi = __syncthreads_and(my_hi ? 1 : 0) != 0 && hi32_layer_ok(p.m_r, p.S, kRes);
-    const int mode = all_hi ? 2 : (all_fast ? 1 : 0);
+    const bool fold = __syncthreads_and(my_fold ? 1 : 0) != 0 && all_hi;
+    const int mode = all_hi ? (fold ? 3 : 2) : (all_fast ? 1 : 0);
+    if (fold) {
+        // constant A tile (every row [1, 127 x 15, 1, 127 x 15]) and digit rows
+        uint4 *ta = reinterpret_cast<uint4 *>(smem + p.off_ba);
+        for (int i = threadIdx.x; i < kTileRows * 2; i += blockDim.x)
+            ta[i] = make_uint4(0x7F7F7F01u, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        for (int n = threadIdx.x; n < p.NC; n += blockDim.x) {
+            uint32_t w[8];
+            bias_digits(bias[group * p.NC + n], w);
+            uint4 *tb = reinterpret_cast<uint4 *>(smem + p.off_bb + n * 32);
+            tb[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            tb[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        fence_proxy_async_smem();  // the MMA reads these through the async proxy
+    }
     int32_t *cb = reinterpret_cast<int32_t *>(cC);  // bias, in the all-32-bit form
     for (int n = threadIdx.x; n < p.NC; n += blockDim.x) {
         const int o = group * p.NC + n;
         const long long mm = mult[o];
-        if (mode == 2) {
+        if (mode == 3) {
+            cm[n] = static_cast<int32_t>(mm * (1ll << (33 - p.S)));  // bias is in the MMA
+        } else if (mode == 2) {
             cm[n] = static_cast<int32_t>(mm * (1ll << (33 - p.S)));
             cb[n] = bias[o];
         } else if (mode == 1) {
@@ -620,6 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!ok)
                         break;
+                    if (fold)  // + bias: constant A tile x digit rows of this slot's channels
+                        mma_i8(d_tmem, smem_desc_sw32(sbase + p.off_ba),
+                               smem_desc_sw32(sbase + p.off_bb + j * p.nmma * 32), idesc, 1u);
                     mma_commit(bars.acc_full(acc));
                     if (++acc == n_slots) {
                         acc = 0;
@@ -639,7 +702,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- epilogue ---------------------------------------------------------------
         const EpiCtx cx{&p, bars, ctl, tmem_base, smem + p.off_r, cm, cC,
                         group, mt_first, mt_step};
-        if (mode == 2)
+        if (mode == 3)
+            epilogue_warp<kRes, 3>(cx, warp, lane);
+        else if (mode == 2)
             epilogue_warp<kRes, 2>(cx, warp, lane);
         else if (mode == 1)
             epilogue_warp<kRes, 1>(cx, warp, lane);
@@ -798,27 +863,40 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
 
     const int wbytes = p.kb_per_tile * p.NC * 32;
     const int a_min = p.n_subs > 1 ? p.kb_per_tile + 2 : 4;
-    const int rem = kSmemLimit - fixed - wbytes - p.NC * 12;
-    // Split what is left between the two rings: the activation ring first gets
-    // a tile's K blocks plus a few (capped), the shortcut ring the rest.
+    // The activation ring gets a tile's K blocks plus a couple (capped); the
+    // I/O ring (shortcut in, result out) gets as many 16 KB stages as fit --
+    // its depth sets how many bytes are in flight.  Without a shortcut the
+    // stages only stage results, so fewer are needed.  The bias-fold tiles are
+    // reserved when the rings still reach their minimum beside them.
     const int a_want = std::max(a_min, std::min(p.kb_per_tile + 2, 8));
-    // I/O stages carry the shortcut in and the result out; without a shortcut
-    // they only stage results for the TMA store, so fewer are needed.
     const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 6;
-    p.r_stages = std::max(r_lo, std::min(r_hi, (rem - a_want * kASlotBytes) / kRSlotBytes));
-    p.a_stages = std::max(a_min, std::min(48, (rem - p.r_stages * kRSlotBytes) / kASlotBytes));
-
-    p.io_wide = p.tw * 4 <= 256 ? 1 : 0;  // TMA box dimensions are at most 256 elements
-    p.off_w = 0;
-    p.off_a = p.off_w + wbytes;
-    p.off_r = p.off_a + p.a_stages * kASlotBytes;
-    p.off_cc = p.off_r + p.r_stages * kRSlotBytes;
-    p.off_cm = p.off_cc + p.NC * 8;
-    p.off_bar = (p.off_cm + p.NC * 4 + 7) & ~7;
-    p.off_misc = p.off_bar + Bars::count(p.a_stages, p.r_stages) * 8;
-    p.smem_bytes = p.off_misc + 16 + 1024;
-    if (p.smem_bytes > kSmemLimit)
+    auto layout = [&](int fold, int a, int r) {
+        p.fold_room = fold;
+        p.a_stages = a;
+        p.r_stages = r;
+        p.off_w = 0;
+        p.off_ba = p.off_w + wbytes;
+        p.off_bb = p.off_ba + (fold ? kTileRows * 32 : 0);
+        p.off_a = p.off_bb + (fold ? p.NC * 32 : 0);
+        p.off_r = p.off_a + a * kASlotBytes;
+        // The per-channel bias/offset table (modes 0-2) and the fold digit rows
+        // (mode 3) are never used together, so they share space when folding
+        // is possible.
+        p.off_cc = fold ? p.off_bb : p.off_r + r * kRSlotBytes;
+        p.off_cm = (fold ? p.off_r + r * kRSlotBytes : p.off_cc + p.NC * 8);
+        p.off_bar = (p.off_cm + p.NC * 4 + 7) & ~7;
+        p.off_misc = p.off_bar + Bars::count(a, r) * 8;
+        p.smem_bytes = p.off_misc + 16 + 1024;  // + alignment slack of the base
+        return p.smem_bytes <= kSmemLimit;
+    };
+    bool placed = false;
+    for (int fold = 1; fold >= 0 && !placed; --fold)
+        for (int a = a_want; a >= a_min && !placed; --a)
+            for (int r = r_hi; r >= r_lo && !placed; --r)
+                placed = layout(fold, a, r);
+    if (!placed)
         return X1CB_ERR_SHAPE;
+    p.io_wide = p.tw * 4 <= 256 ? 1 : 0;  // TMA box dimensions are at most 256 elements
 
     const long long work = mtiles * p.n_groups;
     long long grid = std::min<long long>(num_sms, work);

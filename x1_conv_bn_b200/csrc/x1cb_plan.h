@@ -44,6 +44,10 @@ struct ConvPlan {
     int off_w, off_a, off_r, off_cc, off_cm, off_bar, off_misc;
     int smem_bytes;  // including alignment slack
     int io_wide;  // shortcut/output maps use 8-byte elements (box rows of tw*32 bytes)
+    // Shared memory reserved for folding the bias into the MMA (0 = no room):
+    // a constant 128 x 32-byte A tile at off_ba and NC x 32 bytes of per-channel
+    // digit rows at off_bb.
+    int fold_room, off_ba, off_bb;
     // control
     int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
     unsigned long long wait_limit_ns;
