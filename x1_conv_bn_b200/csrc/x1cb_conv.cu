@@ -508,9 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < p.kb_per_tile; ++kb)
                 tma_load_4d(sw + kb * p.NC * 32, &tmW, bars.w_full(), 0, 0, kb,
                             group * (p.NC / 128));
-            const uint32_t abytes = static_cast<uint32_t>(p.rows * 32);
+            // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
+            // one filter tap), each a 128-row x 32-byte tile, back to back.
+            const uint32_t abytes = static_cast<uint32_t>(p.a_kc * p.rows * 32);
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
+            const int boxes = p.kb_per_tile / p.a_kc;
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
@@ -518,7 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
                 tile_origin(p, mt, w0, h0, b0);
-                for (int kb = 0; kb < p.kb_per_tile; ++kb) {
+                for (int bx = 0; bx < boxes; ++bx) {
+                    const int kb = bx * p.a_kc;
                     const int tap = kb / p.C1, c1 = kb % p.C1;
                     const int dr = tap / p.R, ds = tap % p.R;
                     if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
@@ -526,8 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes);
-                    tma_load_5d_hint(sa + stage * kASlotBytes, &tmA, bars.a_full(stage), 0,
-                                     w0 + ds - p.pad, h0 + dr - p.pad, c1, b0, pol);
+                    tma_load_5d_hint(sa + stage * p.a_slot, &tmA, bars.a_full(stage), 0,
+                                     w0 + ds - p.pad, h0 + dr - p.pad, b0, c1, pol);
                     ++issued;
                     if (++stage == p.a_stages) {
                         stage = 0;
@@ -596,12 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 3) {
         // ---- TMA store of finished I/O stages ----------------------------------------
-        // After issuing the store of stage i it waits until the store of stage
-        // i-1 has read its shared memory, then hands stage i-1 back.
+        // Each stage goes back to the producer as soon as its store has read it
+        // (the global writes complete in the background).
         if (lane == 0) {
             const uint32_t sio = sbase + p.off_r;
             const uint64_t pol = policy_evict_first();
-            int stage = 0, prev = -1;
+            int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
@@ -618,11 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0, h0, o1, b0, pol);
                     bulk_commit();
-                    if (prev >= 0) {
-                        bulk_wait_read<1>();
-                        mbar_arrive(bars.io_empty(prev));
-                    }
-                    prev = stage;
+                    bulk_wait_read<0>();
+                    mbar_arrive(bars.io_empty(stage));
                     if (++stage == p.r_stages) {
                         stage = 0;
                         phase ^= 1u;
@@ -660,22 +661,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     st = a_stage;
                     ph = a_phase;
                     for (int kb = 0; kb < p.kb_per_tile; ++kb) {
-                        if (j == 0) {
+                        const int sub = kb % p.a_kc;  // K block within the slot's box
+                        if (j == 0 && sub == 0) {
                             if (!mbar_wait(bars.a_full(st), ph, ctl, kDevTimeoutMma)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after();
                         }
-                        const uint64_t adesc = smem_desc_sw32(sa + st * kASlotBytes);
+                        const uint64_t adesc =
+                            smem_desc_sw32(sa + st * p.a_slot + sub * p.rows * 32);
                         const uint64_t bdesc =
                             smem_desc_sw32(sw + (kb * p.NC + j * p.nmma) * 32);
                         mma_i8(d_tmem, adesc, bdesc, idesc, kb > 0 ? 1u : 0u);
-                        if (j == p.n_subs - 1)
-                            mma_commit(bars.a_empty(st));  // slot free once these MMAs finish
-                        if (++st == p.a_stages) {
-                            st = 0;
-                            ph ^= 1u;
+                        if (sub == p.a_kc - 1) {
+                            if (j == p.n_subs - 1)
+                                mma_commit(bars.a_empty(st));  // slot free once these MMAs finish
+                            if (++st == p.a_stages) {
+                                st = 0;
+                                ph ^= 1u;
+                            }
                         }
                     }
                     if (!ok)
@@ -862,14 +867,30 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     p.n_subs = p.NC / p.nmma;
 
     const int wbytes = p.kb_per_tile * p.NC * 32;
-    const int a_min = p.n_subs > 1 ? p.kb_per_tile + 2 : 4;
-    // The activation ring gets a tile's K blocks plus a couple (capped); the
-    // I/O ring (shortcut in, result out) gets as many 16 KB stages as fit --
-    // its depth sets how many bytes are in flight.  Without a shortcut the
-    // stages only stage results, so fewer are needed.  The bias-fold tiles are
-    // reserved when the rings still reach their minimum beside them.
-    const int a_want = std::max(a_min, std::min(p.kb_per_tile + 2, 8));
-    const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 6;
+    // The activation ring budget: with a shortcut the I/O ring (shortcut in,
+    // result out) needs the space -- its depth sets the bytes in flight -- so
+    // about a tile's K blocks plus two; without one the activations are most
+    // of the traffic and get up to 128 KB in flight while the I/O stages only
+    // stage results.  The bias-fold tiles are reserved when the rings still
+    // reach their minimum beside them.
+    const int a_bytes_want = has_res ? std::min(p.kb_per_tile + 2, 8) * kASlotBytes
+                                     : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
+    // Several K blocks per activation box (fewer, larger copies) when each
+    // K-block tile starts on a 256-byte swizzle atom (row count a multiple of
+    // 8) and the ring's minimum still fits the budget.  With two accumulator
+    // slots per tile the whole tile's K blocks stay in the ring until the
+    // second slot's MMAs are done.
+    auto ring_min = [&](int kc) { return p.n_subs > 1 ? p.kb_per_tile / kc + 1 : 2; };
+    p.a_kc = 1;
+    for (int kc = 4; kc > 1; kc /= 2)
+        if (p.C1 % kc == 0 && p.rows % 8 == 0 && ring_min(kc) * kc * kASlotBytes <= a_bytes_want) {
+            p.a_kc = kc;
+            break;
+        }
+    p.a_slot = p.a_kc * kASlotBytes;
+    const int a_min = ring_min(p.a_kc);
+    const int a_want = std::max(a_min, a_bytes_want / p.a_slot);
+    const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 4;
     auto layout = [&](int fold, int a, int r) {
         p.fold_room = fold;
         p.a_stages = a;
@@ -878,7 +899,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
         p.off_ba = p.off_w + wbytes;
         p.off_bb = p.off_ba + (fold ? kTileRows * 32 : 0);
         p.off_a = p.off_bb + (fold ? p.NC * 32 : 0);
-        p.off_r = p.off_a + a * kASlotBytes;
+        p.off_r = p.off_a + a * p.a_slot;
         // The per-channel bias/offset table (modes 0-2) and the fold digit rows
         // (mode 3) are never used together, so they share space when folding
         // is possible.
@@ -912,13 +933,15 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
                 const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream)
 {
     CUtensorMap tmA, tmW, tmR, tmO;
-    // Activations: dims (32 ch, Wp, Hp, C1, B); box (32, tw, th, 1, tg).
+    // Activations: dims (32 ch, Wp, Hp, B, C1) -- channel blocks outermost so a
+    // box (32, tw, th, tg, a_kc) lands as a_kc K-block tiles one after another.
     {
-        const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.C1,
-                                  (uint64_t)p.B};
-        const uint64_t str[4] = {32, (uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
-                                 (uint64_t)p.C1 * p.Hp * p.Wp * 32};
-        const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)p.th, 1, (uint32_t)p.tg};
+        const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.B,
+                                  (uint64_t)p.C1};
+        const uint64_t str[4] = {32, (uint64_t)p.Wp * 32, (uint64_t)p.C1 * p.Hp * p.Wp * 32,
+                                 (uint64_t)p.Hp * p.Wp * 32};
+        const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)p.th, (uint32_t)p.tg,
+                                 (uint32_t)p.a_kc};
         if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }

@@ -38,6 +38,8 @@ struct ConvPlan {
     // N split: each CTA keeps NC output channels' weights resident
     int NC, n_groups, nmma, n_subs;
     int kb_per_tile;  // R*R*C1
+    int a_kc;         // K blocks per activation TMA box (divides C1)
+    int a_slot;       // bytes per activation ring slot = a_kc * 4 KB
     // rings
     int a_stages, r_stages;
     // shared memory offsets from the 1024-aligned base
