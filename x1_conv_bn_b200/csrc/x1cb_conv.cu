@@ -514,28 +514,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
             const int boxes = p.kb_per_tile / p.a_kc;
+            const uint32_t a_slot = static_cast<uint32_t>(p.a_slot);
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t slot = sa;
             long long issued = 0;
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
                 tile_origin(p, mt, w0, h0, b0);
+                // K blocks run channel block fastest, then filter column, then
+                // filter row; counters instead of divisions keep the issue cheap.
+                int c1 = 0, ds = 0, dr = 0;
                 for (int bx = 0; bx < boxes; ++bx) {
-                    const int kb = bx * p.a_kc;
-                    const int tap = kb / p.C1, c1 = kb % p.C1;
-                    const int dr = tap / p.R, ds = tap % p.R;
                     if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes);
-                    tma_load_5d_hint(sa + stage * p.a_slot, &tmA, bars.a_full(stage), 0,
+                    tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0,
                                      w0 + ds - p.pad, h0 + dr - p.pad, b0, c1, pol);
                     ++issued;
                     if (++stage == p.a_stages) {
                         stage = 0;
                         phase ^= 1u;
+                        slot = sa;
+                    } else {
+                        slot += a_slot;
+                    }
+                    c1 += p.a_kc;
+                    if (c1 == p.C1) {
+                        c1 = 0;
+                        if (++ds == p.R) {
+                            ds = 0;
+                            ++dr;
+                        }
                     }
                 }
             }
@@ -637,12 +650,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---- MMA issuer -----------------------------------------------------------
         if (lane == 0) {
+            // The issue loop is kept free of divisions and descriptor rebuilds:
+            // a single thread's dependent integer work between two MMAs costs
+            // more than the MMA itself (64-128 tensor cycles).  A descriptor's
+            // start-address field is the byte address / 16 and every operand
+            // lies below 256 KB, so moving an operand by `b` bytes is adding
+            // b / 16 to its descriptor.
             const uint32_t idesc = idesc_i8(kTileRows, p.nmma);
-            const uint32_t sa = sbase + p.off_a;
-            const uint32_t sw = sbase + p.off_w;
+            const uint64_t a_desc0 = smem_desc_sw32(sbase + p.off_a);
+            const uint64_t b_desc0 = smem_desc_sw32(sbase + p.off_w);
+            const uint64_t fold_a = smem_desc_sw32(sbase + p.off_ba);
+            const uint64_t fold_b0 = smem_desc_sw32(sbase + p.off_bb);
+            const uint32_t a_sub_step = static_cast<uint32_t>(p.rows * 32) >> 4;  // next K block in a box
+            const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
+            const uint32_t b_kb_step = static_cast<uint32_t>(p.NC * 32) >> 4;     // next K block of weights
+            const uint32_t b_sub_step = static_cast<uint32_t>(p.nmma * 32) >> 4;  // next N slice
+            const int boxes = p.kb_per_tile / p.a_kc;
+            const int kc = p.a_kc;
             const int n_slots = kTmemCols / p.nmma;
             int a_stage = 0;
             uint32_t a_phase = 0;
+            uint64_t a_slot_desc = a_desc0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma);
@@ -651,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int st = a_stage;
                 uint32_t ph = a_phase;
+                uint64_t sd = a_slot_desc;
                 for (int j = 0; ok && j < p.n_subs; ++j) {
                     if (!mbar_wait(bars.acc_empty(acc), acc_phase ^ 1u, ctl, kDevTimeoutMma)) {
                         ok = false;
@@ -658,36 +687,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * p.nmma);
+                    const bool last_sub = j == p.n_subs - 1;
                     st = a_stage;
                     ph = a_phase;
-                    for (int kb = 0; kb < p.kb_per_tile; ++kb) {
-                        const int sub = kb % p.a_kc;  // K block within the slot's box
-                        if (j == 0 && sub == 0) {
+                    sd = a_slot_desc;
+                    uint64_t bd = b_desc0 + static_cast<uint64_t>(j) * b_sub_step;
+                    uint32_t accumulate = 0;
+                    for (int box = 0; box < boxes; ++box) {
+                        if (j == 0) {
                             if (!mbar_wait(bars.a_full(st), ph, ctl, kDevTimeoutMma)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after();
                         }
-                        const uint64_t adesc =
-                            smem_desc_sw32(sa + st * p.a_slot + sub * p.rows * 32);
-                        const uint64_t bdesc =
-                            smem_desc_sw32(sw + (kb * p.NC + j * p.nmma) * 32);
-                        mma_i8(d_tmem, adesc, bdesc, idesc, kb > 0 ? 1u : 0u);
-                        if (sub == p.a_kc - 1) {
-                            if (j == p.n_subs - 1)
-                                mma_commit(bars.a_empty(st));  // slot free once these MMAs finish
-                            if (++st == p.a_stages) {
-                                st = 0;
-                                ph ^= 1u;
-                            }
+                        uint64_t ad = sd;
+                        if (kc == 4) {
+                            mma_i8(d_tmem, ad, bd, idesc, accumulate);
+                            mma_i8(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
+                            mma_i8(d_tmem, ad + 2 * a_sub_step, bd + 2 * b_kb_step, idesc, 1u);
+                            mma_i8(d_tmem, ad + 3 * a_sub_step, bd + 3 * b_kb_step, idesc, 1u);
+                            bd += 4 * b_kb_step;
+                        } else if (kc == 2) {
+                            mma_i8(d_tmem, ad, bd, idesc, accumulate);
+                            mma_i8(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
+                            bd += 2 * b_kb_step;
+                        } else {
+                            mma_i8(d_tmem, ad, bd, idesc, accumulate);
+                            bd += b_kb_step;
+                        }
+                        accumulate = 1u;
+                        if (last_sub)
+                            mma_commit(bars.a_empty(st));  // slot free once these MMAs finish
+                        if (++st == p.a_stages) {
+                            st = 0;
+                            ph ^= 1u;
+                            sd = a_desc0;
+                        } else {
+                            sd += a_slot_step;
                         }
                     }
                     if (!ok)
                         break;
                     if (fold)  // + bias: constant A tile x digit rows of this slot's channels
-                        mma_i8(d_tmem, smem_desc_sw32(sbase + p.off_ba),
-                               smem_desc_sw32(sbase + p.off_bb + j * p.nmma * 32), idesc, 1u);
+                        mma_i8(d_tmem, fold_a, fold_b0 + static_cast<uint64_t>(j) * b_sub_step,
+                               idesc, 1u);
                     mma_commit(bars.acc_full(acc));
                     if (++acc == n_slots) {
                         acc = 0;
@@ -696,6 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 a_stage = st;
                 a_phase = ph;
+                a_slot_desc = sd;
             }
             // Make sure no MMA is still reading shared memory or writing TMEM.
             mma_commit(bars.mma_done());
