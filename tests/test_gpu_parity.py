@@ -178,12 +178,17 @@ def test_conv1x1_mixed_epilogue_forms_across_ctas(oracle):
 
 # ---- fused 3x3 ------------------------------------------------------------------
 
+# The halo form covers W+2 <= 128 (tiles of th rows x tg images, ragged in H
+# and B); (1, 3, 130, ...) takes the per-tap form.
 SMALL_3X3 = [
     (1, 1, 1, 32, 128),
     (2, 28, 28, 128, 128),
     (3, 5, 7, 64, 256),
     (1, 3, 130, 32, 128),
     (11, 6, 6, 128, 128),
+    (2, 30, 28, 128, 128),
+    (5, 3, 5, 64, 128),
+    (4, 13, 21, 96, 384),
 ]
 
 

@@ -261,11 +261,12 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     const int q = warp & 3;                               // TMEM lane quarter this warp may access
     const int c0 = kCPW * ((warp - kEpiWarp0) >> 2);      // first chunk it takes per stage
     const int row = q * 32 + lane;                        // GEMM row = pixel of the tile
-    const int plane_t = p.tw * p.th;
-    const int xi = row % p.tw;
-    const int yi = (row / p.tw) % p.th;
-    const int gi = row / plane_t;
-    const bool in_box = row < p.rows;
+    const int plane_t = p.tw * p.th;                      // pixels per image in the I/O box
+    const int xi = row % p.row_pitch;
+    const int yi = (row % p.plane_m) / p.row_pitch;
+    const int gi = row / p.plane_m;
+    // Rows past the tile, and the halo form's frame columns/rows, are not pixels.
+    const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
     // This row's 32 bytes inside chunk 0 of an I/O stage ([tg][4][th][tw][32]);
     // rows outside the box read row 0's bytes and write nothing.
     const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
@@ -510,10 +511,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             group * (p.NC / 128));
             // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
             // one filter tap), each a 128-row x 32-byte tile, back to back.
-            const uint32_t abytes = static_cast<uint32_t>(p.a_kc * p.rows * 32);
+            const uint32_t abytes =
+                p.halo ? static_cast<uint32_t>(2 * 16 * p.plane_m * p.tg)  // two K halves
+                       : static_cast<uint32_t>(p.a_kc * p.rows * 32);
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
-            const int boxes = p.kb_per_tile / p.a_kc;
+            const int boxes = p.kb_per_tile / p.a_kc;  // unused in the halo form
             const uint32_t a_slot = static_cast<uint32_t>(p.a_slot);
             int stage = 0;
             uint32_t phase = 0;
@@ -523,6 +526,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
                 tile_origin(p, mt, w0, h0, b0);
+                if (p.halo) {
+                    // One slot per channel block: the tile's pixels plus a one-pixel
+                    // frame (zeros outside the image), each K half as one box.
+                    for (int c1 = 0; c1 < p.C1; ++c1) {
+                        if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl,
+                                       kDevTimeoutProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bars.a_full(stage), abytes);
+                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
+                                         h0 - p.pad, c1, b0, pol);
+                        tma_load_5d_hint(slot + static_cast<uint32_t>(p.a_half), &tmA,
+                                         bars.a_full(stage), 16, w0 - p.pad, h0 - p.pad, c1, b0,
+                                         pol);
+                        ++issued;
+                        if (++stage == p.a_stages) {
+                            stage = 0;
+                            phase ^= 1u;
+                            slot = sa;
+                        } else {
+                            slot += a_slot;
+                        }
+                    }
+                    continue;
+                }
                 // K blocks run channel block fastest, then filter column, then
                 // filter row; counters instead of divisions keep the issue cheap.
                 int c1 = 0, ds = 0, dr = 0;
@@ -657,7 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // lies below 256 KB, so moving an operand by `b` bytes is adding
             // b / 16 to its descriptor.
             const uint32_t idesc = idesc_i8(kTileRows, p.nmma);
-            const uint64_t a_desc0 = smem_desc_sw32(sbase + p.off_a);
+            const uint64_t a_desc0 =
+                p.halo ? smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half))
+                       : smem_desc_sw32(sbase + p.off_a);
             const uint64_t b_desc0 = smem_desc_sw32(sbase + p.off_w);
             const uint64_t fold_a = smem_desc_sw32(sbase + p.off_ba);
             const uint64_t fold_b0 = smem_desc_sw32(sbase + p.off_bb);
@@ -665,8 +696,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
             const uint32_t b_kb_step = static_cast<uint32_t>(p.NC * 32) >> 4;     // next K block of weights
             const uint32_t b_sub_step = static_cast<uint32_t>(p.nmma * 32) >> 4;  // next N slice
-            const int boxes = p.kb_per_tile / p.a_kc;
+            const int boxes = p.halo ? p.C1 : p.kb_per_tile / p.a_kc;
             const int kc = p.a_kc;
+            // Halo form: tap (dr, ds) reads the slot dr*row_pitch + ds rows on and
+            // the weights of K block (dr*3 + ds)*C1 + c1.
+            const uint32_t hp = static_cast<uint32_t>(p.row_pitch);
+            const uint64_t b_tap_step = static_cast<uint64_t>(p.C1) * b_kb_step;
             const int n_slots = kTmemCols / p.nmma;
             int a_stage = 0;
             uint32_t a_phase = 0;
@@ -702,7 +737,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                         }
                         uint64_t ad = sd;
-                        if (kc == 4) {
+                        if (p.halo) {
+#pragma unroll
+                            for (int t = 0; t < 9; ++t)
+                                mma_i8(d_tmem, ad + (t / 3) * hp + (t % 3),
+                                       bd + static_cast<uint64_t>(t) * b_tap_step, idesc,
+                                       t == 0 ? accumulate : 1u);
+                            bd += b_kb_step;
+                        } else if (kc == 4) {
                             mma_i8(d_tmem, ad, bd, idesc, accumulate);
                             mma_i8(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
                             mma_i8(d_tmem, ad + 2 * a_sub_step, bd + 2 * b_kb_step, idesc, 1u);
@@ -848,6 +890,31 @@ void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg)
     }
 }
 
+// Halo form of the 3x3 convolution: th rows of tg images per tile, each image
+// row with its one-pixel frame taking W+2 GEMM rows and each image th+2 rows
+// of them.  Every pixel of the tile must land in the 128 GEMM rows; fewest
+// tiles wins, ties go to taller tiles (longer contiguous runs).
+void choose_halo_tile(int B, int H, int W, int &th, int &tg)
+{
+    const int pitch = W + 2;
+    long long best = -1;
+    th = tg = 1;
+    for (int h = 1; h <= H; ++h) {
+        for (int g = 1; g <= B; ++g) {
+            const long long last = static_cast<long long>(g - 1) * (h + 2) * pitch +
+                                   static_cast<long long>(h - 1) * pitch + (W - 1);
+            if (last >= kTileRows)
+                break;
+            const long long tiles = static_cast<long long>((H + h - 1) / h) * ((B + g - 1) / g);
+            if (best < 0 || tiles < best || (tiles == best && h > th)) {
+                best = tiles;
+                th = h;
+                tg = g;
+            }
+        }
+    }
+}
+
 int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
               int m_r, int num_sms)
 {
@@ -871,7 +938,24 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
         p.Wp = W;
         p.Hp = H;
     }
-    choose_tile(B, p.Wp, p.Hp, p.tw, p.th, p.tg);
+    // The 3x3 convolution uses the halo form whenever one framed image row fits
+    // in the 128 GEMM rows.
+    p.halo = (R == 3 && p.pad == 1 && W + 2 <= kTileRows) ? 1 : 0;
+    if (p.halo) {
+        choose_halo_tile(B, H, W, p.th, p.tg);
+        p.tw = W;
+        p.row_pitch = W + 2;
+        p.plane_m = (p.th + 2) * (W + 2);
+        // Slot rows: the framed tile, and every row a shifted 128-row view can
+        // touch (rows past the frame only feed GEMM rows that are not pixels).
+        const int need_rows = std::max(p.tg * p.plane_m, kTileRows + 2 * p.row_pitch + 2);
+        p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+    } else {
+        choose_tile(B, p.Wp, p.Hp, p.tw, p.th, p.tg);
+        p.row_pitch = p.tw;
+        p.plane_m = p.tw * p.th;
+        p.a_half = 0;
+    }
     p.rows = p.tw * p.th * p.tg;
     p.nTw = (p.Wp + p.tw - 1) / p.tw;
     p.nTh = (p.Hp + p.th - 1) / p.th;
@@ -883,6 +967,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     p.kb_per_tile = R * R * p.C1;
 
     const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 12) * 8 + 64;
+    const int min_slot = p.halo ? 2 * p.a_half : kASlotBytes;
     int chosen = 0;
     long long chosen_work = -1;
     for (int NC = std::min(Oc, 512); NC >= 128; NC -= 128) {
@@ -890,10 +975,11 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
             continue;
         const int nmma = NC >= 256 ? 256 : 128;
         const int n_subs = NC / nmma;
-        const int a_min = n_subs > 1 ? p.kb_per_tile + 2 : 4;
+        const int a_min = n_subs > 1 ? (p.halo ? p.C1 : p.kb_per_tile) + 2 : (p.halo ? 2 : 4);
         const int r_min = has_res ? 4 : 2;
         const long long need = static_cast<long long>(p.kb_per_tile) * NC * 32 + NC * 12 +
-                               a_min * kASlotBytes + r_min * kRSlotBytes + fixed;
+                               static_cast<long long>(a_min) * min_slot + r_min * kRSlotBytes +
+                               fixed;
         if (need > kSmemLimit || a_min > 48)
             continue;
         const long long work = mtiles * (Oc / NC);
@@ -927,13 +1013,17 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     // second slot's MMAs are done.
     auto ring_min = [&](int kc) { return p.n_subs > 1 ? p.kb_per_tile / kc + 1 : 2; };
     p.a_kc = 1;
-    for (int kc = 4; kc > 1; kc /= 2)
-        if (p.C1 % kc == 0 && p.rows % 8 == 0 && ring_min(kc) * kc * kASlotBytes <= a_bytes_want) {
-            p.a_kc = kc;
-            break;
-        }
-    p.a_slot = p.a_kc * kASlotBytes;
-    const int a_min = ring_min(p.a_kc);
+    if (!p.halo)
+        for (int kc = 4; kc > 1; kc /= 2)
+            if (p.C1 % kc == 0 && p.rows % 8 == 0 &&
+                ring_min(kc) * kc * kASlotBytes <= a_bytes_want) {
+                p.a_kc = kc;
+                break;
+            }
+    // Halo form: one slot per channel block, all of a tile's blocks in the ring
+    // when two accumulator slots share them.
+    p.a_slot = p.halo ? 2 * p.a_half : p.a_kc * kASlotBytes;
+    const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
     const int a_want = std::max(a_min, a_bytes_want / p.a_slot);
     const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 4;
     auto layout = [&](int fold, int a, int r) {
@@ -980,7 +1070,18 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
     CUtensorMap tmA, tmW, tmR, tmO;
     // Activations: dims (32 ch, Wp, Hp, B, C1) -- channel blocks outermost so a
     // box (32, tw, th, tg, a_kc) lands as a_kc K-block tiles one after another.
-    {
+    // Halo form: dims (32 ch, W, H, C1, B), box (16, tw+2, th+2, 1, tg) -- one K
+    // half of the framed tile as 16-byte rows, zeros outside the image.
+    if (p.halo) {
+        const uint64_t dims[5] = {32, (uint64_t)p.W, (uint64_t)p.H, (uint64_t)p.C1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {32, (uint64_t)p.W * 32, (uint64_t)p.H * p.W * 32,
+                                 (uint64_t)p.C1 * p.H * p.W * 32};
+        const uint32_t box[5] = {16, (uint32_t)p.row_pitch, (uint32_t)(p.th + 2), 1,
+                                 (uint32_t)p.tg};
+        if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return e;
+    } else {
         const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.B,
                                   (uint64_t)p.C1};
         const uint64_t str[4] = {32, (uint64_t)p.Wp * 32, (uint64_t)p.C1 * p.Hp * p.Wp * 32,

@@ -50,6 +50,15 @@ struct ConvPlan {
     // a constant 128 x 32-byte A tile at off_ba and NC x 32 bytes of per-channel
     // digit rows at off_bb.
     int fold_room, off_ba, off_bb;
+    // Halo form of the 3x3 convolution: one activation slot per channel block
+    // holds tg images x (th+2) rows x (tw+2) columns around the tile (no
+    // swizzle, the two 16-byte K halves `a_half` bytes apart), and every
+    // filter tap reads it shifted by dr*(tw+2)+ds rows.  GEMM row m of the
+    // tile is pixel (g, y, x) with m = (g*(th+2) + y)*row_pitch + x.
+    int halo;
+    int row_pitch;  // GEMM rows per image row: tw, or tw+2 in the halo form
+    int plane_m;    // GEMM rows per image of the tile: tw*th, or (th+2)*(tw+2)
+    int a_half;     // halo form: bytes between the two K halves of a slot
     // control
     int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
     unsigned long long wait_limit_ns;

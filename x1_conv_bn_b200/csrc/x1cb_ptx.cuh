@@ -453,6 +453,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr)
     return d;
 }
 
+// Shared-memory matrix descriptor for a K-major operand without swizzle whose
+// rows are 16 bytes apart (8-row core matrices back to back, 128 bytes each)
+// and whose two 16-byte K halves are `half_bytes` apart.  Rows are linear in
+// the address, so a descriptor shifted by n rows is this one plus n.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr, uint32_t half_bytes)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);           // start address
+    d |= static_cast<uint64_t>((half_bytes >> 4) & 0x3FFFu) << 16;  // K-direction core-matrix stride
+    d |= static_cast<uint64_t>(128 >> 4) << 32;                     // M-direction 8-row stride
+    d |= static_cast<uint64_t>(1) << 46;                            // descriptor version
+    return d;                                                       // layout 0: no swizzle
+}
+
 // Instruction descriptor: s8 x s8 -> s32, both operands K-major, M x N.
 __host__ __device__ constexpr uint32_t idesc_i8(uint32_t M, uint32_t N)
 {
