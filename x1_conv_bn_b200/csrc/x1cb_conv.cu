@@ -135,7 +135,7 @@ __device__ __forceinline__ void requant_fast(const uint32_t *v, const int32_t *c
 // so y2 = floor(t * 2^s / 2^32) = hi32((acc + bias) * m') + 1 + r*k exactly
 // (mad.hi), and floor(t / 2^S) = floor(y2 / 2); clamping y2 to [0, 255]
 // before halving gives the [0, 127] clamp.  No 64-bit arithmetic.
-template <bool kRes, bool kAddBias, int kGroups>
+template <bool kRes, bool kAddBias, bool kK1, int kGroups>
 __device__ __forceinline__ void requant_hi32(const uint32_t *v, const int32_t *cm,
                                              const int32_t *cb, const uint32_t *rw, int k,
                                              const uint32_t (&rsel)[4], uint32_t *ow)
@@ -144,7 +144,7 @@ __device__ __forceinline__ void requant_hi32(const uint32_t *v, const int32_t *c
     const int4 *b4 = reinterpret_cast<const int4 *>(cb);
 #pragma unroll
     for (int q = 0; q < kGroups; ++q)
-        ow[q] = requant4_hi32<kRes, kAddBias>(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+        ow[q] = requant4_hi32<kRes, kAddBias, kK1>(v[4 * q], v[4 * q + 1], v[4 * q + 2],
                                               v[4 * q + 3], m4[q],
                                               kAddBias ? b4[q] : make_int4(0, 0, 0, 0),
                                               kRes ? rw[q] : 0u, rsel, k);
@@ -250,16 +250,20 @@ struct EpiCtx {
 };
 
 // kMode: 3 = all-32-bit form with the bias folded into the MMA, 2 = all-32-bit
-// form, 1 = 64-bit fast form, 0 = generic.
-template <bool kRes, int kMode>
+// form, 1 = 64-bit fast form, 0 = generic.  kK1 (modes 2-3 with a shortcut):
+// the shortcut's scale in the all-32-bit form, k = m_r / 2^(S-1), is 1.
+//
+// The warps of one TMEM lane quarter take turns on the I/O stages: turn g
+// handles stages g, g + kTurns, ... (counted over all of the CTA's tiles), all
+// four 32-channel chunks of its 32 rows.  Turns drift apart in time, so while
+// one warp waits for its stage or its TMEM load the others compute.
+template <bool kRes, int kMode, bool kK1 = false>
 __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int lane)
 {
-    constexpr int kPerQuarter = kEpiWarps / 4;           // warps sharing a TMEM lane quarter
-    constexpr int kCPW = kRChunks / kPerQuarter;          // adjacent chunks per warp per stage
-    static_assert(kCPW == 1 || kCPW == 2, "one or two 32-channel chunks per warp and stage");
+    constexpr int kTurns = kEpiWarps / 4;                 // warps per TMEM lane quarter
     const ConvPlan &p = *cx.p;
     const int q = warp & 3;                               // TMEM lane quarter this warp may access
-    const int c0 = kCPW * ((warp - kEpiWarp0) >> 2);      // first chunk it takes per stage
+    const int turn = (warp - kEpiWarp0) >> 2;
     const int row = q * 32 + lane;                        // GEMM row = pixel of the tile
     const int plane_t = p.tw * p.th;                      // pixels per image in the I/O box
     const int xi = row % p.row_pitch;
@@ -274,6 +278,10 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     const int n_slots = kTmemCols / p.nmma;
     const int chunks_per_sub = p.nmma / 32;
     const int stages_per_sub = chunks_per_sub / kRChunks;
+    const long long my_tiles =
+        cx.mt_first < p.num_m_tiles ? (p.num_m_tiles - cx.mt_first + cx.mt_step - 1) / cx.mt_step
+                                    : 0;
+    const long long total = my_tiles * p.n_subs * stages_per_sub;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     // Shortcut operands.  64-bit fast form: r*2^(8*k8) by one byte permute and
     // m_r*2^(s-8*k8).  All-32-bit form: the sign-extended byte (k8 = 0) and
@@ -295,84 +303,74 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         }
         rsel[b] = sel;
     }
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    int st = 0;
-    uint32_t st_phase = 0;
-    for (int mt = cx.mt_first; mt < p.num_m_tiles; mt += cx.mt_step) {
-        for (int j = 0; j < p.n_subs; ++j) {
-            // Every lane waits; the vote keeps the decision warp-uniform so the
-            // .sync.aligned TMEM loads below always run converged.
-            if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.acc_full(acc), acc_phase, cx.ctl,
-                                                   kDevTimeoutEpilogue)))
-                return;
-            tc_fence_after();
-            const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
-            for (int rl = 0; rl < stages_per_sub; ++rl) {
-                if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.io_full(st), st_phase, cx.ctl,
-                                                       kDevTimeoutEpilogue)))
-                    return;
-                uint8_t *stage = cx.io + st * kRSlotBytes + row_off;
-                const int cs = rl * kRChunks + c0;         // chunk within the TMEM slot
-                const int gch = j * chunks_per_sub + cs;   // chunk within the CTA's channels
-                uint32_t v[32 * kCPW];
-                __syncwarp();
-                if (kCPW == 2)
-                    tmem_ld_32x32b_x64_sync(tbase + static_cast<uint32_t>(cs * 32),
-                                            *reinterpret_cast<uint32_t(*)[64]>(v));
-                else
-                    tmem_ld_32x32b_x32_sync(tbase + static_cast<uint32_t>(cs * 32),
-                                            *reinterpret_cast<uint32_t(*)[32]>(v));
-                uint4 *pc[kCPW];
-#pragma unroll
-                for (int i = 0; i < kCPW; ++i)
-                    pc[i] = reinterpret_cast<uint4 *>(stage + (c0 + i) * chunk_stride);
-                uint32_t rw[8 * kCPW];
-                if (kRes) {
-#pragma unroll
-                    for (int i = 0; i < kCPW; ++i) {
-                        const uint4 ra = pc[i][0], rb = pc[i][1];
-                        rw[8 * i + 0] = ra.x; rw[8 * i + 1] = ra.y; rw[8 * i + 2] = ra.z;
-                        rw[8 * i + 3] = ra.w; rw[8 * i + 4] = rb.x; rw[8 * i + 5] = rb.y;
-                        rw[8 * i + 6] = rb.z; rw[8 * i + 7] = rb.w;
-                    }
-                }
-                uint32_t ow[8 * kCPW];
-                if (kMode >= 2) {
-                    requant_hi32<kRes, kMode == 2, 8 * kCPW>(
-                        v, cx.cm + gch * 32, reinterpret_cast<const int32_t *>(cx.cC) + gch * 32,
-                        rw, mr2, rsel, ow);
-                } else if (kMode == 1) {
-                    requant_fast<kRes, 8 * kCPW>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2,
-                                                 rsel, ow);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < kCPW; ++i)
-                        requant32<kRes>(v + 32 * i, cx.cm + gch * 32 + 32 * i,
-                                        cx.cC + gch * 32 + 32 * i, rw + 8 * i, p.m_r, p.S,
-                                        ow + 8 * i);
-                }
-                if (in_box) {
-#pragma unroll
-                    for (int i = 0; i < kCPW; ++i) {
-                        pc[i][0] = make_uint4(ow[8 * i + 0], ow[8 * i + 1], ow[8 * i + 2], ow[8 * i + 3]);
-                        pc[i][1] = make_uint4(ow[8 * i + 4], ow[8 * i + 5], ow[8 * i + 6], ow[8 * i + 7]);
-                    }
-                }
-                // Results must be visible to the TMA store (async proxy).
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(cx.bars.out_ready(st));
-                if (++st == p.r_stages) {
-                    st = 0;
-                    st_phase ^= 1u;
-                }
-            }
-            tc_fence_before();
+    // Position of stage n = turn: I/O ring slot and phase, stage within its
+    // accumulator slot (rl), N slice (j), accumulator slot and phase.
+    int st = turn % p.r_stages;
+    uint32_t st_phase = static_cast<uint32_t>((turn / p.r_stages) & 1);
+    int rl = turn % stages_per_sub;
+    const int sub_n = turn / stages_per_sub;
+    int j = sub_n % p.n_subs;
+    int acc = sub_n % n_slots;
+    uint32_t acc_phase = static_cast<uint32_t>((sub_n / n_slots) & 1);
+    for (long long n = turn; n < total; n += kTurns) {
+        // Every lane waits; the vote keeps the decision warp-uniform so the
+        // .sync.aligned TMEM loads below always run converged.
+        if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.acc_full(acc), acc_phase, cx.ctl,
+                                               kDevTimeoutEpilogue)))
+            return;
+        tc_fence_after();
+        if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.io_full(st), st_phase, cx.ctl,
+                                               kDevTimeoutEpilogue)))
+            return;
+        const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
+        uint8_t *stage = cx.io + st * kRSlotBytes + row_off;
+#pragma unroll 1
+        for (int c = 0; c < kRChunks; ++c) {
+            const int cs = rl * kRChunks + c;          // chunk within the TMEM slot
+            const int gch = j * chunks_per_sub + cs;   // chunk within the CTA's channels
+            uint32_t v[32];
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(cx.bars.acc_empty(acc));
+            tmem_ld_32x32b_x32_sync(tbase + static_cast<uint32_t>(cs * 32), v);
+            uint4 *pc = reinterpret_cast<uint4 *>(stage + c * chunk_stride);
+            uint32_t rw[8];
+            if (kRes) {
+                const uint4 ra = pc[0], rb = pc[1];
+                rw[0] = ra.x; rw[1] = ra.y; rw[2] = ra.z; rw[3] = ra.w;
+                rw[4] = rb.x; rw[5] = rb.y; rw[6] = rb.z; rw[7] = rb.w;
+            }
+            uint32_t ow[8];
+            if (kMode >= 2) {
+                requant_hi32<kRes, kMode == 2, kK1, 8>(
+                    v, cx.cm + gch * 32, reinterpret_cast<const int32_t *>(cx.cC) + gch * 32, rw,
+                    mr2, rsel, ow);
+            } else if (kMode == 1) {
+                requant_fast<kRes, 8>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2, rsel, ow);
+            } else {
+                requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
+            }
+            if (in_box) {
+                pc[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                pc[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+            }
+        }
+        // Results must be visible to the TMA store (async proxy).
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(cx.bars.out_ready(st));
+            mbar_arrive(cx.bars.acc_empty(acc));  // one arrival per stage of the slot
+        }
+        st += kTurns;
+        while (st >= p.r_stages) {
+            st -= p.r_stages;
+            st_phase ^= 1u;
+        }
+        rl += kTurns;
+        while (rl >= stages_per_sub) {
+            rl -= stages_per_sub;
+            if (++j == p.n_subs)
+                j = 0;
             if (++acc == n_slots) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -422,12 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < p.r_stages; ++s) {
             mbar_init(bars.io_full(s), 1);
-            mbar_init(bars.out_ready(s), kEpiWarps);
+            mbar_init(bars.out_ready(s), 4);  // one warp per TMEM lane quarter
             mbar_init(bars.io_empty(s), 1);
         }
         for (int s = 0; s < 4; ++s) {
             mbar_init(bars.acc_full(s), 1);
-            mbar_init(bars.acc_empty(s), kEpiWarps);
+            // every stage of the slot, each from one warp per lane quarter
+            mbar_init(bars.acc_empty(s), 4 * (p.nmma / (32 * kRChunks)));
         }
         fence_mbar_init();
     }
@@ -794,8 +793,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- epilogue ---------------------------------------------------------------
         const EpiCtx cx{&p, bars, ctl, tmem_base, smem + p.off_r, cm, cC,
                         group, mt_first, mt_step};
-        if (mode == 3)
+        const bool k1 = kRes && static_cast<long long>(p.m_r) == (1ll << (p.S - 1));
+        if (mode == 3 && k1)
+            epilogue_warp<kRes, 3, kRes>(cx, warp, lane);
+        else if (mode == 3)
             epilogue_warp<kRes, 3>(cx, warp, lane);
+        else if (mode == 2 && k1)
+            epilogue_warp<kRes, 2, kRes>(cx, warp, lane);
         else if (mode == 2)
             epilogue_warp<kRes, 2>(cx, warp, lane);
         else if (mode == 1)

@@ -238,121 +238,43 @@ __device__ __forceinline__ uint32_t requant4_fast(uint32_t a0, uint32_t a1, uint
 //   y2_e = hi32((acc_e + bias_e) * m_e) + 1 (+ r_e * k),  r_e = shortcut byte e
 //   out_e = min(max(y2_e, 0), 255) >> 1, four bytes packed into one word.
 // kAddBias = false: the accumulator already holds acc + bias (folded into the
-// MMA), so the four additions are skipped and b is ignored.
-template <bool kRes, bool kAddBias = true>
+// MMA), so the four additions are skipped and b is ignored.  kK1: k == 1.
+// The high word is a plain multiply-high and the small addend a separate add
+// (hi32(u*m) + c is what a fused multiply-high-add computes, but written apart
+// the add of r + 1 is one three-input add when k == 1).
+template <bool kRes, bool kAddBias = true, bool kK1 = false>
 __device__ __forceinline__ uint32_t requant4_hi32(uint32_t a0, uint32_t a1, uint32_t a2,
                                                   uint32_t a3, int4 m, int4 b, uint32_t rword,
                                                   const uint32_t (&rsel)[4], int k)
 {
+    const uint32_t av[4] = {a0, a1, a2, a3};
+    const int mv[4] = {m.x, m.y, m.z, m.w};
+    const int bv[4] = {b.x, b.y, b.z, b.w};
+    int y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int u = kAddBias ? static_cast<int>(av[e]) + bv[e] : static_cast<int>(av[e]);
+        const int h = __mulhi(u, mv[e]);
+        int c = 1;
+        if (kRes) {
+            int r;  // the shortcut byte, sign-extended
+            asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(rword), "r"(rsel[e]));
+            c = kK1 ? r + 1 : r * k + 1;
+        }
+        y[e] = h + c;
+        asm("min.relu.s32 %0, %0, 255;" : "+r"(y[e]));
+    }
     uint32_t d;
-    if (!kAddBias) {
-        b = make_int4(0, 0, 0, 0);
-    }
-    if (kRes && !kAddBias) {
-        asm("{\n\t"
-            ".reg .b32 r0, r1, r2, r3, y0, y1, y2, y3, p, q;\n\t"
-            "prmt.b32 r0, %9, 0, %10;\n\t"
-            "prmt.b32 r1, %9, 0, %11;\n\t"
-            "prmt.b32 r2, %9, 0, %12;\n\t"
-            "prmt.b32 r3, %9, 0, %13;\n\t"
-            "mad.lo.s32 r0, r0, %14, 1;\n\t"
-            "mad.lo.s32 r1, r1, %14, 1;\n\t"
-            "mad.lo.s32 r2, r2, %14, 1;\n\t"
-            "mad.lo.s32 r3, r3, %14, 1;\n\t"
-            "mad.hi.s32 y0, %1, %5, r0;\n\t"
-            "mad.hi.s32 y1, %2, %6, r1;\n\t"
-            "mad.hi.s32 y2, %3, %7, r2;\n\t"
-            "mad.hi.s32 y3, %4, %8, r3;\n\t"
-            "min.relu.s32 y0, y0, 255;\n\t"
-            "min.relu.s32 y1, y1, 255;\n\t"
-            "min.relu.s32 y2, y2, 255;\n\t"
-            "min.relu.s32 y3, y3, 255;\n\t"
-            "mad.lo.u32 p, y1, 256, y0;\n\t"
-            "mad.lo.u32 q, y3, 256, y2;\n\t"
-            "mad.lo.u32 p, q, 65536, p;\n\t"
-            "shr.b32 p, p, 1;\n\t"
-            "and.b32 %0, p, 0x7f7f7f7f;\n\t"
-            "}"
-            : "=r"(d)
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
-              "r"(rword), "r"(rsel[0]), "r"(rsel[1]), "r"(rsel[2]), "r"(rsel[3]), "r"(k));
-    } else if (!kRes && !kAddBias) {
-        asm("{\n\t"
-            ".reg .b32 y0, y1, y2, y3, p, q;\n\t"
-            "mad.hi.s32 y0, %1, %5, 1;\n\t"
-            "mad.hi.s32 y1, %2, %6, 1;\n\t"
-            "mad.hi.s32 y2, %3, %7, 1;\n\t"
-            "mad.hi.s32 y3, %4, %8, 1;\n\t"
-            "min.relu.s32 y0, y0, 255;\n\t"
-            "min.relu.s32 y1, y1, 255;\n\t"
-            "min.relu.s32 y2, y2, 255;\n\t"
-            "min.relu.s32 y3, y3, 255;\n\t"
-            "mad.lo.u32 p, y1, 256, y0;\n\t"
-            "mad.lo.u32 q, y3, 256, y2;\n\t"
-            "mad.lo.u32 p, q, 65536, p;\n\t"
-            "shr.b32 p, p, 1;\n\t"
-            "and.b32 %0, p, 0x7f7f7f7f;\n\t"
-            "}"
-            : "=r"(d)
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w));
-    } else if (kRes) {
-        asm("{\n\t"
-            ".reg .b32 u0, u1, u2, u3, r0, r1, r2, r3, y0, y1, y2, y3, p, q;\n\t"
-            "add.s32 u0, %1, %9;\n\t"
-            "add.s32 u1, %2, %10;\n\t"
-            "add.s32 u2, %3, %11;\n\t"
-            "add.s32 u3, %4, %12;\n\t"
-            "prmt.b32 r0, %13, 0, %14;\n\t"
-            "prmt.b32 r1, %13, 0, %15;\n\t"
-            "prmt.b32 r2, %13, 0, %16;\n\t"
-            "prmt.b32 r3, %13, 0, %17;\n\t"
-            "mad.lo.s32 r0, r0, %18, 1;\n\t"
-            "mad.lo.s32 r1, r1, %18, 1;\n\t"
-            "mad.lo.s32 r2, r2, %18, 1;\n\t"
-            "mad.lo.s32 r3, r3, %18, 1;\n\t"
-            "mad.hi.s32 y0, u0, %5, r0;\n\t"
-            "mad.hi.s32 y1, u1, %6, r1;\n\t"
-            "mad.hi.s32 y2, u2, %7, r2;\n\t"
-            "mad.hi.s32 y3, u3, %8, r3;\n\t"
-            "min.relu.s32 y0, y0, 255;\n\t"
-            "min.relu.s32 y1, y1, 255;\n\t"
-            "min.relu.s32 y2, y2, 255;\n\t"
-            "min.relu.s32 y3, y3, 255;\n\t"
-            "mad.lo.u32 p, y1, 256, y0;\n\t"
-            "mad.lo.u32 q, y3, 256, y2;\n\t"
-            "mad.lo.u32 p, q, 65536, p;\n\t"
-            "shr.b32 p, p, 1;\n\t"
-            "and.b32 %0, p, 0x7f7f7f7f;\n\t"
-            "}"
-            : "=r"(d)
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
-              "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(rword), "r"(rsel[0]), "r"(rsel[1]),
-              "r"(rsel[2]), "r"(rsel[3]), "r"(k));
-    } else {
-        asm("{\n\t"
-            ".reg .b32 u0, u1, u2, u3, y0, y1, y2, y3, p, q;\n\t"
-            "add.s32 u0, %1, %9;\n\t"
-            "add.s32 u1, %2, %10;\n\t"
-            "add.s32 u2, %3, %11;\n\t"
-            "add.s32 u3, %4, %12;\n\t"
-            "mad.hi.s32 y0, u0, %5, 1;\n\t"
-            "mad.hi.s32 y1, u1, %6, 1;\n\t"
-            "mad.hi.s32 y2, u2, %7, 1;\n\t"
-            "mad.hi.s32 y3, u3, %8, 1;\n\t"
-            "min.relu.s32 y0, y0, 255;\n\t"
-            "min.relu.s32 y1, y1, 255;\n\t"
-            "min.relu.s32 y2, y2, 255;\n\t"
-            "min.relu.s32 y3, y3, 255;\n\t"
-            "mad.lo.u32 p, y1, 256, y0;\n\t"
-            "mad.lo.u32 q, y3, 256, y2;\n\t"
-            "mad.lo.u32 p, q, 65536, p;\n\t"
-            "shr.b32 p, p, 1;\n\t"
-            "and.b32 %0, p, 0x7f7f7f7f;\n\t"
-            "}"
-            : "=r"(d)
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(m.x), "r"(m.y), "r"(m.z), "r"(m.w),
-              "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
-    }
+    asm("{\n\t"
+        ".reg .b32 p, q;\n\t"
+        "mad.lo.u32 p, %2, 256, %1;\n\t"
+        "mad.lo.u32 q, %4, 256, %3;\n\t"
+        "mad.lo.u32 p, q, 65536, p;\n\t"
+        "shr.b32 p, p, 1;\n\t"
+        "and.b32 %0, p, 0x7f7f7f7f;\n\t"
+        "}"
+        : "=r"(d)
+        : "r"(y[0]), "r"(y[1]), "r"(y[2]), "r"(y[3]));
     return d;
 }
 
