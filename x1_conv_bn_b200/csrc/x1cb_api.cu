@@ -306,10 +306,10 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
         return e;
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
-                  "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d",
+                  "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo);
+                  p.halo, p.io_swz);
     return X1CB_OK;
 }
 

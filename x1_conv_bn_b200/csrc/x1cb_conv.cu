@@ -275,6 +275,8 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     // rows outside the box read row 0's bytes and write nothing.
     const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
     const int chunk_stride = plane_t * 32;
+    // (o >> 3) & 0x70 is bits 7-9 of o moved to bits 4-6: the 128-byte swizzle.
+    const int swz_mask = p.io_swz ? 0x70 : 0;
     const int n_slots = kTmemCols / p.nmma;
     const int chunks_per_sub = p.nmma / 32;
     const int stages_per_sub = chunks_per_sub / kRChunks;
@@ -323,7 +325,7 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                                                kDevTimeoutEpilogue)))
             return;
         const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
-        uint8_t *stage = cx.io + st * kRSlotBytes + row_off;
+        uint8_t *stage = cx.io + st * kRSlotBytes;
 #pragma unroll 1
         for (int c = 0; c < kRChunks; ++c) {
             const int cs = rl * kRChunks + c;          // chunk within the TMEM slot
@@ -331,10 +333,15 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             uint32_t v[32];
             __syncwarp();
             tmem_ld_32x32b_x32_sync(tbase + static_cast<uint32_t>(cs * 32), v);
-            uint4 *pc = reinterpret_cast<uint4 *>(stage + c * chunk_stride);
+            // This pixel's two 16-byte halves (swizzled stages: the 16-byte unit
+            // index within each 128-byte row is XORed with the row index).
+            const int o = row_off + c * chunk_stride;
+            const int sw = swz_mask & (o >> 3);
+            uint4 *pa = reinterpret_cast<uint4 *>(stage + (o ^ sw));
+            uint4 *pb = reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw));
             uint32_t rw[8];
             if (kRes) {
-                const uint4 ra = pc[0], rb = pc[1];
+                const uint4 ra = *pa, rb = *pb;
                 rw[0] = ra.x; rw[1] = ra.y; rw[2] = ra.z; rw[3] = ra.w;
                 rw[4] = rb.x; rw[5] = rb.y; rw[6] = rb.z; rw[7] = rb.w;
             }
@@ -349,8 +356,8 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                 requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
             }
             if (in_box) {
-                pc[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                pc[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
             }
         }
         // Results must be visible to the TMA store (async proxy).
@@ -614,7 +621,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (kRes) {
                         mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
                         const int o1 = group * (p.NC / 32) + rs * kRChunks;
-                        if (p.io_wide)
+                        if (p.io_swz)
+                            tma_load_5d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
+                                             0, w0 / 4, h0, o1, b0, pol);
+                        else if (p.io_wide)
                             tma_load_4d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
                                              w0 * 4, h0, o1, b0, pol);
                         else
@@ -658,7 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     const int o1 = group * (p.NC / 32) + rs * kRChunks;
-                    if (p.io_wide)
+                    if (p.io_swz)
+                        tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0 / 4, h0, o1, b0,
+                                          pol);
+                    else if (p.io_wide)
                         tma_store_4d_hint(&tmO, sio + stage * kRSlotBytes, w0 * 4, h0, o1, b0, pol);
                     else
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0, h0, o1, b0, pol);
@@ -1025,8 +1038,8 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
                 break;
             }
     // Halo form: one slot per channel block, all of a tile's blocks in the ring
-    // when two accumulator slots share them.
-    p.a_slot = p.halo ? 2 * p.a_half : p.a_kc * kASlotBytes;
+    // when two accumulator slots share them; slots stay 1024-byte aligned.
+    p.a_slot = p.halo ? (2 * p.a_half + 1023) / 1024 * 1024 : p.a_kc * kASlotBytes;
     const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
     const int a_want = std::max(a_min, a_bytes_want / p.a_slot);
     const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 4;
@@ -1057,6 +1070,8 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     if (!placed)
         return X1CB_ERR_SHAPE;
     p.io_wide = p.tw * 4 <= 256 ? 1 : 0;  // TMA box dimensions are at most 256 elements
+    // The swizzled stages need whole 4-pixel groups and 1024-byte aligned stages.
+    p.io_swz = (p.tw % 4 == 0 && p.Wp % 4 == 0 && p.off_r % 1024 == 0) ? 1 : 0;
 
     const long long work = mtiles * p.n_groups;
     long long grid = std::min<long long>(num_sms, work);
@@ -1106,7 +1121,25 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
     // Shortcut and output, no swizzle: one box is one I/O stage [tg][4][th][tw][32].
     // Wide form: the same bytes as 8-byte elements, dims (4*Wp, Hp, O1, B) and
     // box (4*tw, th, 4, tg), so a box row is one contiguous run of tw*32 bytes.
-    if (p.io_wide) {
+    if (p.io_swz) {
+        // 128-byte rows: dims (16 x 8 bytes, Wp/4, Hp, O1, B), box (16, tw/4, th, 4, tg).
+        const uint64_t dims[5] = {16, (uint64_t)p.Wp / 4, (uint64_t)p.Hp, (uint64_t)p.O1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {128, (uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
+                                 (uint64_t)p.O1 * p.Hp * p.Wp * 32};
+        const uint32_t box[5] = {16, (uint32_t)p.tw / 4, (uint32_t)p.th, (uint32_t)kRChunks,
+                                 (uint32_t)p.tg};
+        if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+            return e;
+        if (p.has_res) {
+            if (int e = encode_map(&tmR, r, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_DATA_TYPE_UINT64))
+                return e;
+        } else {
+            tmR = tmO;  // unused
+        }
+    } else if (p.io_wide) {
         const uint64_t dims[4] = {(uint64_t)p.Wp * 4, (uint64_t)p.Hp, (uint64_t)p.O1,
                                   (uint64_t)p.B};
         const uint64_t str[3] = {(uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,

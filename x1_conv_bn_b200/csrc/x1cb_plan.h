@@ -46,6 +46,11 @@ struct ConvPlan {
     int off_w, off_a, off_r, off_cc, off_cm, off_bar, off_misc;
     int smem_bytes;  // including alignment slack
     int io_wide;  // shortcut/output maps use 8-byte elements (box rows of tw*32 bytes)
+    // Shortcut/output stages use the TMA's 128-byte swizzle: box rows of 128
+    // bytes (4 pixels of one chunk) whose 16-byte units are permuted by the
+    // row index, so the epilogue's per-pixel 32-byte accesses avoid bank
+    // conflicts.  Needs tw and the stored row length to be multiples of 4.
+    int io_swz;
     // Shared memory reserved for folding the bias into the MMA (0 = no room):
     // a constant 128 x 32-byte A tile at off_ba and NC x 32 bytes of per-channel
     // digit rows at off_bb.
