@@ -407,7 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_misc + 4);
     Bars bars{sbase + static_cast<uint32_t>(p.off_bar), p.a_stages, p.r_stages};
-    const WaitCtl ctl{abort_flag, &g_dev_status, p.wait_limit_ns};
+    // With the test hook armed, the MMA warp's planted wait has the limit and
+    // every other wait four times it, so the planted one is the wait that runs
+    // out and the others leave on the abort flag.
+    const WaitCtl ctl{abort_flag, &g_dev_status,
+                      p.inject == 1 ? 4 * p.wait_limit_ns : p.wait_limit_ns};
     const uint64_t drain_ns = 200000000ull;  // 0.2 s for copies/MMAs already issued
 
     const int group = blockIdx.x % p.n_groups;
@@ -722,7 +726,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool ok = mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma);
             if (ok && p.inject == 1)
-                ok = mbar_wait(bars.never(), 0, ctl, kDevTimeoutMma);  // test hook
+                ok = mbar_wait(bars.never(), 0,  // test hook
+                               WaitCtl{abort_flag, &g_dev_status, p.wait_limit_ns},
+                               kDevTimeoutMma);
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int st = a_stage;
                 uint32_t ph = a_phase;
@@ -741,12 +747,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint64_t bd = b_desc0 + static_cast<uint64_t>(j) * b_sub_step;
                     uint32_t accumulate = 0;
                     for (int box = 0; box < boxes; ++box) {
-                        if (j == 0) {
-                            if (!mbar_wait(bars.a_full(st), ph, ctl, kDevTimeoutMma)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
+                        // The slot was written by TMA and is read by the MMA, both in the
+                        // async proxy; the barrier's transaction count orders them.
+                        if (j == 0 && !mbar_wait(bars.a_full(st), ph, ctl, kDevTimeoutMma)) {
+                            ok = false;
+                            break;
                         }
                         uint64_t ad = sd;
                         if (p.halo) {

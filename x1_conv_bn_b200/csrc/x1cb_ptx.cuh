@@ -62,9 +62,28 @@ struct WaitCtl {
     uint64_t limit_ns;
 };
 
+// As mbar_try_wait, but a thread whose phase is not complete is suspended
+// until it completes or about `hint_ns` nanoseconds pass, instead of coming
+// straight back to poll: waiting warps leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of barrier `bar`.  Returns false (and never spins
 // forever) when the CTA was told to abort or when the wait exceeded the
 // limit; in the latter case it raises the abort flag and records `code`.
+// After one plain poll the thread sleeps on the barrier (20 us per try), and
+// the abort flag and the limit are checked every eighth try.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl &ctl,
                                           unsigned int code)
 {
@@ -72,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
         return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity))
+        if (mbar_try_wait_sleep(bar, parity, 20000u))
             return true;
         if ((it & 7u) == 0) {
             if (*ctl.abort_flag)
