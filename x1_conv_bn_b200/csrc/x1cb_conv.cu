@@ -13,21 +13,28 @@
 // article's A100 kernel:
 //  * one persistent CTA per SM, 20 warps, warp-specialised:
 //      warp 0      TMA producer: weights (once, resident in shared memory) and
-//                  the activation tiles (one 128-row x 32-byte K block per slot)
+//                  the activation slots (a_kc K blocks of 128 rows x 32 bytes,
+//                  or for the 3x3 one framed "halo" tile per channel block
+//                  that all nine filter taps read at row offsets)
 //      warp 1      MMA issuer: tcgen05.mma.kind::i8 into TMEM (int32), owner
-//                  of the TMEM allocation
+//                  of the TMEM allocation; the whole warp runs the loop and
+//                  one elected lane issues
 //      warp 2      TMA producer of the I/O stages: each 16 KB stage receives a
 //                  shortcut tile (128 pixels x 128 channels) long before use
 //      warp 3      TMA store of finished I/O stages
 //      warps 4-19  epilogue: tcgen05.ld, exact requantisation; each result
 //                  byte overwrites the shortcut byte of the same (pixel,
-//                  channel) in the stage, which warp 3 then stores whole
+//                  channel) in the stage, which warp 3 then stores whole.
+//                  The four warps of a TMEM lane quarter take turns on stages.
 //  * a tile is 128 GEMM rows = tw x th pixels of tg images, chosen per shape
 //    so that whole TMA boxes cover the image (16 px x 8 images for 28x28 1x1)
+//  * I/O stages use the TMA's 128-byte swizzle where the shape allows, so the
+//    epilogue's per-pixel 32-byte accesses are free of bank conflicts
 //  * TMEM holds 512 int32 columns; the accumulator ring lets the MMA of the
 //    next tile run while the epilogue drains the previous one
-//  * every wait is bounded; on timeout the CTA raises an abort flag, records
-//    a status bit, lets in-flight copies and MMAs land, frees TMEM, and exits.
+//  * every wait is bounded (waiting threads sleep on the barrier); on timeout
+//    the CTA raises an abort flag, records a status bit, lets in-flight copies
+//    and MMAs land, frees TMEM, and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -694,9 +701,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ---- MMA issuer -----------------------------------------------------------
-        if (lane == 0) {
+        // The whole warp runs the loop (waits are warp votes, so it stays
+        // converged) and one elected lane issues each MMA and commit.
+        {
             // The issue loop is kept free of divisions and descriptor rebuilds:
-            // a single thread's dependent integer work between two MMAs costs
+            // the dependent integer work between two MMAs would otherwise cost
             // more than the MMA itself (64-128 tensor cycles).  A descriptor's
             // start-address field is the byte address / 16 and every operand
             // lies below 256 KB, so moving an operand by `b` bytes is adding
@@ -724,17 +733,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t a_slot_desc = a_desc0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            bool ok = mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma);
-            if (ok && p.inject == 1)
-                ok = mbar_wait(bars.never(), 0,  // test hook
-                               WaitCtl{abort_flag, &g_dev_status, p.wait_limit_ns},
-                               kDevTimeoutMma);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma));
+            if (ok && p.inject == 1) {
+                const WaitCtl planted{abort_flag, &g_dev_status, p.wait_limit_ns};
+                ok = __all_sync(0xffffffffu,  // test hook
+                                mbar_wait(bars.never(), 0, planted, kDevTimeoutMma));
+            }
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int st = a_stage;
                 uint32_t ph = a_phase;
                 uint64_t sd = a_slot_desc;
                 for (int j = 0; ok && j < p.n_subs; ++j) {
-                    if (!mbar_wait(bars.acc_empty(acc), acc_phase ^ 1u, ctl, kDevTimeoutMma)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(bars.acc_empty(acc), acc_phase ^ 1u,
+                                                           ctl, kDevTimeoutMma))) {
                         ok = false;
                         break;
                     }
@@ -749,7 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int box = 0; box < boxes; ++box) {
                         // The slot was written by TMA and is read by the MMA, both in the
                         // async proxy; the barrier's transaction count orders them.
-                        if (j == 0 && !mbar_wait(bars.a_full(st), ph, ctl, kDevTimeoutMma)) {
+                        if (j == 0 && !__all_sync(0xffffffffu, mbar_wait(bars.a_full(st), ph, ctl,
+                                                                         kDevTimeoutMma))) {
                             ok = false;
                             break;
                         }
@@ -803,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Make sure no MMA is still reading shared memory or writing TMEM.
             mma_commit(bars.mma_done());
-            if (!mbar_drain(bars.mma_done(), 0, drain_ns))
+            if (lane == 0 && !mbar_drain(bars.mma_done(), 0, drain_ns))
                 atomicOr(&g_dev_status, kDevDrainFailed);
         }
         __syncwarp();

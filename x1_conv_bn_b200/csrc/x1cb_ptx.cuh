@@ -418,22 +418,31 @@ __host__ __device__ constexpr uint32_t idesc_i8(uint32_t M, uint32_t N)
            | ((M >> 4) << 24);  // M
 }
 
+// One MMA step D (+)= A x B, s8 x s8 -> s32 in TMEM.  Warp-wide: every lane
+// of the issuing warp calls it with the same operands and one elected lane
+// issues, so the warp stays converged and its operand arithmetic is
+// warp-uniform.  accumulate = 0 overwrites D.
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
-// Arrive once on `bar` when every MMA issued so far by this thread is done.
+// Arrive once on `bar` when every MMA issued so far by the warp's elected lane
+// is done (warp-wide, like mma_i8).
 __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(bar)
         : "memory");
 }
 
