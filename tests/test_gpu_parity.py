@@ -266,6 +266,45 @@ def test_full_size_1x1_sampled(oracle, cfg):
     _assert_spread(ref)
 
 
+# ---- many launches back to back -----------------------------------------------------
+# The kernel's warps hand ring slots and accumulators to one another through
+# mbarrier phases; an ordering mistake there shows up only now and then, as a
+# wait that runs out (device status) or as a launch that differs from the rest.
+
+STRESS = [
+    (256, 28, 28, 128, 512, 1, True),   # Res3.2 Conv3 (I/O ring of 7 stages)
+    (96, 28, 28, 512, 128, 1, False),   # Res3.2 conv1 (3 stages)
+    (96, 28, 28, 128, 128, 3, False),   # Res3.2 conv2, halo form (2 stages)
+]
+
+
+@pytest.mark.parametrize("shape", STRESS, ids=[str(s) for s in STRESS])
+def test_repeated_launches_stay_exact(oracle, shape):
+    s = synth.ConvShape(*shape)
+    inp = synth.conv_inputs(s, 91)
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    w = X.x1cb_pack_weight(inp.w.to(DEV))
+    bias, m = inp.bias.to(DEV), inp.m.to(DEV)
+    r = X.x1cb_pack_act(inp.r.to(DEV)) if s.has_res else None
+    X.x1cb_last_device_error(clear=True)
+    outs = []
+    for i in range(300):
+        if s.R == 1:
+            out = X.conv1x1_bn_add_relu_i8(x, w, bias, m, inp.m_r, inp.S, r)
+        else:
+            out = X.conv3x3_bn_relu_i8(x, w, bias, m, inp.S)
+        if i % 50 == 0 or i == 299:
+            outs.append(out)
+    torch.cuda.synchronize()
+    st, bits = X.x1cb_last_device_error(clear=True)
+    assert st == 0 and bits == 0, bits
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    pix = _sample_pixels(s.B, s.H, s.W, 600, 3)
+    ref = oracle.conv_pixels(inp.x, inp.w, inp.bias, inp.m, inp.S, pix, inp.r, inp.m_r)
+    assert torch.equal(_gather_nc32(outs[0].cpu(), pix, s.H, s.W), ref)
+
+
 def test_full_size_block_sampled(oracle):
     s = synth.CONFIGS["5"]
     inp = synth.block_inputs(s, synth.CONFIG_SEEDS["5"])

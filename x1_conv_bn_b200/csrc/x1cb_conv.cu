@@ -251,6 +251,7 @@ struct EpiCtx {
     WaitCtl ctl;
     uint32_t tmem_base;
     uint8_t *io;
+    volatile int *io_ticket;  // I/O stages before this one have been seen to arrive
     const int32_t *cm;
     const long long *cC;
     int group, mt_first, mt_step;
@@ -264,10 +265,19 @@ struct EpiCtx {
 // handles stages g, g + kTurns, ... (counted over all of the CTA's tiles), all
 // four 32-channel chunks of its 32 rows.  Turns drift apart in time, so while
 // one warp waits for its stage or its TMEM load the others compute.
+//
+// A parity wait on an mbarrier is only meaningful when the phase before the
+// awaited one is known to be complete.  Accumulator slots: the turns are as
+// many as the I/O stages the TMEM holds, so each turn uses one slot and takes
+// every phase of it.  I/O slots: before awaiting a stage's arrival a turn
+// makes sure the slot's previous stage is complete (see below), so each
+// slot's phases are observed in order whatever the ring depth.
 template <bool kRes, int kMode, bool kK1 = false>
 __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int lane)
 {
     constexpr int kTurns = kEpiWarps / 4;                 // warps per TMEM lane quarter
+    static_assert(kTurns == kTmemCols / (32 * kRChunks),
+                  "one turn per I/O stage held in TMEM: each turn owns one accumulator slot");
     const ConvPlan &p = *cx.p;
     const int q = warp & 3;                               // TMEM lane quarter this warp may access
     const int turn = (warp - kEpiWarp0) >> 2;
@@ -328,9 +338,24 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                                                kDevTimeoutEpilogue)))
             return;
         tc_fence_after();
+        // Before the parity wait on the slot's arrival, make sure its previous
+        // phase (stage n - r_stages, another turn's) is complete.  Ring of at
+        // least kTurns stages: wait, as the producer does, until that stage has
+        // been stored (exact: stage n - 2*r_stages was stored before this
+        // turn's previous stage could be loaded).  Shallower ring: take the
+        // arrivals in stage order with the ticket.
+        const bool deep = p.r_stages >= kTurns;
+        if (deep ? !__all_sync(0xffffffffu, mbar_wait(cx.bars.io_empty(st), st_phase ^ 1u,
+                                                      cx.ctl, kDevTimeoutEpilogue))
+                 : !__all_sync(0xffffffffu, ticket_wait(cx.io_ticket, static_cast<int>(n),
+                                                        cx.ctl, kDevTimeoutEpilogue)))
+            return;
         if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.io_full(st), st_phase, cx.ctl,
                                                kDevTimeoutEpilogue)))
             return;
+        // The four warps of a turn each pass the ticket on; it only moves forward.
+        if (!deep && lane == 0)
+            atomicMax(const_cast<int *>(cx.io_ticket), static_cast<int>(n + 1));
         const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
         uint8_t *stage = cx.io + st * kRSlotBytes;
 #pragma unroll 1
@@ -413,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t *cm = reinterpret_cast<int32_t *>(smem + p.off_cm);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_misc + 4);
+    volatile int *io_ticket = reinterpret_cast<volatile int *>(smem + p.off_misc + 8);
     Bars bars{sbase + static_cast<uint32_t>(p.off_bar), p.a_stages, p.r_stages};
     // With the test hook armed, the MMA warp's planted wait has the limit and
     // every other wait four times it, so the planted one is the wait that runs
@@ -429,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- set-up ---------------------------------------------------------------
     if (threadIdx.x == 0) {
         *abort_flag = 0;
+        *io_ticket = 0;
         mbar_init(bars.w_full(), 1);
         mbar_init(bars.mma_done(), 1);
         mbar_init(bars.never(), 1);
@@ -821,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ---- epilogue ---------------------------------------------------------------
-        const EpiCtx cx{&p, bars, ctl, tmem_base, smem + p.off_r, cm, cC,
+        const EpiCtx cx{&p, bars, ctl, tmem_base, smem + p.off_r, io_ticket, cm, cC,
                         group, mt_first, mt_step};
         const bool k1 = kRes && static_cast<long long>(p.m_r) == (1ll << (p.S - 1));
         if (mode == 3 && k1)

@@ -105,6 +105,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
 }
 
+// Bounded wait until a monotonic shared-memory counter reaches at least
+// `want` (napping between polls); same abort and limit rules as mbar_wait.
+__device__ __forceinline__ bool ticket_wait(const volatile int *ticket, int want,
+                                            const WaitCtl &ctl, unsigned int code)
+{
+    if (*ticket >= want)
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(32);
+        if (*ticket >= want)
+            return true;
+        if ((it & 15u) == 0) {
+            if (*ctl.abort_flag)
+                return false;
+            if (globaltimer_ns() - t0 > ctl.limit_ns) {
+                *ctl.abort_flag = 1;
+                atomicOr(ctl.status, code);
+                return false;
+            }
+        }
+    }
+}
+
 // Bounded wait that ignores the abort flag: used on the way out to let copies
 // and MMAs already in flight land before shared memory and TMEM are released.
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
