@@ -115,6 +115,58 @@ def test_plans(L, shape, expect):
     assert expect in X.x1cb_describe_plan(*shape)
 
 
+def _plan(shape):
+    return dict(kv.split("=") for kv in X.x1cb_describe_plan(*shape).split())
+
+
+@pytest.mark.parametrize("shape,tile", [
+    ((1024, 28, 28, 128, 128, 3, 0), "28x4x1"),   # Res3.2 conv2: 4 rows + frame = 120 GEMM rows
+    ((2, 30, 28, 128, 128, 3, 0), "28x4x1"),      # ragged in H: 8 tiles per image, last one 2 rows
+    ((5, 3, 5, 64, 128, 3, 0), "5x3x3"),          # three framed images in one tile
+    ((11, 6, 6, 128, 128, 3, 0), "6x6x2"),
+    ((1, 1, 1, 32, 128, 3, 0), "1x1x1"),
+])
+def test_halo_tiles(L, shape, tile):
+    """3x3 with W+2 <= 128 uses the halo form: every pixel of the tile lands in
+    the 128 GEMM rows, m = (g*(th+2) + y)*(W+2) + x."""
+    p = _plan(shape)
+    assert p["halo"] == "1" and p["tile"] == tile and p["kc"] == "1"
+    tw, th, tg = (int(v) for v in tile.split("x"))
+    W = shape[2]
+    assert tw == W
+    assert (tg - 1) * (th + 2) * (W + 2) + (th - 1) * (W + 2) + (W - 1) < 128
+    assert int(p["rows"]) == tw * th * tg
+
+
+def test_wide_images_take_the_per_tap_form(L):
+    p = _plan((1, 3, 130, 32, 128, 3, 0))
+    assert p["halo"] == "0"
+
+
+@pytest.mark.parametrize("shape,swz", [
+    ((2048, 28, 28, 128, 512, 1, 1), "1"),    # tw 16, row length 784
+    ((512, 56, 56, 64, 256, 1, 1), "1"),
+    ((1024, 28, 28, 128, 128, 3, 0), "1"),    # halo tile 28 wide
+    ((512, 14, 14, 256, 1024, 1, 1), "0"),    # 14-pixel tiles: not whole 4-pixel groups
+    ((512, 7, 7, 512, 2048, 1, 1), "0"),
+    ((17, 2, 3, 32, 384, 1, 1), "0"),
+])
+def test_swizzled_io_stages_only_for_whole_pixel_groups(L, shape, swz):
+    p = _plan(shape)
+    assert p["swz"] == swz
+    if swz == "1":
+        assert int(p["tile"].split("x")[0]) % 4 == 0
+
+
+@pytest.mark.parametrize("shape", [(2048, 28, 28, 128, 512, 1, 1), (1024, 28, 28, 512, 128, 1, 0),
+                                   (1024, 28, 28, 128, 128, 3, 0), (3, 14, 14, 256, 1024, 1, 1)])
+def test_plans_fit_shared_memory(L, shape):
+    p = _plan(shape)
+    assert int(p["smem"]) <= 232448
+    assert int(p["r_stages"]) >= (4 if shape[-1] else 2)
+    assert int(p["a_stages"]) >= 2
+
+
 def test_plan_rejects_weights_that_do_not_fit(L):
     with pytest.raises(X.X1cbError):
         X.x1cb_describe_plan(8, 14, 14, 1024, 256, 3, 0)
