@@ -36,7 +36,9 @@
  * x1cb_last_device_error().
  * Limits: stride 1; 1 <= S <= 60; Ic and Oc multiples of 32 and 128 with
  * Ic <= 4096; the weights of 128 output channels (R*R*Ic*128 bytes) must fit
- * in shared memory (Ic <= 1280 for 1x1 with a residual, Ic <= 128 for 3x3);
+ * in shared memory beside the rings (Ic <= 1120 for 1x1 with a residual,
+ * Ic <= 1376 for 1x1 without, Ic <= 128 for 3x3); other shapes return
+ * X1CB_ERR_SHAPE;
  * requires an sm_100 device.
  * Errors: a negative X1CB_ERR_* status; nothing is launched in that case.
  */

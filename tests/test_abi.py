@@ -167,6 +167,13 @@ def test_plans_fit_shared_memory(L, shape):
     assert int(p["a_stages"]) >= 2
 
 
+@pytest.mark.parametrize("R,res,max_ic", [(1, 1, 1120), (1, 0, 1376), (3, 0, 128)])
+def test_channel_limits_stated_in_the_header(L, R, res, max_ic):
+    X.x1cb_describe_plan(4, 28, 28, max_ic, 128, R, res)
+    with pytest.raises(X.X1cbError):
+        X.x1cb_describe_plan(4, 28, 28, max_ic + 32, 128, R, res)
+
+
 def test_plan_rejects_weights_that_do_not_fit(L):
     with pytest.raises(X.X1cbError):
         X.x1cb_describe_plan(8, 14, 14, 1024, 256, 3, 0)
