@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="3", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="x1cb", choices=["x1cb", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target length of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -355,42 +355,70 @@ def main():
     tops = value_ops / 1e12
 
     # ---- end to end through the API with host buffers ----
+    # Every step uploads its inputs from pinned host memory, runs the fused op
+    # and reads its result back.  Steps are double-buffered over three streams
+    # (upload, compute, read-back) so that step i+1's upload, step i's kernel
+    # and step i-1's read-back overlap: PCIe is full duplex and the copy
+    # engines run beside the SMs.  Events order each buffer's reuse.
     e2e = None
     if not a.no_e2e:
         host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in ins.items()}
         for k in ins:
             host_in[k].copy_(ins[k])
-        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        dev_in = {k: torch.empty_like(v) for k, v in ins.items()}
-        dev_out = torch.empty_like(out)
+        host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+        dev_in = [{k: torch.empty_like(v) for k, v in ins.items()} for _ in range(2)]
+        dev_out = [torch.empty_like(out) for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-        d2h = host_out.numel() * host_out.element_size()
+        d2h = host_out[0].numel() * host_out[0].element_size()
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        n_e2e = a.e2e_steps
 
-        def e2e_step():
-            for k in dev_in:
-                dev_in[k].copy_(host_in[k], non_blocking=True)
-            if "r" in dev_in:
-                call(x_=dev_in["x"], r_=dev_in["r"], out_=dev_out, stream=stream)
-            else:
-                call(x_=dev_in["x"], out_=dev_out, stream=stream)
-            host_out.copy_(dev_out, non_blocking=True)
+        def e2e_run(n):
+            done_in = [None, None]    # kernel of the buffer's last step has read its inputs
+            done_out = [None, None]   # read-back of the buffer's last step has finished
+            for i in range(n):
+                b = i % 2
+                with torch.cuda.stream(s_in):
+                    if done_in[b] is not None:
+                        s_in.wait_event(done_in[b])
+                    for k in dev_in[b]:
+                        dev_in[b][k].copy_(host_in[k], non_blocking=True)
+                    ev_in = torch.cuda.Event()
+                    ev_in.record(s_in)
+                stream.wait_event(ev_in)
+                if done_out[b] is not None:
+                    stream.wait_event(done_out[b])
+                if "r" in dev_in[b]:
+                    call(x_=dev_in[b]["x"], r_=dev_in[b]["r"], out_=dev_out[b], stream=stream)
+                else:
+                    call(x_=dev_in[b]["x"], out_=dev_out[b], stream=stream)
+                ev_k = torch.cuda.Event()
+                ev_k.record(stream)
+                done_in[b] = ev_k
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_k)
+                    host_out[b].copy_(dev_out[b], non_blocking=True)
+                    ev_o = torch.cuda.Event()
+                    ev_o.record(s_out)
+                done_out[b] = ev_o
 
-        with torch.cuda.stream(stream):
-            e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         barrier()
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(a.e2e_steps):
-                e2e_step()
-            e1.record(stream)
-        e1.synchronize()
+        e0.record(s_in)
+        e2e_run(n_e2e)
+        e1.record(s_out)  # after the last read-back; e0 came before the first upload
+        torch.cuda.synchronize()
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / a.e2e_steps, dist, dev)
+        st, bits = X.x1cb_last_device_error(clear=True)
+        if st != 0:
+            raise RuntimeError(f"device status {bits:#x} in the end-to-end region")
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
         e2e_ops, _ = aggregate([e2e_ms] * world, ops)
         e2e = {"value": e2e_ops / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "how": "pinned host -> device copies, fused op, device -> pinned host, per step"}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e,
+               "how": "per step: pinned host -> device inputs, fused op, device -> pinned "
+                      "host result; double-buffered over upload/compute/read-back streams"}
 
     if dist is not None:
         dist.destroy_process_group()
