@@ -47,6 +47,10 @@ def lib():
                                      + [ctypes.c_int] * 5)
         L.x1o_bottleneck_pixels.argtypes = ([c_i8p] * 10 + [ctypes.c_int32, ctypes.c_int, c_i8p,
                                              ctypes.c_int64, c_i8p] + [ctypes.c_int] * 5)
+        L.x1o_conv_strided.argtypes = ([c_i8p] * 4 + [ctypes.c_int, c_i8p, ctypes.c_int32, c_i8p]
+                                       + [ctypes.c_int] * 8)
+        L.x1o_conv_proj.argtypes = [c_i8p] * 6 + [ctypes.c_int, c_i8p] + [ctypes.c_int] * 9
+        L.x1o_bottleneck_proj.argtypes = [c_i8p] * 11 + [ctypes.c_int, c_i8p] + [ctypes.c_int] * 6
         L.x1o_set_threads.argtypes = [ctypes.c_int]
         L.x1o_set_threads.restype = ctypes.c_int
         _lib = L
@@ -155,4 +159,56 @@ def bottleneck_pixels(x, ws, bs, ms, m_r, S, pix):
     out = torch.empty((pix.numel(), Cin), dtype=torch.int8)
     lib().x1o_bottleneck_pixels(*[_p(a) for a in args], int(m_r), S, _p(pix), pix.numel(),
                                 _p(out), B, H, W, Cin, Cmid)
+    return out
+
+
+def out_extent(n: int, R: int, pad: int, stride: int) -> int:
+    return (n + 2 * pad - R) // stride + 1
+
+
+def conv_strided(x, w, bias, m, S, stride, r=None, m_r=0, pad=None):
+    """Fused conv of any stride + BN (+ residual) + ReLU + requant.  NHWC in,
+    NHWC out of (H + 2 pad - R) / stride + 1 rows and columns."""
+    B, H, W, Ic = x.shape
+    Oc, _, R, _ = w.shape
+    pad = (R - 1) // 2 if pad is None else pad
+    Ho, Wo = out_extent(H, R, pad, stride), out_extent(W, R, pad, stride)
+    x, w = _cpu(x, torch.int8), _cpu(w, torch.int8)
+    bias, m = _cpu(bias, torch.int32), _cpu(m, torch.int32)
+    r = _cpu(r, torch.int8)
+    out = torch.empty((B, Ho, Wo, Oc), dtype=torch.int8)
+    lib().x1o_conv_strided(_p(x), _p(w), _p(bias), _p(m), S, _p(r), int(m_r), _p(out),
+                           B, H, W, Ic, Oc, R, pad, stride)
+    return out
+
+
+def conv_proj(y, w3, x, wp, bias, m, S, stride=2):
+    """Projection block's Conv3: 1x1 of y plus the stride-`stride` 1x1 of x in
+    one accumulator, + BN + ReLU + requant.  y [B,H,W,Cy], x [B,Hx,Wx,Cx]."""
+    B, H, W, Cy = y.shape
+    _, Hx, Wx, Cx = x.shape
+    Oc = w3.shape[0]
+    y, x = _cpu(y, torch.int8), _cpu(x, torch.int8)
+    w3, wp = _cpu(w3, torch.int8), _cpu(wp, torch.int8)
+    bias, m = _cpu(bias, torch.int32), _cpu(m, torch.int32)
+    out = torch.empty((B, H, W, Oc), dtype=torch.int8)
+    lib().x1o_conv_proj(_p(y), _p(w3), _p(x), _p(wp), _p(bias), _p(m), S, _p(out),
+                        B, H, W, Cy, Cx, Oc, Hx, Wx, stride)
+    return out
+
+
+def bottleneck_proj(x, ws, wp, bs, ms, S):
+    """Res3.1 projection block.  ws = (w1, w2, w3) OIHW, wp the projection
+    weight [Cout, Cin, 1, 1]; bs, ms the three layers' bias and multiplier
+    (the third shared by Conv3 and the projection)."""
+    B, H, W, Cin = x.shape
+    Cmid, Cout = ws[0].shape[0], ws[2].shape[0]
+    Ho, Wo = out_extent(H, 3, 1, 2), out_extent(W, 3, 1, 2)
+    args = [_cpu(x, torch.int8)]
+    for w, b, mm in zip(ws[:2], bs[:2], ms[:2]):
+        args += [_cpu(w, torch.int8), _cpu(b, torch.int32), _cpu(mm, torch.int32)]
+    args += [_cpu(ws[2], torch.int8), _cpu(wp, torch.int8), _cpu(bs[2], torch.int32),
+             _cpu(ms[2], torch.int32)]
+    out = torch.empty((B, Ho, Wo, Cout), dtype=torch.int8)
+    lib().x1o_bottleneck_proj(*[_p(a) for a in args], S, _p(out), B, H, W, Cin, Cmid, Cout)
     return out

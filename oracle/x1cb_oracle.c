@@ -270,6 +270,112 @@ void x1o_bottleneck_pixels(const int8_t *x, const int8_t *w1, const int32_t *b1,
     }
 }
 
+/* ---- strided convolution and the projection block (Res3.1) ------------------
+ *
+ * The pages describe Res3.2-Res3.4 and say only that Res3.1's output feeds
+ * Res3.2 (Inspur article, section 2.2).  Res3.1 is the stage's first block:
+ * it halves the image and widens the channels, so its shortcut is a 1x1
+ * projection convolution of stride 2 instead of the identity.  Read here as
+ * in the MLPerf ResNet50 (v1.5) network: conv1 1x1 stride 1, conv2 3x3 pad 1
+ * stride 2, conv3 1x1; shortcut 1x1 stride 2 on the block input.  The
+ * projection's folded BN shares Conv3's per-channel multiplier (its relative
+ * scale folded into its int8 weights), so the two products are summed into
+ * one accumulator before the common bias, multiplier, rounding and ReLU:
+ *
+ *   acc = sum_i Y[b,h,w,i] * W3[o,i] + sum_j X[b, 2h, 2w, j] * WP[o,j]
+ *   out = min(max(floor(((acc + bias[o]) * m[o] + 2^(S-1)) / 2^S), 0), 127)
+ */
+
+/* Output extent of a convolution along one axis. */
+static int64_t conv_out_extent(int64_t in, int64_t R, int64_t pad, int64_t stride)
+{
+    return (in + 2 * pad - R) / stride + 1;
+}
+
+/* Fused convolution of any stride: output pixel (b, ho, wo) reads input
+ * pixels (ho*stride + r - pad, wo*stride + s - pad); taps outside the image
+ * contribute 0.  x: [B,H,W,Ic]; wt: [Oc,Ic,R,R]; r: [B,Ho,Wo,Oc] or NULL;
+ * out: [B,Ho,Wo,Oc]. */
+void x1o_conv_strided(const int8_t *x, const int8_t *wt, const int32_t *bias, const int32_t *m,
+                      int S, const int8_t *r, int32_t m_r, int8_t *out, int B, int H, int W,
+                      int Ic, int Oc, int R, int pad, int stride)
+{
+    int64_t Ho = conv_out_extent(H, R, pad, stride), Wo = conv_out_extent(W, R, pad, stride);
+    int64_t rows = (int64_t)B * Ho;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < rows; ++bh) {
+        int64_t b = bh / Ho, ho = bh % Ho;
+        for (int64_t wo = 0; wo < Wo; ++wo) {
+            size_t q = (size_t)((b * Ho + ho) * Wo + wo) * Oc;
+            for (int64_t o = 0; o < Oc; ++o) {
+                int64_t acc = 0;
+                for (int64_t rr = 0; rr < R; ++rr) {
+                    int64_t hi = ho * stride + rr - pad;
+                    if (hi < 0 || hi >= H)
+                        continue;
+                    for (int64_t ss = 0; ss < R; ++ss) {
+                        int64_t wi = wo * stride + ss - pad;
+                        if (wi < 0 || wi >= W)
+                            continue;
+                        const int8_t *xp = x + nhwc_index(b, hi, wi, 0, H, W, Ic);
+                        for (int64_t i = 0; i < Ic; ++i)
+                            acc += (int64_t)xp[i] * (int64_t)wt[oihw_index(o, i, rr, ss, Ic, R)];
+                    }
+                }
+                out[q + o] = x1o_requant(acc, bias[o], m[o], r != NULL, r ? r[q + o] : 0, m_r, S);
+            }
+        }
+    }
+}
+
+/* Conv3 of the projection block with its shortcut in the same accumulator.
+ * y: [B,H,W,Cy] (Conv2's output); w3: [Oc,Cy] (1x1, OIHW with R = 1);
+ * x: [B,Hx,Wx,Cx] (the block input), sampled at (stride*h, stride*w);
+ * wp: [Oc,Cx]; out: [B,H,W,Oc]. */
+void x1o_conv_proj(const int8_t *y, const int8_t *w3, const int8_t *x, const int8_t *wp,
+                   const int32_t *bias, const int32_t *m, int S, int8_t *out, int B, int H, int W,
+                   int Cy, int Cx, int Oc, int Hx, int Wx, int stride)
+{
+    int64_t rows = (int64_t)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < rows; ++bh) {
+        int64_t b = bh / H, h = bh % H;
+        for (int64_t w = 0; w < W; ++w) {
+            const int8_t *yp = y + nhwc_index(b, h, w, 0, H, W, Cy);
+            const int8_t *xp = x + nhwc_index(b, h * stride, w * stride, 0, Hx, Wx, Cx);
+            size_t q = (size_t)nhwc_index(b, h, w, 0, H, W, Oc);
+            for (int64_t o = 0; o < Oc; ++o) {
+                int64_t acc = 0;
+                for (int64_t i = 0; i < Cy; ++i)
+                    acc += (int64_t)yp[i] * (int64_t)w3[o * Cy + i];
+                for (int64_t j = 0; j < Cx; ++j)
+                    acc += (int64_t)xp[j] * (int64_t)wp[o * Cx + j];
+                out[q + o] = x1o_requant(acc, bias[o], m[o], 0, 0, 0, S);
+            }
+        }
+    }
+}
+
+/* Res3.1 projection block: conv1 1x1 Cin->Cmid +Bn+Relu (H x W), conv2 3x3
+ * pad 1 stride 2 Cmid->Cmid +Bn+Relu (-> Ho x Wo), conv3 1x1 Cmid->Cout plus
+ * the stride-2 1x1 projection Cin->Cout of the block input in one
+ * accumulator, +Bn+Relu.  x: [B,H,W,Cin]; out: [B,Ho,Wo,Cout]. */
+void x1o_bottleneck_proj(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                         const int8_t *w2, const int32_t *b2, const int32_t *m2,
+                         const int8_t *w3, const int8_t *wp, const int32_t *b3,
+                         const int32_t *m3, int S, int8_t *out, int B, int H, int W, int Cin,
+                         int Cmid, int Cout)
+{
+    int64_t Ho = conv_out_extent(H, 3, 1, 2), Wo = conv_out_extent(W, 3, 1, 2);
+    int8_t *y1 = (int8_t *)malloc((size_t)B * H * W * Cmid);
+    int8_t *y2 = (int8_t *)malloc((size_t)B * Ho * Wo * Cmid);
+    x1o_conv_strided(x, w1, b1, m1, S, NULL, 0, y1, B, H, W, Cin, Cmid, 1, 0, 1);
+    x1o_conv_strided(y1, w2, b2, m2, S, NULL, 0, y2, B, H, W, Cmid, Cmid, 3, 1, 2);
+    x1o_conv_proj(y2, w3, x, wp, b3, m3, S, out, B, (int)Ho, (int)Wo, Cmid, Cin, Cout, H, W, 2);
+    free(y1);
+    free(y2);
+}
+
 int x1o_set_threads(int n)
 {
 #ifdef _OPENMP

@@ -112,6 +112,76 @@ class BlockShape:
         return sum(s.bytes_moved() for s in self.stages())
 
 
+@dataclass(frozen=True)
+class ProjBlockShape:
+    """Res3.1-style projection bottleneck on an H x W input: 1x1 Cin->Cmid,
+    3x3 stride 2 Cmid->Cmid, 1x1 Cmid->Cout plus the stride-2 1x1 projection
+    Cin->Cout of the block input in the same accumulator."""
+
+    B: int
+    H: int
+    W: int
+    Cin: int
+    Cmid: int
+    Cout: int
+
+    @property
+    def Ho(self) -> int:
+        return (self.H - 1) // 2 + 1
+
+    @property
+    def Wo(self) -> int:
+        return (self.W - 1) // 2 + 1
+
+    def ops(self) -> int:
+        px_in, px_out = self.B * self.H * self.W, self.B * self.Ho * self.Wo
+        return 2 * (px_in * self.Cmid * self.Cin + px_out * self.Cmid * 9 * self.Cmid
+                    + px_out * self.Cout * (self.Cmid + self.Cin))
+
+    def bytes_moved(self) -> int:
+        px_in, px_out = self.B * self.H * self.W, self.B * self.Ho * self.Wo
+        n = px_in * (self.Cin + self.Cmid)                      # conv1: x in, y1 out
+        n += px_in * self.Cmid + px_out * self.Cmid             # conv2: y1 in, y2 out
+        n += px_out * (self.Cmid + self.Cin + self.Cout)        # conv3: y2, strided x, out
+        n += self.Cmid * self.Cin + 9 * self.Cmid ** 2 + self.Cout * (self.Cmid + self.Cin)
+        n += 8 * (2 * self.Cmid + self.Cout)
+        return n
+
+
+@dataclass
+class ProjBlockInputs:
+    shape: ProjBlockShape
+    x: torch.Tensor  # [B, H, W, Cin] int8
+    w: list = field(default_factory=list)  # conv1, conv2, conv3 OIHW
+    wp: Optional[torch.Tensor] = None      # projection [Cout, Cin, 1, 1]
+    bias: list = field(default_factory=list)
+    m: list = field(default_factory=list)
+    S: int = S_DEFAULT
+
+
+def proj_block_inputs(s: ProjBlockShape, seed: int, device="cpu",
+                      S: int = S_DEFAULT) -> ProjBlockInputs:
+    """Draw x, then (w, bias, m) of conv1 and conv2, then w3, wp, bias3, m3.
+    The third layer's multiplier uses the fan-in of both sources (Cmid + Cin)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = _randint(g, X_LO, X_HI, (s.B, s.H, s.W, s.Cin), torch.int8, device)
+    out = ProjBlockInputs(s, x, S=S)
+    for st in (ConvShape(s.B, s.H, s.W, s.Cin, s.Cmid, 1, False),
+               ConvShape(s.B, s.H, s.W, s.Cmid, s.Cmid, 3, False)):
+        w, bias, m = _draw_layer(g, st, S, device)
+        out.w.append(w)
+        out.bias.append(bias)
+        out.m.append(m)
+    out.w.append(_randint(g, W_LO, W_HI, (s.Cout, s.Cmid, 1, 1), torch.int8, device))
+    out.wp = _randint(g, W_LO, W_HI, (s.Cout, s.Cin, 1, 1), torch.int8, device)
+    out.bias.append(_randint(g, BIAS_LO, BIAS_HI, (s.Cout,), torch.int32, device))
+    c = multiplier_center(s.Cmid + s.Cin, S)
+    out.m.append(_randint(g, int(round(0.9 * c)), int(round(1.1 * c)), (s.Cout,), torch.int32,
+                          device))
+    return out
+
+
 # Named workloads.  Index 1..5 as in the benchmark plan; "4a".."4c" are the
 # three expand convolutions of the sweep.
 CONFIGS: Dict[str, object] = {
@@ -122,8 +192,11 @@ CONFIGS: Dict[str, object] = {
     "4b": ConvShape(512, 14, 14, 256, 1024, 1, True),
     "4c": ConvShape(512, 7, 7, 512, 2048, 1, True),
     "5": BlockShape(1024, 28, 28, 512, 128),
+    # Res3.1 (the stage's projection block), 56x56x256 in, 28x28x512 out.
+    "p31": ProjBlockShape(256, 56, 56, 256, 128, 512),
 }
-CONFIG_SEEDS = {"1": 1001, "2": 1002, "3": 1003, "4a": 1004, "4b": 1004, "4c": 1004, "5": 1005}
+CONFIG_SEEDS = {"1": 1001, "2": 1002, "3": 1003, "4a": 1004, "4b": 1004, "4c": 1004, "5": 1005,
+                "p31": 1031}
 WORKLOAD_NAMES = {
     "1": "res3.2-conv3 1x1 128->512 +bn+sum+relu, 28x28, B=1",
     "2": "res3.2-conv3 1x1 128->512 +bn+sum+relu, 28x28, B=256",
@@ -132,6 +205,8 @@ WORKLOAD_NAMES = {
     "4b": "expand 1x1 256->1024 +bn+sum+relu, 14x14, B=512",
     "4c": "expand 1x1 512->2048 +bn+sum+relu, 7x7, B=512",
     "5": "res3.2 bottleneck block 512->128->128->512, 28x28, B=1024",
+    "p31": "res3.1 projection block 256->128->128(s2)->512 + proj 256->512(s2), 56x56->28x28, "
+           "B=256",
 }
 
 
