@@ -7,8 +7,12 @@ One step = one pass of the fused op over one batch (config 3: B=2048).
 Timing: CUDA events on the launching stream around exactly K launches,
 bracketed by a barrier and a device synchronise on both sides; the max over
 ranks.  Inputs (1.85 GB per step at B=2048) are larger than the 126 MB L2,
-so no flush is needed.  With N > 1 every rank runs its own batch (weak
-scaling, batches are independent; no collective on the data path).
+so no flush is needed; smaller workloads rotate over enough input/output
+sets to span three times the L2.  With N > 1 every rank runs its own batch
+(weak scaling, batches are independent; no collective on the data path):
+launched under torch.distributed.run (WORLD_SIZE = N) each process drives
+its LOCAL_RANK GPU; started plainly with --gpus N, bench.py launches the N
+ranks itself.  --dry-run runs the same rank logic on the CPU over gloo.
 
 Prints one JSON line (rank 0).  The oracle (plain C on the host cores) is
 timed on a bounded sample as the CPU baseline; ``--impl reference`` times it
@@ -36,9 +40,21 @@ from x1_conv_bn_b200 import synth  # noqa: E402
 METRIC = "fused int8 conv TOPS and HBM GB/s (% of roofline) at Res3.2 Conv3, B=2048"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+# Dense int8 tensor throughput is twice dense bf16 on B200 (4.5 vs 2.25 POPS
+# nominal); the int8 peak is that ratio times the measured bf16 GEMM figure.
+INT8_PER_BF16 = 2.0
+L2_BYTES = 126 * 2 ** 20
 
 
-def parse():
+def metric_for(cfg):
+    """The headline metric string for config 3; the same metric on the named
+    workload for the others."""
+    if cfg == "3":
+        return METRIC
+    return "fused int8 conv TOPS and HBM GB/s (% of roofline) at " + synth.WORKLOAD_NAMES[cfg]
+
+
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -49,8 +65,13 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target length of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-1thread", action="store_true",
+                    help="also time the oracle sample on one host thread")
     ap.add_argument("--no-e2e", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--dry-run", action="store_true",
+                    help="CPU only: run the rank/timing logic over gloo with a host stand-in "
+                         "for the kernel (tests the multi-process path without a GPU)")
+    return ap.parse_args(argv)
 
 
 # ---- small helpers (also exercised by the CPU tests) ---------------------------------
@@ -61,6 +82,50 @@ def peaks():
         d = json.load(open(path))
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def roofline(ops, nbytes, seconds, hbm_gbs, bf16_tflops, kind):
+    """Roofline of one launch: the bound is the larger of bytes / HBM bandwidth
+    and ops / int8 dense peak; `frac` = achieved / peak in the bound's unit
+    (= roofline time / measured time)."""
+    int8_tops = INT8_PER_BF16 * bf16_tflops
+    t_hbm = nbytes / (hbm_gbs * 1e9)
+    t_tc = ops / (int8_tops * 1e12)
+    gbs = nbytes / seconds / 1e9
+    tops = ops / seconds / 1e12
+    if t_hbm >= t_tc:
+        r = {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s",
+             "frac": gbs / hbm_gbs, "peak_source": f"{kind} copy bandwidth (hbm_gbs)"}
+    else:
+        r = {"bound": "tensor", "achieved": tops, "peak": int8_tops, "unit": "TOPS",
+             "frac": tops / int8_tops,
+             "peak_source": f"{INT8_PER_BF16:g} x {kind} dense bf16 GEMM (int8:bf16 = 2:1)"}
+    r["roofline_time_us"] = max(t_hbm, t_tc) * 1e6
+    r["hbm_time_us"] = t_hbm * 1e6
+    r["int8_time_us"] = t_tc * 1e6
+    r["int8_tensor"] = {"achieved_tops": tops, "peak_tops": int8_tops, "frac": tops / int8_tops,
+                        "peak_source": f"{INT8_PER_BF16:g} x {kind} dense bf16 GEMM burst "
+                                       f"({bf16_tflops:g} TFLOP/s), nominal int8:bf16 = 2:1"}
+    r["hbm"] = {"achieved_gbs": gbs, "peak_gbs": hbm_gbs, "frac": gbs / hbm_gbs}
+    return r
+
+
+def rotation_sets(bytes_per_step, l2_bytes=L2_BYTES, cap=512):
+    """Input/output sets to cycle through so that no launch finds its operands
+    in L2: enough sets to span three times the L2 (1 when one step alone does)."""
+    if bytes_per_step >= 3 * l2_bytes:
+        return 1
+    return int(min(cap, -(-3 * l2_bytes // max(1, bytes_per_step))))
+
+
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def aggregate(per_rank_ms, units_per_rank):
@@ -172,7 +237,11 @@ def kernel_source_sha():
 
 # ---- inputs on the device -----------------------------------------------------------
 
-def device_inputs(cfg, dev, seed):
+def device_inputs(cfg, dev, seed, n_sets=1):
+    """Packed operands of one step on the device, plus (n_sets - 1) more copies
+    of the streamed tensors (activations, shortcut, output) so that the timed
+    loop can rotate over sets larger than the L2.  Returns (call, ins, out):
+    call(i) launches the op on set i; ins/out are set 0's tensors."""
     import x1_conv_bn_b200 as X
 
     s = synth.CONFIGS[cfg]
@@ -182,28 +251,33 @@ def device_inputs(cfg, dev, seed):
         ws = [X.x1cb_pack_weight(w) for w in inp.w]
         ws_bytes = X.bottleneck_i8_workspace_size(s.B, s.H, s.W, s.Cmid)
         work = torch.empty(ws_bytes, dtype=torch.int8, device=dev)
-        out = torch.empty_like(x)
+        xs = [x] + [x.clone() for _ in range(n_sets - 1)]
+        outs = [torch.empty_like(x) for _ in range(n_sets)]
         del inp.x
 
-        def call(x_=None, out_=None, stream=None):
-            X.bottleneck_i8(x if x_ is None else x_, ws[0], inp.bias[0], inp.m[0], ws[1],
+        def call(i=0, x_=None, out_=None, stream=None):
+            X.bottleneck_i8(xs[i] if x_ is None else x_, ws[0], inp.bias[0], inp.m[0], ws[1],
                             inp.bias[1], inp.m[1], ws[2], inp.bias[2], inp.m[2], inp.m_r, inp.S,
-                            out=out if out_ is None else out_, workspace=work, stream=stream)
+                            out=outs[i] if out_ is None else out_, workspace=work,
+                            stream=stream)
 
-        return call, {"x": x}, out
+        return call, {"x": x}, outs[0]
     inp = synth.conv_inputs(s, seed, device=dev)
     x = X.x1cb_pack_act(inp.x)
     w = X.x1cb_pack_weight(inp.w)
     r = X.x1cb_pack_act(inp.r)
     del inp.x, inp.r
-    out = torch.empty((s.B, s.Oc // 32, s.H, s.W, 32), dtype=torch.int8, device=dev)
+    xs = [x] + [x.clone() for _ in range(n_sets - 1)]
+    rs = [r] + [r.clone() for _ in range(n_sets - 1)]
+    outs = [torch.empty((s.B, s.Oc // 32, s.H, s.W, 32), dtype=torch.int8, device=dev)
+            for _ in range(n_sets)]
 
-    def call(x_=None, r_=None, out_=None, stream=None):
-        X.conv1x1_bn_add_relu_i8(x if x_ is None else x_, w, inp.bias, inp.m, inp.m_r, inp.S,
-                                 r if r_ is None else r_, out=out if out_ is None else out_,
-                                 stream=stream)
+    def call(i=0, x_=None, r_=None, out_=None, stream=None):
+        X.conv1x1_bn_add_relu_i8(xs[i] if x_ is None else x_, w, inp.bias, inp.m, inp.m_r,
+                                 inp.S, rs[i] if r_ is None else r_,
+                                 out=outs[i] if out_ is None else out_, stream=stream)
 
-    return call, {"x": x, "r": r}, out
+    return call, {"x": x, "r": r}, outs[0]
 
 
 # ---- CPU oracle (baseline / reference arm) ---------------------------------------------
@@ -266,23 +340,140 @@ class OracleSample:
 
 # ---- main ------------------------------------------------------------------------------
 
-def main():
-    a = parse()
+def free_port():
+    import socket
+
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    return port
+
+
+def spawn_ranks(n, argv):
+    """`--gpus N` (N > 1) started without a launcher: run N ranks, one process
+    per GPU, through torch.distributed.run on this node and return its exit
+    status.  Rank 0 prints the JSON line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+def clocks_verdict(summary):
+    """A run is rejected when a slowdown other than the power cap was active,
+    or when the SM clock sat well below its maximum with no reason given (a
+    leftover clock lock)."""
+    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+    reasons = set(summary.get("reasons") or [])
+    sm, mx = summary.get("sm_mhz"), summary.get("sm_max_mhz")
+    stuck = sm is not None and mx and sm < 0.8 * mx and not reasons
+    return bool(reasons & bad) or bool(stuck)
+
+
+def dry_run(a, rank, world):
+    """The rank/timing logic of a GPU run, on the CPU over gloo: each rank
+    times a host stand-in for its kernel, the slowest rank's time is taken,
+    rank 0 prints the line (marked dry_run; not a measurement)."""
+    import torch.distributed as dist
+
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    dd = dist if world > 1 else None
+    a_ = torch.randn(256, 256)
+    for _ in range(max(3, a.warmup)):
+        a_ @ a_
+    if dd is not None:
+        dd.barrier()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        a_ @ a_
+    ms = (time.perf_counter() - t0) * 1e3 / max(1, a.steps)
+    ms_max = max_over_ranks(ms, dd, "cpu")
+    ops = 2 * 256 ** 3
+    value, _ = aggregate([ms_max] * world, ops)
+    if dd is not None:
+        dd.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"metric": "dry run (host stand-in, not a measurement)",
+                          "value": value / 1e12, "unit": "TOPS", "n_gpus": world,
+                          "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max,
+                          "dry_run": True, "scaling": "weak"}), flush=True)
+
+
+def block_stage_calls(cfg, dev, seed):
+    """For the block workload: the three stages as separate calls on the same
+    buffers (conv1 x -> y1, conv2 y1 -> y2, conv3 y2 (+x) -> out), for
+    per-stage timing."""
+    import x1_conv_bn_b200 as X
+
+    s = synth.CONFIGS[cfg]
+    inp = synth.block_inputs(s, seed, device=dev)
+    x = X.x1cb_pack_act(inp.x)
+    ws = [X.x1cb_pack_weight(w) for w in inp.w]
+    y1 = torch.empty((s.B, s.Cmid // 32, s.H, s.W, 32), dtype=torch.int8, device=dev)
+    y2 = torch.empty_like(y1)
+    out = torch.empty_like(x)
+    st = s.stages()
+    return [
+        (st[0], lambda stream: X.conv1x1_bn_add_relu_i8(x, ws[0], inp.bias[0], inp.m[0], 0,
+                                                        inp.S, None, out=y1, stream=stream)),
+        (st[1], lambda stream: X.conv3x3_bn_relu_i8(y1, ws[1], inp.bias[1], inp.m[1], inp.S,
+                                                    out=y2, stream=stream)),
+        (st[2], lambda stream: X.conv1x1_bn_add_relu_i8(y2, ws[2], inp.bias[2], inp.m[2],
+                                                        inp.m_r, inp.S, x, out=out,
+                                                        stream=stream)),
+    ]
+
+
+def time_launches(fn, stream, n, warm=5):
+    for _ in range(warm):
+        fn(stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        fn(stream)
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
+    a = parse(argv)
+    launched = "WORLD_SIZE" in os.environ
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.gpus > 1 and not launched:
+        return spawn_ranks(a.gpus, argv)
+    if launched and world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
+    if a.dry_run:
+        return dry_run(a, rank, world)
     cfg = a.config
     s = synth.CONFIGS[cfg]
+    metric = metric_for(cfg)
     ops, nbytes = workload_units(cfg)
+    n_sets = rotation_sets(nbytes)
+    l2 = ("inputs larger than L2 (no flush): %.2f GB per step vs 126 MB" % (nbytes / 1e9)
+          if n_sets == 1 else
+          "rotating over %d input/output sets (%.0f MB in all, %.1f MB per step) so that no "
+          "launch finds its operands in the 126 MB L2" % (n_sets, n_sets * nbytes / 2 ** 20,
+                                                          nbytes / 2 ** 20))
     cfg_json = {"workload": synth.WORKLOAD_NAMES[cfg],
                 "shape": {k: getattr(s, k) for k in s.__dataclass_fields__},
                 "layout": "NC/32HW32 activations, blocked [O1,I1,O2,I2] weights",
-                "l2": "inputs larger than L2 (no flush): %.2f GB per step vs 126 MB" % (nbytes / 1e9),
-                "parallelism": f"replicas x{a.gpus} (independent batches)"}
+                "l2": l2,
+                "parallelism": (f"replicas x{world} (independent batches, one process per GPU)"
+                                if world > 1 else "1 GPU")}
 
     if a.impl == "reference":
         if rank != 0:
-            return
+            return 0
         per_step = min(5.0, max(0.05, 90.0 / max(1, a.steps + a.warmup)))
         smp = OracleSample(cfg, per_step)
         vals = []
@@ -292,16 +483,17 @@ def main():
                 vals.append((v, dt))
         v = smp.ops() * len(vals) / sum(dt for _, dt in vals) / 1e12
         ms = 1e3 * sum(dt for _, dt in vals) / len(vals)
-        line = {"metric": METRIC, "value": v, "unit": "TOPS", "impl": "reference",
+        line = {"metric": metric, "value": v, "unit": "TOPS", "impl": "reference",
                 "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "int64", "data": "synthetic", "config": cfg_json,
                 "cpu_baseline": {"value": v, "unit": "TOPS", "cores": smp.cores,
-                                 "kind": "oracle", "sample": smp.describe() + ", per step"},
+                                 "cpu_model": cpu_model(), "kind": "oracle",
+                                 "sample": smp.describe() + ", per step"},
                 "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
-        return
+        return 0
 
     import x1_conv_bn_b200 as X
     from x1_conv_bn_b200 import _build
@@ -321,16 +513,17 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    call, ins, out = device_inputs(cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank))
+    call, ins, out = device_inputs(cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank), n_sets)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        for _ in range(max(3, a.warmup)):
-            call(stream=stream)
+        for k in range(max(3, a.warmup)):
+            call(k % n_sets, stream=stream)
     torch.cuda.synchronize()
     st, bits = X.x1cb_last_device_error(clear=True)
     if st != 0:
         raise RuntimeError(f"device status {bits:#x} during warm-up")
+    forms = X.x1cb_last_epilogue_forms(clear=True)
 
     # ---- timed region (device time, CUDA events on the launching stream) ----
     e0 = torch.cuda.Event(enable_timing=True)
@@ -340,8 +533,8 @@ def main():
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             e0.record(stream)
-            for _ in range(a.steps):
-                call(stream=stream)
+            for k in range(a.steps):
+                call(k % n_sets, stream=stream)
             e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
@@ -353,6 +546,22 @@ def main():
     ms_max = max_over_ranks(ms_step, dist, dev)
     value_ops, _ = aggregate([ms_max] * world, ops)
     tops = value_ops / 1e12
+
+    # ---- per-stage times of the block (its dominant kernel gets the roofline) ----
+    stages = None
+    if isinstance(s, synth.BlockShape):
+        stages = []
+        with torch.cuda.stream(stream):
+            for shp, fn in block_stage_calls(cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank)):
+                t = time_launches(fn, stream, max(20, min(200, a.steps)))
+                stages.append({"stage": f"{shp.R}x{shp.R} {shp.Ic}->{shp.Oc}"
+                                        + (" +res" if shp.has_res else ""),
+                               "us": t * 1e3, "ops": shp.ops(), "bytes": shp.bytes_moved()})
+        torch.cuda.synchronize()
+        if X.x1cb_last_device_error(clear=True)[0] != 0:
+            raise RuntimeError("device status set in the per-stage timing")
+        for stg in stages:
+            stg["us"] = max_over_ranks(stg["us"], dist, dev)
 
     # ---- end to end through the API with host buffers ----
     # Every step uploads its inputs from pinned host memory, runs the fused op
@@ -389,9 +598,9 @@ def main():
                 if done_out[b] is not None:
                     stream.wait_event(done_out[b])
                 if "r" in dev_in[b]:
-                    call(x_=dev_in[b]["x"], r_=dev_in[b]["r"], out_=dev_out[b], stream=stream)
+                    call(0, x_=dev_in[b]["x"], r_=dev_in[b]["r"], out_=dev_out[b], stream=stream)
                 else:
-                    call(x_=dev_in[b]["x"], out_=dev_out[b], stream=stream)
+                    call(0, x_=dev_in[b]["x"], out_=dev_out[b], stream=stream)
                 ev_k = torch.cuda.Event()
                 ev_k.record(stream)
                 done_in[b] = ev_k
@@ -423,29 +632,58 @@ def main():
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
-        return
+        return 0
 
-    hbm, _, peak_kind = peaks()
+    hbm, bf16, peak_kind = peaks()
     launches = launches_per_step(cfg)
     gbs = nbytes / (ms_max * 1e-3) / 1e9
-    roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-            "frac": gbs / hbm, "peak_source": peak_kind + " (hbm_gbs)",
-            "traffic": read_traffic(f"conv1x1_res32_b{s.B}.md" if launches == 1 else
-                                    f"bottleneck_b{s.B}.md", kernel_source_sha()),
-            "algorithmic_bytes_per_launch": nbytes if launches == 1 else None,
-            "kernel": "conv_bn_act_kernel<true>" if launches == 1 else "3 launches"}
-    line = {"metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world, "steps": a.steps,
+    if stages is None:
+        roof = roofline(ops, nbytes, ms_max * 1e-3, hbm, bf16, peak_kind)
+        roof["kernel"] = "conv_bn_act_kernel<1> (1x1 with shortcut)"
+        roof["algorithmic_bytes_per_launch"] = nbytes
+        roof["algorithmic_ops_per_launch"] = ops
+        prof = f"conv1x1_res32_b{s.B}.md" if cfg in ("2", "3") else f"conv1x1_{cfg}.md"
+    else:
+        for stg in stages:
+            stg["roofline"] = roofline(stg["ops"], stg["bytes"], stg["us"] * 1e-6, hbm, bf16,
+                                       peak_kind)
+        top = max(stages, key=lambda t: t["us"])
+        roof = dict(top["roofline"])
+        roof["kernel"] = "stage " + top["stage"] + " (the block's slowest launch)"
+        roof["algorithmic_bytes_per_launch"] = top["bytes"]
+        roof["algorithmic_ops_per_launch"] = top["ops"]
+        prof = f"bottleneck_b{s.B}.md"
+    roof["traffic"] = read_traffic(prof, kernel_source_sha())
+    roof["traffic_source"] = (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
+                              f"profiles/{prof}, taken on this kernel source"
+                              if roof["traffic"] is not None else
+                              "no ncu capture of this kernel source")
+    clocks = clk.summary()
+    clocks["rejected"] = clocks_verdict(clocks)
+    line = {"metric": metric, "value": tops, "unit": "TOPS", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": cfg_json, "hbm_gbs": gbs, "roofline": roof,
-            "gpu_launches": a.steps * launches, "clocks": clk.summary(), "e2e": e2e}
+            "gpu_launches": a.steps * launches, "epilogue_forms": forms, "clocks": clocks,
+            "e2e": e2e}
+    if stages is not None:
+        line["stages"] = stages
     if world == 1 and not a.no_cpu_baseline:
         smp = OracleSample(cfg, a.cpu_seconds)
         v, dt = smp.time()
         line["cpu_baseline"] = {"value": v / 1e12, "unit": "TOPS", "cores": smp.cores,
-                                "kind": "oracle", "sample": smp.describe(), "seconds": dt}
+                                "cpu_model": cpu_model(), "kind": "oracle",
+                                "sample": smp.describe(), "seconds": dt}
+        if a.cpu_1thread:
+            from oracle import oracle as O
+
+            O.set_threads(1)
+            v1, dt1 = smp.time()
+            O.set_threads(smp.cores)
+            line["cpu_baseline"]["one_thread"] = {"value": v1 / 1e12, "seconds": dt1}
     print(json.dumps(line), flush=True)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

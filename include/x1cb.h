@@ -26,15 +26,19 @@
  * where acc is the exact int32 sum of x*w over the receptive field and the
  * r*m_r term is present only when a residual tensor is passed.
  *
- * Memory: every pointer is DEVICE memory owned by the caller, 16-byte
- * aligned.  Inputs and outputs must not overlap.  The library never
- * allocates device memory in any call.
+ * Memory: every pointer is DEVICE memory of the CURRENT device (cudaSetDevice),
+ * owned by the caller, 16-byte aligned (bias and multipliers: 4-byte).
+ * Inputs and outputs must not overlap.  Every call checks where its operands
+ * live (cudaPointerGetAttributes) and returns X1CB_ERR_DEVICE for host memory
+ * or another GPU's memory.  The library never allocates device memory in any
+ * call.  Calls are thread-safe: host-side caches are locked, and per-device
+ * state (the kernels' shared-memory opt-in) is set once per device.
  * Execution: every call only enqueues work on `stream` and returns after the
  * argument checks and the launch; results are ready when the stream is
  * synchronised.  A bounded-wait timeout inside a kernel (which never happens
  * in normal operation) is recorded in a sticky device status word, read with
  * x1cb_last_device_error().
- * Limits: stride 1; 1 <= S <= 60; Ic and Oc multiples of 32 and 128 with
+ * Limits: stride 1 (the stride-2 entry points below excepted); 1 <= S <= 60; Ic and Oc multiples of 32 and 128 with
  * Ic <= 4096; the weights of 128 output channels (R*R*Ic*128 bytes) must fit
  * in shared memory beside the rings (Ic <= 1120 for 1x1 with a residual,
  * Ic <= 1376 for 1x1 without, Ic <= 128 for 3x3); other shapes return
@@ -61,6 +65,7 @@ extern "C" {
 #define X1CB_ERR_TIMEOUT (-6)   /* a kernel gave up a bounded wait */
 #define X1CB_ERR_WORKSPACE (-7) /* workspace missing or too small */
 #define X1CB_ERR_OVERLAP (-8)   /* an output overlaps an input */
+#define X1CB_ERR_DEVICE (-9)    /* an operand is not memory of the current device */
 
 /*
  * Fused 1x1 Conv3 + folded BN + shortcut Sum + ReLU + int8 requantisation
@@ -91,6 +96,62 @@ int conv1x1_bn_add_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias
 int conv3x3_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
                        int32_t S, int8_t *out, int B, int H, int W, int Ic, int Oc, int pad,
                        void *stream);
+
+/*
+ * Fused 3x3 convolution of stride 2 (zero padding 1) + folded BN + ReLU +
+ * int8 requantisation: Conv2 of a downsampling (projection) block such as
+ * Res3.1.  The Inspur article (section 2.2) says only that Res3.1's output
+ * feeds Res3.2; the block's layers are read as in the MLPerf ResNet50 (v1.5)
+ * network, whose stride-2 step is this 3x3.
+ *   x   [B, Ic/32, H, W, 32]        input (read)
+ *   w   [Oc/128, 3, 3, Ic/32, 128, 32]
+ *   out [B, Oc/32, Ho, Wo, 32] with Ho = (H - 1)/2 + 1, Wo = (W - 1)/2 + 1;
+ *       output pixel (h, w) reads input rows 2h-1..2h+1, columns 2w-1..2w+1.
+ * Same requantisation as above without the r term.
+ */
+int conv3x3s2_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
+                         const int32_t *m, int32_t S, int8_t *out, int B, int H, int W, int Ic,
+                         int Oc, void *stream);
+
+/*
+ * Conv3 of a projection block with its shortcut fused in: the 1x1 Conv3 of
+ * y and the stride-2 1x1 projection of the block input x are accumulated into
+ * the same int32 accumulator (the projection's folded BN shares Conv3's
+ * multiplier, its relative scale folded into its int8 weights), then BN, ReLU
+ * and requantisation as above (no separate r term):
+ *   acc = sum_i y[b,h,w,i]*w3[o,i] + sum_j x[b,2h,2w,j]*wp[o,j]
+ *   y   [B, Cy/32, H, W, 32]; w3 [Oc/128, Cy/32, 128, 32]
+ *   x   [B, Cx/32, Hx, Wx, 32] with 2(H-1) < Hx and 2(W-1) < Wx
+ *   wp  [Oc/128, Cx/32, 128, 32]; bias, m [Oc]; out [B, Oc/32, H, W, 32]
+ * The shared-memory limit applies to the combined weights (Cy + Cx per output
+ * channel).
+ */
+int conv1x1_proj_bn_relu_i8(const int8_t *y, const int8_t *w3, const int8_t *x,
+                            const int8_t *wp, const int32_t *bias, const int32_t *m, int32_t S,
+                            int8_t *out, int B, int H, int W, int Cy, int Hx, int Wx, int Cx,
+                            int Oc, void *stream);
+
+/* Bytes of device workspace bottleneck_proj_i8 needs for an H x W input:
+ * [B, Cmid/32, H, W, 32] and [B, Cmid/32, Ho, Wo, 32]. */
+size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid);
+
+/*
+ * Projection bottleneck block (Res3.1 of ResNet50 in the MLPerf v1.5 form):
+ * conv1 1x1 Cin->Cmid +BN+ReLU on H x W; conv2 3x3 stride 2 Cmid->Cmid
+ * +BN+ReLU to Ho x Wo; conv3 1x1 Cmid->Cout plus the stride-2 1x1 projection
+ * Cin->Cout of the block input in one accumulator, +BN+ReLU.  Three launches
+ * on `stream`.
+ *   x  [B, Cin/32, H, W, 32]; out [B, Cout/32, Ho, Wo, 32]
+ *   w1 [Cmid/128, Cin/32, 128, 32]; w2 [Cmid/128, 3, 3, Cmid/32, 128, 32];
+ *   w3 [Cout/128, Cmid/32, 128, 32]; wp [Cout/128, Cin/32, 128, 32];
+ *   b1, m1, b2, m2 [Cmid]; b3, m3 [Cout] (shared by Conv3 and the projection)
+ *   workspace: caller-owned, >= bottleneck_proj_i8_workspace_size() bytes
+ */
+int bottleneck_proj_i8(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                       const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                       const int8_t *wp, const int32_t *b3, const int32_t *m3, int32_t S,
+                       int8_t *out, void *workspace, size_t ws_bytes, int B, int H, int W,
+                       int Cin, int Cmid, int Cout, void *stream);
 
 /* Bytes of device workspace bottleneck_i8 needs: two [B, Cmid/32, H, W, 32]
  * intermediates. */
@@ -160,6 +221,15 @@ const char *x1cb_status_string(int status);
  * when bits is not NULL.  clear != 0 resets the word. */
 int x1cb_last_device_error(unsigned int *bits, int clear);
 
+/* Synchronises the current device, then writes to *bits which exact
+ * epilogue forms the kernels launched since the last clear ran (bit 0: the
+ * generic 64-bit definition, 1: the 64-bit high-word form, 2: the all-32-bit
+ * form, 3: the all-32-bit form with the bias added by the tensor core).  Every
+ * form gives the same bytes; this only shows which arithmetic a shape and its
+ * constants reached.  clear != 0 resets the record.  Returns X1CB_OK or an
+ * error. */
+int x1cb_last_epilogue_forms(unsigned int *bits, int clear);
+
 /* Limit of every in-kernel wait, in nanoseconds (default 2 s; 0 restores the
  * default).  Applies to launches made after the call. */
 void x1cb_set_wait_limit_ns(unsigned long long ns);
@@ -174,7 +244,13 @@ void x1cb_debug_inject(int mode);
 int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, char *buf,
                        size_t len);
 
-/* Library version, e.g. "x1cb 0.1.0 sm_100a". */
+/* As x1cb_describe_plan for an Hin x Win input at `stride` (R = 3: pad 1),
+ * optionally with a projection source of Ic2 channels (1x1, stride 2, over a
+ * 2H x 2W image; R = 1 and stride = 1 then). */
+int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int stride, int Ic2,
+                          int has_res, char *buf, size_t len);
+
+/* Library version, e.g. "x1cb 0.2.0 sm_100a". */
 const char *x1cb_version(void);
 
 #ifdef __cplusplus

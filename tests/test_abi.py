@@ -37,7 +37,7 @@ def test_python_binding_has_same_names(L):
 
 def test_status_strings(L):
     assert X.x1cb_status_string(0) == "ok"
-    for code in range(-8, 0):
+    for code in range(-9, 0):
         assert X.x1cb_status_string(code) != "unknown status"
     assert "sm_100a" in X.x1cb_version()
 

@@ -66,3 +66,49 @@ def test_workload_numbers_match_the_plan():
     ops, nbytes = bench.workload_units("3")
     assert ops == 2 * 2048 * 784 * 512 * 128  # 210.45 G int-ops
     assert abs(nbytes / 1e9 - 1.8497) < 0.001  # x + r + out + weights (+ bias, m)
+
+
+def test_spawned_dry_run_over_two_ranks():
+    """`bench.py --gpus 2` started without a launcher spawns two ranks (one
+    process per GPU on a GPU machine); --dry-run takes the same rank path on the
+    CPU over gloo and rank 0 prints one line with n_gpus = 2."""
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                          "--dry-run", "--steps", "5", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=240, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["dry_run"] is True and d["steps"] == 5
+
+
+def test_roofline_takes_the_larger_bound():
+    ops, nbytes = bench.workload_units("3")
+    r = bench.roofline(ops, nbytes, 350e-6, 6533.5, 1673.6, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["frac"] == pytest.approx(nbytes / 350e-6 / 1e9 / 6533.5)
+    assert r["int8_tensor"]["peak_tops"] == pytest.approx(2 * 1673.6)
+    assert r["roofline_time_us"] == pytest.approx(nbytes / 6533.5e9 * 1e6)
+    # the block's 3x3 stage: 1151 ops per byte, above the ridge -> tensor-bound
+    conv2 = bench.synth.CONFIGS["5"].stages()[1]
+    r2 = bench.roofline(conv2.ops(), conv2.bytes_moved(), 125e-6, 6533.5, 1673.6, "measured")
+    assert r2["bound"] == "tensor" and r2["unit"] == "TOPS"
+    assert r2["frac"] == pytest.approx(conv2.ops() / 125e-6 / 1e12 / (2 * 1673.6))
+
+
+def test_rotation_and_metric_per_config():
+    assert bench.rotation_sets(2 * 10 ** 9) == 1
+    n1 = bench.rotation_sets(bench.workload_units("1")[1])
+    assert n1 * bench.workload_units("1")[1] >= 3 * bench.L2_BYTES
+    assert bench.metric_for("3") == bench.METRIC
+    assert "B=2048" not in bench.metric_for("1") and "B=1" in bench.metric_for("1")
+
+
+def test_clock_verdict():
+    assert not bench.clocks_verdict({"sm_mhz": 1800, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]})
+    assert bench.clocks_verdict({"sm_mhz": 1800, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]})
+    assert bench.clocks_verdict({"sm_mhz": 900, "sm_max_mhz": 1965, "reasons": []})

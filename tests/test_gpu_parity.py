@@ -176,6 +176,70 @@ def test_conv1x1_mixed_epilogue_forms_across_ctas(oracle):
     assert torch.equal(got, ref)
 
 
+# The all-32-bit forms fold the shortcut in as y2 = hi32((acc + bias) * m'') + 1
+# + r * k with k = m_r / 2^(S-1).  These cases drive k != 1 (negative, odd,
+# and the extremes the form admits), with the bias folded into the MMA and
+# added in the epilogue, and check that the intended form really ran.
+K_CASES = [(2, -1), (2, 3), (2, -(1 << 23) + 1), (2, 1 << 23),
+           (24, -1), (24, 3), (24, -256), (24, 255)]
+
+
+@pytest.mark.parametrize("S,k", K_CASES, ids=[f"S{S}_k{k}" for S, k in K_CASES])
+@pytest.mark.parametrize("fold", [True, False], ids=["fold", "nofold"])
+@pytest.mark.parametrize("mag", ["full", "small"])
+def test_all32_forms_with_shortcut_scale(oracle, S, k, fold, mag):
+    s = synth.ConvShape(3, 9, 13, 96, 256, 1, True)
+    g = torch.Generator().manual_seed(S * 7 + (k & 0xFFFF) + (1000 if fold else 0))
+    lo, hi = (-128, 127) if mag == "full" else (-3, 3)
+    x = torch.randint(lo, hi + 1, (s.B, s.H, s.W, s.Ic), generator=g, dtype=torch.int8)
+    w = torch.randint(-128, 128, (s.Oc, s.Ic, 1, 1), generator=g, dtype=torch.int8)
+    r = torch.randint(-128, 128, (s.B, s.H, s.W, s.Oc), generator=g, dtype=torch.int8)
+    if fold:
+        bias = torch.randint(-(1 << 12), (1 << 12) + 1, (s.Oc,), generator=g, dtype=torch.int32)
+    else:  # every channel beyond the foldable range
+        mag_b = torch.randint((1 << 18) + 1, 1 << 20, (s.Oc,), generator=g, dtype=torch.int32)
+        sign = torch.randint(0, 2, (s.Oc,), generator=g, dtype=torch.int32) * 2 - 1
+        bias = mag_b * sign
+    if S == 2:  # m * 2^31 must fit int32
+        m = torch.randint(-1, 1, (s.Oc,), generator=g, dtype=torch.int32)
+    else:
+        m = torch.randint(-(1 << 21), (1 << 21) + 1, (s.Oc,), generator=g, dtype=torch.int32)
+    m_r = k * (1 << (S - 1))
+    assert -(1 << 31) <= m_r < (1 << 31)
+    inp = synth.ConvInputs(s, x, w, bias, m, r, m_r, S)
+    ref = _oracle_conv(oracle, inp)
+    X.x1cb_last_epilogue_forms(clear=True)
+    got = _nhwc(_gpu_conv(inp))
+    forms = X.x1cb_last_epilogue_forms(clear=True)
+    assert forms == (1 << (3 if fold else 2)), forms
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
+    assert ref.unique().numel() >= 2
+
+
+@pytest.mark.parametrize("k,form", [(-(1 << 23), 0), (-(1 << 23) + 1, 2)])
+def test_all32_form_bound_on_the_shortcut_scale(oracle, k, form):
+    """At S = 9, m_r = k * 2^8.  With (acc + bias) near -2^31 and m'' = -2^31
+    the high word is near 2^30; r = -128 adds -128 * k.  For k = -2^23 that
+    sum is 2^31, outside int32, so the all-32-bit form must not be taken (the
+    generic form runs); k = -2^23 + 1 still fits and keeps the form.  Either
+    way every output is the exact 127."""
+    s = synth.ConvShape(1, 2, 4, 32, 128, 1, True)
+    x = torch.zeros(s.B, s.H, s.W, s.Ic, dtype=torch.int8)
+    x[..., 0] = 1
+    w = torch.zeros(s.Oc, s.Ic, 1, 1, dtype=torch.int8)
+    w[:, 0, 0, 0] = -128                     # acc = -128
+    bias = torch.full((s.Oc,), -(1 << 31) + (1 << 21), dtype=torch.int32)
+    m = torch.full((s.Oc,), -128, dtype=torch.int32)  # m * 2^(33-9) = -2^31
+    r = torch.full((s.B, s.H, s.W, s.Oc), -128, dtype=torch.int8)
+    inp = synth.ConvInputs(s, x, w, bias, m, r, k * 256, 9)
+    ref = _oracle_conv(oracle, inp)
+    assert (ref == 127).all()
+    X.x1cb_last_epilogue_forms(clear=True)
+    got = _nhwc(_gpu_conv(inp))
+    assert X.x1cb_last_epilogue_forms(clear=True) == 1 << form
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
+
+
 # ---- fused 3x3 ------------------------------------------------------------------
 
 # The halo form covers W+2 <= 128 (tiles of th rows x tg images, ragged in H
@@ -238,7 +302,7 @@ def test_bottleneck_parity(oracle, shape):
     _assert_spread(ref)
 
 
-# ---- full-size workloads, sampled --------------------------------------------------
+# ---- full-size workloads, every output byte -------------------------------------
 
 def _sample_pixels(B, H, W, n, seed):
     g = torch.Generator().manual_seed(seed)
@@ -255,14 +319,27 @@ def _gather_nc32(t_nc32_cpu, pix, H, W):
     return flat[pix]
 
 
+def _nhwc(t_nc32_cpu):
+    """[B, C/32, H, W, 32] -> [B, H, W, C] (a layout view, no arithmetic)."""
+    B, C1, H, W, _ = t_nc32_cpu.shape
+    return t_nc32_cpu.permute(0, 2, 3, 1, 4).reshape(B, H, W, C1 * 32)
+
+
+def _first_mismatch(got, ref):
+    bad = (got != ref).nonzero()
+    return f"{bad.shape[0]} bytes differ, first at {bad[0].tolist()}" if bad.numel() else ""
+
+
 @pytest.mark.parametrize("cfg", ["1", "2", "3", "4a", "4b", "4c"])
-def test_full_size_1x1_sampled(oracle, cfg):
+def test_full_size_1x1_every_output(oracle, cfg):
+    """The benchmark workloads at full size, compared byte for byte with the
+    whole oracle output (B=2048: 822 MB of results, 12544 tiles over the
+    persistent grid, including the last partial wave)."""
     s = synth.CONFIGS[cfg]
     inp = synth.conv_inputs(s, synth.CONFIG_SEEDS[cfg])
-    got = _gpu_conv(inp)
-    pix = _sample_pixels(s.B, s.H, s.W, 1500, 7)
-    ref = oracle.conv_pixels(inp.x, inp.w, inp.bias, inp.m, inp.S, pix, inp.r, inp.m_r)
-    assert torch.equal(_gather_nc32(got, pix, s.H, s.W), ref)
+    got = _nhwc(_gpu_conv(inp))
+    ref = _oracle_conv(oracle, inp)
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
     _assert_spread(ref)
 
 
@@ -305,19 +382,25 @@ def test_repeated_launches_stay_exact(oracle, shape):
     assert torch.equal(_gather_nc32(outs[0].cpu(), pix, s.H, s.W), ref)
 
 
-def test_full_size_block_sampled(oracle):
+def test_full_size_block_every_output(oracle):
+    """The Res3.2 bottleneck block at B=1024, every output byte against the
+    oracle's three composed layers."""
     s = synth.CONFIGS["5"]
     inp = synth.block_inputs(s, synth.CONFIG_SEEDS["5"])
     x = X.x1cb_pack_act(inp.x.to(DEV))
     ws = [X.x1cb_pack_weight(w.to(DEV)) for w in inp.w]
     bs = [b.to(DEV) for b in inp.bias]
     ms = [m.to(DEV) for m in inp.m]
+    X.x1cb_last_device_error(clear=True)
     out = X.bottleneck_i8(x, ws[0], bs[0], ms[0], ws[1], bs[1], ms[1], ws[2], bs[2], ms[2],
                           inp.m_r, inp.S)
     torch.cuda.synchronize()
-    pix = _sample_pixels(s.B, s.H, s.W, 400, 8)
-    ref = oracle.bottleneck_pixels(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S, pix)
-    assert torch.equal(_gather_nc32(out.cpu(), pix, s.H, s.W), ref)
+    st, bits = X.x1cb_last_device_error(clear=True)
+    assert st == 0, bits
+    got = _nhwc(out.cpu())
+    del out, x
+    ref = oracle.bottleneck(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S)
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
     _assert_spread(ref)
 
 
@@ -381,3 +464,72 @@ def test_empty_batch_is_noop():
     b = torch.zeros(512, dtype=torch.int32, device=DEV)
     out = X.conv1x1_bn_add_relu_i8(x, w, b, b, 0, 24, None)
     assert out.shape == (0, 16, 28, 28, 32)
+
+
+def test_two_threads_on_one_device_stay_exact(oracle):
+    """Two host threads call the library at once, each on its own stream, on
+    shapes whose plans differ (the plan cache and the per-device kernel set-up
+    are shared); both results stay bit-exact."""
+    import threading
+
+    cases = [synth.conv_inputs(synth.ConvShape(8, 28, 28, 128, 512, 1, True), 61),
+             synth.conv_inputs(synth.ConvShape(6, 14, 14, 256, 1024, 1, True), 62),
+             synth.conv_inputs(synth.ConvShape(5, 28, 28, 128, 128, 3, False), 63)]
+    refs = [_oracle_conv(oracle, c) for c in cases]
+    got = [[None] * 20 for _ in cases]
+    errors = []
+
+    def worker(i):
+        try:
+            torch.cuda.set_device(0)
+            c = cases[i]
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                x = X.x1cb_pack_act(c.x.to(DEV))
+                w = X.x1cb_pack_weight(c.w.to(DEV))
+                b, m = c.bias.to(DEV), c.m.to(DEV)
+                r = X.x1cb_pack_act(c.r.to(DEV)) if c.r is not None else None
+                for j in range(20):
+                    if c.shape.R == 1:
+                        got[i][j] = X.conv1x1_bn_add_relu_i8(x, w, b, m, c.m_r, c.S, r)
+                    else:
+                        got[i][j] = X.conv3x3_bn_relu_i8(x, w, b, m, c.S)
+            st.synchronize()
+        except Exception as e:  # reported on the main thread
+            errors.append(e)
+
+    ts = [threading.Thread(target=worker, args=(i,)) for i in range(len(cases))]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    assert X.x1cb_last_device_error(clear=True)[0] == 0
+    for i, ref in enumerate(refs):
+        for o in got[i]:
+            assert torch.equal(_nhwc(o.cpu()), ref)
+
+
+def test_operands_must_be_memory_of_the_current_device():
+    """Host memory handed to the C ABI is refused before anything launches."""
+    import ctypes
+
+    s = synth.ConvShape(1, 4, 4, 32, 128, 1, False)
+    inp = synth.conv_inputs(s, 5)
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    w = X.x1cb_pack_weight(inp.w.to(DEV))
+    b, m = inp.bias.to(DEV), inp.m.to(DEV)
+    out = torch.empty((1, 4, 4, 4, 32), dtype=torch.int8, device=DEV)
+    host = torch.empty_like(out, device="cpu").pin_memory()
+    v = ctypes.c_void_p
+    L = X.lib()
+    args = lambda xp, op: (v(xp), v(w.data_ptr()), v(b.data_ptr()), v(m.data_ptr()), 0, 24,
+                           None, v(op), 1, 4, 4, 32, 128, None)
+    assert L.conv1x1_bn_add_relu_i8(*args(x.data_ptr(), host.data_ptr())) == X.X1CB_ERR_DEVICE
+    hx = x.cpu().pin_memory()
+    assert L.conv1x1_bn_add_relu_i8(*args(hx.data_ptr(), out.data_ptr())) == X.X1CB_ERR_DEVICE
+    assert L.conv1x1_bn_add_relu_i8(*args(x.data_ptr(), out.data_ptr())) == X.X1CB_OK
+    torch.cuda.synchronize()
+    with pytest.raises(ValueError):
+        X.conv1x1_bn_add_relu_i8(x, w.cpu(), b, m, 0, 24)

@@ -27,6 +27,7 @@ X1CB_ERR_CUDA = -5
 X1CB_ERR_TIMEOUT = -6
 X1CB_ERR_WORKSPACE = -7
 X1CB_ERR_OVERLAP = -8
+X1CB_ERR_DEVICE = -9
 
 
 class X1cbError(RuntimeError):
@@ -58,12 +59,19 @@ def lib() -> ctypes.CDLL:
         L.x1cb_status_string.argtypes = [i]
         L.x1cb_status_string.restype = ctypes.c_char_p
         L.x1cb_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+        L.x1cb_last_epilogue_forms.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
         L.x1cb_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.x1cb_set_wait_limit_ns.restype = None
         L.x1cb_debug_inject.argtypes = [i]
         L.x1cb_debug_inject.restype = None
         L.x1cb_describe_plan.argtypes = [i, i, i, i, i, i, i, ctypes.c_char_p, sz]
         L.x1cb_version.restype = ctypes.c_char_p
+        L.conv3x3s2_bn_relu_i8.argtypes = [vp] * 4 + [i32, vp] + [i] * 5 + [vp]
+        L.conv1x1_proj_bn_relu_i8.argtypes = [vp] * 6 + [i32, vp] + [i] * 9 + [vp]
+        L.bottleneck_proj_i8_workspace_size.argtypes = [i, i, i, i]
+        L.bottleneck_proj_i8_workspace_size.restype = sz
+        L.bottleneck_proj_i8.argtypes = [vp] * 11 + [i32, vp, vp, sz] + [i] * 6 + [vp]
+        L.x1cb_describe_plan_ex.argtypes = [i] * 9 + [ctypes.c_char_p, sz]
         _lib = L
     return _lib
 
@@ -92,10 +100,23 @@ def _dev(t: Optional[torch.Tensor], dtype, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device) -> ctypes.c_void_p:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif isinstance(stream, torch.cuda.Stream) and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, operands on {device}")
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _same_device(first: torch.Tensor, *others):
+    """Every operand must live on the first one's GPU; the call then runs with
+    that GPU current (the library launches on the current device)."""
+    if not isinstance(first, torch.Tensor) or first.device.type != "cuda":
+        raise ValueError("operands must be CUDA tensors")
+    for t in others:
+        if t is not None and isinstance(t, torch.Tensor) and t.device != first.device:
+            raise ValueError(f"operand on {t.device}, expected {first.device}")
+    return torch.cuda.device(first.device)
 
 
 def _act_shape(x: torch.Tensor, name: str):
@@ -114,10 +135,11 @@ def conv1x1_bn_add_relu_i8(x, w, bias, m, m_r: int, S: int, r=None, out=None, st
     Oc = bias.numel()
     if out is None:
         out = torch.empty((B, Oc // 32, H, W, 32), dtype=torch.int8, device=x.device)
-    st = lib().conv1x1_bn_add_relu_i8(
-        _dev(x, torch.int8, "x"), _dev(w, torch.int8, "w"), _dev(bias, torch.int32, "bias"),
-        _dev(m, torch.int32, "m"), int(m_r), int(S), _dev(r, torch.int8, "r"),
-        _dev(out, torch.int8, "out"), B, H, W, Ic, Oc, _stream(stream))
+    with _same_device(x, w, bias, m, r, out):
+        st = lib().conv1x1_bn_add_relu_i8(
+            _dev(x, torch.int8, "x"), _dev(w, torch.int8, "w"), _dev(bias, torch.int32, "bias"),
+            _dev(m, torch.int32, "m"), int(m_r), int(S), _dev(r, torch.int8, "r"),
+            _dev(out, torch.int8, "out"), B, H, W, Ic, Oc, _stream(stream, x.device))
     _check(st, "conv1x1_bn_add_relu_i8")
     return out
 
@@ -130,10 +152,11 @@ def conv3x3_bn_relu_i8(x, w, bias, m, S: int, out=None, pad: int = 1, stream=Non
     Oc = bias.numel()
     if out is None:
         out = torch.empty((B, Oc // 32, H, W, 32), dtype=torch.int8, device=x.device)
-    st = lib().conv3x3_bn_relu_i8(
-        _dev(x, torch.int8, "x"), _dev(w, torch.int8, "w"), _dev(bias, torch.int32, "bias"),
-        _dev(m, torch.int32, "m"), int(S), _dev(out, torch.int8, "out"), B, H, W, Ic, Oc,
-        int(pad), _stream(stream))
+    with _same_device(x, w, bias, m, out):
+        st = lib().conv3x3_bn_relu_i8(
+            _dev(x, torch.int8, "x"), _dev(w, torch.int8, "w"), _dev(bias, torch.int32, "bias"),
+            _dev(m, torch.int32, "m"), int(S), _dev(out, torch.int8, "out"), B, H, W, Ic, Oc,
+            int(pad), _stream(stream, x.device))
     _check(st, "conv3x3_bn_relu_i8")
     return out
 
@@ -152,13 +175,14 @@ def bottleneck_i8(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r: int, S: int, out=N
     need = bottleneck_i8_workspace_size(B, H, W, Cmid)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.int8, device=x.device)
-    st = lib().bottleneck_i8(
-        _dev(x, torch.int8, "x"), _dev(w1, torch.int8, "w1"), _dev(b1, torch.int32, "b1"),
-        _dev(m1, torch.int32, "m1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
-        _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(b3, torch.int32, "b3"),
-        _dev(m3, torch.int32, "m3"), int(m_r), int(S), _dev(out, torch.int8, "out"),
-        _dev(workspace, torch.int8, "workspace"), workspace.numel(), B, H, W, Cin, Cmid,
-        _stream(stream))
+    with _same_device(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, out, workspace):
+        st = lib().bottleneck_i8(
+            _dev(x, torch.int8, "x"), _dev(w1, torch.int8, "w1"), _dev(b1, torch.int32, "b1"),
+            _dev(m1, torch.int32, "m1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
+            _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(b3, torch.int32, "b3"),
+            _dev(m3, torch.int32, "m3"), int(m_r), int(S), _dev(out, torch.int8, "out"),
+            _dev(workspace, torch.int8, "workspace"), workspace.numel(), B, H, W, Cin, Cmid,
+            _stream(stream, x.device))
     _check(st, "bottleneck_i8")
     return out
 
@@ -173,13 +197,85 @@ def bottleneck_i8_noalloc(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r: int, S: in
     Cmid = b1.numel()
     if out is None:
         out = torch.empty_like(x)
-    st = lib().bottleneck_i8_noalloc(
-        _dev(x, torch.int8, "x"), _dev(w1, torch.int8, "w1"), _dev(b1, torch.int32, "b1"),
-        _dev(m1, torch.int32, "m1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
-        _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(b3, torch.int32, "b3"),
-        _dev(m3, torch.int32, "m3"), int(m_r), int(S), _dev(out, torch.int8, "out"),
-        B, H, W, Cin, Cmid, _stream(stream))
+    with _same_device(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, out):
+        st = lib().bottleneck_i8_noalloc(
+            _dev(x, torch.int8, "x"), _dev(w1, torch.int8, "w1"), _dev(b1, torch.int32, "b1"),
+            _dev(m1, torch.int32, "m1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
+            _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(b3, torch.int32, "b3"),
+            _dev(m3, torch.int32, "m3"), int(m_r), int(S), _dev(out, torch.int8, "out"),
+            B, H, W, Cin, Cmid, _stream(stream, x.device))
     _check(st, "bottleneck_i8_noalloc")
+    return out
+
+
+def _half(n: int) -> int:
+    """Output extent of a stride-2 3x3 (pad 1) over n pixels."""
+    return (n - 1) // 2 + 1 if n > 0 else 0
+
+
+def conv3x3s2_bn_relu_i8(x, w, bias, m, S: int, out=None, stream=None):
+    """Fused 3x3 stride-2 conv (pad 1) + BN + ReLU + int8 (a projection
+    block's Conv2).  x [B, Ic/32, H, W, 32] -> out [B, Oc/32, Ho, Wo, 32]."""
+    B, Ic, H, W = _act_shape(x, "x")
+    Oc = bias.numel()
+    if out is None:
+        out = torch.empty((B, Oc // 32, _half(H), _half(W), 32), dtype=torch.int8,
+                          device=x.device)
+    with _same_device(x, w, bias, m, out):
+        st = lib().conv3x3s2_bn_relu_i8(
+            _dev(x, torch.int8, "x"), _dev(w, torch.int8, "w"), _dev(bias, torch.int32, "bias"),
+            _dev(m, torch.int32, "m"), int(S), _dev(out, torch.int8, "out"), B, H, W, Ic, Oc,
+            _stream(stream, x.device))
+    _check(st, "conv3x3s2_bn_relu_i8")
+    return out
+
+
+def conv1x1_proj_bn_relu_i8(y, w3, x, wp, bias, m, S: int, out=None, stream=None):
+    """Projection block's Conv3: 1x1 of y plus the stride-2 1x1 of the block
+    input x in one accumulator, + BN + ReLU + int8.
+    y [B, Cy/32, H, W, 32]; x [B, Cx/32, Hx, Wx, 32]; out [B, Oc/32, H, W, 32]."""
+    B, Cy, H, W = _act_shape(y, "y")
+    B2, Cx, Hx, Wx = _act_shape(x, "x")
+    if B2 != B:
+        raise ValueError("y and x must have the same batch")
+    Oc = bias.numel()
+    if out is None:
+        out = torch.empty((B, Oc // 32, H, W, 32), dtype=torch.int8, device=y.device)
+    with _same_device(y, w3, x, wp, bias, m, out):
+        st = lib().conv1x1_proj_bn_relu_i8(
+            _dev(y, torch.int8, "y"), _dev(w3, torch.int8, "w3"), _dev(x, torch.int8, "x"),
+            _dev(wp, torch.int8, "wp"), _dev(bias, torch.int32, "bias"),
+            _dev(m, torch.int32, "m"), int(S), _dev(out, torch.int8, "out"),
+            B, H, W, Cy, Hx, Wx, Cx, Oc, _stream(stream, y.device))
+    _check(st, "conv1x1_proj_bn_relu_i8")
+    return out
+
+
+def bottleneck_proj_i8_workspace_size(B: int, H: int, W: int, Cmid: int) -> int:
+    return int(lib().bottleneck_proj_i8_workspace_size(B, H, W, Cmid))
+
+
+def bottleneck_proj_i8(x, w1, b1, m1, w2, b2, m2, w3, wp, b3, m3, S: int, out=None,
+                       workspace=None, stream=None):
+    """Projection bottleneck (Res3.1): 1x1, 3x3 stride 2, 1x1 + stride-2 1x1
+    projection of x in one accumulator; BN + ReLU after each."""
+    B, Cin, H, W = _act_shape(x, "x")
+    Cmid, Cout = b1.numel(), b3.numel()
+    if out is None:
+        out = torch.empty((B, Cout // 32, _half(H), _half(W), 32), dtype=torch.int8,
+                          device=x.device)
+    need = bottleneck_proj_i8_workspace_size(B, H, W, Cmid)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.int8, device=x.device)
+    with _same_device(x, w1, b1, m1, w2, b2, m2, w3, wp, b3, m3, out, workspace):
+        st = lib().bottleneck_proj_i8(
+            _dev(x, torch.int8, "x"), _dev(w1, torch.int8, "w1"), _dev(b1, torch.int32, "b1"),
+            _dev(m1, torch.int32, "m1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
+            _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(wp, torch.int8, "wp"),
+            _dev(b3, torch.int32, "b3"), _dev(m3, torch.int32, "m3"), int(S),
+            _dev(out, torch.int8, "out"), _dev(workspace, torch.int8, "workspace"),
+            workspace.numel(), B, H, W, Cin, Cmid, Cout, _stream(stream, x.device))
+    _check(st, "bottleneck_proj_i8")
     return out
 
 
@@ -188,8 +284,10 @@ def x1cb_pack_act(nhwc, out=None, stream=None):
     B, H, W, C = nhwc.shape
     if out is None:
         out = torch.empty((B, C // 32, H, W, 32), dtype=torch.int8, device=nhwc.device)
-    _check(lib().x1cb_pack_act(_dev(nhwc, torch.int8, "nhwc"), _dev(out, torch.int8, "out"),
-                               B, H, W, C, _stream(stream)), "x1cb_pack_act")
+    with _same_device(nhwc, out):
+        st = lib().x1cb_pack_act(_dev(nhwc, torch.int8, "nhwc"), _dev(out, torch.int8, "out"),
+                                 B, H, W, C, _stream(stream, nhwc.device))
+    _check(st, "x1cb_pack_act")
     return out
 
 
@@ -197,8 +295,10 @@ def x1cb_unpack_act(nc32, out=None, stream=None):
     B, C, H, W = _act_shape(nc32, "nc32")
     if out is None:
         out = torch.empty((B, H, W, C), dtype=torch.int8, device=nc32.device)
-    _check(lib().x1cb_unpack_act(_dev(nc32, torch.int8, "nc32"), _dev(out, torch.int8, "out"),
-                                 B, H, W, C, _stream(stream)), "x1cb_unpack_act")
+    with _same_device(nc32, out):
+        st = lib().x1cb_unpack_act(_dev(nc32, torch.int8, "nc32"), _dev(out, torch.int8, "out"),
+                                   B, H, W, C, _stream(stream, nc32.device))
+    _check(st, "x1cb_unpack_act")
     return out
 
 
@@ -208,8 +308,11 @@ def x1cb_pack_weight(oihw, out=None, stream=None):
     if out is None:
         out = torch.empty((Oc // 128, R, R, Ic // 32, 128, 32), dtype=torch.int8,
                           device=oihw.device)
-    _check(lib().x1cb_pack_weight(_dev(oihw, torch.int8, "oihw"), _dev(out, torch.int8, "out"),
-                                  Oc, Ic, R, _stream(stream)), "x1cb_pack_weight")
+    with _same_device(oihw, out):
+        st = lib().x1cb_pack_weight(_dev(oihw, torch.int8, "oihw"),
+                                    _dev(out, torch.int8, "out"), Oc, Ic, R,
+                                    _stream(stream, oihw.device))
+    _check(st, "x1cb_pack_weight")
     return out
 
 
@@ -224,6 +327,16 @@ def x1cb_last_device_error(clear: bool = True):
     return st, bits.value
 
 
+def x1cb_last_epilogue_forms(clear: bool = True) -> int:
+    """Bit set of the exact epilogue forms run since the last clear (bit 0
+    generic, 1 64-bit high word, 2 all-32-bit, 3 all-32-bit with the bias in
+    the MMA); synchronises."""
+    bits = ctypes.c_uint(0)
+    _check(lib().x1cb_last_epilogue_forms(ctypes.byref(bits), int(clear)),
+           "x1cb_last_epilogue_forms")
+    return bits.value
+
+
 def x1cb_set_wait_limit_ns(ns: int):
     lib().x1cb_set_wait_limit_ns(int(ns))
 
@@ -236,6 +349,13 @@ def x1cb_describe_plan(B, H, W, Ic, Oc, R=1, has_res=True) -> str:
     buf = ctypes.create_string_buffer(512)
     _check(lib().x1cb_describe_plan(B, H, W, Ic, Oc, R, int(has_res), buf, 512),
            "x1cb_describe_plan")
+    return buf.value.decode()
+
+
+def x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R=1, stride=1, Ic2=0, has_res=False) -> str:
+    buf = ctypes.create_string_buffer(512)
+    _check(lib().x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R, stride, Ic2, int(has_res), buf,
+                                       512), "x1cb_describe_plan_ex")
     return buf.value.decode()
 
 

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "x1cb_internal.h"
@@ -50,11 +51,12 @@ int device_info(int &sms)
 // a B=1 call is latency-bound).
 struct PlanKey {
     int B, H, W, Ic, Oc, R, has_res, sms;
+    int stride, Hin, Win, Ic2, stride2, Hin2, Win2;
     bool operator==(const PlanKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
 
 int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
-             int m_r, int sms)
+             int m_r, int sms, const ConvGeom &g = ConvGeom{})
 {
     static std::mutex mu;
     static PlanKey keys[32];
@@ -62,7 +64,8 @@ int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_re
     static int used = 0, next = 0;
     PlanKey k;
     std::memset(&k, 0, sizeof(k));
-    k = PlanKey{B, H, W, Ic, Oc, R, has_res, sms};
+    k = PlanKey{B, H, W, Ic, Oc, R, has_res, sms,
+                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2};
     {
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < used; ++i)
@@ -71,7 +74,7 @@ int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_re
                 goto found;
             }
     }
-    if (int e = plan_conv(p, B, H, W, Ic, Oc, R, has_res, S, m_r, sms))
+    if (int e = plan_conv_ex(p, B, H, W, Ic, Oc, R, has_res, S, m_r, sms, g))
         return e;
     {
         std::lock_guard<std::mutex> lk(mu);
@@ -91,6 +94,29 @@ found:
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Every operand must be memory of the current device: the kernels launch on
+// the current device, and a pointer into another GPU (or into host memory)
+// would be read through a peer or host mapping, or fault.  NULL entries are
+// skipped (optional operands).
+int check_resident(std::initializer_list<const void *> ptrs)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return X1CB_ERR_CUDA;
+    for (const void *q : ptrs) {
+        if (!q)
+            continue;
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, q) != cudaSuccess) {
+            cudaGetLastError();  // not sticky: clear it for later calls
+            return X1CB_ERR_DEVICE;
+        }
+        if ((a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) || a.device != dev)
+            return X1CB_ERR_DEVICE;
+    }
+    return X1CB_OK;
+}
 
 bool overlap(const void *a, size_t na, const void *b, size_t nb)
 {
@@ -120,7 +146,7 @@ int check_conv_shape(int B, int H, int W, int Ic, int Oc, int S)
 
 int conv_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
                 int32_t m_r, int32_t S, const int8_t *r, int8_t *out, int B, int H, int W, int Ic,
-                int Oc, int R, void *stream)
+                int Oc, int R, void *stream, bool check_ptrs = true)
 {
     if (int e = check_conv_shape(B, H, W, Ic, Oc, S))
         return e;
@@ -140,13 +166,130 @@ int conv_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int
     int sms = 0;
     if (int e = device_info(sms))
         return e;
+    if (check_ptrs)
+        if (int e = check_resident({x, w, bias, m, r, out}))
+            return e;
     ConvPlan p;
     if (int e = get_plan(p, B, H, W, Ic, Oc, R, r != nullptr, S, m_r, sms))
         return e;
     return launch_conv(p, x, w, bias, m, r, out, static_cast<cudaStream_t>(stream));
 }
 
+// Convolutions whose input differs from their output grid: stride > 1, and
+// optionally a second 1x1 source (the projection shortcut) accumulated into
+// the same outputs.  x is [B, Ic/32, Hin, Win, 32]; out is [B, Oc/32, H, W,
+// 32] with H, W the convolution's output extent; x2 is [B, Ic2/32, Hin2,
+// Win2, 32] read at (stride2*h, stride2*w).
+int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
+                     int32_t S, int8_t *out, int B, int Hin, int Win, int Ic, int Oc, int R,
+                     int stride, const int8_t *x2, const int8_t *w2, int Ic2, int Hin2,
+                     int Win2, int stride2, void *stream, bool check_ptrs = true)
+{
+    const int pad = (R - 1) / 2;
+    if (Hin < 0 || Win < 0 || stride < 1 || stride > 8 || stride2 < 1 || stride2 > 8)
+        return X1CB_ERR_SHAPE;
+    const int H = Hin + 2 * pad >= R ? (Hin + 2 * pad - R) / stride + 1 : 0;
+    const int W = Win + 2 * pad >= R ? (Win + 2 * pad - R) / stride + 1 : 0;
+    if (int e = check_conv_shape(B, Hin, Win, Ic, Oc, S))
+        return e;
+    if (Ic2) {
+        if (Ic2 < 32 || Ic2 % 32 || Ic2 > 4096 || Hin2 < 0 || Win2 < 0)
+            return X1CB_ERR_SHAPE;
+        if (int e = check_conv_shape(B, Hin2, Win2, Ic2, Oc, S))
+            return e;
+    }
+    const size_t px = static_cast<size_t>(B) * H * W;
+    if (px == 0)
+        return X1CB_OK;
+    if (Ic2 && ((H - 1) * static_cast<long long>(stride2) >= Hin2 ||
+                (W - 1) * static_cast<long long>(stride2) >= Win2))
+        return X1CB_ERR_SHAPE;
+    if (!x || !w || !bias || !m || !out || (Ic2 && (!x2 || !w2)))
+        return X1CB_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out) || (x2 && !aligned16(x2)) ||
+        (w2 && !aligned16(w2)) || (reinterpret_cast<uintptr_t>(bias) & 3u) ||
+        (reinterpret_cast<uintptr_t>(m) & 3u))
+        return X1CB_ERR_ALIGN;
+    const size_t out_bytes = px * Oc;
+    const size_t in_bytes = static_cast<size_t>(B) * Hin * Win * Ic;
+    const size_t in2_bytes = static_cast<size_t>(B) * Hin2 * Win2 * Ic2;
+    if (overlap(out, out_bytes, x, in_bytes) || overlap(out, out_bytes, x2, in2_bytes) ||
+        overlap(out, out_bytes, w, static_cast<size_t>(Oc) * Ic * R * R) ||
+        overlap(out, out_bytes, w2, static_cast<size_t>(Oc) * Ic2) ||
+        overlap(out, out_bytes, bias, Oc * 4u) || overlap(out, out_bytes, m, Oc * 4u))
+        return X1CB_ERR_OVERLAP;
+    int sms = 0;
+    if (int e = device_info(sms))
+        return e;
+    if (check_ptrs)
+        if (int e = check_resident({x, w, bias, m, out, x2, w2}))
+            return e;
+    ConvGeom g;
+    g.stride = stride;
+    g.Hin = Hin;
+    g.Win = Win;
+    g.Ic2 = Ic2;
+    g.stride2 = stride2;
+    g.Hin2 = Hin2;
+    g.Win2 = Win2;
+    ConvPlan p;
+    if (int e = get_plan(p, B, H, W, Ic, Oc, R, 0, S, 0, sms, g))
+        return e;
+    return launch_conv(p, x, w, bias, m, nullptr, out, static_cast<cudaStream_t>(stream), x2, w2);
+}
+
+int device_info_check()
+{
+    int sms = 0;
+    return device_info(sms);
+}
+
 }  // namespace
+
+int bottleneck_chain(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                     const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                     const int32_t *b3, const int32_t *m3, int32_t m_r, int32_t S, int8_t *out,
+                     void *workspace, size_t ws_bytes, int B, int H, int W, int Cin, int Cmid,
+                     void *stream, bool ws_trusted)
+{
+    if (int e = check_conv_shape(B, H, W, Cin, Cmid, S))
+        return e;
+    if (int e = check_conv_shape(B, H, W, Cmid, Cin, S))
+        return e;
+    if (static_cast<size_t>(B) * H * W == 0)
+        return X1CB_OK;
+    if (!x || !w1 || !b1 || !m1 || !w2 || !b2 || !m2 || !w3 || !b3 || !m3 || !out)
+        return X1CB_ERR_NULL;
+    const size_t need = bottleneck_i8_workspace_size(B, H, W, Cmid);
+    if (need > 0 && (!workspace || ws_bytes < need))
+        return X1CB_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace))
+        return X1CB_ERR_ALIGN;
+    const size_t px = static_cast<size_t>(B) * H * W;
+    if (overlap(out, px * Cin, x, px * Cin) || overlap(workspace, need, x, px * Cin) ||
+        overlap(workspace, need, out, px * Cin))
+        return X1CB_ERR_OVERLAP;
+    if (px == 0)
+        return X1CB_OK;
+    if (int e = device_info_check())
+        return e;
+    if (int e = check_resident({x, w1, b1, m1, w2, b2, m2, w3, b3, m3, out}))
+        return e;
+    if (!ws_trusted)
+        if (int e = check_resident({workspace}))
+            return e;
+    int8_t *y1 = static_cast<int8_t *>(workspace);
+    int8_t *y2 = y1 + need / 2;
+    // Operands were checked above; the intermediates are the workspace.
+    if (int e = conv_common(x, w1, b1, m1, 0, S, nullptr, y1, B, H, W, Cin, Cmid, 1, stream,
+                            false))
+        return e;
+    if (int e = conv_common(y1, w2, b2, m2, 0, S, nullptr, y2, B, H, W, Cmid, Cmid, 3, stream,
+                            false))
+        return e;
+    return conv_common(y2, w3, b3, m3, m_r, S, x, out, B, H, W, Cmid, Cin, 1, stream, false);
+}
+
 }  // namespace x1cb
 
 using namespace x1cb;
@@ -169,6 +312,76 @@ int conv3x3_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias, co
     return conv_common(x, w, bias, m, 0, S, nullptr, out, B, H, W, Ic, Oc, 3, stream);
 }
 
+int conv3x3s2_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
+                         const int32_t *m, int32_t S, int8_t *out, int B, int H, int W, int Ic,
+                         int Oc, void *stream)
+{
+    return conv_geom_common(x, w, bias, m, S, out, B, H, W, Ic, Oc, 3, 2, nullptr, nullptr, 0, 0,
+                            0, 1, stream);
+}
+
+int conv1x1_proj_bn_relu_i8(const int8_t *y, const int8_t *w3, const int8_t *x,
+                            const int8_t *wp, const int32_t *bias, const int32_t *m, int32_t S,
+                            int8_t *out, int B, int H, int W, int Cy, int Hx, int Wx, int Cx,
+                            int Oc, void *stream)
+{
+    if (Cx <= 0)
+        return X1CB_ERR_SHAPE;
+    return conv_geom_common(y, w3, bias, m, S, out, B, H, W, Cy, Oc, 1, 1, x, wp, Cx, Hx, Wx, 2,
+                            stream);
+}
+
+size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid)
+{
+    if (B < 0 || H < 0 || W < 0 || Cmid < 0)
+        return 0;
+    const size_t Ho = H > 0 ? (H - 1) / 2 + 1 : 0, Wo = W > 0 ? (W - 1) / 2 + 1 : 0;
+    const size_t y1 = static_cast<size_t>(B) * H * W * Cmid;
+    const size_t y2 = static_cast<size_t>(B) * Ho * Wo * Cmid;
+    return ((y1 + 255) & ~static_cast<size_t>(255)) + ((y2 + 255) & ~static_cast<size_t>(255));
+}
+
+int bottleneck_proj_i8(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                       const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                       const int8_t *wp, const int32_t *b3, const int32_t *m3, int32_t S,
+                       int8_t *out, void *workspace, size_t ws_bytes, int B, int H, int W,
+                       int Cin, int Cmid, int Cout, void *stream)
+{
+    if (int e = check_conv_shape(B, H, W, Cin, Cmid, S))
+        return e;
+    if (int e = check_conv_shape(B, H, W, Cmid, Cout, S))
+        return e;
+    const int Ho = H > 0 ? (H - 1) / 2 + 1 : 0, Wo = W > 0 ? (W - 1) / 2 + 1 : 0;
+    const size_t px_in = static_cast<size_t>(B) * H * W;
+    const size_t px_out = static_cast<size_t>(B) * Ho * Wo;
+    if (px_in == 0)
+        return X1CB_OK;
+    if (!x || !w1 || !b1 || !m1 || !w2 || !b2 || !m2 || !w3 || !wp || !b3 || !m3 || !out)
+        return X1CB_ERR_NULL;
+    const size_t need = bottleneck_proj_i8_workspace_size(B, H, W, Cmid);
+    if (!workspace || ws_bytes < need)
+        return X1CB_ERR_WORKSPACE;
+    if (!aligned16(workspace))
+        return X1CB_ERR_ALIGN;
+    if (overlap(out, px_out * Cout, x, px_in * Cin) || overlap(workspace, need, x, px_in * Cin) ||
+        overlap(workspace, need, out, px_out * Cout))
+        return X1CB_ERR_OVERLAP;
+    if (int e = device_info_check())
+        return e;
+    if (int e = check_resident({x, w1, b1, m1, w2, b2, m2, w3, wp, b3, m3, out, workspace}))
+        return e;
+    int8_t *y1 = static_cast<int8_t *>(workspace);
+    int8_t *y2 = y1 + ((px_in * Cmid + 255) & ~static_cast<size_t>(255));
+    if (int e = conv_common(x, w1, b1, m1, 0, S, nullptr, y1, B, H, W, Cin, Cmid, 1, stream,
+                            false))
+        return e;
+    if (int e = conv_geom_common(y1, w2, b2, m2, S, y2, B, H, W, Cmid, Cmid, 3, 2, nullptr,
+                                 nullptr, 0, 0, 0, 1, stream, false))
+        return e;
+    return conv_geom_common(y2, w3, b3, m3, S, out, B, Ho, Wo, Cmid, Cout, 1, 1, x, wp, Cin, H, W,
+                            2, stream, false);
+}
+
 size_t bottleneck_i8_workspace_size(int B, int H, int W, int Cmid)
 {
     if (B < 0 || H < 0 || W < 0 || Cmid < 0)
@@ -183,34 +396,9 @@ int bottleneck_i8(const int8_t *x, const int8_t *w1, const int32_t *b1, const in
                   void *workspace, size_t ws_bytes, int B, int H, int W, int Cin, int Cmid,
                   void *stream)
 {
-    if (int e = check_conv_shape(B, H, W, Cin, Cmid, S))
-        return e;
-    if (int e = check_conv_shape(B, H, W, Cmid, Cin, S))
-        return e;
-    if (static_cast<size_t>(B) * H * W == 0)
-        return X1CB_OK;
-    if (!x || !w1 || !b1 || !m1 || !w2 || !b2 || !m2 || !w3 || !b3 || !m3 || !out)
-        return X1CB_ERR_NULL;
-    const size_t need = bottleneck_i8_workspace_size(B, H, W, Cmid);
-    if (need > 0 && (!workspace || ws_bytes < need))
-        return X1CB_ERR_WORKSPACE;
-    if (workspace && !aligned16(workspace))
-        return X1CB_ERR_ALIGN;
-    const size_t px = static_cast<size_t>(B) * H * W;
-    if (overlap(out, px * Cin, x, px * Cin) || overlap(workspace, need, x, px * Cin) ||
-        overlap(workspace, need, out, px * Cin))
-        return X1CB_ERR_OVERLAP;
-    if (px == 0)
-        return X1CB_OK;
-    int8_t *y1 = static_cast<int8_t *>(workspace);
-    int8_t *y2 = y1 + need / 2;
-    if (int e = conv_common(x, w1, b1, m1, 0, S, nullptr, y1, B, H, W, Cin, Cmid, 1, stream))
-        return e;
-    if (int e = conv_common(y1, w2, b2, m2, 0, S, nullptr, y2, B, H, W, Cmid, Cmid, 3, stream))
-        return e;
-    return conv_common(y2, w3, b3, m3, m_r, S, x, out, B, H, W, Cmid, Cin, 1, stream);
+    return bottleneck_chain(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r, S, out, workspace,
+                            ws_bytes, B, H, W, Cin, Cmid, stream, false);
 }
-
 int x1cb_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, void *stream)
 {
     if (B < 0 || H < 0 || W < 0 || C < 32 || C % 32)
@@ -224,6 +412,8 @@ int x1cb_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, 
     const size_t n = static_cast<size_t>(B) * H * W * C;
     if (overlap(nhwc, n, nc32, n))
         return X1CB_ERR_OVERLAP;
+    if (int e = check_resident({nhwc, nc32}))
+        return e;
     return launch_pack_act(nhwc, nc32, B, H, W, C, static_cast<cudaStream_t>(stream));
 }
 
@@ -240,6 +430,8 @@ int x1cb_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C
     const size_t n = static_cast<size_t>(B) * H * W * C;
     if (overlap(nhwc, n, nc32, n))
         return X1CB_ERR_OVERLAP;
+    if (int e = check_resident({nhwc, nc32}))
+        return e;
     return launch_unpack_act(nc32, nhwc, B, H, W, C, static_cast<cudaStream_t>(stream));
 }
 
@@ -252,6 +444,8 @@ int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R,
     const size_t n = static_cast<size_t>(Oc) * Ic * R * R;
     if (overlap(oihw, n, blocked, n))
         return X1CB_ERR_OVERLAP;
+    if (int e = check_resident({oihw, blocked}))
+        return e;
     return launch_pack_weight(oihw, blocked, Oc, Ic, R, static_cast<cudaStream_t>(stream));
 }
 
@@ -267,6 +461,7 @@ const char *x1cb_status_string(int s)
     case X1CB_ERR_TIMEOUT: return "kernel wait timed out";
     case X1CB_ERR_WORKSPACE: return "workspace missing or too small";
     case X1CB_ERR_OVERLAP: return "output overlaps an input";
+    case X1CB_ERR_DEVICE: return "operand is not memory of the current device";
     default: return "unknown status";
     }
 }
@@ -281,6 +476,16 @@ int x1cb_last_device_error(unsigned int *bits, int clear)
     if (bits)
         *bits = v;
     return v ? X1CB_ERR_TIMEOUT : X1CB_OK;
+}
+
+int x1cb_last_epilogue_forms(unsigned int *bits, int clear)
+{
+    if (!bits)
+        return X1CB_ERR_NULL;
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return X1CB_ERR_CUDA;
+    *bits = read_and_clear_dev_forms(clear != 0);
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 
 void x1cb_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns); }
@@ -313,6 +518,48 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
     return X1CB_OK;
 }
 
-const char *x1cb_version(void) { return "x1cb 0.1.0 sm_100a"; }
+int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int stride, int Ic2,
+                          int has_res, char *buf, size_t len)
+{
+    if (!buf || len == 0)
+        return X1CB_ERR_NULL;
+    if (R != 1 && R != 3)
+        return X1CB_ERR_SHAPE;
+    if (int e = check_conv_shape(B, Hin, Win, Ic, Oc, 24))
+        return e;
+    const int pad = (R - 1) / 2;
+    if (stride < 1 || stride > 8 || Hin + 2 * pad < R || Win + 2 * pad < R || Ic2 < 0 ||
+        Ic2 % 32 || (Ic2 && (R != 1 || stride != 1)))
+        return X1CB_ERR_SHAPE;
+    const int H = (Hin + 2 * pad - R) / stride + 1, W = (Win + 2 * pad - R) / stride + 1;
+    if (static_cast<long long>(B) * H * W == 0)
+        return X1CB_ERR_SHAPE;
+    int sms = 148;
+    if (device_info(sms) != X1CB_OK)
+        sms = 148;
+    ConvGeom g;
+    g.stride = stride;
+    g.Hin = Hin;
+    g.Win = Win;
+    if (Ic2) {  // the projection source: the stride-2 1x1 over a 2H x 2W image
+        g.Ic2 = Ic2;
+        g.stride2 = 2;
+        g.Hin2 = 2 * H;
+        g.Win2 = 2 * W;
+    }
+    ConvPlan p;
+    if (int e = plan_conv_ex(p, B, H, W, Ic, Oc, R, has_res, 24, 0, sms, g))
+        return e;
+    std::snprintf(buf, len,
+                  "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
+                  "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
+                  "out=%dx%d stride=%d kb2=%d",
+                  p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
+                  p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
+                  p.halo, p.io_swz, H, W, p.stride, p.C1b);
+    return X1CB_OK;
+}
+
+const char *x1cb_version(void) { return "x1cb 0.2.0 sm_100a"; }
 
 }  // extern "C"

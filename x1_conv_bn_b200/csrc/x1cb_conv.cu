@@ -43,6 +43,7 @@
 #include <climits>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "x1cb_internal.h"
 #include "x1cb_plan.h"
@@ -52,6 +53,10 @@ namespace x1cb {
 
 // Sticky device status word (timeouts).  Read and cleared by the API.
 __device__ unsigned int g_dev_status;
+// Epilogue forms chosen since the last clear: bit f set when a CTA ran form f
+// (0 generic, 1 64-bit high word, 2 all-32-bit, 3 all-32-bit with the bias in
+// the MMA).  Observability for tests and benchmarks; one atomic per CTA.
+__device__ unsigned int g_dev_forms;
 
 namespace {
 
@@ -202,8 +207,11 @@ __device__ __forceinline__ bool hi32_layer_ok(int m_r, int S, bool res)
     const long long q = 1ll << (S - 1);
     if (static_cast<long long>(m_r) % q != 0)
         return false;
+    // y2 = h + 1 + r*k with -2^30 <= h <= 2^30 - 1 and r in [-128, 127]
+    // stays inside int32 while -2^30 - 1 <= r*k <= 2^30 - 1: k = -2^23 with
+    // r = -128 would reach 2^31, so the lower bound is exclusive.
     const long long k = static_cast<long long>(m_r) / q;
-    return k >= -(1ll << 23) && k <= (1ll << 23);
+    return k > -(1ll << 23) && k <= (1ll << 23);
 }
 
 // Per-channel conditions: m * 2^(33-S) fits int32, and acc + bias cannot
@@ -424,6 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmR,
                        const __grid_constant__ CUtensorMap tmO,
+                       const __grid_constant__ CUtensorMap tmA2,
+                       const __grid_constant__ CUtensorMap tmW2,
                        const int32_t *__restrict__ bias, const int32_t *__restrict__ mult,
                        const ConvPlan p)
 {
@@ -481,6 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmO);
         if (kRes)
             tma_prefetch_desc(&tmR);
+        if (p.C1b) {
+            tma_prefetch_desc(&tmA2);
+            tma_prefetch_desc(&tmW2);
+        }
     }
     // Folded-BN constants of this CTA's channels.  Generic form:
     // C = bias*m + 2^(S-1), so that t = acc*m + C (+ r*m_r) is one wide
@@ -503,6 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool all_hi = __syncthreads_and(my_hi ? 1 : 0) != 0 && hi32_layer_ok(p.m_r, p.S, kRes);
     const bool fold = __syncthreads_and(my_fold ? 1 : 0) != 0 && all_hi;
     const int mode = all_hi ? (fold ? 3 : 2) : (all_fast ? 1 : 0);
+    if (threadIdx.x == 0)
+        atomicOr(&g_dev_forms, 1u << mode);
     if (fold) {
         // constant A tile (every row [1, 127 x 15, 1, 127 x 15]) and digit rows
         uint4 *ta = reinterpret_cast<uint4 *>(smem + p.off_ba);
@@ -550,9 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sw = sbase + p.off_w;
             const uint32_t wbytes = static_cast<uint32_t>(p.kb_per_tile * p.NC * 32);
             mbar_arrive_expect_tx(bars.w_full(), wbytes);
-            for (int kb = 0; kb < p.kb_per_tile; ++kb)
-                tma_load_4d(sw + kb * p.NC * 32, &tmW, bars.w_full(), 0, 0, kb,
-                            group * (p.NC / 128));
+            // The second source's weights (if any) follow the first's K blocks.
+            for (int kb = 0; kb < p.kb_per_tile; ++kb) {
+                if (kb < p.kb_a)
+                    tma_load_4d(sw + kb * p.NC * 32, &tmW, bars.w_full(), 0, 0, kb,
+                                group * (p.NC / 128));
+                else
+                    tma_load_4d(sw + kb * p.NC * 32, &tmW2, bars.w_full(), 0, 0, kb - p.kb_a,
+                                group * (p.NC / 128));
+            }
             // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
             // one filter tap), each a 128-row x 32-byte tile, back to back.
             const uint32_t abytes =
@@ -597,16 +619,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 // K blocks run channel block fastest, then filter column, then
-                // filter row; counters instead of divisions keep the issue cheap.
+                // filter row, then (if present) the second source's channel
+                // blocks; counters instead of divisions keep the issue cheap.
+                // Output pixel (w0, h0) reads input (w0*stride + ds - pad, ...);
+                // a strided map steps `stride` input pixels per loaded pixel.
+                const int wi0 = w0 * p.stride - p.pad, hi0 = h0 * p.stride - p.pad;
                 int c1 = 0, ds = 0, dr = 0;
+                bool second = false;
                 for (int bx = 0; bx < boxes; ++bx) {
                     if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes);
-                    tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0,
-                                     w0 + ds - p.pad, h0 + dr - p.pad, b0, c1, pol);
+                    if (!second)
+                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, wi0 + ds, hi0 + dr,
+                                         b0, c1, pol);
+                    else
+                        tma_load_5d_hint(slot, &tmA2, bars.a_full(stage), 0, w0 * p.stride2,
+                                         h0 * p.stride2, b0, c1, pol);
                     ++issued;
                     if (++stage == p.a_stages) {
                         stage = 0;
@@ -616,11 +647,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         slot += a_slot;
                     }
                     c1 += p.a_kc;
-                    if (c1 == p.C1) {
+                    if (!second && c1 == p.C1) {
                         c1 = 0;
                         if (++ds == p.R) {
                             ds = 0;
-                            ++dr;
+                            if (++dr == p.R)
+                                second = true;  // only reached when C1b > 0
                         }
                     }
                 }
@@ -891,9 +923,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode()
     return fn;
 }
 
+// elem_strides (optional): the traversal step per dimension; a box of
+// n * step elements along a strided dimension loads n of them.
 int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
                const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz,
-               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8)
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8,
+               const uint32_t *elem_strides = nullptr)
 {
     auto fn = get_encode();
     if (!fn)
@@ -904,7 +939,7 @@ int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
     for (int i = 0; i < rank; ++i) {
         d[i] = dims[i];
         bx[i] = box[i];
-        es[i] = 1;
+        es[i] = elem_strides ? elem_strides[i] : 1;
     }
     for (int i = 0; i < rank - 1; ++i)
         s[i] = strides_bytes[i];
@@ -912,6 +947,28 @@ int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
                     const_cast<void *>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+// Function attributes are per device: the dynamic shared-memory opt-in is set
+// once for every (device, kernel) pair, under a lock, before the first launch
+// of that kernel on that device.
+int opt_in_smem(const void *kern, int which)
+{
+    constexpr int kMaxDev = 64, kKinds = 8;
+    static std::mutex mu;
+    static bool done[kMaxDev][kKinds] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev || which < 0 ||
+        which >= kKinds)
+        return X1CB_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev][which]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+            cudaSuccess)
+            return X1CB_ERR_CUDA;
+        done[dev][which] = true;
+    }
+    return X1CB_OK;
 }
 
 }  // namespace
@@ -979,6 +1036,12 @@ void choose_halo_tile(int B, int H, int W, int &th, int &tg)
 int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
               int m_r, int num_sms)
 {
+    return plan_conv_ex(p, B, H, W, Ic, Oc, R, has_res, S, m_r, num_sms, ConvGeom{});
+}
+
+int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
+                 int m_r, int num_sms, const ConvGeom &g)
+{
     std::memset(&p, 0, sizeof(p));
     p.B = B;
     p.H = H;
@@ -992,16 +1055,38 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     p.has_res = has_res;
     p.S = S;
     p.m_r = m_r;
-    if (R == 1) {
+    p.stride = g.stride < 1 ? 1 : g.stride;
+    p.Hin = g.Hin ? g.Hin : H;
+    p.Win = g.Win ? g.Win : W;
+    p.C1b = g.Ic2 / 32;
+    p.stride2 = g.stride2 < 1 ? 1 : g.stride2;
+    p.Hin2 = g.Hin2;
+    p.Win2 = g.Win2;
+    if (p.stride > 8 || p.stride2 > 8 || g.Ic2 % 32 || g.Ic2 < 0)
+        return X1CB_ERR_SHAPE;  // the TMA's traversal step is at most 8
+    // Every tapped input pixel must exist for some output: (H-1)*stride + R - 1
+    // - pad < Hin + pad, and the output extent is the convolution's.
+    if ((p.Hin + 2 * p.pad - R) / p.stride + 1 != H || (p.Win + 2 * p.pad - R) / p.stride + 1 != W)
+        return X1CB_ERR_SHAPE;
+    if (p.C1b && ((H - 1) * p.stride2 >= p.Hin2 || (W - 1) * p.stride2 >= p.Win2))
+        return X1CB_ERR_SHAPE;
+    // A stride-1 1x1 without a second source sees the image as one row of H*W
+    // pixels (tiles may span image rows); otherwise tiles are 2-D.
+    const bool flat = R == 1 && p.stride == 1 && p.C1b == 0;
+    if (flat) {
         p.Wp = H * W;
         p.Hp = 1;
+        p.Wpi = H * W;
+        p.Hpi = 1;
     } else {
         p.Wp = W;
         p.Hp = H;
+        p.Wpi = p.Win;
+        p.Hpi = p.Hin;
     }
     // The 3x3 convolution uses the halo form whenever one framed image row fits
-    // in the 128 GEMM rows.
-    p.halo = (R == 3 && p.pad == 1 && W + 2 <= kTileRows) ? 1 : 0;
+    // in the 128 GEMM rows (stride 1).
+    p.halo = (R == 3 && p.pad == 1 && p.stride == 1 && p.C1b == 0 && W + 2 <= kTileRows) ? 1 : 0;
     if (p.halo) {
         choose_halo_tile(B, H, W, p.th, p.tg);
         p.tw = W;
@@ -1025,7 +1110,8 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     if (mtiles > INT_MAX / 2)
         return X1CB_ERR_SHAPE;
     p.num_m_tiles = static_cast<int>(mtiles);
-    p.kb_per_tile = R * R * p.C1;
+    p.kb_a = R * R * p.C1;
+    p.kb_per_tile = p.kb_a + p.C1b;
 
     const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 12) * 8 + 64;
     const int min_slot = p.halo ? 2 * p.a_half : kASlotBytes;
@@ -1076,7 +1162,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
     p.a_kc = 1;
     if (!p.halo)
         for (int kc = 4; kc > 1; kc /= 2)
-            if (p.C1 % kc == 0 && p.rows % 8 == 0 &&
+            if (p.C1 % kc == 0 && p.C1b % kc == 0 && p.rows % 8 == 0 &&
                 ring_min(kc) * kc * kASlotBytes <= a_bytes_want) {
                 p.a_kc = kc;
                 break;
@@ -1128,9 +1214,12 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
 }
 
 int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32_t *bias,
-                const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream)
+                const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream,
+                const int8_t *x2, const int8_t *w2)
 {
-    CUtensorMap tmA, tmW, tmR, tmO;
+    if (p.C1b && (!x2 || !w2))
+        return X1CB_ERR_NULL;
+    CUtensorMap tmA, tmW, tmR, tmO, tmA2, tmW2;
     // Activations: dims (32 ch, Wp, Hp, B, C1) -- channel blocks outermost so a
     // box (32, tw, th, tg, a_kc) lands as a_kc K-block tiles one after another.
     // Halo form: dims (32 ch, W, H, C1, B), box (16, tw+2, th+2, 1, tg) -- one K
@@ -1145,21 +1234,49 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return e;
     } else {
-        const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.B,
+        // Input extent (Wpi, Hpi); a strided map loads every stride-th pixel,
+        // so a box of tw*stride x th*stride elements lands tw x th pixels.
+        const uint64_t dims[5] = {32, (uint64_t)p.Wpi, (uint64_t)p.Hpi, (uint64_t)p.B,
                                   (uint64_t)p.C1};
-        const uint64_t str[4] = {32, (uint64_t)p.Wp * 32, (uint64_t)p.C1 * p.Hp * p.Wp * 32,
-                                 (uint64_t)p.Hp * p.Wp * 32};
-        const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)p.th, (uint32_t)p.tg,
-                                 (uint32_t)p.a_kc};
-        if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
+        const uint64_t str[4] = {32, (uint64_t)p.Wpi * 32, (uint64_t)p.C1 * p.Hpi * p.Wpi * 32,
+                                 (uint64_t)p.Hpi * p.Wpi * 32};
+        const uint32_t box[5] = {32, (uint32_t)(p.tw * p.stride), (uint32_t)(p.th * p.stride),
+                                 (uint32_t)p.tg, (uint32_t)p.a_kc};
+        const uint32_t es[5] = {1, (uint32_t)p.stride, (uint32_t)p.stride, 1, 1};
+        if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT8, es))
+            return e;
+    }
+    // Second source (projection shortcut): dims (32, Win2, Hin2, B, C1b), the
+    // same box at its own stride.
+    tmA2 = tmA;
+    if (p.C1b) {
+        const uint64_t dims[5] = {32, (uint64_t)p.Win2, (uint64_t)p.Hin2, (uint64_t)p.B,
+                                  (uint64_t)p.C1b};
+        const uint64_t str[4] = {32, (uint64_t)p.Win2 * 32,
+                                 (uint64_t)p.C1b * p.Hin2 * p.Win2 * 32,
+                                 (uint64_t)p.Hin2 * p.Win2 * 32};
+        const uint32_t box[5] = {32, (uint32_t)(p.tw * p.stride2), (uint32_t)(p.th * p.stride2),
+                                 (uint32_t)p.tg, (uint32_t)p.a_kc};
+        const uint32_t es[5] = {1, (uint32_t)p.stride2, (uint32_t)p.stride2, 1, 1};
+        if (int e = encode_map(&tmA2, x2, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT8, es))
             return e;
     }
     // Weights [Oc/128][KB][128][32]: dims (32, 128, KB, Oc/128); box (32,128,1,NC/128).
     {
-        const uint64_t dims[4] = {32, 128, (uint64_t)p.kb_per_tile, (uint64_t)(p.Oc / 128)};
-        const uint64_t str[3] = {32, 4096, (uint64_t)p.kb_per_tile * 4096};
+        const uint64_t dims[4] = {32, 128, (uint64_t)p.kb_a, (uint64_t)(p.Oc / 128)};
+        const uint64_t str[3] = {32, 4096, (uint64_t)p.kb_a * 4096};
         const uint32_t box[4] = {32, 128, 1, (uint32_t)(p.NC / 128)};
         if (int e = encode_map(&tmW, w, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
+            return e;
+    }
+    tmW2 = tmW;
+    if (p.C1b) {
+        const uint64_t dims[4] = {32, 128, (uint64_t)p.C1b, (uint64_t)(p.Oc / 128)};
+        const uint64_t str[3] = {32, 4096, (uint64_t)p.C1b * 4096};
+        const uint32_t box[4] = {32, 128, 1, (uint32_t)(p.NC / 128)};
+        if (int e = encode_map(&tmW2, w2, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }
     // Shortcut and output, no swizzle: one box is one I/O stage [tg][4][th][tw][32].
@@ -1217,14 +1334,10 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         }
     }
     auto kern = p.has_res ? conv_bn_act_kernel<true> : conv_bn_act_kernel<false>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[p.has_res]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
-            cudaSuccess)
-            return X1CB_ERR_CUDA;
-        attr_set[p.has_res] = true;
-    }
-    kern<<<p.grid, kThreads, p.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, bias, mult, p);
+    if (int e = opt_in_smem(reinterpret_cast<const void *>(kern), p.has_res))
+        return e;
+    kern<<<p.grid, kThreads, p.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, tmA2, tmW2, bias, mult,
+                                                      p);
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 
@@ -1235,6 +1348,17 @@ unsigned int read_and_clear_dev_status(bool clear)
     if (clear) {
         const unsigned int z = 0;
         cudaMemcpyToSymbol(g_dev_status, &z, sizeof(z));
+    }
+    return v;
+}
+
+unsigned int read_and_clear_dev_forms(bool clear)
+{
+    unsigned int v = 0;
+    cudaMemcpyFromSymbol(&v, g_dev_forms, sizeof(v));
+    if (clear) {
+        const unsigned int z = 0;
+        cudaMemcpyToSymbol(g_dev_forms, &z, sizeof(z));
     }
     return v;
 }

@@ -12,9 +12,30 @@ namespace x1cb {
 void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg);
 int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
               int m_r, int num_sms);
+// Geometry beyond the plain stride-1 layer: the input image is Hin x Win and
+// the stride `stride` (output H x W); optionally a second 1x1 source of Ic2
+// channels at stride `stride2` over a Hin2 x Win2 image, accumulated into the
+// same outputs (Ic2 = 0: none).
+struct ConvGeom {
+    int stride = 1, Hin = 0, Win = 0;
+    int Ic2 = 0, stride2 = 1, Hin2 = 0, Win2 = 0;
+};
+int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
+                 int m_r, int num_sms, const ConvGeom &g);
 int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32_t *bias,
-                const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream);
+                const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream,
+                const int8_t *x2 = nullptr, const int8_t *w2 = nullptr);
 unsigned int read_and_clear_dev_status(bool clear);
+unsigned int read_and_clear_dev_forms(bool clear);
+
+// The bottleneck chain behind bottleneck_i8 and bottleneck_i8_noalloc.
+// ws_checked: the workspace was supplied by the library itself (its own
+// device array), so its residency is not re-checked.
+int bottleneck_chain(const int8_t *x, const int8_t *w1, const int32_t *b1, const int32_t *m1,
+                     const int8_t *w2, const int32_t *b2, const int32_t *m2, const int8_t *w3,
+                     const int32_t *b3, const int32_t *m3, int32_t m_r, int32_t S, int8_t *out,
+                     void *workspace, size_t ws_bytes, int B, int H, int W, int Cin, int Cmid,
+                     void *stream, bool ws_trusted);
 
 int launch_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C,
                     cudaStream_t s);

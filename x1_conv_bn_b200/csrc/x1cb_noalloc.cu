@@ -65,13 +65,13 @@ extern "C" int bottleneck_i8_noalloc(const int8_t *x, const int8_t *w1, const in
     if (need > x1cb::kNoAllocScratchBytes)
         return X1CB_ERR_WORKSPACE;  // the two intermediates do not fit the built-in scratch
     if (need == 0)
-        return bottleneck_i8(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r, S, out, nullptr, 0, B,
-                             H, W, Cin, Cmid, stream);
+        return x1cb::bottleneck_chain(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r, S, out,
+                                      nullptr, 0, B, H, W, Cin, Cmid, stream, true);
     void *scratch = nullptr;
     if (int e = x1cb::scratch_address(&scratch))
         return e;
     // The intermediates are written in full by conv1 and conv2 before they are
     // read, so nothing in the scratch has to start at zero.
-    return bottleneck_i8(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r, S, out, scratch,
-                         x1cb::kNoAllocScratchBytes, B, H, W, Cin, Cmid, stream);
+    return x1cb::bottleneck_chain(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r, S, out, scratch,
+                                  x1cb::kNoAllocScratchBytes, B, H, W, Cin, Cmid, stream, true);
 }

@@ -27,7 +27,16 @@ struct ConvPlan {
     // problem
     int B, H, W, Ic, Oc, R, pad;
     int C1, O1;       // Ic/32, Oc/32
-    int Wp, Hp;       // spatial dims seen by the tensor maps (1x1: H*W and 1)
+    int Wp, Hp;       // output spatial dims seen by the tensor maps (1x1: H*W and 1)
+    // Convolution stride and the input image the activation map covers
+    // (Wpi, Hpi: the input's dims as the map sees them; H*W and 1 for a
+    // stride-1 1x1).  Output pixel (h, w) reads input rows h*stride + dr - pad.
+    int stride, Hin, Win, Wpi, Hpi;
+    // Optional second activation source whose K blocks follow the first's in
+    // the same accumulator (the projection shortcut of a downsampling block):
+    // a 1x1 at stride `stride2` over a Hin2 x Win2 image of C1b channel blocks.
+    // kb_a = R*R*C1 blocks come from the first source, C1b from the second.
+    int C1b, kb_a, stride2, Hin2, Win2;
     int has_res;
     int S;
     int m_r;
