@@ -152,8 +152,12 @@ def workload_units(cfg):
     return s.ops(), s.bytes_moved()
 
 
+def is_block(s):
+    return isinstance(s, (synth.BlockShape, synth.ProjBlockShape))
+
+
 def launches_per_step(cfg):
-    return 3 if isinstance(synth.CONFIGS[cfg], synth.BlockShape) else 1
+    return 3 if is_block(synth.CONFIGS[cfg]) else 1
 
 
 class ClockSampler:
@@ -245,6 +249,25 @@ def device_inputs(cfg, dev, seed, n_sets=1):
     import x1_conv_bn_b200 as X
 
     s = synth.CONFIGS[cfg]
+    if isinstance(s, synth.ProjBlockShape):
+        inp = synth.proj_block_inputs(s, seed, device=dev)
+        x = X.x1cb_pack_act(inp.x)
+        ws = [X.x1cb_pack_weight(w) for w in inp.w]
+        wp = X.x1cb_pack_weight(inp.wp)
+        work = torch.empty(X.bottleneck_proj_i8_workspace_size(s.B, s.H, s.W, s.Cmid),
+                           dtype=torch.int8, device=dev)
+        xs = [x] + [x.clone() for _ in range(n_sets - 1)]
+        outs = [torch.empty((s.B, s.Cout // 32, s.Ho, s.Wo, 32), dtype=torch.int8, device=dev)
+                for _ in range(n_sets)]
+        del inp.x
+
+        def call(i=0, x_=None, out_=None, stream=None):
+            X.bottleneck_proj_i8(xs[i] if x_ is None else x_, ws[0], inp.bias[0], inp.m[0],
+                                 ws[1], inp.bias[1], inp.m[1], ws[2], wp, inp.bias[2], inp.m[2],
+                                 inp.S, out=outs[i] if out_ is None else out_, workspace=work,
+                                 stream=stream)
+
+        return call, {"x": x}, outs[0]
     if isinstance(s, synth.BlockShape):
         inp = synth.block_inputs(s, seed, device=dev)
         x = X.x1cb_pack_act(inp.x)
@@ -295,12 +318,17 @@ class OracleSample:
         self.s = synth.CONFIGS[cfg]
         self.cores = O.set_threads(0)
         s = self.s
-        self.hw = s.H * s.W
+        # output pixels per image (the projection block halves the image; its
+        # oracle runs whole images, so its sample is whole images)
+        self.proj = isinstance(s, synth.ProjBlockShape)
+        self.hw = s.Ho * s.Wo if self.proj else s.H * s.W
         self._make(1, seed)
         t = self._run(self.hw)
         per_px = t / self.hw
         n = int(max(1, min(s.B * self.hw, seconds / max(per_px, 1e-9))))
         imgs = (n + self.hw - 1) // self.hw
+        if self.proj:
+            n = imgs * self.hw
         if imgs > 1:
             self._make(imgs, seed)
         self.n = n
@@ -308,7 +336,10 @@ class OracleSample:
 
     def _make(self, imgs, seed):
         s = self.s
-        if isinstance(s, synth.BlockShape):
+        if isinstance(s, synth.ProjBlockShape):
+            self.inp = synth.proj_block_inputs(
+                synth.ProjBlockShape(imgs, s.H, s.W, s.Cin, s.Cmid, s.Cout), seed)
+        elif isinstance(s, synth.BlockShape):
             self.inp = synth.block_inputs(synth.BlockShape(imgs, s.H, s.W, s.Cin, s.Cmid), seed)
         else:
             self.inp = synth.conv_inputs(
@@ -318,7 +349,9 @@ class OracleSample:
         inp, O = self.inp, self.O
         pix = torch.arange(n, dtype=torch.int64)
         t0 = time.perf_counter()
-        if isinstance(self.s, synth.BlockShape):
+        if self.proj:
+            O.bottleneck_proj(inp.x, inp.w, inp.wp, inp.bias, inp.m, inp.S)
+        elif isinstance(self.s, synth.BlockShape):
             O.bottleneck_pixels(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S, pix)
         else:
             O.conv_pixels(inp.x, inp.w, inp.bias, inp.m, inp.S, pix, inp.r, inp.m_r)
@@ -403,12 +436,36 @@ def dry_run(a, rank, world):
 
 
 def block_stage_calls(cfg, dev, seed):
-    """For the block workload: the three stages as separate calls on the same
+    """For the block workloads: the three stages as separate calls on the same
     buffers (conv1 x -> y1, conv2 y1 -> y2, conv3 y2 (+x) -> out), for
-    per-stage timing."""
+    per-stage timing.  Returns (label, ops, bytes, call) per stage."""
     import x1_conv_bn_b200 as X
 
     s = synth.CONFIGS[cfg]
+    if isinstance(s, synth.ProjBlockShape):
+        inp = synth.proj_block_inputs(s, seed, device=dev)
+        x = X.x1cb_pack_act(inp.x)
+        ws = [X.x1cb_pack_weight(w) for w in inp.w]
+        wp = X.x1cb_pack_weight(inp.wp)
+        y1 = torch.empty((s.B, s.Cmid // 32, s.H, s.W, 32), dtype=torch.int8, device=dev)
+        y2 = torch.empty((s.B, s.Cmid // 32, s.Ho, s.Wo, 32), dtype=torch.int8, device=dev)
+        out = torch.empty((s.B, s.Cout // 32, s.Ho, s.Wo, 32), dtype=torch.int8, device=dev)
+        c1 = synth.ConvShape(s.B, s.H, s.W, s.Cin, s.Cmid, 1, False)
+        px = s.B * s.Ho * s.Wo
+        return [
+            ("1x1 %d->%d" % (s.Cin, s.Cmid), c1.ops(), c1.bytes_moved(),
+             lambda stream: X.conv1x1_bn_add_relu_i8(x, ws[0], inp.bias[0], inp.m[0], 0, inp.S,
+                                                     None, out=y1, stream=stream)),
+            ("3x3/2 %d->%d" % (s.Cmid, s.Cmid), 2 * px * s.Cmid * 9 * s.Cmid,
+             s.B * s.H * s.W * s.Cmid + px * s.Cmid + 9 * s.Cmid ** 2 + 8 * s.Cmid,
+             lambda stream: X.conv3x3s2_bn_relu_i8(y1, ws[1], inp.bias[1], inp.m[1], inp.S,
+                                                   out=y2, stream=stream)),
+            ("1x1 %d->%d + proj %d/2" % (s.Cmid, s.Cout, s.Cin),
+             2 * px * s.Cout * (s.Cmid + s.Cin),
+             px * (s.Cmid + s.Cin + s.Cout) + s.Cout * (s.Cmid + s.Cin) + 8 * s.Cout,
+             lambda stream: X.conv1x1_proj_bn_relu_i8(y2, ws[2], x, wp, inp.bias[2], inp.m[2],
+                                                      inp.S, out=out, stream=stream)),
+        ]
     inp = synth.block_inputs(s, seed, device=dev)
     x = X.x1cb_pack_act(inp.x)
     ws = [X.x1cb_pack_weight(w) for w in inp.w]
@@ -416,14 +473,20 @@ def block_stage_calls(cfg, dev, seed):
     y2 = torch.empty_like(y1)
     out = torch.empty_like(x)
     st = s.stages()
+
+    def label(c):
+        return f"{c.R}x{c.R} {c.Ic}->{c.Oc}" + (" +res" if c.has_res else "")
+
     return [
-        (st[0], lambda stream: X.conv1x1_bn_add_relu_i8(x, ws[0], inp.bias[0], inp.m[0], 0,
-                                                        inp.S, None, out=y1, stream=stream)),
-        (st[1], lambda stream: X.conv3x3_bn_relu_i8(y1, ws[1], inp.bias[1], inp.m[1], inp.S,
-                                                    out=y2, stream=stream)),
-        (st[2], lambda stream: X.conv1x1_bn_add_relu_i8(y2, ws[2], inp.bias[2], inp.m[2],
-                                                        inp.m_r, inp.S, x, out=out,
-                                                        stream=stream)),
+        (label(st[0]), st[0].ops(), st[0].bytes_moved(),
+         lambda stream: X.conv1x1_bn_add_relu_i8(x, ws[0], inp.bias[0], inp.m[0], 0, inp.S, None,
+                                                 out=y1, stream=stream)),
+        (label(st[1]), st[1].ops(), st[1].bytes_moved(),
+         lambda stream: X.conv3x3_bn_relu_i8(y1, ws[1], inp.bias[1], inp.m[1], inp.S, out=y2,
+                                             stream=stream)),
+        (label(st[2]), st[2].ops(), st[2].bytes_moved(),
+         lambda stream: X.conv1x1_bn_add_relu_i8(y2, ws[2], inp.bias[2], inp.m[2], inp.m_r,
+                                                 inp.S, x, out=out, stream=stream)),
     ]
 
 
@@ -549,14 +612,13 @@ def main(argv=None):
 
     # ---- per-stage times of the block (its dominant kernel gets the roofline) ----
     stages = None
-    if isinstance(s, synth.BlockShape):
+    if is_block(s):
         stages = []
         with torch.cuda.stream(stream):
-            for shp, fn in block_stage_calls(cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank)):
+            for lab, s_ops, s_bytes, fn in block_stage_calls(
+                    cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank)):
                 t = time_launches(fn, stream, max(20, min(200, a.steps)))
-                stages.append({"stage": f"{shp.R}x{shp.R} {shp.Ic}->{shp.Oc}"
-                                        + (" +res" if shp.has_res else ""),
-                               "us": t * 1e3, "ops": shp.ops(), "bytes": shp.bytes_moved()})
+                stages.append({"stage": lab, "us": t * 1e3, "ops": s_ops, "bytes": s_bytes})
         torch.cuda.synchronize()
         if X.x1cb_last_device_error(clear=True)[0] != 0:
             raise RuntimeError("device status set in the per-stage timing")
@@ -652,7 +714,7 @@ def main(argv=None):
         roof["kernel"] = "stage " + top["stage"] + " (the block's slowest launch)"
         roof["algorithmic_bytes_per_launch"] = top["bytes"]
         roof["algorithmic_ops_per_launch"] = top["ops"]
-        prof = f"bottleneck_b{s.B}.md"
+        prof = f"bottleneck_{cfg}_b{s.B}.md"
     roof["traffic"] = read_traffic(prof, kernel_source_sha())
     roof["traffic_source"] = (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
                               f"profiles/{prof}, taken on this kernel source"

@@ -160,8 +160,12 @@ size_t bottleneck_i8_workspace_size(int B, int H, int W, int Cmid);
 /*
  * Res3.x bottleneck block (Inspur article section 2.2): conv1 1x1 Cin->Cmid
  * +BN+ReLU, conv2 3x3 pad 1 Cmid->Cmid +BN+ReLU, conv3 1x1 Cmid->Cin +BN +
- * Sum with the block input + ReLU.  Three launches on `stream`, no host
- * synchronisation between them.
+ * Sum with the block input + ReLU.  With Cmid = 128, Cin <= 1024 and W <= 126
+ * conv2 and conv3 run as one kernel on pairs of SMs (the merge of two
+ * consecutive convolutions of the article's section 2.1): conv2's output
+ * stays on chip, so the block is two launches and only conv1's output goes
+ * through the workspace.  Other shapes take three launches.  No host
+ * synchronisation between launches.
  *   x   [B, Cin/32, H, W, 32] block input, also the shortcut (read)
  *   w1  [Cmid/128, Cin/32, 128, 32]; w2 [Cmid/128, 3, 3, Cmid/32, 128, 32];
  *   w3  [Cin/128, Cmid/32, 128, 32]; b*, m* [Cmid], [Cmid], [Cin]
@@ -229,6 +233,12 @@ int x1cb_last_device_error(unsigned int *bits, int clear);
  * constants reached.  clear != 0 resets the record.  Returns X1CB_OK or an
  * error. */
 int x1cb_last_epilogue_forms(unsigned int *bits, int clear);
+
+/* enable = 0 makes bottleneck_i8 (and bottleneck_i8_noalloc) run conv2 and
+ * conv3 as two separate launches even where the fused form applies (for
+ * comparisons); 1 (the default) restores the fused form.  Same results
+ * either way. */
+void x1cb_set_block_fusion(int enable);
 
 /* Limit of every in-kernel wait, in nanoseconds (default 2 s; 0 restores the
  * default).  Applies to launches made after the call. */

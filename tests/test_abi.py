@@ -167,13 +167,47 @@ def test_plans_fit_shared_memory(L, shape):
     assert int(p["a_stages"]) >= 2
 
 
+def _stream(shape):
+    return _plan(shape)["wstream"]
+
+
 @pytest.mark.parametrize("R,res,max_ic", [(1, 1, 1120), (1, 0, 1376), (3, 0, 128)])
-def test_channel_limits_stated_in_the_header(L, R, res, max_ic):
-    X.x1cb_describe_plan(4, 28, 28, max_ic, 128, R, res)
-    with pytest.raises(X.X1cbError):
-        X.x1cb_describe_plan(4, 28, 28, max_ic + 32, 128, R, res)
+def test_weights_stay_resident_up_to_the_stated_fan_in(L, R, res, max_ic):
+    """Up to these fan-ins the weights of 128 output channels stay resident in
+    shared memory; beyond them they are streamed with the activations."""
+    assert _stream((4, 28, 28, max_ic, 128, R, res)) == "0"
+    assert _stream((4, 28, 28, max_ic + 32, 128, R, res)) == "1"
 
 
-def test_plan_rejects_weights_that_do_not_fit(L):
-    with pytest.raises(X.X1cbError):
-        X.x1cb_describe_plan(8, 14, 14, 1024, 256, 3, 0)
+@pytest.mark.parametrize("shape", [(8, 14, 14, 1024, 256, 3, 0), (512, 7, 7, 512, 512, 3, 0),
+                                   (4, 28, 28, 4096, 128, 1, 1), (2, 7, 7, 4096, 128, 3, 0)])
+def test_large_fan_in_streams_weights(L, shape):
+    p = _plan(shape)
+    assert p["wstream"] == "1" and p["NC"] == "128" and p["subs"] == "1"
+    assert int(p["smem"]) <= 232448 and int(p["a_stages"]) >= 2
+
+
+def _header_param_counts():
+    import re
+
+    text = open(X.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(\w+)\s*\(([^()]*)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_header(L):
+    """Every declared function's ctypes signature has as many arguments as
+    its C declaration (a missing or extra one would shift every later
+    argument)."""
+    counts = _header_param_counts()
+    assert len(counts) == len(X.header_functions())
+    for name, n in counts.items():
+        at = getattr(L, name).argtypes
+        if at is None:  # argument-less helpers
+            assert n == 0, name
+        else:
+            assert len(at) == n, (name, len(at), n)

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.x1cb_status_string.restype = ctypes.c_char_p
         L.x1cb_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
         L.x1cb_last_epilogue_forms.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+        L.x1cb_set_block_fusion.argtypes = [i]
+        L.x1cb_set_block_fusion.restype = None
         L.x1cb_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.x1cb_set_wait_limit_ns.restype = None
         L.x1cb_debug_inject.argtypes = [i]
@@ -67,7 +69,7 @@ def lib() -> ctypes.CDLL:
         L.x1cb_describe_plan.argtypes = [i, i, i, i, i, i, i, ctypes.c_char_p, sz]
         L.x1cb_version.restype = ctypes.c_char_p
         L.conv3x3s2_bn_relu_i8.argtypes = [vp] * 4 + [i32, vp] + [i] * 5 + [vp]
-        L.conv1x1_proj_bn_relu_i8.argtypes = [vp] * 6 + [i32, vp] + [i] * 9 + [vp]
+        L.conv1x1_proj_bn_relu_i8.argtypes = [vp] * 6 + [i32, vp] + [i] * 8 + [vp]
         L.bottleneck_proj_i8_workspace_size.argtypes = [i, i, i, i]
         L.bottleneck_proj_i8_workspace_size.restype = sz
         L.bottleneck_proj_i8.argtypes = [vp] * 11 + [i32, vp, vp, sz] + [i] * 6 + [vp]
@@ -335,6 +337,12 @@ def x1cb_last_epilogue_forms(clear: bool = True) -> int:
     _check(lib().x1cb_last_epilogue_forms(ctypes.byref(bits), int(clear)),
            "x1cb_last_epilogue_forms")
     return bits.value
+
+
+def x1cb_set_block_fusion(enable: bool):
+    """Fused conv2 -> conv3 in bottleneck_i8 where the shape allows (default
+    on); off runs them as separate launches.  Same results either way."""
+    lib().x1cb_set_block_fusion(int(bool(enable)))
 
 
 def x1cb_set_wait_limit_ns(ns: int):

@@ -18,6 +18,7 @@ namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{0};
 std::atomic<int> g_inject{0};
+std::atomic<int> g_block_fusion{1};
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 
 struct DevInfo {
@@ -280,6 +281,17 @@ int bottleneck_chain(const int8_t *x, const int8_t *w1, const int32_t *b1, const
             return e;
     int8_t *y1 = static_cast<int8_t *>(workspace);
     int8_t *y2 = y1 + need / 2;
+    // Conv2 -> Conv3 in one kernel where the shape has the fused form: Conv2's
+    // output stays on chip and only Conv1's output goes through the workspace.
+    ChainPlan cp;
+    if (g_block_fusion.load() && plan_chain(cp, B, H, W, Cmid, Cin, S, m_r) == X1CB_OK) {
+        if (int e = conv_common(x, w1, b1, m1, 0, S, nullptr, y1, B, H, W, Cin, Cmid, 1, stream,
+                                false))
+            return e;
+        cp.wait_limit_ns = g_wait_limit_ns.load() ? g_wait_limit_ns.load() : kDefaultWaitNs;
+        return launch_chain(cp, y1, w2, b2, m2, w3, b3, m3, x, out,
+                            static_cast<cudaStream_t>(stream));
+    }
     // Operands were checked above; the intermediates are the workspace.
     if (int e = conv_common(x, w1, b1, m1, 0, S, nullptr, y1, B, H, W, Cin, Cmid, 1, stream,
                             false))
@@ -488,6 +500,8 @@ int x1cb_last_epilogue_forms(unsigned int *bits, int clear)
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 
+void x1cb_set_block_fusion(int enable) { g_block_fusion.store(enable ? 1 : 0); }
+
 void x1cb_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns); }
 
 void x1cb_debug_inject(int mode) { g_inject.store(mode); }
@@ -511,10 +525,11 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
         return e;
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
-                  "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d",
+                  "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
+                  "wstream=%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo, p.io_swz);
+                  p.halo, p.io_swz, p.wstream);
     return X1CB_OK;
 }
 
@@ -553,10 +568,10 @@ int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int st
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
                   "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
-                  "out=%dx%d stride=%d kb2=%d",
+                  "out=%dx%d stride=%d kb2=%d wstream=%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo, p.io_swz, H, W, p.stride, p.C1b);
+                  p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream);
     return X1CB_OK;
 }
 

@@ -1,0 +1,743 @@
+// Conv2 -> Conv3 of the Res3.x bottleneck in one kernel: the 3x3 convolution
+// (+ folded BN + ReLU, requantised to int8) feeds the 1x1 convolution (+ folded
+// BN + shortcut Sum + ReLU) through on-chip memory, so Conv2's output never
+// travels through HBM.  This is the merge of two consecutive convolutions
+// that the Inspur MLPerf ResNet50 convolution-merge article names in section
+// 2.1 (its A100 kernel merged only Conv3 with the shortcut, section 2.2).
+//
+// Both weight sets must stay on chip (3x3: 144 KB for 128 channels, 1x1: up to
+// 64 KB), more than one SM's shared memory next to the rings, so the kernel
+// runs on pairs of CTAs (a cluster of two) that share every MMA
+// (tcgen05 cta_group::2): A is split by rows -- each CTA loads its own halo
+// tile and keeps its own Conv2 output as Conv3's A operand -- and B by
+// columns, so each CTA holds half of each weight set.  Rank 0 issues every
+// MMA (M = 256: 128 rows per CTA); each CTA's TMEM receives its own rows.
+//
+// Per CTA (20 warps):
+//   warp 0      TMA producer: its weight halves once, then the halo tile of
+//               each channel block (one 3x3 A slot, nine row-shifted views),
+//               completion counted on rank 0's barriers
+//   warp 1      TMEM owner (both ranks); MMA issuer (rank 0): Conv2 of pair
+//               tile i, then Conv3 of pair tile i-1 in 128-channel chunks
+//   warp 2      TMA producer of the shortcut stages (own rows)
+//   warp 3      TMA store of finished output stages (own rows)
+//   warps 4-15  Conv3 epilogue: 3 turns per TMEM lane quarter, one per
+//               Conv3 accumulator slot; shortcut Sum, requantisation, ReLU
+//   warps 16-19 Conv2 epilogue (one per lane quarter, every tile): requantises
+//               Conv2 and writes the int8 result into this CTA's Conv3 A
+//               buffer in shared memory
+// TMEM (512 columns per CTA): Conv2's accumulator (128) and three Conv3
+// accumulator slots of 128 output channels.  Conv3's epilogue is the heavy
+// one (the shortcut and 4x the channels), so it gets 12 of the 16 epilogue
+// warps.
+// Every wait is bounded; a wait that runs out raises the CTA's abort flag and
+// a status bit, and both CTAs leave through a bounded exit handshake.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "x1cb_epi.cuh"
+#include "x1cb_internal.h"
+#include "x1cb_ptx.cuh"
+
+namespace x1cb {
+
+extern __device__ unsigned int g_dev_status;
+extern __device__ unsigned int g_dev_forms;
+
+namespace {
+
+constexpr int kA3Bufs = 2;          // Conv3 A buffers (Conv2 results) in shared memory
+constexpr int kAcc3 = 3;            // Conv3 accumulator slots (= Conv3 epilogue turns)
+constexpr int kE2Warp0 = 4, kE1Warp0 = 16;
+constexpr int kA3Bytes = 128 * 128;  // Conv3 A buffer: 128 rows x 128 channels
+static_assert(kE1Warp0 - kE2Warp0 == 4 * kAcc3, "one Conv3 turn per accumulator slot");
+static_assert(kThreads == 32 * (kE1Warp0 + 4), "20 warps");
+constexpr int kHalfRows = 64;      // B rows (output channels) each CTA holds per MMA
+
+struct ChainBars {
+    uint32_t base;
+    int a_stages, r_stages;
+    __device__ uint32_t at(int i) const { return base + 8u * static_cast<uint32_t>(i); }
+    __device__ uint32_t w_full() const { return at(0); }
+    __device__ uint32_t mma_done() const { return at(1); }
+    __device__ uint32_t exit_bar() const { return at(2); }
+    __device__ uint32_t a_full(int s) const { return at(3 + s); }
+    __device__ uint32_t a_empty(int s) const { return at(3 + a_stages + s); }
+    __device__ uint32_t acc2_full() const { return at(3 + 2 * a_stages); }
+    __device__ uint32_t acc2_empty() const { return at(4 + 2 * a_stages); }
+    __device__ uint32_t a3_full(int k) const { return at(5 + 2 * a_stages + k); }
+    __device__ uint32_t a3_empty(int k) const { return at(7 + 2 * a_stages + k); }
+    __device__ uint32_t acc3_full(int k) const { return at(9 + 2 * a_stages + k); }
+    __device__ uint32_t acc3_empty(int k) const { return at(12 + 2 * a_stages + k); }
+    __device__ uint32_t io_full(int s) const { return at(15 + 2 * a_stages + s); }
+    __device__ uint32_t out_ready(int s) const { return at(15 + 2 * a_stages + r_stages + s); }
+    __device__ uint32_t io_empty(int s) const { return at(15 + 2 * a_stages + 2 * r_stages + s); }
+    static int count(int a, int r) { return 15 + 2 * a + 3 * r; }
+};
+
+// Own halo tile of pair tile `pt`: tile 2*pt + rank of the halo tiling (full
+// image width, th rows of tg images).  Past the last tile the origin lies
+// beyond the batch: loads read zeros and nothing is stored.
+__device__ __forceinline__ void chain_origin(const ChainPlan &p, int mt, int &h0, int &b0)
+{
+    h0 = (mt % p.nTh) * p.th;
+    b0 = (mt / p.nTh) * p.tg;
+}
+
+// Requantisation of 32 accumulators in the form chosen for the layer.
+template <bool kRes>
+__device__ __forceinline__ void requant_any(int mode, const uint32_t *v, const int32_t *cm,
+                                            const long long *cC, const uint32_t *rw, int m_r,
+                                            int S, int mr2, const uint32_t (&rsel)[4],
+                                            uint32_t *ow)
+{
+    if (mode == 2)
+        requant_hi32<kRes, true, false, 8>(v, cm, reinterpret_cast<const int32_t *>(cC), rw, mr2,
+                                           rsel, ow);
+    else if (mode == 1)
+        requant_fast<kRes, 8>(v, cm, cC, rw, mr2, rsel, ow);
+    else
+        requant32<kRes>(v, cm, cC, rw, m_r, S, ow);
+}
+
+// Per-layer constants of the chosen form into shared memory (see the
+// convolution kernel's prologue): mode 2: m*2^(33-S) and the bias; mode 1:
+// m*2^(32-S) and bias*m' + 2^31; mode 0: m and bias*m + 2^(S-1).
+__device__ __forceinline__ int pick_form(const int32_t *bias, const int32_t *mult, int n, int m_r,
+                                         int S, int K, bool res)
+{
+    bool fast = true, hi = true;
+    for (int o = threadIdx.x; o < n; o += blockDim.x) {
+        fast = fast && fast_form_ok(mult[o], bias[o], m_r, S, K, res);
+        hi = hi && hi32_ok(mult[o], bias[o], S, K);
+    }
+    const bool all_fast = __syncthreads_and(fast ? 1 : 0) != 0;
+    const bool all_hi = __syncthreads_and(hi ? 1 : 0) != 0 && hi32_layer_ok(m_r, S, res);
+    return all_hi ? 2 : (all_fast ? 1 : 0);
+}
+
+__device__ __forceinline__ void fill_consts(int mode, const int32_t *bias, const int32_t *mult,
+                                            int n, int S, int32_t *cm, long long *cC)
+{
+    int32_t *cb = reinterpret_cast<int32_t *>(cC);
+    for (int o = threadIdx.x; o < n; o += blockDim.x) {
+        const long long mm = mult[o];
+        if (mode == 2) {
+            cm[o] = static_cast<int32_t>(mm * (1ll << (33 - S)));
+            cb[o] = bias[o];
+        } else if (mode == 1) {
+            const long long mp = mm * (1ll << (32 - S));
+            cm[o] = static_cast<int32_t>(mp);
+            cC[o] = static_cast<long long>(bias[o]) * mp + (1ll << 31);
+        } else {
+            cm[o] = static_cast<int32_t>(mm);
+            cC[o] = static_cast<long long>(bias[o]) * mm + (1ll << (S - 1));
+        }
+    }
+}
+
+// Shortcut operands of the chosen Conv3 form (see the convolution kernel).
+__device__ __forceinline__ int shortcut_operands(int mode, int m_r, int S, uint32_t (&rsel)[4])
+{
+    const int sh = 32 - S;
+    const int k8 = mode >= 2 ? 0 : (sh < 0 ? 0 : (sh / 8 < 3 ? sh / 8 : 3));
+    const int mr2 =
+        mode == 1 ? static_cast<int>(static_cast<long long>(m_r) * (1ll << (sh - 8 * k8)))
+                  : (mode >= 2 ? static_cast<int>(static_cast<long long>(m_r) / (1ll << (S - 1)))
+                               : 0);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        uint32_t sel = 0;
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t nib = i < k8 ? 4u : (i == k8 ? static_cast<uint32_t>(b) : 8u | b);
+            sel |= nib << (4 * i);
+        }
+        rsel[b] = sel;
+    }
+    return mr2;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chain23_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW2,
+                   const __grid_constant__ CUtensorMap tmW3,
+                   const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmO,
+                   const int32_t *__restrict__ b2, const int32_t *__restrict__ m2,
+                   const int32_t *__restrict__ b3, const int32_t *__restrict__ m3,
+                   const ChainPlan p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_misc + 4);
+    ChainBars bars{sbase + static_cast<uint32_t>(p.off_bar), p.a_stages, p.r_stages};
+    const WaitCtl ctl{abort_flag, &g_dev_status, p.wait_limit_ns};
+    const uint64_t drain_ns = 200000000ull;
+    const int pair0 = blockIdx.x / 2;
+    const int pair_step = gridDim.x / 2;
+    const int n_my = pair0 < p.n_pairs ? (p.n_pairs - pair0 + pair_step - 1) / pair_step : 0;
+
+    // ---- set-up -----------------------------------------------------------------
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bars.w_full(), 1);
+        mbar_init(bars.mma_done(), 1);
+        mbar_init(bars.exit_bar(), 1);
+        for (int s = 0; s < p.a_stages; ++s) {
+            mbar_init(bars.a_full(s), 1);
+            mbar_init(bars.a_empty(s), 1);
+        }
+        // Arrival counts: commits arrive once (multicast to both CTAs); the
+        // epilogue barriers on rank 0 take one arrival per warp of a lane
+        // quarter from each CTA (4 x 2).
+        mbar_init(bars.acc2_full(), 1);
+        mbar_init(bars.acc2_empty(), 8);
+        for (int k = 0; k < kA3Bufs; ++k) {
+            mbar_init(bars.a3_full(k), 8);
+            mbar_init(bars.a3_empty(k), 1);
+        }
+        for (int k = 0; k < kAcc3; ++k) {
+            mbar_init(bars.acc3_full(k), 1);
+            mbar_init(bars.acc3_empty(k), 8);
+        }
+        for (int s = 0; s < p.r_stages; ++s) {
+            mbar_init(bars.io_full(s), 1);
+            mbar_init(bars.out_ready(s), 4);
+            mbar_init(bars.io_empty(s), 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmW2);
+        tma_prefetch_desc(&tmW3);
+        tma_prefetch_desc(&tmR);
+        tma_prefetch_desc(&tmO);
+    }
+    // Exact forms of the two layers (every CTA takes the same decision).
+    int32_t *cm2 = reinterpret_cast<int32_t *>(smem + p.off_cm2);
+    long long *cc2 = reinterpret_cast<long long *>(smem + p.off_cc2);
+    int32_t *cm3 = reinterpret_cast<int32_t *>(smem + p.off_cm3);
+    long long *cc3 = reinterpret_cast<long long *>(smem + p.off_cc3);
+    const int mode2 = pick_form(b2, m2, p.Cm, 0, p.S, 9 * p.Cm, false);
+    const int mode3 = pick_form(b3, m3, p.Cout, p.m_r, p.S, p.Cm, true);
+    fill_consts(mode2, b2, m2, p.Cm, p.S, cm2, cc2);
+    fill_consts(mode3, b3, m3, p.Cout, p.S, cm3, cc3);
+    if (threadIdx.x == 0)
+        atomicOr(&g_dev_forms, (1u << mode2) | (1u << mode3));
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish_pair();
+        tc_fence_before();
+    }
+    __syncthreads();
+    // Both CTAs' barriers are initialised and their TMEM allocated before any
+    // traffic crosses between them.
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- producer: weight halves, then halo tiles --------------------------------
+        if (lane == 0) {
+            const uint32_t wfull0 = mapa_shared(bars.w_full(), 0);
+            const int half = static_cast<int>(rank) * kHalfRows;
+            const uint32_t w2_bytes = 9 * p.C1 * kHalfRows * 32;
+            const uint32_t w3_bytes = p.n_chunks * p.C1 * kHalfRows * 32;
+            if (leader)  // both CTAs' halves complete on rank 0's barrier
+                mbar_arrive_expect_tx(bars.w_full(), 2 * (w2_bytes + w3_bytes));
+            for (int kb = 0; kb < 9 * p.C1; ++kb)
+                tma2_load_4d(sbase + p.off_w2 + kb * kHalfRows * 32, &tmW2, wfull0, 0, half, kb,
+                             0);
+            for (int c = 0; c < p.n_chunks; ++c)
+                for (int kb = 0; kb < p.C1; ++kb)
+                    tma2_load_4d(sbase + p.off_w3 + (c * p.C1 + kb) * kHalfRows * 32, &tmW3,
+                                 wfull0, 0, half, kb, c);
+            const uint32_t abytes = static_cast<uint32_t>(2 * 16 * p.plane_m * p.tg);
+            const uint64_t pol = policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_my; ++i) {
+                const int mt = 2 * (pair0 + i * pair_step) + static_cast<int>(rank);
+                int h0, b0;
+                chain_origin(p, mt, h0, b0);
+                for (int c1 = 0; c1 < p.C1; ++c1) {
+                    if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader)
+                        mbar_arrive_expect_tx(bars.a_full(stage), 2 * abytes);
+                    const uint32_t slot = sbase + p.off_a + stage * p.a_slot;
+                    const uint32_t full0 = mapa_shared(bars.a_full(stage), 0);
+                    tma2_load_5d_hint(slot, &tmA, full0, 0, -1, h0 - 1, c1, b0, pol);
+                    tma2_load_5d_hint(slot + p.a_half, &tmA, full0, 16, -1, h0 - 1, c1, b0, pol);
+                    if (++stage == p.a_stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---- shortcut stages (own rows) ------------------------------------------------
+        if (lane == 0) {
+            const uint32_t rbytes = static_cast<uint32_t>(kRChunks * p.rows * 32);
+            const uint64_t pol = policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_my; ++i) {
+                const int mt = 2 * (pair0 + i * pair_step) + static_cast<int>(rank);
+                int h0, b0;
+                chain_origin(p, mt, h0, b0);
+                for (int c = 0; c < p.n_chunks; ++c) {
+                    if (!mbar_wait(bars.io_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
+                    const uint32_t dst = sbase + p.off_r + stage * kRSlotBytes;
+                    if (p.io_swz)
+                        tma_load_5d_hint(dst, &tmR, bars.io_full(stage), 0, 0, h0, c * kRChunks,
+                                         b0, pol);
+                    else
+                        tma_load_4d_hint(dst, &tmR, bars.io_full(stage), 0, h0, c * kRChunks, b0,
+                                         pol);
+                    ++issued;
+                    if (++stage == p.r_stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            const long long last = issued < p.r_stages ? issued : p.r_stages;
+            for (long long k = issued - last; k < issued; ++k)
+                if (!mbar_drain(bars.io_full(static_cast<int>(k % p.r_stages)),
+                                static_cast<uint32_t>((k / p.r_stages) & 1), drain_ns))
+                    atomicOr(&g_dev_status, kDevDrainFailed);
+        }
+        __syncwarp();
+    } else if (warp == 3) {
+        // ---- stores of finished output stages (own rows) -------------------------------
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_my; ++i) {
+                const int mt = 2 * (pair0 + i * pair_step) + static_cast<int>(rank);
+                int h0, b0;
+                chain_origin(p, mt, h0, b0);
+                for (int c = 0; c < p.n_chunks; ++c) {
+                    if (!mbar_wait(bars.out_ready(stage), phase, ctl, kDevTimeoutProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t src = sbase + p.off_r + stage * kRSlotBytes;
+                    if (mt < p.num_m_tiles) {
+                        if (p.io_swz)
+                            tma_store_5d_hint(&tmO, src, 0, 0, h0, c * kRChunks, b0, pol);
+                        else
+                            tma_store_4d_hint(&tmO, src, 0, h0, c * kRChunks, b0, pol);
+                        bulk_commit();
+                        bulk_wait_read<0>();
+                    }
+                    mbar_arrive(bars.io_empty(stage));
+                    if (++stage == p.r_stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            bulk_wait_all();
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---- MMA issuer (rank 0) -------------------------------------------------------
+        if (leader) {
+            const uint32_t idesc = idesc_i8(256, 128);
+            const uint64_t a_desc0 =
+                smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half));
+            const uint64_t w2_desc0 = smem_desc_sw32(sbase + p.off_w2);
+            const uint64_t w3_desc0 = smem_desc_sw32(sbase + p.off_w3);
+            const uint64_t a3_desc0 = smem_desc_rows16(sbase + p.off_a3, kA3Bytes / 8);
+            const uint32_t kb_step = (kHalfRows * 32) >> 4;      // next K block of a weight half
+            const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
+            const uint32_t a3_kb_step = (kA3Bytes / 4) >> 4;     // next K block of an A buffer
+            const uint32_t a3_buf_step = kA3Bytes >> 4;
+            const uint32_t hp = static_cast<uint32_t>(p.row_pitch);
+            int st = 0;
+            uint32_t ph = 0;
+            uint64_t sd = a_desc0;
+            int n3_slot = 0;        // Conv3 accumulator slot of the next chunk
+            uint32_t n3_phase = 0;  // and its use parity
+            bool ok = __all_sync(0xffffffffu, mbar_wait_cl(bars.w_full(), 0, ctl, kDevTimeoutMma));
+            for (int i = 0; ok && i <= n_my; ++i) {
+                if (i < n_my) {
+                    // Conv2 of pair tile i (TMEM columns 0-127): 4 channel blocks x 9 taps,
+                    // once the Conv2 epilogue has drained tile i - 1.
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait_cl(bars.acc2_empty(), (i & 1) ^ 1u, ctl,
+                                                 kDevTimeoutMma))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base;
+                    for (int c1 = 0; c1 < p.C1; ++c1) {
+                        if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.a_full(st), ph, ctl,
+                                                                  kDevTimeoutMma))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int t = 0; t < 9; ++t)
+                            mma_i8_pair(d, sd + (t / 3) * hp + (t % 3),
+                                        w2_desc0 + static_cast<uint64_t>(t * p.C1 + c1) * kb_step,
+                                        idesc, (c1 | t) ? 1u : 0u);
+                        mma_commit_pair(bars.a_empty(st));
+                        if (++st == p.a_stages) {
+                            st = 0;
+                            ph ^= 1u;
+                            sd = a_desc0;
+                        } else {
+                            sd += a_slot_step;
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    mma_commit_pair(bars.acc2_full());
+                }
+                if (i >= 1) {
+                    // Conv3 of pair tile i - 1: A = its Conv2 result (buffer (i-1) % 2).
+                    const int j = i - 1, b = j & 1;
+                    if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.a3_full(b), (j >> 1) & 1, ctl,
+                                                              kDevTimeoutMma))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = a3_desc0 + static_cast<uint64_t>(b) * a3_buf_step;
+                    for (int c = 0; c < p.n_chunks; ++c) {
+                        // chunk n3 -> slot n3 % 3 (TMEM columns 128 + 128 * slot)
+                        const int k = n3_slot;
+                        if (!__all_sync(0xffffffffu,
+                                        mbar_wait_cl(bars.acc3_empty(k), n3_phase ^ 1u, ctl,
+                                                     kDevTimeoutMma))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d = tmem_base + static_cast<uint32_t>(128 + k * 128);
+                        for (int kb = 0; kb < p.C1; ++kb)
+                            mma_i8_pair(d, ad + static_cast<uint64_t>(kb) * a3_kb_step,
+                                        w3_desc0 +
+                                            static_cast<uint64_t>(c * p.C1 + kb) * kb_step,
+                                        idesc, kb ? 1u : 0u);
+                        mma_commit_pair(bars.acc3_full(k));
+                        if (++n3_slot == kAcc3) {
+                            n3_slot = 0;
+                            n3_phase ^= 1u;
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    mma_commit_pair(bars.a3_empty(b));
+                }
+            }
+            mma_commit_pair(bars.mma_done());
+            if (lane == 0 && !mbar_drain(bars.mma_done(), 0, drain_ns))
+                atomicOr(&g_dev_status, kDevDrainFailed);
+        }
+        __syncwarp();
+    } else if (warp >= kE1Warp0) {
+        // ---- Conv2 epilogue: accumulator -> int8 -> this CTA's Conv3 A buffer ------
+        // One warp per lane quarter takes every tile, so it sees every phase of
+        // the Conv2 accumulator and of both A buffers in order.
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t e2_0 = mapa_shared(bars.acc2_empty(), 0);
+        uint32_t rsel[4] = {0, 0, 0, 0};
+        for (int i = 0; i < n_my; ++i) {
+            const int b = i & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(bars.acc2_full(), static_cast<uint32_t>(i & 1),
+                                                   ctl, kDevTimeoutEpilogue)))
+                break;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(bars.a3_empty(b), static_cast<uint32_t>((i >> 1) & 1) ^ 1u,
+                                      ctl, kDevTimeoutEpilogue)))
+                break;
+            tc_fence_after();
+            uint8_t *a3 = smem + p.off_a3 + b * kA3Bytes;
+            const uint32_t tb = tmem_base + lane_addr;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32], ow[8];
+                __syncwarp();
+                tmem_ld_32x32b_x32_sync(tb + static_cast<uint32_t>(c * 32), v);
+                requant_any<false>(mode2, v, cm2 + c * 32, cc2 + c * 32, nullptr, 0, p.S, 0, rsel,
+                                   ow);
+                // K block c of the A buffer: two 16-byte halves, rows 16 bytes apart.
+                uint4 *dst = reinterpret_cast<uint4 *>(a3 + c * (kA3Bytes / 4) + row * 16);
+                dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                dst[(kA3Bytes / 8) / 16] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+            }
+            fence_proxy_async_smem();  // the MMA (async proxy, issued by rank 0) reads it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_cluster(e2_0);
+                mbar_arrive_cluster(mapa_shared(bars.a3_full(b), 0));
+            }
+        }
+    } else {
+        // ---- Conv3 epilogue: shortcut Sum + requantisation into the output stage --------
+        const int q = warp & 3;
+        const int turn = (warp - kE2Warp0) >> 2;  // owns Conv3 slot `turn`
+        const int row = q * 32 + lane;
+        const int plane_t = p.tw * p.th;
+        const int xi = row % p.row_pitch;
+        const int yi = (row % p.plane_m) / p.row_pitch;
+        const int gi = row / p.plane_m;
+        const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
+        const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
+        const int chunk_stride = plane_t * 32;
+        const int swz_mask = p.io_swz ? 0x70 : 0;
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t e3_0 = mapa_shared(bars.acc3_empty(turn), 0);
+        uint32_t rsel[4];
+        const int mr2 = shortcut_operands(mode3, p.m_r, p.S, rsel);
+        const long long total = static_cast<long long>(n_my) * p.n_chunks;
+        for (long long n = turn; n < total; n += kAcc3) {
+            const int c = static_cast<int>(n % p.n_chunks);
+            const int st = static_cast<int>(n % p.r_stages);
+            const uint32_t st_phase = static_cast<uint32_t>((n / p.r_stages) & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(bars.acc3_full(turn),
+                                                   static_cast<uint32_t>((n / kAcc3) & 1), ctl,
+                                                   kDevTimeoutEpilogue)))
+                break;
+            tc_fence_after();
+            // The stage's previous use (stage n - r_stages, another turn's) must be
+            // complete before its arrival is awaited: wait until it was stored, as
+            // the producer does (exact with at least as many stages as turns).
+            if (!__all_sync(0xffffffffu, mbar_wait(bars.io_empty(st), st_phase ^ 1u, ctl,
+                                                   kDevTimeoutEpilogue)))
+                break;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(bars.io_full(st), st_phase, ctl, kDevTimeoutEpilogue)))
+                break;
+            const uint32_t tb = tmem_base + lane_addr + static_cast<uint32_t>(128 + turn * 128);
+            uint8_t *stage = smem + p.off_r + st * kRSlotBytes;
+#pragma unroll 1
+            for (int cs = 0; cs < kRChunks; ++cs) {
+                const int ch = c * 128 + cs * 32;
+                uint32_t v[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32_sync(tb + static_cast<uint32_t>(cs * 32), v);
+                const int o = row_off + cs * chunk_stride;
+                const int sw = swz_mask & (o >> 3);
+                uint4 *pa = reinterpret_cast<uint4 *>(stage + (o ^ sw));
+                uint4 *pb = reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw));
+                const uint4 ra = *pa, rb = *pb;
+                const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+                uint32_t ow[8];
+                requant_any<true>(mode3, v, cm3 + ch, cc3 + ch, rw, p.m_r, p.S, mr2, rsel, ow);
+                if (in_box) {
+                    *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bars.out_ready(st));
+                mbar_arrive_cluster(e3_0);
+            }
+        }
+    }
+
+    // ---- tear-down: neither CTA leaves while the other may still reach it ----------
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_cluster(mapa_shared(bars.exit_bar(), rank ^ 1u));
+        if (!mbar_drain(bars.exit_bar(), 0, 2 * p.wait_limit_ns + drain_ns))
+            atomicOr(&g_dev_status, kDevDrainFailed);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+// ---- host side --------------------------------------------------------------
+
+int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r)
+{
+    std::memset(&p, 0, sizeof(p));
+    // The fused form: one 128-channel Conv2 (its output is Conv3's whole K), a
+    // halo tile row that fits the 128 GEMM rows, and output rows that the I/O
+    // maps can move whole (4-pixel groups, or rows of at most 256 8-byte units).
+    if (Cm != 128 || Cout < 128 || Cout % 128 || Cout > 1024 || W + 2 > kTileRows || H < 1 ||
+        W < 1 || B < 1)
+        return X1CB_ERR_SHAPE;
+    if (W % 4 != 0 && 4 * W > 256)
+        return X1CB_ERR_SHAPE;
+    p.B = B;
+    p.H = H;
+    p.W = W;
+    p.Cm = Cm;
+    p.Cout = Cout;
+    p.S = S;
+    p.m_r = m_r;
+    p.C1 = Cm / 32;
+    p.n_chunks = Cout / 128;
+    choose_halo_tile(B, H, W, p.th, p.tg);
+    p.tw = W;
+    p.row_pitch = W + 2;
+    p.plane_m = (p.th + 2) * (W + 2);
+    const int need_rows = std::max(p.tg * p.plane_m, kTileRows + 2 * p.row_pitch + 2);
+    p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+    p.a_slot = (2 * p.a_half + 1023) / 1024 * 1024;
+    p.rows = p.tw * p.th * p.tg;
+    p.nTh = (H + p.th - 1) / p.th;
+    p.nTg = (B + p.tg - 1) / p.tg;
+    const long long tiles = static_cast<long long>(p.nTh) * p.nTg;
+    if (tiles > INT_MAX / 4)
+        return X1CB_ERR_SHAPE;
+    p.num_m_tiles = static_cast<int>(tiles);
+    p.n_pairs = (p.num_m_tiles + 1) / 2;
+    p.io_swz = W % 4 == 0 ? 1 : 0;
+
+    const int w2_bytes = 9 * p.C1 * kHalfRows * 32;
+    const int w3_bytes = p.n_chunks * p.C1 * kHalfRows * 32;
+    auto layout = [&](int a, int r) {
+        p.a_stages = a;
+        p.r_stages = r;
+        p.off_w2 = 0;
+        p.off_w3 = w2_bytes;
+        p.off_a3 = (p.off_w3 + w3_bytes + 1023) / 1024 * 1024;
+        p.off_a = p.off_a3 + kA3Bufs * kA3Bytes;
+        p.off_r = p.off_a + a * p.a_slot;
+        p.off_cm2 = p.off_r + r * kRSlotBytes;
+        p.off_cc2 = p.off_cm2 + p.Cm * 4;
+        p.off_cm3 = p.off_cc2 + p.Cm * 8;
+        p.off_cc3 = p.off_cm3 + p.Cout * 4;
+        p.off_bar = (p.off_cc3 + p.Cout * 8 + 7) & ~7;
+        p.off_misc = p.off_bar + ChainBars::count(a, r) * 8;
+        p.smem_bytes = p.off_misc + 16 + 1024;
+        return p.smem_bytes <= kSmemLimit;
+    };
+    // Deepest shortcut ring beside at least four halo slots (fewer if needed).
+    // (the shortcut ring needs at least one stage per Conv3 epilogue turn)
+    bool placed = false;
+    for (int a = 4; a >= 2 && !placed; --a)
+        for (int r = 8; r >= kAcc3 && !placed; --r)
+            placed = layout(a, r);
+    if (!placed)
+        return X1CB_ERR_SHAPE;
+    p.grid = 2 * std::max(1, std::min(74, p.n_pairs));
+    p.wait_limit_ns = 2000000000ull;
+    return X1CB_OK;
+}
+
+int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const int32_t *b2,
+                 const int32_t *m2, const int8_t *w3, const int32_t *b3, const int32_t *m3,
+                 const int8_t *x, int8_t *out, cudaStream_t stream)
+{
+    CUtensorMap tmA, tmW2, tmW3, tmR, tmO;
+    {  // Conv2 input, halo form: dims (32, W, H, C1, B), box (16, W+2, th+2, 1, tg)
+        const uint64_t dims[5] = {32, (uint64_t)p.W, (uint64_t)p.H, (uint64_t)p.C1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {32, (uint64_t)p.W * 32, (uint64_t)p.H * p.W * 32,
+                                 (uint64_t)p.C1 * p.H * p.W * 32};
+        const uint32_t box[5] = {16, (uint32_t)p.row_pitch, (uint32_t)(p.th + 2), 1,
+                                 (uint32_t)p.tg};
+        if (int e = encode_map(&tmA, y1, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return e;
+    }
+    {  // Conv2 weights [1][9*C1][128][32]: one CTA's half = 64 rows of a K block
+        const uint64_t dims[4] = {32, 128, (uint64_t)(9 * p.C1), 1};
+        const uint64_t str[3] = {32, 4096, (uint64_t)(9 * p.C1) * 4096};
+        const uint32_t box[4] = {32, kHalfRows, 1, 1};
+        if (int e = encode_map(&tmW2, w2, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
+            return e;
+    }
+    {  // Conv3 weights [Cout/128][C1][128][32]
+        const uint64_t dims[4] = {32, 128, (uint64_t)p.C1, (uint64_t)p.n_chunks};
+        const uint64_t str[3] = {32, 4096, (uint64_t)p.C1 * 4096};
+        const uint32_t box[4] = {32, kHalfRows, 1, 1};
+        if (int e = encode_map(&tmW3, w3, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
+            return e;
+    }
+    const uint64_t O1 = p.Cout / 32;
+    if (p.io_swz) {  // 128-byte rows of 4 pixels: (16 x 8 B, W/4, H, O1, B)
+        const uint64_t dims[5] = {16, (uint64_t)p.W / 4, (uint64_t)p.H, O1, (uint64_t)p.B};
+        const uint64_t str[4] = {128, (uint64_t)p.W * 32, (uint64_t)p.H * p.W * 32,
+                                 O1 * p.H * p.W * 32};
+        const uint32_t box[5] = {16, (uint32_t)p.W / 4, (uint32_t)p.th, (uint32_t)kRChunks,
+                                 (uint32_t)p.tg};
+        if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+            return e;
+        if (int e = encode_map(&tmR, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+            return e;
+    } else {  // whole rows of W*32 bytes as 8-byte units: (4W, H, O1, B)
+        const uint64_t dims[4] = {(uint64_t)p.W * 4, (uint64_t)p.H, O1, (uint64_t)p.B};
+        const uint64_t str[3] = {(uint64_t)p.W * 32, (uint64_t)p.H * p.W * 32,
+                                 O1 * p.H * p.W * 32};
+        const uint32_t box[4] = {(uint32_t)p.W * 4, (uint32_t)p.th, (uint32_t)kRChunks,
+                                 (uint32_t)p.tg};
+        if (int e = encode_map(&tmO, out, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+            return e;
+        if (int e = encode_map(&tmR, x, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+            return e;
+    }
+    if (int e = opt_in_smem(reinterpret_cast<const void *>(chain23_kernel), 2))
+        return e;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(p.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = p.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, chain23_kernel, tmA, tmW2, tmW3, tmR, tmO, b2, m2, b3, m3, p) !=
+        cudaSuccess)
+        return X1CB_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+}  // namespace x1cb

@@ -47,6 +47,7 @@
 
 #include "x1cb_internal.h"
 #include "x1cb_plan.h"
+#include "x1cb_epi.cuh"
 #include "x1cb_ptx.cuh"
 
 namespace x1cb {
@@ -91,162 +92,6 @@ __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, 
     w0 = iw * p.tw;
     h0 = ih * p.th;
     b0 = ig * p.tg;
-}
-
-// Generic exact requantisation of 32 accumulators of one pixel (channels
-// n0..n0+31 of this CTA's group), packed as 32 int8 bytes:
-//   t = acc*m + C (+ r*m_r),  C = bias*m + 2^(S-1),  y = clamp(t >> S, 0, 127).
-template <bool kRes>
-__device__ __forceinline__ void requant32(const uint32_t *v, const int32_t *cm,
-                                          const long long *cC, const uint32_t *rw, int m_r,
-                                          int S, uint32_t *ow)
-{
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-        ow[q] = 0u;
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-        long long t = static_cast<long long>(static_cast<int>(v[k])) * cm[k] + cC[k];
-        if (kRes) {
-            const int r = static_cast<int>(static_cast<int8_t>((rw[k >> 2] >> (8 * (k & 3))) & 0xFF));
-            t += static_cast<long long>(r) * m_r;
-        }
-        const long long y = t >> S;  // arithmetic shift: floor(t / 2^S)
-        const int yc = y < 0 ? 0 : (y > 127 ? 127 : static_cast<int>(y));
-        ow[k >> 2] |= static_cast<uint32_t>(yc) << (8 * (k & 3));
-    }
-}
-
-// Exact fast form of the same requantisation, used when the CTA's constants
-// allow it (checked in the prologue).  With s = 32 - S >= 0 every term is
-// pre-scaled by 2^s: m' = m*2^s, C' = bias*m' + 2^31, and the residual term
-// becomes (r*2^(8*k8)) * (m_r*2^(s - 8*k8)).  Then
-//     t' = acc*m' + C' + r*m_r*2^s = t * 2^s,
-// so floor(t / 2^S) = floor(t' / 2^32) is exactly the high word of t' (no
-// shift, no 64-bit compare).  All three products fit their 32-bit operands and
-// the sum stays below 2^63 (prologue check), so nothing is approximated.
-// Processes n4 groups of 4 channels.
-template <bool kRes, int kGroups>
-__device__ __forceinline__ void requant_fast(const uint32_t *v, const int32_t *cm,
-                                             const long long *cC, const uint32_t *rw, int mr2,
-                                             const uint32_t (&rsel)[4], uint32_t *ow)
-{
-    const int4 *m4 = reinterpret_cast<const int4 *>(cm);
-    const longlong2 *c2 = reinterpret_cast<const longlong2 *>(cC);
-#pragma unroll
-    for (int q = 0; q < kGroups; ++q)
-        ow[q] = requant4_fast<kRes>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], m4[q],
-                                    c2[2 * q], c2[2 * q + 1], kRes ? rw[q] : 0u, rsel, mr2);
-}
-
-// Exact all-32-bit form, used when the shortcut multiplier is a multiple of
-// 2^(S-1) (m_r = k * 2^(S-1)) and the CTA's constants allow it.  With
-// s = 33 - S >= 0 and m' = m * 2^s, every term of t * 2^s except the product
-// is a multiple of 2^32:
-//     t * 2^s = (acc + bias) * m' + 2^32 * (1 + r*k),
-// so y2 = floor(t * 2^s / 2^32) = hi32((acc + bias) * m') + 1 + r*k exactly
-// (mad.hi), and floor(t / 2^S) = floor(y2 / 2); clamping y2 to [0, 255]
-// before halving gives the [0, 127] clamp.  No 64-bit arithmetic.
-template <bool kRes, bool kAddBias, bool kK1, int kGroups>
-__device__ __forceinline__ void requant_hi32(const uint32_t *v, const int32_t *cm,
-                                             const int32_t *cb, const uint32_t *rw, int k,
-                                             const uint32_t (&rsel)[4], uint32_t *ow)
-{
-    const int4 *m4 = reinterpret_cast<const int4 *>(cm);
-    const int4 *b4 = reinterpret_cast<const int4 *>(cb);
-#pragma unroll
-    for (int q = 0; q < kGroups; ++q)
-        ow[q] = requant4_hi32<kRes, kAddBias, kK1>(v[4 * q], v[4 * q + 1], v[4 * q + 2],
-                                              v[4 * q + 3], m4[q],
-                                              kAddBias ? b4[q] : make_int4(0, 0, 0, 0),
-                                              kRes ? rw[q] : 0u, rsel, k);
-}
-
-// Bias folded into the MMA: one extra K step of 32 columns adds
-//   sum_c A[c] * D_n[c] = bias[n]
-// to every row of the accumulator, with the constant A row
-//   [1, 127 x 15, 1, 127 x 15]
-// and per-channel int8 digits D_n: D_n[0] = bias mod 127 (centred), the other
-// 30 digits (columns 1-15, 17-31) carry (bias - D_n[0]) / 127 in steps of at
-// most 127 in magnitude, D_n[16] = 0.  Exact for |bias| <= 30*127*127 + 63;
-// used for |bias| <= 2^18.  Because the two 16-byte halves of the A row are
-// equal, the sum does not depend on which half of a 32-byte row the 32-byte
-// swizzle presents first, so both tiles are written without swizzling.
-constexpr int kBiasFoldMax = 1 << 18;
-
-__device__ __forceinline__ void bias_digits(int bias, uint32_t (&w)[8])
-{
-    int8_t d[32];
-    const int d0 = ((bias + 63) % 127 + 127) % 127 - 63;  // bias mod 127 in [-63, 63]
-    int D = (bias - d0) / 127;
-    d[0] = static_cast<int8_t>(d0);
-    d[16] = 0;
-#pragma unroll
-    for (int c = 1; c < 32; ++c) {
-        if (c == 16)
-            continue;
-        const int step = D > 127 ? 127 : (D < -127 ? -127 : D);
-        d[c] = static_cast<int8_t>(step);
-        D -= step;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        w[i] = static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i])) |
-               static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i + 1])) << 8 |
-               static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i + 2])) << 16 |
-               static_cast<uint32_t>(static_cast<uint8_t>(d[4 * i + 3])) << 24;
-}
-
-// Layer-wide conditions of the all-32-bit form (per channel: hi32_ok).
-__device__ __forceinline__ bool hi32_layer_ok(int m_r, int S, bool res)
-{
-    if (S < 2 || S > 33)
-        return false;
-    if (!res)
-        return true;
-    const long long q = 1ll << (S - 1);
-    if (static_cast<long long>(m_r) % q != 0)
-        return false;
-    // y2 = h + 1 + r*k with -2^30 <= h <= 2^30 - 1 and r in [-128, 127]
-    // stays inside int32 while -2^30 - 1 <= r*k <= 2^30 - 1: k = -2^23 with
-    // r = -128 would reach 2^31, so the lower bound is exclusive.
-    const long long k = static_cast<long long>(m_r) / q;
-    return k > -(1ll << 23) && k <= (1ll << 23);
-}
-
-// Per-channel conditions: m * 2^(33-S) fits int32, and acc + bias cannot
-// overflow int32 (|acc| <= K * 2^14).
-__device__ __forceinline__ bool hi32_ok(long long m, long long bias, int S, int K)
-{
-    if (S < 2 || S > 33)
-        return false;
-    const long long mp = m * (1ll << (33 - S));
-    if (mp < INT_MIN || mp > INT_MAX)
-        return false;
-    return (bias < 0 ? -bias : bias) + static_cast<long long>(K) * 16384 < (1ll << 31);
-}
-
-// Whether the fast form is exact for output channel o of a layer of fan-in K
-// (every |x|, |w| <= 128, so |acc| <= K * 2^14).
-__device__ __forceinline__ bool fast_form_ok(long long m, long long bias, int m_r, int S, int K,
-                                             bool res)
-{
-    if (S > 32)
-        return false;
-    const int sh = 32 - S;
-    const long long mp = m * (1ll << sh);
-    if (mp < INT_MIN || mp > INT_MAX)
-        return false;
-    double bound = static_cast<double>(K) * 16384.0 * fabs(static_cast<double>(mp)) +
-                   fabs(static_cast<double>(bias) * static_cast<double>(mp)) + 2147483648.0;
-    if (res) {
-        const int k8 = sh / 8 < 3 ? sh / 8 : 3;
-        const long long mr2 = static_cast<long long>(m_r) * (1ll << (sh - 8 * k8));
-        if (mr2 < INT_MIN || mr2 > INT_MAX)
-            return false;
-        bound += 128.0 * fabs(static_cast<double>(m_r)) * static_cast<double>(1ll << sh);
-    }
-    return bound < 4.0e18;  // < 2^62 with margin for the double rounding
 }
 
 // Epilogue of one warp.  For every tile of this CTA and every accumulator
@@ -564,17 +409,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- producer: resident weights, then activation K blocks ---------------
         if (lane == 0) {
             const uint32_t sw = sbase + p.off_w;
-            const uint32_t wbytes = static_cast<uint32_t>(p.kb_per_tile * p.NC * 32);
-            mbar_arrive_expect_tx(bars.w_full(), wbytes);
-            // The second source's weights (if any) follow the first's K blocks.
-            for (int kb = 0; kb < p.kb_per_tile; ++kb) {
-                if (kb < p.kb_a)
-                    tma_load_4d(sw + kb * p.NC * 32, &tmW, bars.w_full(), 0, 0, kb,
-                                group * (p.NC / 128));
-                else
-                    tma_load_4d(sw + kb * p.NC * 32, &tmW2, bars.w_full(), 0, 0, kb - p.kb_a,
-                                group * (p.NC / 128));
+            const int o1 = group * (p.NC / 128);
+            if (!p.wstream) {
+                const uint32_t wbytes = static_cast<uint32_t>(p.kb_per_tile * p.NC * 32);
+                mbar_arrive_expect_tx(bars.w_full(), wbytes);
+                // The second source's weights (if any) follow the first's K blocks.
+                for (int kb = 0; kb < p.kb_per_tile; ++kb) {
+                    if (kb < p.kb_a)
+                        tma_load_4d(sw + kb * p.NC * 32, &tmW, bars.w_full(), 0, 0, kb, o1);
+                    else
+                        tma_load_4d(sw + kb * p.NC * 32, &tmW2, bars.w_full(), 0, 0,
+                                    kb - p.kb_a, o1);
+                }
+            } else {
+                mbar_arrive(bars.w_full());  // weights travel with the activation stages
             }
+            // Streamed weights: bytes per stage, each K block NC rows x 32 bytes.
+            const uint32_t wpart = static_cast<uint32_t>(p.w_part);
+            const uint32_t wkb = static_cast<uint32_t>(p.NC * 32);
             // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
             // one filter tap), each a 128-row x 32-byte tile, back to back.
             const uint32_t abytes =
@@ -601,12 +453,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(bars.a_full(stage), abytes);
+                        mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
                         tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
                                          h0 - p.pad, c1, b0, pol);
                         tma_load_5d_hint(slot + static_cast<uint32_t>(p.a_half), &tmA,
                                          bars.a_full(stage), 16, w0 - p.pad, h0 - p.pad, c1, b0,
                                          pol);
+                        if (wpart) {  // the nine taps' weights of channel block c1
+                            const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
+                            for (int t = 0; t < 9; ++t)
+                                tma_load_4d(wdst + t * wkb, &tmW, bars.a_full(stage), 0, 0,
+                                            t * p.C1 + c1, o1);
+                        }
                         ++issued;
                         if (++stage == p.a_stages) {
                             stage = 0;
@@ -631,13 +489,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(bars.a_full(stage), abytes);
+                    mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
                     if (!second)
                         tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, wi0 + ds, hi0 + dr,
                                          b0, c1, pol);
                     else
                         tma_load_5d_hint(slot, &tmA2, bars.a_full(stage), 0, w0 * p.stride2,
                                          h0 * p.stride2, b0, c1, pol);
+                    if (wpart) {  // the box's K blocks' weights
+                        const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
+                        const int kb0 = second ? c1 : (dr * p.R + ds) * p.C1 + c1;
+                        for (int i = 0; i < p.a_kc; ++i) {
+                            if (!second)
+                                tma_load_4d(wdst + i * wkb, &tmW, bars.a_full(stage), 0, 0,
+                                            kb0 + i, o1);
+                            else
+                                tma_load_4d(wdst + i * wkb, &tmW2, bars.a_full(stage), 0, 0,
+                                            kb0 + i, o1);
+                        }
+                    }
                     ++issued;
                     if (++stage == p.a_stages) {
                         stage = 0;
@@ -774,6 +644,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 p.halo ? smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half))
                        : smem_desc_sw32(sbase + p.off_a);
             const uint64_t b_desc0 = smem_desc_sw32(sbase + p.off_w);
+            // Streamed weights: each ring stage carries its K blocks' weights
+            // right after its activation part (same 32-byte swizzle layout as the
+            // resident weights), so the stage's weight descriptor is the first
+            // stage's plus the stage offset.
+            const uint64_t w_desc0 = smem_desc_sw32(sbase + p.off_a + p.a_part);
             const uint64_t fold_a = smem_desc_sw32(sbase + p.off_ba);
             const uint64_t fold_b0 = smem_desc_sw32(sbase + p.off_bb);
             const uint32_t a_sub_step = static_cast<uint32_t>(p.rows * 32) >> 4;  // next K block in a box
@@ -785,7 +660,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Halo form: tap (dr, ds) reads the slot dr*row_pitch + ds rows on and
             // the weights of K block (dr*3 + ds)*C1 + c1.
             const uint32_t hp = static_cast<uint32_t>(p.row_pitch);
-            const uint64_t b_tap_step = static_cast<uint64_t>(p.C1) * b_kb_step;
+            // (streamed: the nine taps of one channel block are consecutive)
+            const uint64_t b_tap_step =
+                p.wstream ? b_kb_step : static_cast<uint64_t>(p.C1) * b_kb_step;
             const int n_slots = kTmemCols / p.nmma;
             int a_stage = 0;
             uint32_t a_phase = 0;
@@ -825,6 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         uint64_t ad = sd;
+                        if (p.wstream)  // this stage's own weights (one N slice: j == 0)
+                            bd = w_desc0 + (sd - a_desc0);
                         if (p.halo) {
 #pragma unroll
                             for (int t = 0; t < 9; ++t)
@@ -907,6 +786,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+}  // namespace
+
 // ---- host side --------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode()
@@ -927,8 +808,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode()
 // n * step elements along a strided dimension loads n of them.
 int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
                const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz,
-               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8,
-               const uint32_t *elem_strides = nullptr)
+               CUtensorMapDataType dtype, const uint32_t *elem_strides)
 {
     auto fn = get_encode();
     if (!fn)
@@ -971,7 +851,6 @@ int opt_in_smem(const void *kern, int which)
     return X1CB_OK;
 }
 
-}  // namespace
 
 // Choose the pixel tile: tw x th pixels of tg images, at most 128 GEMM rows.
 // Cost = MMA rows issued over the whole problem, with a mild penalty for
@@ -1137,22 +1016,27 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         if (work >= num_sms)
             break;
     }
-    if (chosen == 0)
-        return X1CB_ERR_SHAPE;  // weights of 128 output channels do not fit on chip
+    // When no resident copy fits (large fan-in), the weights are streamed:
+    // 128 output channels per CTA, each ring stage bringing its K blocks'
+    // weights from L2 next to its activations.
+    p.wstream = chosen == 0 ? 1 : 0;
+    if (p.wstream)
+        chosen = 128;
     p.NC = chosen;
     p.n_groups = Oc / p.NC;
     p.nmma = p.NC >= 256 ? 256 : 128;
     p.n_subs = p.NC / p.nmma;
 
-    const int wbytes = p.kb_per_tile * p.NC * 32;
+    const int wbytes = p.wstream ? 0 : p.kb_per_tile * p.NC * 32;
     // The activation ring budget: with a shortcut the I/O ring (shortcut in,
     // result out) needs the space -- its depth sets the bytes in flight -- so
     // about a tile's K blocks plus two; without one the activations are most
     // of the traffic and get up to 128 KB in flight while the I/O stages only
     // stage results.  The bias-fold tiles are reserved when the rings still
     // reach their minimum beside them.
-    const int a_bytes_want = has_res ? std::min(p.kb_per_tile + 2, 8) * kASlotBytes
-                                     : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
+    const int a_bytes_want = p.wstream ? 4 * 4 * kASlotBytes
+                             : has_res ? std::min(p.kb_per_tile + 2, 8) * kASlotBytes
+                                       : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
     // Several K blocks per activation box (fewer, larger copies) when each
     // K-block tile starts on a 256-byte swizzle atom (row count a multiple of
     // 8) and the ring's minimum still fits the budget.  With two accumulator
@@ -1169,9 +1053,11 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
             }
     // Halo form: one slot per channel block, all of a tile's blocks in the ring
     // when two accumulator slots share them; slots stay 1024-byte aligned.
-    p.a_slot = p.halo ? (2 * p.a_half + 1023) / 1024 * 1024 : p.a_kc * kASlotBytes;
+    p.a_part = p.halo ? (2 * p.a_half + 1023) / 1024 * 1024 : p.a_kc * kASlotBytes;
+    p.w_part = p.wstream ? (p.halo ? 9 : p.a_kc) * p.NC * 32 : 0;
+    p.a_slot = p.a_part + p.w_part;
     const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
-    const int a_want = std::max(a_min, a_bytes_want / p.a_slot);
+    const int a_want = std::max(a_min, p.wstream ? 4 : a_bytes_want / p.a_slot);
     const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 4;
     auto layout = [&](int fold, int a, int r) {
         p.fold_room = fold;

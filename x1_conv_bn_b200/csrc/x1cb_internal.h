@@ -1,5 +1,6 @@
 // Internal host-side interfaces between the API layer and the kernels.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -10,6 +11,12 @@
 namespace x1cb {
 
 void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg);
+void choose_halo_tile(int B, int H, int W, int &th, int &tg);
+int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
+               const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8,
+               const uint32_t *elem_strides = nullptr);
+int opt_in_smem(const void *kern, int which);
 int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
               int m_r, int num_sms);
 // Geometry beyond the plain stride-1 layer: the input image is Hin x Win and
@@ -25,6 +32,14 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
 int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32_t *bias,
                 const int32_t *mult, const int8_t *r, int8_t *out, cudaStream_t stream,
                 const int8_t *x2 = nullptr, const int8_t *w2 = nullptr);
+// Fused Conv2 -> Conv3: plan (X1CB_ERR_SHAPE when the shape has no fused
+// form) and launch.  y1 [B, Cm/32, H, W, 32] is Conv1's output, x the block
+// input (the shortcut), out the block output.
+int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r);
+int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const int32_t *b2,
+                 const int32_t *m2, const int8_t *w3, const int32_t *b3, const int32_t *m3,
+                 const int8_t *x, int8_t *out, cudaStream_t stream);
+
 unsigned int read_and_clear_dev_status(bool clear);
 unsigned int read_and_clear_dev_forms(bool clear);
 

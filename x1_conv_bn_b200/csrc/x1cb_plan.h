@@ -48,7 +48,13 @@ struct ConvPlan {
     int NC, n_groups, nmma, n_subs;
     int kb_per_tile;  // R*R*C1
     int a_kc;         // K blocks per activation TMA box (divides C1)
-    int a_slot;       // bytes per activation ring slot = a_kc * 4 KB
+    int a_slot;       // bytes per ring stage: activation part + streamed weights
+    int a_part;       // bytes of the activation part of a stage (a_kc * 4 KB, or the halo tile)
+    // Streamed weights (when a resident copy of NC channels does not fit):
+    // every stage also carries its K blocks' weights, w_part bytes right after
+    // the activation part (each K block NC rows x 32 bytes; the halo form: all
+    // nine taps of the stage's channel block).  0 = weights resident.
+    int wstream, w_part;
     // rings
     int a_stages, r_stages;
     // shared memory offsets from the 1024-aligned base
@@ -77,6 +83,23 @@ struct ConvPlan {
     int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
     unsigned long long wait_limit_ns;
     int grid;
+};
+
+// Launch plan of the fused Conv2 -> Conv3 kernel (pairs of CTAs; see
+// x1cb_chain.cu).  Conv2 is the 3x3 (pad 1, halo tiles of th rows x tg
+// images, full width); Conv3 the 1x1 with the shortcut.
+struct ChainPlan {
+    int B, H, W, Cm, Cout, S, m_r;
+    int C1, n_chunks;  // Cm/32 channel blocks, Cout/128 output chunks
+    int th, tg, tw, row_pitch, plane_m, a_half, rows;
+    int nTh, nTg, num_m_tiles, n_pairs;
+    int a_stages, a_slot, r_stages;
+    int off_w2, off_w3, off_a, off_a3, off_r, off_cm2, off_cc2, off_cm3, off_cc3, off_bar,
+        off_misc;
+    int smem_bytes;
+    int io_swz;  // output/shortcut stages in the 128-byte swizzle (else 8-byte-element rows)
+    int grid;    // CTAs (two per cluster)
+    unsigned long long wait_limit_ns;
 };
 
 }  // namespace x1cb
