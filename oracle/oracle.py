@@ -51,6 +51,8 @@ def lib():
                                        + [ctypes.c_int] * 8)
         L.x1o_conv_proj.argtypes = [c_i8p] * 6 + [ctypes.c_int, c_i8p] + [ctypes.c_int] * 9
         L.x1o_bottleneck_proj.argtypes = [c_i8p] * 11 + [ctypes.c_int, c_i8p] + [ctypes.c_int] * 6
+        L.x1o_maxpool3s2.argtypes = [c_i8p, c_i8p] + [ctypes.c_int] * 4
+        L.x1o_conv_pool.argtypes = [c_i8p] * 4 + [ctypes.c_int, c_i8p] + [ctypes.c_int] * 8
         L.x1o_set_threads.argtypes = [ctypes.c_int]
         L.x1o_set_threads.restype = ctypes.c_int
         _lib = L
@@ -96,7 +98,8 @@ def unpack_act(nc32: torch.Tensor) -> torch.Tensor:
 def pack_weight(oihw: torch.Tensor) -> torch.Tensor:
     Oc, Ic, R, _ = oihw.shape
     w = _cpu(oihw, torch.int8)
-    out = torch.empty((Oc // 128, R, R, Ic // 32, 128, 32), dtype=torch.int8)
+    O2 = min(Oc, 128)
+    out = torch.empty((Oc // O2, R, R, Ic // 32, O2, 32), dtype=torch.int8)
     lib().x1o_pack_weight(_p(w), _p(out), Oc, Ic, R)
     return out
 
@@ -211,4 +214,29 @@ def bottleneck_proj(x, ws, wp, bs, ms, S):
              _cpu(ms[2], torch.int32)]
     out = torch.empty((B, Ho, Wo, Cout), dtype=torch.int8)
     lib().x1o_bottleneck_proj(*[_p(a) for a in args], S, _p(out), B, H, W, Cin, Cmid, Cout)
+    return out
+
+
+def maxpool3s2(y):
+    """3x3 stride-2 max pooling (pad 1, padding never wins).  NHWC in and out."""
+    B, H, W, C = y.shape
+    y = _cpu(y, torch.int8)
+    out = torch.empty((B, out_extent(H, 3, 1, 2), out_extent(W, 3, 1, 2), C), dtype=torch.int8)
+    lib().x1o_maxpool3s2(_p(y), _p(out), B, H, W, C)
+    return out
+
+
+def conv_pool(x, w, bias, m, S, stride=2, pad=None):
+    """Stem: conv (R x R, pad (R-1)/2, stride) + BN + ReLU, then 3x3 stride-2
+    max pooling.  NHWC in and out."""
+    B, H, W, Ic = x.shape
+    Oc, _, R, _ = w.shape
+    pad = (R - 1) // 2 if pad is None else pad
+    Hc, Wc = out_extent(H, R, pad, stride), out_extent(W, R, pad, stride)
+    x, w = _cpu(x, torch.int8), _cpu(w, torch.int8)
+    bias, m = _cpu(bias, torch.int32), _cpu(m, torch.int32)
+    out = torch.empty((B, out_extent(Hc, 3, 1, 2), out_extent(Wc, 3, 1, 2), Oc),
+                      dtype=torch.int8)
+    lib().x1o_conv_pool(_p(x), _p(w), _p(bias), _p(m), S, _p(out), B, H, W, Ic, Oc, R, pad,
+                        stride)
     return out

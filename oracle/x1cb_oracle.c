@@ -88,13 +88,16 @@ static size_t nhwc_index(int64_t b, int64_t h, int64_t w, int64_t c, int64_t H, 
     return (size_t)(((b * H + h) * W + w) * C + c);
 }
 
-/* Blocked weight [O1, R, S, I1, O2=128, I2=32]: element (o, i, r, s).  For
- * R = S = 1 this is the article's [O1, I1, O2, I2]. */
-static size_t wblk_index(int64_t o, int64_t i, int64_t r, int64_t s, int64_t Ic, int64_t R)
+/* Blocked weight [O1, R, S, I1, O2, I2=32]: element (o, i, r, s).  O2 = 128
+ * (the article's block of output channels); a layer of fewer than 128 output
+ * channels (64: the network's stem) is one block of O2 = Oc.  For R = S = 1
+ * this is the article's [O1, I1, O2, I2]. */
+static size_t wblk_index(int64_t o, int64_t i, int64_t r, int64_t s, int64_t Ic, int64_t R,
+                         int64_t Oc)
 {
     int64_t I1 = Ic / 32;
-    return (size_t)((((((o / 128) * R + r) * R + s) * I1 + i / 32) * 128 + o % 128) * 32 +
-                    i % 32);
+    int64_t O2 = Oc < 128 ? Oc : 128;
+    return (size_t)((((((o / O2) * R + r) * R + s) * I1 + i / 32) * O2 + o % O2) * 32 + i % 32);
 }
 
 /* OIHW (PyTorch convolution weight order): element (o, i, r, s). */
@@ -127,7 +130,7 @@ void x1o_pack_weight(const int8_t *oihw, int8_t *blk, int Oc, int Ic, int R)
         for (int64_t i = 0; i < Ic; ++i)
             for (int64_t r = 0; r < R; ++r)
                 for (int64_t s = 0; s < R; ++s)
-                    blk[wblk_index(o, i, r, s, Ic, R)] = oihw[oihw_index(o, i, r, s, Ic, R)];
+                    blk[wblk_index(o, i, r, s, Ic, R, Oc)] = oihw[oihw_index(o, i, r, s, Ic, R)];
 }
 
 void x1o_unpack_weight(const int8_t *blk, int8_t *oihw, int Oc, int Ic, int R)
@@ -136,7 +139,7 @@ void x1o_unpack_weight(const int8_t *blk, int8_t *oihw, int Oc, int Ic, int R)
         for (int64_t i = 0; i < Ic; ++i)
             for (int64_t r = 0; r < R; ++r)
                 for (int64_t s = 0; s < R; ++s)
-                    oihw[oihw_index(o, i, r, s, Ic, R)] = blk[wblk_index(o, i, r, s, Ic, R)];
+                    oihw[oihw_index(o, i, r, s, Ic, R)] = blk[wblk_index(o, i, r, s, Ic, R, Oc)];
 }
 
 /* ---- the fused convolution ---------------------------------------------- */
@@ -374,6 +377,51 @@ void x1o_bottleneck_proj(const int8_t *x, const int8_t *w1, const int32_t *b1, c
     x1o_conv_proj(y2, w3, x, wp, b3, m3, S, out, B, (int)Ho, (int)Wo, Cmid, Cin, Cout, H, W, 2);
     free(y1);
     free(y2);
+}
+
+/* ---- the stem: convolution + BN + ReLU + max pooling --------------------------
+ *
+ * The Didi Cloud IFX article (inference-optimisation section) fuses
+ * CONV+BN+RELU+MAXPOOL into one function; in ResNet50 that is the stem: the
+ * 7x7 stride-2 convolution (pad 3) of the image, its BN and ReLU, then a 3x3
+ * stride-2 max pooling (pad 1).  Max pooling takes, per channel, the largest
+ * value of the window's in-image pixels (padding never wins).
+ */
+
+/* y: [B,H,W,C]; out: [B,Ho,Wo,C] with Ho = (H - 1)/2 + 1, Wo = (W - 1)/2 + 1:
+ * out[b,i,j,c] = max of y[b, 2i+r-1, 2j+s-1, c] over r, s in 0..2 inside. */
+void x1o_maxpool3s2(const int8_t *y, int8_t *out, int B, int H, int W, int C)
+{
+    int64_t Ho = conv_out_extent(H, 3, 1, 2), Wo = conv_out_extent(W, 3, 1, 2);
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t i = 0; i < Ho; ++i)
+            for (int64_t j = 0; j < Wo; ++j)
+                for (int64_t c = 0; c < C; ++c) {
+                    int best = -129; /* below every int8 */
+                    for (int64_t r = 0; r < 3; ++r)
+                        for (int64_t s = 0; s < 3; ++s) {
+                            int64_t h = 2 * i + r - 1, w = 2 * j + s - 1;
+                            if (h < 0 || h >= H || w < 0 || w >= W)
+                                continue;
+                            int v = y[nhwc_index(b, h, w, c, H, W, C)];
+                            if (v > best)
+                                best = v;
+                        }
+                    out[nhwc_index(b, i, j, c, Ho, Wo, C)] = (int8_t)best;
+                }
+}
+
+/* Stem: x1o_conv_strided (R x R, pad, stride) + BN + ReLU, then
+ * x1o_maxpool3s2.  x: [B,H,W,Ic]; out: [B,Hp,Wp,Oc]. */
+void x1o_conv_pool(const int8_t *x, const int8_t *wt, const int32_t *bias, const int32_t *m,
+                   int S, int8_t *out, int B, int H, int W, int Ic, int Oc, int R, int pad,
+                   int stride)
+{
+    int64_t Hc = conv_out_extent(H, R, pad, stride), Wc = conv_out_extent(W, R, pad, stride);
+    int8_t *y = (int8_t *)malloc((size_t)B * Hc * Wc * Oc);
+    x1o_conv_strided(x, wt, bias, m, S, NULL, 0, y, B, H, W, Ic, Oc, R, pad, stride);
+    x1o_maxpool3s2(y, out, B, (int)Hc, (int)Wc, Oc);
+    free(y);
 }
 
 int x1o_set_threads(int n)
