@@ -68,6 +68,8 @@ def parse(argv=None):
     ap.add_argument("--cpu-1thread", action="store_true",
                     help="also time the oracle sample on one host thread")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fusion", action="store_true",
+                    help="block workloads: run conv2 and conv3 as separate launches")
     ap.add_argument("--dry-run", action="store_true",
                     help="CPU only: run the rank/timing logic over gloo with a host stand-in "
                          "for the kernel (tests the multi-process path without a GPU)")
@@ -156,8 +158,13 @@ def is_block(s):
     return isinstance(s, (synth.BlockShape, synth.ProjBlockShape))
 
 
-def launches_per_step(cfg):
-    return 3 if is_block(synth.CONFIGS[cfg]) else 1
+def launches_per_step(cfg, fused=True):
+    """Kernel launches of one step: the Res3.2 block fuses conv2 and conv3 into
+    one launch (Cmid = 128); the projection block takes three."""
+    s = synth.CONFIGS[cfg]
+    if isinstance(s, synth.BlockShape):
+        return 2 if fused and s.Cmid == 128 and s.W + 2 <= 128 and s.Cin <= 1024 else 3
+    return 3 if is_block(s) else 1
 
 
 class ClockSampler:
@@ -564,6 +571,7 @@ def main(argv=None):
     if not os.path.exists(X.LIB_PATH):
         _build.build()
     X.lib()
+    X.x1cb_set_block_fusion(not a.no_fusion)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = None
@@ -697,7 +705,7 @@ def main(argv=None):
         return 0
 
     hbm, bf16, peak_kind = peaks()
-    launches = launches_per_step(cfg)
+    launches = launches_per_step(cfg, not a.no_fusion)
     gbs = nbytes / (ms_max * 1e-3) / 1e9
     if stages is None:
         roof = roofline(ops, nbytes, ms_max * 1e-3, hbm, bf16, peak_kind)

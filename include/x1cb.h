@@ -131,6 +131,25 @@ int conv1x1_proj_bn_relu_i8(const int8_t *y, const int8_t *w3, const int8_t *x,
                             int8_t *out, int B, int H, int W, int Cy, int Hx, int Wx, int Cx,
                             int Oc, void *stream);
 
+/*
+ * The stem's CONV+BN+RELU+MAXPOOL as one launch (the fusion the Didi Cloud
+ * IFX article's inference-optimisation section lists): an R x R convolution
+ * (R in {1, 3, 5, 7}, zero padding (R-1)/2, stride 1 or 2) + folded BN + ReLU,
+ * requantised as above (no r term), then 3x3 stride-2 max pooling (pad 1;
+ * padding never wins) -- ResNet50's 7x7 stride-2 stem with R = 7, stride = 2.
+ *   x   [B, Ic/32, H, W, 32]: an image of fewer channels (3) is given as one
+ *       32-channel block with the unused channels zero
+ *   w   [1, R, R, Ic/32, 64, 32] (x1cb_pack_weight of [64, Ic, R, R])
+ *   out [B, 2, Hp, Wp, 32]: Hc = (H + 2*((R-1)/2) - R)/stride + 1 conv rows,
+ *       Hp = (Hc - 1)/2 + 1 pooled rows (likewise W)
+ * Oc must be 64 (the stem's width).  Each CTA computes a tile of
+ * (2pw+1) x (2ph+1) conv pixels and pools it to pw x ph; neighbouring tiles
+ * recompute one shared conv row or column.
+ */
+int conv_bn_relu_maxpool_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
+                            const int32_t *m, int32_t S, int8_t *out, int B, int H, int W, int Ic,
+                            int Oc, int R, int stride, void *stream);
+
 /* Bytes of device workspace bottleneck_proj_i8 needs for an H x W input:
  * [B, Cmid/32, H, W, 32] and [B, Cmid/32, Ho, Wo, 32]. */
 size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid);
@@ -213,7 +232,8 @@ int x1cb_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C, 
 int x1cb_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C, void *stream);
 
 /* oihw [Oc, Ic, R, R] (the usual convolution weight order) -> blocked
- * [Oc/128, R, R, Ic/32, 128, 32]; R in {1, 3}. */
+ * [Oc/O2, R, R, Ic/32, O2, 32] with O2 = 128 (O2 = 64 for a 64-channel
+ * layer); R in {1, 3, 5, 7}. */
 int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R, void *stream);
 
 /* Human-readable name of a status code (static storage). */
@@ -254,11 +274,12 @@ void x1cb_debug_inject(int mode);
 int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, char *buf,
                        size_t len);
 
-/* As x1cb_describe_plan for an Hin x Win input at `stride` (R = 3: pad 1),
+/* As x1cb_describe_plan for an Hin x Win input at `stride` (pad (R-1)/2),
  * optionally with a projection source of Ic2 channels (1x1, stride 2, over a
- * 2H x 2W image; R = 1 and stride = 1 then). */
+ * 2H x 2W image; R = 1 and stride = 1 then) or with max pooling (pool != 0;
+ * Oc = 64). */
 int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int stride, int Ic2,
-                          int has_res, char *buf, size_t len);
+                          int has_res, int pool, char *buf, size_t len);
 
 /* Library version, e.g. "x1cb 0.2.0 sm_100a". */
 const char *x1cb_version(void);

@@ -102,7 +102,8 @@ def test_pack_argument_checks(L):
     assert L.x1cb_pack_act(None, None, 0, 2, 2, 32, None) == X.X1CB_OK
     assert L.x1cb_pack_act(v(P), v(2 * P), 1, 2, 2, 40, None) == X.X1CB_ERR_SHAPE
     assert L.x1cb_pack_act(v(P + 1), v(2 * P), 1, 2, 2, 32, None) == X.X1CB_ERR_ALIGN
-    assert L.x1cb_pack_weight(v(P), v(2 * P), 128, 32, 5, None) == X.X1CB_ERR_SHAPE
+    assert L.x1cb_pack_weight(v(P), v(2 * P), 128, 32, 4, None) == X.X1CB_ERR_SHAPE
+    assert L.x1cb_pack_weight(v(P), v(2 * P), 192, 32, 3, None) == X.X1CB_ERR_SHAPE
     assert L.x1cb_pack_weight(v(P), v(P), 128, 32, 1, None) == X.X1CB_ERR_OVERLAP
 
 

@@ -73,7 +73,8 @@ def lib() -> ctypes.CDLL:
         L.bottleneck_proj_i8_workspace_size.argtypes = [i, i, i, i]
         L.bottleneck_proj_i8_workspace_size.restype = sz
         L.bottleneck_proj_i8.argtypes = [vp] * 11 + [i32, vp, vp, sz] + [i] * 6 + [vp]
-        L.x1cb_describe_plan_ex.argtypes = [i] * 9 + [ctypes.c_char_p, sz]
+        L.x1cb_describe_plan_ex.argtypes = [i] * 10 + [ctypes.c_char_p, sz]
+        L.conv_bn_relu_maxpool_i8.argtypes = [vp] * 4 + [i32, vp] + [i] * 7 + [vp]
         _lib = L
     return _lib
 
@@ -253,6 +254,27 @@ def conv1x1_proj_bn_relu_i8(y, w3, x, wp, bias, m, S: int, out=None, stream=None
     return out
 
 
+def conv_bn_relu_maxpool_i8(x, w, bias, m, S: int, R: int = 7, stride: int = 2, out=None,
+                            stream=None):
+    """The stem's conv (R x R, pad (R-1)/2, stride) + BN + ReLU + 3x3 stride-2
+    max pooling in one launch; 64 output channels.
+    x [B, Ic/32, H, W, 32] -> out [B, 2, Hp, Wp, 32]."""
+    B, Ic, H, W = _act_shape(x, "x")
+    Oc = bias.numel()
+    pad = (R - 1) // 2
+    Hc, Wc = (H + 2 * pad - R) // stride + 1, (W + 2 * pad - R) // stride + 1
+    if out is None:
+        out = torch.empty((B, Oc // 32, _half(Hc), _half(Wc), 32), dtype=torch.int8,
+                          device=x.device)
+    with _same_device(x, w, bias, m, out):
+        st = lib().conv_bn_relu_maxpool_i8(
+            _dev(x, torch.int8, "x"), _dev(w, torch.int8, "w"), _dev(bias, torch.int32, "bias"),
+            _dev(m, torch.int32, "m"), int(S), _dev(out, torch.int8, "out"), B, H, W, Ic, Oc,
+            int(R), int(stride), _stream(stream, x.device))
+    _check(st, "conv_bn_relu_maxpool_i8")
+    return out
+
+
 def bottleneck_proj_i8_workspace_size(B: int, H: int, W: int, Cmid: int) -> int:
     return int(lib().bottleneck_proj_i8_workspace_size(B, H, W, Cmid))
 
@@ -305,10 +327,11 @@ def x1cb_unpack_act(nc32, out=None, stream=None):
 
 
 def x1cb_pack_weight(oihw, out=None, stream=None):
-    """[Oc, Ic, R, R] int8 -> blocked [Oc/128, R, R, Ic/32, 128, 32]."""
+    """[Oc, Ic, R, R] int8 -> blocked [Oc/O2, R, R, Ic/32, O2, 32], O2 = min(Oc, 128)."""
     Oc, Ic, R, R2 = oihw.shape
+    O2 = min(Oc, 128)
     if out is None:
-        out = torch.empty((Oc // 128, R, R, Ic // 32, 128, 32), dtype=torch.int8,
+        out = torch.empty((Oc // O2, R, R, Ic // 32, O2, 32), dtype=torch.int8,
                           device=oihw.device)
     with _same_device(oihw, out):
         st = lib().x1cb_pack_weight(_dev(oihw, torch.int8, "oihw"),
@@ -360,10 +383,11 @@ def x1cb_describe_plan(B, H, W, Ic, Oc, R=1, has_res=True) -> str:
     return buf.value.decode()
 
 
-def x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R=1, stride=1, Ic2=0, has_res=False) -> str:
+def x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R=1, stride=1, Ic2=0, has_res=False,
+                          pool=False) -> str:
     buf = ctypes.create_string_buffer(512)
-    _check(lib().x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R, stride, Ic2, int(has_res), buf,
-                                       512), "x1cb_describe_plan_ex")
+    _check(lib().x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R, stride, Ic2, int(has_res),
+                                       int(pool), buf, 512), "x1cb_describe_plan_ex")
     return buf.value.decode()
 
 

@@ -52,7 +52,7 @@ int device_info(int &sms)
 // a B=1 call is latency-bound).
 struct PlanKey {
     int B, H, W, Ic, Oc, R, has_res, sms;
-    int stride, Hin, Win, Ic2, stride2, Hin2, Win2;
+    int stride, Hin, Win, Ic2, stride2, Hin2, Win2, pool;
     bool operator==(const PlanKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
 
@@ -66,7 +66,7 @@ int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_re
     PlanKey k;
     std::memset(&k, 0, sizeof(k));
     k = PlanKey{B, H, W, Ic, Oc, R, has_res, sms,
-                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2};
+                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2, g.pool};
     {
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < used; ++i)
@@ -184,15 +184,19 @@ int conv_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int
 int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int32_t *m,
                      int32_t S, int8_t *out, int B, int Hin, int Win, int Ic, int Oc, int R,
                      int stride, const int8_t *x2, const int8_t *w2, int Ic2, int Hin2,
-                     int Win2, int stride2, void *stream, bool check_ptrs = true)
+                     int Win2, int stride2, void *stream, bool check_ptrs = true,
+                     bool pool = false)
 {
     const int pad = (R - 1) / 2;
     if (Hin < 0 || Win < 0 || stride < 1 || stride > 8 || stride2 < 1 || stride2 > 8)
         return X1CB_ERR_SHAPE;
     const int H = Hin + 2 * pad >= R ? (Hin + 2 * pad - R) / stride + 1 : 0;
     const int W = Win + 2 * pad >= R ? (Win + 2 * pad - R) / stride + 1 : 0;
-    if (int e = check_conv_shape(B, Hin, Win, Ic, Oc, S))
+    // (a pooled layer has 64 output channels: checked as 128 here, exactly below)
+    if (int e = check_conv_shape(B, Hin, Win, Ic, pool ? 128 : Oc, S))
         return e;
+    if (pool && Oc != 64)
+        return X1CB_ERR_SHAPE;
     if (Ic2) {
         if (Ic2 < 32 || Ic2 % 32 || Ic2 > 4096 || Hin2 < 0 || Win2 < 0)
             return X1CB_ERR_SHAPE;
@@ -202,6 +206,9 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
     const size_t px = static_cast<size_t>(B) * H * W;
     if (px == 0)
         return X1CB_OK;
+    // the written output: the pooled image when pooling
+    const size_t px_out =
+        pool ? static_cast<size_t>(B) * ((H - 1) / 2 + 1) * ((W - 1) / 2 + 1) : px;
     if (Ic2 && ((H - 1) * static_cast<long long>(stride2) >= Hin2 ||
                 (W - 1) * static_cast<long long>(stride2) >= Win2))
         return X1CB_ERR_SHAPE;
@@ -211,7 +218,7 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
         (w2 && !aligned16(w2)) || (reinterpret_cast<uintptr_t>(bias) & 3u) ||
         (reinterpret_cast<uintptr_t>(m) & 3u))
         return X1CB_ERR_ALIGN;
-    const size_t out_bytes = px * Oc;
+    const size_t out_bytes = px_out * Oc;
     const size_t in_bytes = static_cast<size_t>(B) * Hin * Win * Ic;
     const size_t in2_bytes = static_cast<size_t>(B) * Hin2 * Win2 * Ic2;
     if (overlap(out, out_bytes, x, in_bytes) || overlap(out, out_bytes, x2, in2_bytes) ||
@@ -233,6 +240,7 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
     g.stride2 = stride2;
     g.Hin2 = Hin2;
     g.Win2 = Win2;
+    g.pool = pool ? 1 : 0;
     ConvPlan p;
     if (int e = get_plan(p, B, H, W, Ic, Oc, R, 0, S, 0, sms, g))
         return e;
@@ -343,6 +351,16 @@ int conv1x1_proj_bn_relu_i8(const int8_t *y, const int8_t *w3, const int8_t *x,
                             stream);
 }
 
+int conv_bn_relu_maxpool_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
+                            const int32_t *m, int32_t S, int8_t *out, int B, int H, int W, int Ic,
+                            int Oc, int R, int stride, void *stream)
+{
+    if ((R != 1 && R != 3 && R != 5 && R != 7) || (stride != 1 && stride != 2))
+        return X1CB_ERR_SHAPE;
+    return conv_geom_common(x, w, bias, m, S, out, B, H, W, Ic, Oc, R, stride, nullptr, nullptr,
+                            0, 0, 0, 1, stream, true, true);
+}
+
 size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid)
 {
     if (B < 0 || H < 0 || W < 0 || Cmid < 0)
@@ -451,7 +469,8 @@ int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R,
 {
     if (!oihw || !blocked)
         return X1CB_ERR_NULL;
-    if (Oc < 128 || Oc % 128 || Ic < 32 || Ic % 32 || (R != 1 && R != 3))
+    if ((Oc != 64 && (Oc < 128 || Oc % 128)) || Ic < 32 || Ic % 32 ||
+        (R != 1 && R != 3 && R != 5 && R != 7))
         return X1CB_ERR_SHAPE;
     const size_t n = static_cast<size_t>(Oc) * Ic * R * R;
     if (overlap(oihw, n, blocked, n))
@@ -534,13 +553,13 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
 }
 
 int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int stride, int Ic2,
-                          int has_res, char *buf, size_t len)
+                          int has_res, int pool, char *buf, size_t len)
 {
     if (!buf || len == 0)
         return X1CB_ERR_NULL;
-    if (R != 1 && R != 3)
+    if (R != 1 && R != 3 && R != 5 && R != 7)
         return X1CB_ERR_SHAPE;
-    if (int e = check_conv_shape(B, Hin, Win, Ic, Oc, 24))
+    if (int e = check_conv_shape(B, Hin, Win, Ic, pool ? 128 : Oc, 24))
         return e;
     const int pad = (R - 1) / 2;
     if (stride < 1 || stride > 8 || Hin + 2 * pad < R || Win + 2 * pad < R || Ic2 < 0 ||
@@ -562,16 +581,17 @@ int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int st
         g.Hin2 = 2 * H;
         g.Win2 = 2 * W;
     }
+    g.pool = pool ? 1 : 0;
     ConvPlan p;
     if (int e = plan_conv_ex(p, B, H, W, Ic, Oc, R, has_res, 24, 0, sms, g))
         return e;
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
                   "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
-                  "out=%dx%d stride=%d kb2=%d wstream=%d",
+                  "out=%dx%d stride=%d kb2=%d wstream=%d pool=%dx%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream);
+                  p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream, p.pw, p.ph);
     return X1CB_OK;
 }
 

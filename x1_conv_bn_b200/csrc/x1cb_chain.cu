@@ -91,20 +91,23 @@ __device__ __forceinline__ void chain_origin(const ChainPlan &p, int mt, int &h0
     b0 = (mt / p.nTh) * p.tg;
 }
 
-// Requantisation of 32 accumulators in the form chosen for the layer.
+// Requantisation of 32 accumulators (channels ch..ch+31) in the form chosen
+// for the layer.  The constant table holds int32 biases in the all-32-bit
+// form and int64 offsets otherwise, so the channel offset is applied per form.
 template <bool kRes>
 __device__ __forceinline__ void requant_any(int mode, const uint32_t *v, const int32_t *cm,
-                                            const long long *cC, const uint32_t *rw, int m_r,
-                                            int S, int mr2, const uint32_t (&rsel)[4],
+                                            const long long *cC, int ch, const uint32_t *rw,
+                                            int m_r, int S, int mr2, const uint32_t (&rsel)[4],
                                             uint32_t *ow)
 {
     if (mode == 2)
-        requant_hi32<kRes, true, false, 8>(v, cm, reinterpret_cast<const int32_t *>(cC), rw, mr2,
+        requant_hi32<kRes, true, false, 8>(v, cm + ch,
+                                           reinterpret_cast<const int32_t *>(cC) + ch, rw, mr2,
                                            rsel, ow);
     else if (mode == 1)
-        requant_fast<kRes, 8>(v, cm, cC, rw, mr2, rsel, ow);
+        requant_fast<kRes, 8>(v, cm + ch, cC + ch, rw, mr2, rsel, ow);
     else
-        requant32<kRes>(v, cm, cC, rw, m_r, S, ow);
+        requant32<kRes>(v, cm + ch, cC + ch, rw, m_r, S, ow);
 }
 
 // Per-layer constants of the chosen form into shared memory (see the
@@ -494,8 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t v[32], ow[8];
                 __syncwarp();
                 tmem_ld_32x32b_x32_sync(tb + static_cast<uint32_t>(c * 32), v);
-                requant_any<false>(mode2, v, cm2 + c * 32, cc2 + c * 32, nullptr, 0, p.S, 0, rsel,
-                                   ow);
+                requant_any<false>(mode2, v, cm2, cc2, c * 32, nullptr, 0, p.S, 0, rsel, ow);
                 // K block c of the A buffer: two 16-byte halves, rows 16 bytes apart.
                 uint4 *dst = reinterpret_cast<uint4 *>(a3 + c * (kA3Bytes / 4) + row * 16);
                 dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
@@ -560,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint4 ra = *pa, rb = *pb;
                 const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
                 uint32_t ow[8];
-                requant_any<true>(mode3, v, cm3 + ch, cc3 + ch, rw, p.m_r, p.S, mr2, rsel, ow);
+                requant_any<true>(mode3, v, cm3, cc3, ch, rw, p.m_r, p.S, mr2, rsel, ow);
                 if (in_box) {
                     *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                     *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);

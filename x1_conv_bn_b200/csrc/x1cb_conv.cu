@@ -76,12 +76,18 @@ struct Bars {
     __device__ uint32_t io_full(int s) const { return at(3 + 2 * a_stages + s); }
     __device__ uint32_t out_ready(int s) const { return at(3 + 2 * a_stages + r_stages + s); }
     __device__ uint32_t io_empty(int s) const { return at(3 + 2 * a_stages + 2 * r_stages + s); }
+    // Accumulator slots: up to 8 (64-column accumulators of a 64-channel layer).
     __device__ uint32_t acc_full(int s) const { return at(3 + 2 * a_stages + 3 * r_stages + s); }
     __device__ uint32_t acc_empty(int s) const
     {
-        return at(3 + 2 * a_stages + 3 * r_stages + 4 + s);
+        return at(3 + 2 * a_stages + 3 * r_stages + 8 + s);
     }
-    static int count(int a, int r) { return 3 + 2 * a + 3 * r + 8; }
+    // Pool mode: the four warps of a turn meet here before pooling their tile.
+    __device__ uint32_t pool_bar(int turn) const
+    {
+        return at(3 + 2 * a_stages + 3 * r_stages + 16 + turn);
+    }
+    static int count(int a, int r) { return 3 + 2 * a + 3 * r + 16 + 4; }
 };
 
 __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, int &h0, int &b0)
@@ -89,8 +95,13 @@ __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, 
     const int iw = mt % p.nTw;
     const int ih = (mt / p.nTw) % p.nTh;
     const int ig = mt / (p.nTw * p.nTh);
-    w0 = iw * p.tw;
-    h0 = ih * p.th;
+    if (p.pool) {  // conv origin of pooled tile (iw, ih): one pixel before 2 * pooled origin
+        w0 = 2 * iw * p.pw - 1;
+        h0 = 2 * ih * p.ph - 1;
+    } else {
+        w0 = iw * p.tw;
+        h0 = ih * p.th;
+    }
     b0 = ig * p.tg;
 }
 
@@ -131,6 +142,8 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     constexpr int kTurns = kEpiWarps / 4;                 // warps per TMEM lane quarter
     static_assert(kTurns == kTmemCols / (32 * kRChunks),
                   "one turn per I/O stage held in TMEM: each turn owns one accumulator slot");
+    // (64-channel layers: stages of two chunks, eight 64-column slots; turn g
+    // then owns slots g and g + 4, still seeing each slot's phases in order)
     const ConvPlan &p = *cx.p;
     const int q = warp & 3;                               // TMEM lane quarter this warp may access
     const int turn = (warp - kEpiWarp0) >> 2;
@@ -143,13 +156,13 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
     // This row's 32 bytes inside chunk 0 of an I/O stage ([tg][4][th][tw][32]);
     // rows outside the box read row 0's bytes and write nothing.
-    const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
+    const int row_off = in_box ? ((gi * p.stage_ch) * plane_t + yi * p.tw + xi) * 32 : 0;
     const int chunk_stride = plane_t * 32;
     // (o >> 3) & 0x70 is bits 7-9 of o moved to bits 4-6: the 128-byte swizzle.
     const int swz_mask = p.io_swz ? 0x70 : 0;
-    const int n_slots = kTmemCols / p.nmma;
+    const int n_slots = p.n_slots;
     const int chunks_per_sub = p.nmma / 32;
-    const int stages_per_sub = chunks_per_sub / kRChunks;
+    const int stages_per_sub = chunks_per_sub / p.stage_ch;
     const long long my_tiles =
         cx.mt_first < p.num_m_tiles ? (p.num_m_tiles - cx.mt_first + cx.mt_step - 1) / cx.mt_step
                                     : 0;
@@ -184,6 +197,7 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     int j = sub_n % p.n_subs;
     int acc = sub_n % n_slots;
     uint32_t acc_phase = static_cast<uint32_t>((sub_n / n_slots) & 1);
+    uint32_t pool_phase = 0;
     for (long long n = turn; n < total; n += kTurns) {
         // Every lane waits; the vote keeps the decision warp-uniform so the
         // .sync.aligned TMEM loads below always run converged.
@@ -211,9 +225,17 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             atomicMax(const_cast<int *>(cx.io_ticket), static_cast<int>(n + 1));
         const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
         uint8_t *stage = cx.io + st * kRSlotBytes;
+        bool conv_px = true;  // pool mode: this row is a pixel of the conv output
+        if (p.pool) {
+            const int mt = cx.mt_first + static_cast<int>(n / (p.n_subs * stages_per_sub)) *
+                                             cx.mt_step;
+            int w0, h0, b0;
+            tile_origin(p, mt, w0, h0, b0);
+            conv_px = w0 + xi >= 0 && w0 + xi < p.W && h0 + yi >= 0 && h0 + yi < p.H;
+        }
 #pragma unroll 1
-        for (int c = 0; c < kRChunks; ++c) {
-            const int cs = rl * kRChunks + c;          // chunk within the TMEM slot
+        for (int c = 0; c < p.stage_ch; ++c) {
+            const int cs = rl * p.stage_ch + c;        // chunk within the TMEM slot
             const int gch = j * chunks_per_sub + cs;   // chunk within the CTA's channels
             uint32_t v[32];
             __syncwarp();
@@ -241,8 +263,48 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                 requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
             }
             if (in_box) {
+                if (p.pool && !conv_px)  // outside the conv output: never the maximum
+                    ow[0] = ow[1] = ow[2] = ow[3] = ow[4] = ow[5] = ow[6] = ow[7] = 0u;
                 *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+            }
+        }
+        if (p.pool) {
+            // Every conv pixel of the tile is in the stage once the turn's four
+            // warps are here; then each thread pools 16-byte pieces (16 channels)
+            // of pooled pixels into the upper half of the stage.
+            // (an mbarrier, so that a turn whose wait ran out cannot strand the
+            // others: this wait is bounded like every other)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(cx.bars.pool_bar(turn));
+            if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.pool_bar(turn), pool_phase, cx.ctl,
+                                                   kDevTimeoutEpilogue)))
+                return;
+            pool_phase ^= 1u;
+            const int tid = q * 32 + lane;
+            const int np = p.pw * p.ph;
+            uint8_t *pooled = stage + kRSlotBytes / 2;
+            for (int k = tid; k < np * p.stage_ch * 2; k += 128) {
+                const int half = k & 1;
+                const int c = (k >> 1) / np;
+                const int pix = (k >> 1) % np;
+                const int pi = pix / p.pw, pj = pix % p.pw;
+                const uint8_t *src = stage + c * chunk_stride + half * 16;
+                uint4 mx = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int r = 0; r < 3; ++r)
+#pragma unroll
+                    for (int t = 0; t < 3; ++t) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(
+                            src + ((2 * pi + r) * p.tw + 2 * pj + t) * 32);
+                        mx.x = __vmaxu4(mx.x, v.x);
+                        mx.y = __vmaxu4(mx.y, v.y);
+                        mx.z = __vmaxu4(mx.z, v.z);
+                        mx.w = __vmaxu4(mx.w, v.w);
+                    }
+                *reinterpret_cast<uint4 *>(pooled + (c * np + pix) * 32 + half * 16) = mx;
             }
         }
         // Results must be visible to the TMA store (async proxy).
@@ -305,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int group = blockIdx.x % p.n_groups;
     const int mt_first = blockIdx.x / p.n_groups;
     const int mt_step = gridDim.x / p.n_groups;
-    const int stages_per_tile = p.NC / (32 * kRChunks);
+    const int stages_per_tile = p.NC / (32 * p.stage_ch);
 
     // ---- set-up ---------------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -323,10 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bars.out_ready(s), 4);  // one warp per TMEM lane quarter
             mbar_init(bars.io_empty(s), 1);
         }
-        for (int s = 0; s < 4; ++s) {
+        for (int t = 0; t < 4; ++t)
+            mbar_init(bars.pool_bar(t), 4);
+        for (int s = 0; s < 8; ++s) {
             mbar_init(bars.acc_full(s), 1);
             // every stage of the slot, each from one warp per lane quarter
-            mbar_init(bars.acc_empty(s), 4 * (p.nmma / (32 * kRChunks)));
+            mbar_init(bars.acc_empty(s), 4 * (p.nmma / (32 * p.stage_ch)));
         }
         fence_mbar_init();
     }
@@ -409,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- producer: resident weights, then activation K blocks ---------------
         if (lane == 0) {
             const uint32_t sw = sbase + p.off_w;
-            const int o1 = group * (p.NC / 128);
+            const int o1 = group * (p.NC / p.O2);  // weight block of this CTA's channels
             if (!p.wstream) {
                 const uint32_t wbytes = static_cast<uint32_t>(p.kb_per_tile * p.NC * 32);
                 mbar_arrive_expect_tx(bars.w_full(), wbytes);
@@ -543,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- producer of I/O stages: shortcut tiles, issued as early as the ring
         // allows; without a shortcut it only hands out free stages ----------------
         if (lane == 0) {
-            const uint32_t rbytes = static_cast<uint32_t>(kRChunks * p.rows * 32);
+            const uint32_t rbytes = static_cast<uint32_t>(p.stage_ch * p.rows * 32);
             const uint32_t sio = sbase + p.off_r;
             const uint64_t pol = policy_evict_first();
             int stage = 0;
@@ -560,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (kRes) {
                         mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
-                        const int o1 = group * (p.NC / 32) + rs * kRChunks;
+                        const int o1 = group * (p.NC / 32) + rs * p.stage_ch;
                         if (p.io_swz)
                             tma_load_5d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
                                              0, w0 / 4, h0, o1, b0, pol);
@@ -607,8 +671,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    const int o1 = group * (p.NC / 32) + rs * kRChunks;
-                    if (p.io_swz)
+                    const int o1 = group * (p.NC / 32) + rs * p.stage_ch;
+                    if (p.pool)  // pooled tile at pooled coordinates ((w0 + 1) / 2, ...)
+                        tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes + kRSlotBytes / 2, 0,
+                                          (w0 + 1) / 2, (h0 + 1) / 2, o1, b0, pol);
+                    else if (p.io_swz)
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0 / 4, h0, o1, b0,
                                           pol);
                     else if (p.io_wide)
@@ -663,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (streamed: the nine taps of one channel block are consecutive)
             const uint64_t b_tap_step =
                 p.wstream ? b_kb_step : static_cast<uint64_t>(p.C1) * b_kb_step;
-            const int n_slots = kTmemCols / p.nmma;
+            const int n_slots = p.n_slots;
             int a_stage = 0;
             uint32_t a_phase = 0;
             uint64_t a_slot_desc = a_desc0;
@@ -949,9 +1016,14 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         return X1CB_ERR_SHAPE;
     if (p.C1b && ((H - 1) * p.stride2 >= p.Hin2 || (W - 1) * p.stride2 >= p.Win2))
         return X1CB_ERR_SHAPE;
+    p.pool = g.pool ? 1 : 0;
+    if (p.pool && (Oc != 64 || has_res || p.C1b))
+        return X1CB_ERR_SHAPE;  // pooled tiles use the upper half of 64-channel stages
+    p.Hpo = p.pool ? (H - 1) / 2 + 1 : 0;
+    p.Wpo = p.pool ? (W - 1) / 2 + 1 : 0;
     // A stride-1 1x1 without a second source sees the image as one row of H*W
     // pixels (tiles may span image rows); otherwise tiles are 2-D.
-    const bool flat = R == 1 && p.stride == 1 && p.C1b == 0;
+    const bool flat = R == 1 && p.stride == 1 && p.C1b == 0 && !p.pool;
     if (flat) {
         p.Wp = H * W;
         p.Hp = 1;
@@ -965,7 +1037,8 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     }
     // The 3x3 convolution uses the halo form whenever one framed image row fits
     // in the 128 GEMM rows (stride 1).
-    p.halo = (R == 3 && p.pad == 1 && p.stride == 1 && p.C1b == 0 && W + 2 <= kTileRows) ? 1 : 0;
+    p.halo = (R == 3 && p.pad == 1 && p.stride == 1 && p.C1b == 0 && !p.pool &&
+              W + 2 <= kTileRows) ? 1 : 0;
     if (p.halo) {
         choose_halo_tile(B, H, W, p.th, p.tg);
         p.tw = W;
@@ -975,6 +1048,26 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         // touch (rows past the frame only feed GEMM rows that are not pixels).
         const int need_rows = std::max(p.tg * p.plane_m, kTileRows + 2 * p.row_pitch + 2);
         p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+    } else if (p.pool) {
+        // pw x ph pooled pixels per tile, (2pw+1) x (2ph+1) conv pixels: fewest
+        // tiles, ties to more pooled pixels per tile.
+        long long best = -1;
+        for (int pw = 1; 2 * pw + 1 <= kTileRows; ++pw)
+            for (int ph = 1; (2 * pw + 1) * (2 * ph + 1) <= kTileRows; ++ph) {
+                const long long t = static_cast<long long>((p.Wpo + pw - 1) / pw) *
+                                    ((p.Hpo + ph - 1) / ph);
+                if (best < 0 || t < best || (t == best && pw * ph > p.pw * p.ph)) {
+                    best = t;
+                    p.pw = pw;
+                    p.ph = ph;
+                }
+            }
+        p.tw = 2 * p.pw + 1;
+        p.th = 2 * p.ph + 1;
+        p.tg = 1;
+        p.row_pitch = p.tw;
+        p.plane_m = p.tw * p.th;
+        p.a_half = 0;
     } else {
         choose_tile(B, p.Wp, p.Hp, p.tw, p.th, p.tg);
         p.row_pitch = p.tw;
@@ -982,8 +1075,8 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.a_half = 0;
     }
     p.rows = p.tw * p.th * p.tg;
-    p.nTw = (p.Wp + p.tw - 1) / p.tw;
-    p.nTh = (p.Hp + p.th - 1) / p.th;
+    p.nTw = p.pool ? (p.Wpo + p.pw - 1) / p.pw : (p.Wp + p.tw - 1) / p.tw;
+    p.nTh = p.pool ? (p.Hpo + p.ph - 1) / p.ph : (p.Hp + p.th - 1) / p.th;
     p.nTg = (B + p.tg - 1) / p.tg;
     const long long mtiles = static_cast<long long>(p.nTw) * p.nTh * p.nTg;
     if (mtiles > INT_MAX / 2)
@@ -996,10 +1089,11 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     const int min_slot = p.halo ? 2 * p.a_half : kASlotBytes;
     int chosen = 0;
     long long chosen_work = -1;
-    for (int NC = std::min(Oc, 512); NC >= 128; NC -= 128) {
-        if (Oc % NC)
+    // A 64-channel layer (the stem) is one CTA group of N = 64.
+    for (int NC = std::min(Oc, 512); NC >= 64; NC -= (NC > 128 ? 128 : 64)) {
+        if (Oc % NC || (NC == 64 && Oc != 64))
             continue;
-        const int nmma = NC >= 256 ? 256 : 128;
+        const int nmma = NC >= 256 ? 256 : (NC >= 128 ? 128 : 64);
         const int n_subs = NC / nmma;
         const int a_min = n_subs > 1 ? (p.halo ? p.C1 : p.kb_per_tile) + 2 : (p.halo ? 2 : 4);
         const int r_min = has_res ? 4 : 2;
@@ -1021,11 +1115,14 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // weights from L2 next to its activations.
     p.wstream = chosen == 0 ? 1 : 0;
     if (p.wstream)
-        chosen = 128;
+        chosen = Oc == 64 ? 64 : 128;
     p.NC = chosen;
     p.n_groups = Oc / p.NC;
-    p.nmma = p.NC >= 256 ? 256 : 128;
+    p.nmma = p.NC >= 256 ? 256 : (p.NC >= 128 ? 128 : 64);
     p.n_subs = p.NC / p.nmma;
+    p.O2 = Oc < 128 ? Oc : 128;
+    p.stage_ch = p.NC >= 128 ? kRChunks : p.NC / 32;
+    p.n_slots = kTmemCols / p.nmma;
 
     const int wbytes = p.wstream ? 0 : p.kb_per_tile * p.NC * 32;
     // The activation ring budget: with a shortcut the I/O ring (shortcut in,
@@ -1085,9 +1182,9 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
                 placed = layout(fold, a, r);
     if (!placed)
         return X1CB_ERR_SHAPE;
-    p.io_wide = p.tw * 4 <= 256 ? 1 : 0;  // TMA box dimensions are at most 256 elements
+    p.io_wide = p.tw * 4 <= 256 && !p.pool ? 1 : 0;  // TMA boxes span at most 256 elements
     // The swizzled stages need whole 4-pixel groups and 1024-byte aligned stages.
-    p.io_swz = (p.tw % 4 == 0 && p.Wp % 4 == 0 && p.off_r % 1024 == 0) ? 1 : 0;
+    p.io_swz = (p.tw % 4 == 0 && p.Wp % 4 == 0 && p.off_r % 1024 == 0 && !p.pool) ? 1 : 0;
 
     const long long work = mtiles * p.n_groups;
     long long grid = std::min<long long>(num_sms, work);
@@ -1151,17 +1248,17 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
     }
     // Weights [Oc/128][KB][128][32]: dims (32, 128, KB, Oc/128); box (32,128,1,NC/128).
     {
-        const uint64_t dims[4] = {32, 128, (uint64_t)p.kb_a, (uint64_t)(p.Oc / 128)};
-        const uint64_t str[3] = {32, 4096, (uint64_t)p.kb_a * 4096};
-        const uint32_t box[4] = {32, 128, 1, (uint32_t)(p.NC / 128)};
+        const uint64_t dims[4] = {32, (uint64_t)p.O2, (uint64_t)p.kb_a, (uint64_t)(p.Oc / p.O2)};
+        const uint64_t str[3] = {32, (uint64_t)p.O2 * 32, (uint64_t)p.kb_a * p.O2 * 32};
+        const uint32_t box[4] = {32, (uint32_t)p.O2, 1, (uint32_t)(p.NC / p.O2)};
         if (int e = encode_map(&tmW, w, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }
     tmW2 = tmW;
     if (p.C1b) {
-        const uint64_t dims[4] = {32, 128, (uint64_t)p.C1b, (uint64_t)(p.Oc / 128)};
-        const uint64_t str[3] = {32, 4096, (uint64_t)p.C1b * 4096};
-        const uint32_t box[4] = {32, 128, 1, (uint32_t)(p.NC / 128)};
+        const uint64_t dims[4] = {32, (uint64_t)p.O2, (uint64_t)p.C1b, (uint64_t)(p.Oc / p.O2)};
+        const uint64_t str[3] = {32, (uint64_t)p.O2 * 32, (uint64_t)p.C1b * p.O2 * 32};
+        const uint32_t box[4] = {32, (uint32_t)p.O2, 1, (uint32_t)(p.NC / p.O2)};
         if (int e = encode_map(&tmW2, w2, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }
@@ -1174,7 +1271,7 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
                                   (uint64_t)p.B};
         const uint64_t str[4] = {128, (uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
                                  (uint64_t)p.O1 * p.Hp * p.Wp * 32};
-        const uint32_t box[5] = {16, (uint32_t)p.tw / 4, (uint32_t)p.th, (uint32_t)kRChunks,
+        const uint32_t box[5] = {16, (uint32_t)p.tw / 4, (uint32_t)p.th, (uint32_t)p.stage_ch,
                                  (uint32_t)p.tg};
         if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_DATA_TYPE_UINT64))
@@ -1191,7 +1288,7 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
                                   (uint64_t)p.B};
         const uint64_t str[3] = {(uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
                                  (uint64_t)p.O1 * p.Hp * p.Wp * 32};
-        const uint32_t box[4] = {(uint32_t)p.tw * 4, (uint32_t)p.th, (uint32_t)kRChunks,
+        const uint32_t box[4] = {(uint32_t)p.tw * 4, (uint32_t)p.th, (uint32_t)p.stage_ch,
                                  (uint32_t)p.tg};
         if (int e = encode_map(&tmO, out, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
                                CU_TENSOR_MAP_DATA_TYPE_UINT64))
@@ -1203,12 +1300,22 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         } else {
             tmR = tmO;  // unused
         }
+    } else if (p.pool) {
+        // pooled output [B, Oc/32, Hpo, Wpo, 32]: box of the tile's pooled pixels
+        const uint64_t dims[5] = {32, (uint64_t)p.Wpo, (uint64_t)p.Hpo, (uint64_t)p.O1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {32, (uint64_t)p.Wpo * 32, (uint64_t)p.Hpo * p.Wpo * 32,
+                                 (uint64_t)p.O1 * p.Hpo * p.Wpo * 32};
+        const uint32_t box[5] = {32, (uint32_t)p.pw, (uint32_t)p.ph, (uint32_t)p.stage_ch, 1};
+        if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return e;
+        tmR = tmO;  // unused
     } else {
         const uint64_t dims[5] = {32, (uint64_t)p.Wp, (uint64_t)p.Hp, (uint64_t)p.O1,
                                   (uint64_t)p.B};
         const uint64_t str[4] = {32, (uint64_t)p.Wp * 32, (uint64_t)p.Hp * p.Wp * 32,
                                  (uint64_t)p.O1 * p.Hp * p.Wp * 32};
-        const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)p.th, (uint32_t)kRChunks,
+        const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)p.th, (uint32_t)p.stage_ch,
                                  (uint32_t)p.tg};
         if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return e;

@@ -26,6 +26,7 @@ int plan_conv(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_r
 struct ConvGeom {
     int stride = 1, Hin = 0, Win = 0;
     int Ic2 = 0, stride2 = 1, Hin2 = 0, Win2 = 0;
+    int pool = 0;  // 3x3 stride-2 max pooling after the ReLU (64-channel layers)
 };
 int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
                  int m_r, int num_sms, const ConvGeom &g);

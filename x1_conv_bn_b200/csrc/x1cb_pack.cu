@@ -1,6 +1,6 @@
 // Layout conversions (Inspur MLPerf ResNet50 convolution-merge article,
 // news.cnblogs.com/n/719672, section 3.1): NHWC <-> NC/32HW32 activations and
-// OIHW -> blocked [O1, R, S, I1, O2=128, I2=32] weights.  These are the
+// OIHW -> blocked [O1, R, S, I1, O2, I2=32] weights (O2 = 128, or Oc below 128).  These are the
 // article's offline preparation steps; they move 32-byte channel chunks with
 // 16-byte vector accesses.
 #include <cuda_runtime.h>
@@ -57,21 +57,22 @@ __global__ void pack_weight_kernel(const int8_t *__restrict__ oihw, int8_t *__re
 {
     const long long n = static_cast<long long>(Oc) * Ic * R * R;
     const int I1 = Ic / 32;
+    const int O2 = Oc < 128 ? Oc : 128;  // a 64-channel layer is one block of 64
     for (long long d = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; d < n;
          d += static_cast<long long>(gridDim.x) * blockDim.x) {
-        // d = ((((ob*R + r)*R + s)*I1 + i1)*128 + o2)*32 + i2
+        // d = ((((ob*R + r)*R + s)*I1 + i1)*O2 + o2)*32 + i2
         long long t = d;
         const int i2 = static_cast<int>(t % 32);
         t /= 32;
-        const int o2 = static_cast<int>(t % 128);
-        t /= 128;
+        const int o2 = static_cast<int>(t % O2);
+        t /= O2;
         const int i1 = static_cast<int>(t % I1);
         t /= I1;
         const int s = static_cast<int>(t % R);
         t /= R;
         const int r = static_cast<int>(t % R);
         const int ob = static_cast<int>(t / R);
-        const long long o = static_cast<long long>(ob) * 128 + o2;
+        const long long o = static_cast<long long>(ob) * O2 + o2;
         const long long i = static_cast<long long>(i1) * 32 + i2;
         blk[d] = oihw[((o * Ic + i) * R + r) * R + s];
     }

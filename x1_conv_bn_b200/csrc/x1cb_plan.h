@@ -46,6 +46,9 @@ struct ConvPlan {
     int num_m_tiles;
     // N split: each CTA keeps NC output channels' weights resident
     int NC, n_groups, nmma, n_subs;
+    int O2;        // output channels per weight block: 128, or Oc for a 64-channel layer
+    int stage_ch;  // 32-channel chunks per I/O stage: 4, or 2 for a 64-channel layer
+    int n_slots;   // accumulator slots in TMEM (512 columns / nmma)
     int kb_per_tile;  // R*R*C1
     int a_kc;         // K blocks per activation TMA box (divides C1)
     int a_slot;       // bytes per ring stage: activation part + streamed weights
@@ -79,6 +82,13 @@ struct ConvPlan {
     int row_pitch;  // GEMM rows per image row: tw, or tw+2 in the halo form
     int plane_m;    // GEMM rows per image of the tile: tw*th, or (th+2)*(tw+2)
     int a_half;     // halo form: bytes between the two K halves of a slot
+    // Max pooling fused after the ReLU (3x3, stride 2, pad 1): tiles cover
+    // pw x ph pooled pixels; their conv tile is (2pw+1) x (2ph+1) pixels from
+    // conv pixel (2*pooled origin - 1), so neighbouring tiles share one conv
+    // row/column.  Conv pixels outside the conv output count as 0, which never
+    // wins over a ReLU output.  The pooled tile is staged in the upper half of
+    // the I/O stage and stored to the pooled tensor (Hpo x Wpo).
+    int pool, pw, ph, Hpo, Wpo;
     // control
     int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
     unsigned long long wait_limit_ns;
