@@ -70,6 +70,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fusion", action="store_true",
                     help="block workloads: run conv2 and conv3 as separate launches")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--dry-run", action="store_true",
                     help="CPU only: run the rank/timing logic over gloo with a host stand-in "
                          "for the kernel (tests the multi-process path without a GPU)")
@@ -158,12 +160,19 @@ def is_block(s):
     return isinstance(s, (synth.BlockShape, synth.ProjBlockShape))
 
 
+def block_fused(s, fused=True):
+    """Whether the library runs this bottleneck's conv2 and conv3 as one
+    launch (its fused form: Cmid = 128, Cout up to 1024, whole-row I/O)."""
+    return (fused and isinstance(s, synth.BlockShape) and s.Cmid == 128 and s.Cin % 128 == 0
+            and s.Cin <= 1024 and s.W + 2 <= 128 and (s.W % 4 == 0 or 4 * s.W <= 256))
+
+
 def launches_per_step(cfg, fused=True):
     """Kernel launches of one step: the Res3.2 block fuses conv2 and conv3 into
     one launch (Cmid = 128); the projection block takes three."""
     s = synth.CONFIGS[cfg]
     if isinstance(s, synth.BlockShape):
-        return 2 if fused and s.Cmid == 128 and s.W + 2 <= 128 and s.Cin <= 1024 else 3
+        return 2 if block_fused(s, fused) else 3
     return 3 if is_block(s) else 1
 
 
@@ -442,7 +451,7 @@ def dry_run(a, rank, world):
                           "dry_run": True, "scaling": "weak"}), flush=True)
 
 
-def block_stage_calls(cfg, dev, seed):
+def block_stage_calls(cfg, dev, seed, fusion=True):
     """For the block workloads: the three stages as separate calls on the same
     buffers (conv1 x -> y1, conv2 y1 -> y2, conv3 y2 (+x) -> out), for
     per-stage timing.  Returns (label, ops, bytes, call) per stage."""
@@ -480,14 +489,26 @@ def block_stage_calls(cfg, dev, seed):
     y2 = torch.empty_like(y1)
     out = torch.empty_like(x)
     st = s.stages()
+    fused = block_fused(s, fusion)
 
     def label(c):
         return f"{c.R}x{c.R} {c.Ic}->{c.Oc}" + (" +res" if c.has_res else "")
 
+    conv1 = (label(st[0]), st[0].ops(), st[0].bytes_moved(),
+             lambda stream: X.conv1x1_bn_add_relu_i8(x, ws[0], inp.bias[0], inp.m[0], 0, inp.S,
+                                                     None, out=y1, stream=stream))
+    if fused:
+        # conv2 -> conv3 fused: y1 and the shortcut in, out out; no y2 round trip
+        px = s.B * s.H * s.W
+        return [conv1, ("3x3 %d->%d -> 1x1 %d->%d +res (fused)" % (s.Cmid, s.Cmid, s.Cmid, s.Cin),
+                        st[1].ops() + st[2].ops(),
+                        px * (s.Cmid + 2 * s.Cin) + 9 * s.Cmid ** 2 + s.Cin * s.Cmid
+                        + 8 * (s.Cmid + s.Cin),
+                        lambda stream: X.conv3x3_conv1x1_bn_add_relu_i8(
+                            y1, ws[1], inp.bias[1], inp.m[1], ws[2], inp.bias[2], inp.m[2],
+                            inp.m_r, inp.S, x, out=out, stream=stream))]
     return [
-        (label(st[0]), st[0].ops(), st[0].bytes_moved(),
-         lambda stream: X.conv1x1_bn_add_relu_i8(x, ws[0], inp.bias[0], inp.m[0], 0, inp.S, None,
-                                                 out=y1, stream=stream)),
+        conv1,
         (label(st[1]), st[1].ops(), st[1].bytes_moved(),
          lambda stream: X.conv3x3_bn_relu_i8(y1, ws[1], inp.bias[1], inp.m[1], inp.S, out=y2,
                                              stream=stream)),
@@ -525,6 +546,11 @@ def main(argv=None):
     if a.dry_run:
         return dry_run(a, rank, world)
     cfg = a.config
+    if a.batch:
+        import dataclasses
+
+        synth.CONFIGS[cfg] = dataclasses.replace(synth.CONFIGS[cfg], B=a.batch)
+        synth.WORKLOAD_NAMES[cfg] = re.sub(r"B=\d+", f"B={a.batch}", synth.WORKLOAD_NAMES[cfg])
     s = synth.CONFIGS[cfg]
     metric = metric_for(cfg)
     ops, nbytes = workload_units(cfg)
@@ -624,7 +650,7 @@ def main(argv=None):
         stages = []
         with torch.cuda.stream(stream):
             for lab, s_ops, s_bytes, fn in block_stage_calls(
-                    cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank)):
+                    cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank), not a.no_fusion):
                 t = time_launches(fn, stream, max(20, min(200, a.steps)))
                 stages.append({"stage": lab, "us": t * 1e3, "ops": s_ops, "bytes": s_bytes})
         torch.cuda.synchronize()

@@ -98,6 +98,26 @@ int conv3x3_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias, co
                        void *stream);
 
 /*
+ * Conv2 -> Conv3 of the Res3.x bottleneck as one launch (the merge of two
+ * consecutive convolutions, Inspur article section 2.1): the 3x3 pad-1
+ * convolution of y1 + BN + ReLU, requantised to int8, stays on chip as the A
+ * operand of the 1x1 convolution + BN + shortcut Sum with r + ReLU.  Runs on
+ * pairs of SMs sharing each MMA (both weight sets on chip).
+ *   y1  [B, Cmid/32, H, W, 32] (Conv1's output); w2 [Cmid/128, 3, 3, Cmid/32, 128, 32]
+ *   b2, m2 [Cmid]; w3 [Cout/128, Cmid/32, 128, 32]; b3, m3 [Cout]; m_r, S
+ *   r   [B, Cout/32, H, W, 32] shortcut; out [B, Cout/32, H, W, 32]
+ * Requires Cmid = 128, Cout a multiple of 128 up to 1024, W <= 126 and
+ * (W % 4 == 0 or W <= 64); otherwise X1CB_ERR_SHAPE (use the two separate
+ * calls).  Bit-identical to conv3x3_bn_relu_i8 followed by
+ * conv1x1_bn_add_relu_i8.
+ */
+int conv3x3_conv1x1_bn_add_relu_i8(const int8_t *y1, const int8_t *w2, const int32_t *b2,
+                                   const int32_t *m2, const int8_t *w3, const int32_t *b3,
+                                   const int32_t *m3, int32_t m_r, int32_t S, const int8_t *r,
+                                   int8_t *out, int B, int H, int W, int Cmid, int Cout,
+                                   void *stream);
+
+/*
  * Fused 3x3 convolution of stride 2 (zero padding 1) + folded BN + ReLU +
  * int8 requantisation: Conv2 of a downsampling (projection) block such as
  * Res3.1.  The Inspur article (section 2.2) says only that Res3.1's output
@@ -280,6 +300,12 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
  * Oc = 64). */
 int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int stride, int Ic2,
                           int has_res, int pool, char *buf, size_t len);
+
+/* Describes the fused conv2 -> conv3 plan of a bottleneck block (tiles, ring
+ * depths, shared memory, and the clusters of two CTAs the current device can
+ * hold at once; 0 without a device).  X1CB_ERR_SHAPE when the block has no
+ * fused form. */
+int x1cb_describe_chain(int B, int H, int W, int Cmid, int Cout, char *buf, size_t len);
 
 /* Library version, e.g. "x1cb 0.2.0 sm_100a". */
 const char *x1cb_version(void);

@@ -131,3 +131,20 @@ def test_fused_block_repeated_launches(oracle):
     ref = oracle.bottleneck_pixels(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S, pix)
     got = _nhwc(outs[-1].cpu()).reshape(-1, 512)[pix]
     assert torch.equal(got, ref)
+
+
+def test_fused_entry_point_equals_the_two_layers():
+    """conv3x3_conv1x1_bn_add_relu_i8 against conv3x3_bn_relu_i8 followed by
+    conv1x1_bn_add_relu_i8 (both oracle-checked elsewhere), bit for bit."""
+    s = synth.BlockShape(6, 28, 28, 512, 128)
+    inp = synth.block_inputs(s, 17)
+    x, args = _packed(inp)
+    y1 = X.conv1x1_bn_add_relu_i8(x, args[0], args[1], args[2], 0, inp.S)
+    fused = X.conv3x3_conv1x1_bn_add_relu_i8(y1, args[3], args[4], args[5], args[6], args[7],
+                                             args[8], inp.m_r, inp.S, x)
+    y2 = X.conv3x3_bn_relu_i8(y1, args[3], args[4], args[5], inp.S)
+    two = X.conv1x1_bn_add_relu_i8(y2, args[6], args[7], args[8], inp.m_r, inp.S, x)
+    torch.cuda.synchronize()
+    assert X.x1cb_last_device_error(clear=True)[0] == 0
+    assert torch.equal(fused, two)
+    assert "resident_clusters=" in X.x1cb_describe_chain(6, 28, 28)

@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.bottleneck_proj_i8.argtypes = [vp] * 11 + [i32, vp, vp, sz] + [i] * 6 + [vp]
         L.x1cb_describe_plan_ex.argtypes = [i] * 10 + [ctypes.c_char_p, sz]
         L.conv_bn_relu_maxpool_i8.argtypes = [vp] * 4 + [i32, vp] + [i] * 7 + [vp]
+        L.x1cb_describe_chain.argtypes = [i] * 5 + [ctypes.c_char_p, sz]
+        L.conv3x3_conv1x1_bn_add_relu_i8.argtypes = [vp] * 7 + [i32, i32, vp, vp] + [i] * 5 + [vp]
         _lib = L
     return _lib
 
@@ -214,6 +216,25 @@ def bottleneck_i8_noalloc(x, w1, b1, m1, w2, b2, m2, w3, b3, m3, m_r: int, S: in
 def _half(n: int) -> int:
     """Output extent of a stride-2 3x3 (pad 1) over n pixels."""
     return (n - 1) // 2 + 1 if n > 0 else 0
+
+
+def conv3x3_conv1x1_bn_add_relu_i8(y1, w2, b2, m2, w3, b3, m3, m_r: int, S: int, r,
+                                   out=None, stream=None):
+    """Conv2 (3x3 + BN + ReLU) -> Conv3 (1x1 + BN + shortcut r + ReLU) of the
+    bottleneck in one launch; conv2's output stays on chip.
+    y1 [B, Cmid/32, H, W, 32]; r, out [B, Cout/32, H, W, 32]."""
+    B, Cmid, H, W = _act_shape(y1, "y1")
+    Cout = b3.numel()
+    if out is None:
+        out = torch.empty((B, Cout // 32, H, W, 32), dtype=torch.int8, device=y1.device)
+    with _same_device(y1, w2, b2, m2, w3, b3, m3, r, out):
+        st = lib().conv3x3_conv1x1_bn_add_relu_i8(
+            _dev(y1, torch.int8, "y1"), _dev(w2, torch.int8, "w2"), _dev(b2, torch.int32, "b2"),
+            _dev(m2, torch.int32, "m2"), _dev(w3, torch.int8, "w3"), _dev(b3, torch.int32, "b3"),
+            _dev(m3, torch.int32, "m3"), int(m_r), int(S), _dev(r, torch.int8, "r"),
+            _dev(out, torch.int8, "out"), B, H, W, Cmid, Cout, _stream(stream, y1.device))
+    _check(st, "conv3x3_conv1x1_bn_add_relu_i8")
+    return out
 
 
 def conv3x3s2_bn_relu_i8(x, w, bias, m, S: int, out=None, stream=None):
@@ -388,6 +409,12 @@ def x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R=1, stride=1, Ic2=0, has_res=Fal
     buf = ctypes.create_string_buffer(512)
     _check(lib().x1cb_describe_plan_ex(B, Hin, Win, Ic, Oc, R, stride, Ic2, int(has_res),
                                        int(pool), buf, 512), "x1cb_describe_plan_ex")
+    return buf.value.decode()
+
+
+def x1cb_describe_chain(B, H, W, Cmid=128, Cout=512) -> str:
+    buf = ctypes.create_string_buffer(512)
+    _check(lib().x1cb_describe_chain(B, H, W, Cmid, Cout, buf, 512), "x1cb_describe_chain")
     return buf.value.decode()
 
 

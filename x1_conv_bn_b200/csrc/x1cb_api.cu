@@ -332,6 +332,39 @@ int conv3x3_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias, co
     return conv_common(x, w, bias, m, 0, S, nullptr, out, B, H, W, Ic, Oc, 3, stream);
 }
 
+int conv3x3_conv1x1_bn_add_relu_i8(const int8_t *y1, const int8_t *w2, const int32_t *b2,
+                                   const int32_t *m2, const int8_t *w3, const int32_t *b3,
+                                   const int32_t *m3, int32_t m_r, int32_t S, const int8_t *r,
+                                   int8_t *out, int B, int H, int W, int Cmid, int Cout,
+                                   void *stream)
+{
+    if (int e = check_conv_shape(B, H, W, Cmid, Cout, S))
+        return e;
+    const size_t px = static_cast<size_t>(B) * H * W;
+    if (px == 0)
+        return X1CB_OK;
+    if (!y1 || !w2 || !b2 || !m2 || !w3 || !b3 || !m3 || !r || !out)
+        return X1CB_ERR_NULL;
+    if (!aligned16(y1) || !aligned16(w2) || !aligned16(w3) || !aligned16(r) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(b2) & 3u) || (reinterpret_cast<uintptr_t>(m2) & 3u) ||
+        (reinterpret_cast<uintptr_t>(b3) & 3u) || (reinterpret_cast<uintptr_t>(m3) & 3u))
+        return X1CB_ERR_ALIGN;
+    const size_t ob = px * Cout;
+    if (overlap(out, ob, y1, px * Cmid) || overlap(out, ob, r, ob) ||
+        overlap(out, ob, w2, static_cast<size_t>(Cmid) * Cmid * 9) ||
+        overlap(out, ob, w3, static_cast<size_t>(Cout) * Cmid))
+        return X1CB_ERR_OVERLAP;
+    ChainPlan cp;
+    if (int e = plan_chain(cp, B, H, W, Cmid, Cout, S, m_r))
+        return e;
+    if (int e = device_info_check())
+        return e;
+    if (int e = check_resident({y1, w2, b2, m2, w3, b3, m3, r, out}))
+        return e;
+    cp.wait_limit_ns = g_wait_limit_ns.load() ? g_wait_limit_ns.load() : kDefaultWaitNs;
+    return launch_chain(cp, y1, w2, b2, m2, w3, b3, m3, r, out, static_cast<cudaStream_t>(stream));
+}
+
 int conv3x3s2_bn_relu_i8(const int8_t *x, const int8_t *w, const int32_t *bias,
                          const int32_t *m, int32_t S, int8_t *out, int B, int H, int W, int Ic,
                          int Oc, void *stream)
@@ -592,6 +625,24 @@ int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int st
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
                   p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream, p.pw, p.ph);
+    return X1CB_OK;
+}
+
+int x1cb_describe_chain(int B, int H, int W, int Cmid, int Cout, char *buf, size_t len)
+{
+    if (!buf || len == 0)
+        return X1CB_ERR_NULL;
+    ChainPlan p;
+    if (int e = plan_chain(p, B, H, W, Cmid, Cout, 24, 1 << 23))
+        return e;
+    int clusters = 0;
+    if (resident_clusters(p.smem_bytes, clusters) != X1CB_OK)
+        clusters = 0;  // no device: the plan alone
+    std::snprintf(buf, len,
+                  "tile=%dx%dx%d rows=%d m_tiles=%d pairs=%d a_stages=%d r_stages=%d smem=%d "
+                  "resident_clusters=%d swz=%d",
+                  p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.n_pairs, p.a_stages, p.r_stages,
+                  p.smem_bytes, clusters, p.io_swz);
     return X1CB_OK;
 }
 

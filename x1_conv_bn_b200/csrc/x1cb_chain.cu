@@ -666,6 +666,43 @@ int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m
     return X1CB_OK;
 }
 
+// Clusters of two CTAs of chain23_kernel that fit on the current device at
+// once with `smem` bytes of shared memory each (cached per device and size).
+int resident_clusters(int smem, int &clusters)
+{
+    static std::mutex mu;
+    static int cached[64] = {}, cached_smem[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return X1CB_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[dev] == 0 || cached_smem[dev] != smem) {
+        if (int e = opt_in_smem(reinterpret_cast<const void *>(chain23_kernel), 2))
+            return e;
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, chain23_kernel, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return X1CB_ERR_CUDA;
+        }
+        cached[dev] = n;
+        cached_smem[dev] = smem;
+    }
+    clusters = cached[dev];
+    return X1CB_OK;
+}
+
 int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const int32_t *b2,
                  const int32_t *m2, const int8_t *w3, const int32_t *b3, const int32_t *m3,
                  const int8_t *x, int8_t *out, cudaStream_t stream)
@@ -723,9 +760,17 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
     }
     if (int e = opt_in_smem(reinterpret_cast<const void *>(chain23_kernel), 2))
         return e;
+    // The kernel is persistent with a static assignment of pair tiles, so it
+    // must not launch more clusters than can be resident at once: a cluster
+    // needs two SMs of one GPC, and a GPC with an odd number of free SMs
+    // leaves one over.
+    int clusters = 0;
+    if (int e = resident_clusters(p.smem_bytes, clusters))
+        return e;
+    const int grid = 2 * std::max(1, std::min(clusters, p.n_pairs));
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(p.grid, 1, 1);
+    cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = p.smem_bytes;
     cfg.stream = stream;
