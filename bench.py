@@ -244,14 +244,22 @@ def read_traffic(profile_name, src_sha):
     return float(m.group(1))
 
 
-def kernel_source_sha():
+KERNEL_SOURCES = {
+    # the files that define each kernel's device code and launch plan
+    "conv": ("x1cb_conv.cu", "x1cb_epi.cuh", "x1cb_ptx.cuh", "x1cb_plan.h"),
+    "chain": ("x1cb_chain.cu", "x1cb_epi.cuh", "x1cb_ptx.cuh", "x1cb_plan.h"),
+}
+
+
+def kernel_source_sha(kernel="conv"):
+    """Short hash of one kernel's sources: a profile's counters are used only
+    while the kernel they were taken on is unchanged."""
     import hashlib
 
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "x1_conv_bn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:12]
 
 
@@ -749,7 +757,8 @@ def main(argv=None):
         roof["algorithmic_bytes_per_launch"] = top["bytes"]
         roof["algorithmic_ops_per_launch"] = top["ops"]
         prof = f"bottleneck_{cfg}_b{s.B}.md"
-    roof["traffic"] = read_traffic(prof, kernel_source_sha())
+    roof["traffic"] = read_traffic(prof, kernel_source_sha("chain" if stages and
+                                                           "fused" in roof["kernel"] else "conv"))
     roof["traffic_source"] = (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
                               f"profiles/{prof}, taken on this kernel source"
                               if roof["traffic"] is not None else

@@ -21,15 +21,14 @@
 //               tile i, then Conv3 of pair tile i-1 in 128-channel chunks
 //   warp 2      TMA producer of the shortcut stages (own rows)
 //   warp 3      TMA store of finished output stages (own rows)
-//   warps 4-15  Conv3 epilogue: 3 turns per TMEM lane quarter, one per
-//               Conv3 accumulator slot; shortcut Sum, requantisation, ReLU
-//   warps 16-19 Conv2 epilogue (one per lane quarter, every tile): requantises
-//               Conv2 and writes the int8 result into this CTA's Conv3 A
-//               buffer in shared memory
-// TMEM (512 columns per CTA): Conv2's accumulator (128) and three Conv3
-// accumulator slots of 128 output channels.  Conv3's epilogue is the heavy
-// one (the shortcut and 4x the channels), so it gets 12 of the 16 epilogue
-// warps.
+//   warps 4-19  epilogue, 4 turns per TMEM lane quarter over one ring of
+//               accumulators: the MMA issuer fills four 128-column TMEM slots
+//               in issue order with Conv2 tiles and Conv3 chunks (item k in
+//               slot k % 4), and turn g takes items g, g+4, ...: a Conv2 item
+//               is requantised into this CTA's Conv3 A buffer in shared
+//               memory, a Conv3 item gets the shortcut Sum and is
+//               requantised into an output stage.  All 16 warps share both
+//               kinds of work (Conv3's is ~4x Conv2's per tile).
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
 // a status bit, and both CTAs leave through a bounded exit handshake.
 #include <cuda.h>
@@ -53,12 +52,11 @@ extern __device__ unsigned int g_dev_forms;
 
 namespace {
 
-constexpr int kA3Bufs = 2;          // Conv3 A buffers (Conv2 results) in shared memory
-constexpr int kAcc3 = 3;            // Conv3 accumulator slots (= Conv3 epilogue turns)
-constexpr int kE2Warp0 = 4, kE1Warp0 = 16;
+constexpr int kA3Bufs = 2;           // Conv3 A buffers (Conv2 results) in shared memory
+constexpr int kSlots = 4;            // 128-column accumulator slots (= epilogue turns)
 constexpr int kA3Bytes = 128 * 128;  // Conv3 A buffer: 128 rows x 128 channels
-static_assert(kE1Warp0 - kE2Warp0 == 4 * kAcc3, "one Conv3 turn per accumulator slot");
-static_assert(kThreads == 32 * (kE1Warp0 + 4), "20 warps");
+static_assert(kEpiWarps == 4 * kSlots, "one epilogue turn per accumulator slot");
+static_assert(kSlots * 128 == kTmemCols, "the slots fill the TMEM");
 constexpr int kHalfRows = 64;      // B rows (output channels) each CTA holds per MMA
 
 struct ChainBars {
@@ -70,12 +68,10 @@ struct ChainBars {
     __device__ uint32_t exit_bar() const { return at(2); }
     __device__ uint32_t a_full(int s) const { return at(3 + s); }
     __device__ uint32_t a_empty(int s) const { return at(3 + a_stages + s); }
-    __device__ uint32_t acc2_full() const { return at(3 + 2 * a_stages); }
-    __device__ uint32_t acc2_empty() const { return at(4 + 2 * a_stages); }
-    __device__ uint32_t a3_full(int k) const { return at(5 + 2 * a_stages + k); }
-    __device__ uint32_t a3_empty(int k) const { return at(7 + 2 * a_stages + k); }
-    __device__ uint32_t acc3_full(int k) const { return at(9 + 2 * a_stages + k); }
-    __device__ uint32_t acc3_empty(int k) const { return at(12 + 2 * a_stages + k); }
+    __device__ uint32_t acc_full(int k) const { return at(3 + 2 * a_stages + k); }
+    __device__ uint32_t acc_empty(int k) const { return at(7 + 2 * a_stages + k); }
+    __device__ uint32_t a3_full(int k) const { return at(11 + 2 * a_stages + k); }
+    __device__ uint32_t a3_empty(int k) const { return at(13 + 2 * a_stages + k); }
     __device__ uint32_t io_full(int s) const { return at(15 + 2 * a_stages + s); }
     __device__ uint32_t out_ready(int s) const { return at(15 + 2 * a_stages + r_stages + s); }
     __device__ uint32_t io_empty(int s) const { return at(15 + 2 * a_stages + 2 * r_stages + s); }
@@ -186,6 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + p.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + p.off_misc + 4);
+    // Conv3 items take the shortcut stages' arrivals in stage order (ticket).
+    volatile int *io_ticket = reinterpret_cast<volatile int *>(smem + p.off_misc + 8);
     ChainBars bars{sbase + static_cast<uint32_t>(p.off_bar), p.a_stages, p.r_stages};
     const WaitCtl ctl{abort_flag, &g_dev_status, p.wait_limit_ns};
     const uint64_t drain_ns = 200000000ull;
@@ -196,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- set-up -----------------------------------------------------------------
     if (threadIdx.x == 0) {
         *abort_flag = 0;
+        *io_ticket = 0;
         mbar_init(bars.w_full(), 1);
         mbar_init(bars.mma_done(), 1);
         mbar_init(bars.exit_bar(), 1);
@@ -206,15 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Arrival counts: commits arrive once (multicast to both CTAs); the
         // epilogue barriers on rank 0 take one arrival per warp of a lane
         // quarter from each CTA (4 x 2).
-        mbar_init(bars.acc2_full(), 1);
-        mbar_init(bars.acc2_empty(), 8);
+        for (int k = 0; k < kSlots; ++k) {
+            mbar_init(bars.acc_full(k), 1);
+            mbar_init(bars.acc_empty(k), 8);
+        }
         for (int k = 0; k < kA3Bufs; ++k) {
             mbar_init(bars.a3_full(k), 8);
             mbar_init(bars.a3_empty(k), 1);
-        }
-        for (int k = 0; k < kAcc3; ++k) {
-            mbar_init(bars.acc3_full(k), 1);
-            mbar_init(bars.acc3_empty(k), 8);
         }
         for (int s = 0; s < p.r_stages; ++s) {
             mbar_init(bars.io_full(s), 1);
@@ -389,21 +386,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             int st = 0;
             uint32_t ph = 0;
             uint64_t sd = a_desc0;
-            int n3_slot = 0;        // Conv3 accumulator slot of the next chunk
-            uint32_t n3_phase = 0;  // and its use parity
+            int slot = 0;        // accumulator slot of the next item (Conv2 tile or Conv3 chunk)
+            uint32_t sph = 0;    // and its use parity
             bool ok = __all_sync(0xffffffffu, mbar_wait_cl(bars.w_full(), 0, ctl, kDevTimeoutMma));
             for (int i = 0; ok && i <= n_my; ++i) {
                 if (i < n_my) {
-                    // Conv2 of pair tile i (TMEM columns 0-127): 4 channel blocks x 9 taps,
-                    // once the Conv2 epilogue has drained tile i - 1.
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait_cl(bars.acc2_empty(), (i & 1) ^ 1u, ctl,
-                                                 kDevTimeoutMma))) {
+                    // Conv2 of pair tile i: 4 channel blocks x 9 taps into the next slot.
+                    if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.acc_empty(slot), sph ^ 1u, ctl,
+                                                              kDevTimeoutMma))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d = tmem_base;
+                    const uint32_t d = tmem_base + static_cast<uint32_t>(slot * 128);
                     for (int c1 = 0; c1 < p.C1; ++c1) {
                         if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.a_full(st), ph, ctl,
                                                                   kDevTimeoutMma))) {
@@ -427,10 +422,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!ok)
                         break;
-                    mma_commit_pair(bars.acc2_full());
+                    mma_commit_pair(bars.acc_full(slot));
+                    if (++slot == kSlots) {
+                        slot = 0;
+                        sph ^= 1u;
+                    }
                 }
                 if (i >= 1) {
-                    // Conv3 of pair tile i - 1: A = its Conv2 result (buffer (i-1) % 2).
+                    // Conv3 of pair tile i - 1: A = its Conv2 result (buffer (i-1) % 2),
+                    // one 128-channel chunk per slot.
                     const int j = i - 1, b = j & 1;
                     if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.a3_full(b), (j >> 1) & 1, ctl,
                                                               kDevTimeoutMma))) {
@@ -440,25 +440,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint64_t ad = a3_desc0 + static_cast<uint64_t>(b) * a3_buf_step;
                     for (int c = 0; c < p.n_chunks; ++c) {
-                        // chunk n3 -> slot n3 % 3 (TMEM columns 128 + 128 * slot)
-                        const int k = n3_slot;
-                        if (!__all_sync(0xffffffffu,
-                                        mbar_wait_cl(bars.acc3_empty(k), n3_phase ^ 1u, ctl,
-                                                     kDevTimeoutMma))) {
+                        if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.acc_empty(slot), sph ^ 1u,
+                                                                  ctl, kDevTimeoutMma))) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t d = tmem_base + static_cast<uint32_t>(128 + k * 128);
+                        const uint32_t d = tmem_base + static_cast<uint32_t>(slot * 128);
                         for (int kb = 0; kb < p.C1; ++kb)
                             mma_i8_pair(d, ad + static_cast<uint64_t>(kb) * a3_kb_step,
                                         w3_desc0 +
                                             static_cast<uint64_t>(c * p.C1 + kb) * kb_step,
                                         idesc, kb ? 1u : 0u);
-                        mma_commit_pair(bars.acc3_full(k));
-                        if (++n3_slot == kAcc3) {
-                            n3_slot = 0;
-                            n3_phase ^= 1u;
+                        mma_commit_pair(bars.acc_full(slot));
+                        if (++slot == kSlots) {
+                            slot = 0;
+                            sph ^= 1u;
                         }
                     }
                     if (!ok)
@@ -471,51 +468,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 atomicOr(&g_dev_status, kDevDrainFailed);
         }
         __syncwarp();
-    } else if (warp >= kE1Warp0) {
-        // ---- Conv2 epilogue: accumulator -> int8 -> this CTA's Conv3 A buffer ------
-        // One warp per lane quarter takes every tile, so it sees every phase of
-        // the Conv2 accumulator and of both A buffers in order.
+    } else {
+        // ---- epilogue: items of the accumulator ring, turn g takes items g, g+4, ... --
+        // Item order is the MMA issuer's: Conv2 of tile i, then Conv3 of tile
+        // i - 1 in n_chunks chunks.  Each turn owns slot `turn` (items k with
+        // k % 4 == turn), so it sees every phase of its slot in order.
         const int q = warp & 3;
+        const int turn = (warp - kEpiWarp0) >> 2;
         const int row = q * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        const uint32_t e2_0 = mapa_shared(bars.acc2_empty(), 0);
-        uint32_t rsel[4] = {0, 0, 0, 0};
-        for (int i = 0; i < n_my; ++i) {
-            const int b = i & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(bars.acc2_full(), static_cast<uint32_t>(i & 1),
-                                                   ctl, kDevTimeoutEpilogue)))
-                break;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(bars.a3_empty(b), static_cast<uint32_t>((i >> 1) & 1) ^ 1u,
-                                      ctl, kDevTimeoutEpilogue)))
-                break;
-            tc_fence_after();
-            uint8_t *a3 = smem + p.off_a3 + b * kA3Bytes;
-            const uint32_t tb = tmem_base + lane_addr;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32], ow[8];
-                __syncwarp();
-                tmem_ld_32x32b_x32_sync(tb + static_cast<uint32_t>(c * 32), v);
-                requant_any<false>(mode2, v, cm2, cc2, c * 32, nullptr, 0, p.S, 0, rsel, ow);
-                // K block c of the A buffer: two 16-byte halves, rows 16 bytes apart.
-                uint4 *dst = reinterpret_cast<uint4 *>(a3 + c * (kA3Bytes / 4) + row * 16);
-                dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                dst[(kA3Bytes / 8) / 16] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-            }
-            fence_proxy_async_smem();  // the MMA (async proxy, issued by rank 0) reads it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_cluster(e2_0);
-                mbar_arrive_cluster(mapa_shared(bars.a3_full(b), 0));
-            }
-        }
-    } else {
-        // ---- Conv3 epilogue: shortcut Sum + requantisation into the output stage --------
-        const int q = warp & 3;
-        const int turn = (warp - kE2Warp0) >> 2;  // owns Conv3 slot `turn`
-        const int row = q * 32 + lane;
+        const uint32_t tslot = tmem_base + lane_addr + static_cast<uint32_t>(turn * 128);
+        const uint32_t empty0 = mapa_shared(bars.acc_empty(turn), 0);
+        // Conv3 output rows: this row's place in an output stage (halo rows
+        // outside the image are computed and not stored).
         const int plane_t = p.tw * p.th;
         const int xi = row % p.row_pitch;
         const int yi = (row % p.plane_m) / p.row_pitch;
@@ -524,56 +489,103 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
         const int chunk_stride = plane_t * 32;
         const int swz_mask = p.io_swz ? 0x70 : 0;
-        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        const uint32_t e3_0 = mapa_shared(bars.acc3_empty(turn), 0);
-        uint32_t rsel[4];
-        const int mr2 = shortcut_operands(mode3, p.m_r, p.S, rsel);
-        const long long total = static_cast<long long>(n_my) * p.n_chunks;
-        for (long long n = turn; n < total; n += kAcc3) {
-            const int c = static_cast<int>(n % p.n_chunks);
-            const int st = static_cast<int>(n % p.r_stages);
-            const uint32_t st_phase = static_cast<uint32_t>((n / p.r_stages) & 1);
-            if (!__all_sync(0xffffffffu, mbar_wait(bars.acc3_full(turn),
-                                                   static_cast<uint32_t>((n / kAcc3) & 1), ctl,
-                                                   kDevTimeoutEpilogue)))
-                break;
-            tc_fence_after();
-            // The stage's previous use (stage n - r_stages, another turn's) must be
-            // complete before its arrival is awaited: wait until it was stored, as
-            // the producer does (exact with at least as many stages as turns).
-            if (!__all_sync(0xffffffffu, mbar_wait(bars.io_empty(st), st_phase ^ 1u, ctl,
-                                                   kDevTimeoutEpilogue)))
-                break;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(bars.io_full(st), st_phase, ctl, kDevTimeoutEpilogue)))
-                break;
-            const uint32_t tb = tmem_base + lane_addr + static_cast<uint32_t>(128 + turn * 128);
-            uint8_t *stage = smem + p.off_r + st * kRSlotBytes;
+        uint32_t rsel3[4];
+        const int mr2 = shortcut_operands(mode3, p.m_r, p.S, rsel3);
+        const uint32_t rsel2[4] = {0, 0, 0, 0};
+        int k = 0;             // item index in issue order
+        uint32_t kph = 0;      // parity of this turn's slot at its next item
+        bool ok = true;
+        for (int i = 0; ok && i <= n_my; ++i) {
+            if (i < n_my) {
+                if ((k & 3) == turn) {
+                    // Conv2 of tile i -> int8 -> A buffer i % 2 of this CTA.
+                    const int b = i & 1;
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
+                        !__all_sync(0xffffffffu,
+                                    mbar_wait(bars.a3_empty(b),
+                                              static_cast<uint32_t>((i >> 1) & 1) ^ 1u, ctl,
+                                              kDevTimeoutEpilogue))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *a3 = smem + p.off_a3 + b * kA3Bytes;
 #pragma unroll 1
-            for (int cs = 0; cs < kRChunks; ++cs) {
-                const int ch = c * 128 + cs * 32;
-                uint32_t v[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32_sync(tb + static_cast<uint32_t>(cs * 32), v);
-                const int o = row_off + cs * chunk_stride;
-                const int sw = swz_mask & (o >> 3);
-                uint4 *pa = reinterpret_cast<uint4 *>(stage + (o ^ sw));
-                uint4 *pb = reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw));
-                const uint4 ra = *pa, rb = *pb;
-                const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-                uint32_t ow[8];
-                requant_any<true>(mode3, v, cm3, cc3, ch, rw, p.m_r, p.S, mr2, rsel, ow);
-                if (in_box) {
-                    *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t v[32], ow[8];
+                        __syncwarp();
+                        tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(c * 32), v);
+                        requant_any<false>(mode2, v, cm2, cc2, c * 32, nullptr, 0, p.S, 0, rsel2,
+                                           ow);
+                        // K block c of the A buffer: two 16-byte halves, rows 16 bytes apart.
+                        uint4 *dst = reinterpret_cast<uint4 *>(a3 + c * (kA3Bytes / 4) + row * 16);
+                        dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        dst[(kA3Bytes / 8) / 16] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                    }
+                    fence_proxy_async_smem();  // read by the MMA (async proxy, rank 0's issue)
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_cluster(empty0);
+                        mbar_arrive_cluster(mapa_shared(bars.a3_full(b), 0));
+                    }
+                    kph ^= 1u;
                 }
+                ++k;
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bars.out_ready(st));
-                mbar_arrive_cluster(e3_0);
+            if (i >= 1) {
+                const int j = i - 1;
+                for (int c = 0; c < p.n_chunks; ++c, ++k) {
+                    if ((k & 3) != turn)
+                        continue;
+                    // Conv3 of tile j, output chunk c: shortcut stage n = j*n_chunks + c.
+                    const long long n = static_cast<long long>(j) * p.n_chunks + c;
+                    const int st = static_cast<int>(n % p.r_stages);
+                    const uint32_t st_phase = static_cast<uint32_t>((n / p.r_stages) & 1);
+                    // Stages are taken in order (the ticket), so each stage's
+                    // previous phase is complete before its arrival is awaited.
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
+                        !__all_sync(0xffffffffu, ticket_wait(io_ticket, static_cast<int>(n), ctl,
+                                                             kDevTimeoutEpilogue)) ||
+                        !__all_sync(0xffffffffu, mbar_wait(bars.io_full(st), st_phase, ctl,
+                                                           kDevTimeoutEpilogue))) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0)
+                        atomicMax(const_cast<int *>(io_ticket), static_cast<int>(n + 1));
+                    tc_fence_after();
+                    uint8_t *stage = smem + p.off_r + st * kRSlotBytes;
+#pragma unroll 1
+                    for (int cs = 0; cs < kRChunks; ++cs) {
+                        const int ch = c * 128 + cs * 32;
+                        uint32_t v[32];
+                        __syncwarp();
+                        tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(cs * 32), v);
+                        const int o = row_off + cs * chunk_stride;
+                        const int sw = swz_mask & (o >> 3);
+                        uint4 *pa = reinterpret_cast<uint4 *>(stage + (o ^ sw));
+                        uint4 *pb = reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw));
+                        const uint4 ra = *pa, rb = *pb;
+                        const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+                        uint32_t ow[8];
+                        requant_any<true>(mode3, v, cm3, cc3, ch, rw, p.m_r, p.S, mr2, rsel3, ow);
+                        if (in_box) {
+                            *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                            *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(bars.out_ready(st));
+                        mbar_arrive_cluster(empty0);
+                    }
+                    kph ^= 1u;
+                }
             }
         }
     }
@@ -654,10 +666,9 @@ int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m
         return p.smem_bytes <= kSmemLimit;
     };
     // Deepest shortcut ring beside at least four halo slots (fewer if needed).
-    // (the shortcut ring needs at least one stage per Conv3 epilogue turn)
     bool placed = false;
     for (int a = 4; a >= 2 && !placed; --a)
-        for (int r = 8; r >= kAcc3 && !placed; --r)
+        for (int r = 8; r >= 2 && !placed; --r)
             placed = layout(a, r);
     if (!placed)
         return X1CB_ERR_SHAPE;
