@@ -292,6 +292,37 @@ def device_inputs(cfg, dev, seed, n_sets=1):
                                  stream=stream)
 
         return call, {"x": x}, outs[0]
+    if isinstance(s, synth.StemShape):
+        # the image width-folded (the stem's layout step, not timed): each
+        # pixel carries its filter row's 7 taps x 3 channels
+        inp = synth.stem_inputs(s, seed, device=dev)
+        x = X.x1cb_pack_stem(inp.x, R=s.R)
+        w = X.x1cb_pack_stem_weight(inp.w)
+        del inp.x
+        xs = [x] + [x.clone() for _ in range(n_sets - 1)]
+        outs = [torch.empty((s.B, s.Oc // 32, s.Hp, s.Wp, 32), dtype=torch.int8, device=dev)
+                for _ in range(n_sets)]
+
+        def call(i=0, x_=None, out_=None, stream=None):
+            X.stem_conv_bn_relu_maxpool_i8(xs[i] if x_ is None else x_, w, inp.bias, inp.m,
+                                           inp.S, R=s.R, out=outs[i] if out_ is None else out_,
+                                           stream=stream)
+
+        return call, {"x": x}, outs[0]
+    if isinstance(s, synth.ConvShape) and s.R == 3:
+        inp = synth.conv_inputs(s, seed, device=dev)
+        x = X.x1cb_pack_act(inp.x)
+        w = X.x1cb_pack_weight(inp.w)
+        del inp.x
+        xs = [x] + [x.clone() for _ in range(n_sets - 1)]
+        outs = [torch.empty((s.B, s.Oc // 32, s.H, s.W, 32), dtype=torch.int8, device=dev)
+                for _ in range(n_sets)]
+
+        def call(i=0, x_=None, out_=None, stream=None):
+            X.conv3x3_bn_relu_i8(xs[i] if x_ is None else x_, w, inp.bias, inp.m, inp.S,
+                                 out=outs[i] if out_ is None else out_, stream=stream)
+
+        return call, {"x": x}, outs[0]
     if isinstance(s, synth.BlockShape):
         inp = synth.block_inputs(s, seed, device=dev)
         x = X.x1cb_pack_act(inp.x)
@@ -345,13 +376,14 @@ class OracleSample:
         # output pixels per image (the projection block halves the image; its
         # oracle runs whole images, so its sample is whole images)
         self.proj = isinstance(s, synth.ProjBlockShape)
-        self.hw = s.Ho * s.Wo if self.proj else s.H * s.W
+        self.stem = isinstance(s, synth.StemShape)
+        self.hw = s.Ho * s.Wo if self.proj else (s.Hp * s.Wp if self.stem else s.H * s.W)
         self._make(1, seed)
         t = self._run(self.hw)
         per_px = t / self.hw
         n = int(max(1, min(s.B * self.hw, seconds / max(per_px, 1e-9))))
         imgs = (n + self.hw - 1) // self.hw
-        if self.proj:
+        if self.proj or self.stem:  # whole images
             n = imgs * self.hw
         if imgs > 1:
             self._make(imgs, seed)
@@ -360,7 +392,11 @@ class OracleSample:
 
     def _make(self, imgs, seed):
         s = self.s
-        if isinstance(s, synth.ProjBlockShape):
+        if isinstance(s, synth.StemShape):
+            import dataclasses
+
+            self.inp = synth.stem_inputs(dataclasses.replace(s, B=imgs), seed)
+        elif isinstance(s, synth.ProjBlockShape):
             self.inp = synth.proj_block_inputs(
                 synth.ProjBlockShape(imgs, s.H, s.W, s.Cin, s.Cmid, s.Cout), seed)
         elif isinstance(s, synth.BlockShape):
@@ -373,7 +409,9 @@ class OracleSample:
         inp, O = self.inp, self.O
         pix = torch.arange(n, dtype=torch.int64)
         t0 = time.perf_counter()
-        if self.proj:
+        if self.stem:
+            O.conv_pool(inp.x, inp.w, inp.bias, inp.m, inp.S, stride=self.s.stride)
+        elif self.proj:
             O.bottleneck_proj(inp.x, inp.w, inp.wp, inp.bias, inp.m, inp.S)
         elif isinstance(self.s, synth.BlockShape):
             O.bottleneck_pixels(inp.x, inp.w, inp.bias, inp.m, inp.m_r, inp.S, pix)
@@ -743,10 +781,21 @@ def main(argv=None):
     gbs = nbytes / (ms_max * 1e-3) / 1e9
     if stages is None:
         roof = roofline(ops, nbytes, ms_max * 1e-3, hbm, bf16, peak_kind)
-        roof["kernel"] = "conv_bn_act_kernel<1> (1x1 with shortcut)"
+        if isinstance(s, synth.StemShape):
+            roof["kernel"] = ("conv_bn_act_kernel<0> (pool mode: 7x1/2 conv over the "
+                              "width-folded image + BN + ReLU + max pool)")
+            roof["note"] = ("ops count the image's 3 real channels; the kernel multiplies the "
+                            "folded 32-channel block (21 used)")
+            prof = f"stem_b{s.B}.md"
+        elif s.R == 3:
+            roof["kernel"] = "conv_bn_act_kernel<0> (3x3, halo form)"
+            prof = f"conv3x3_{cfg}_b{s.B}.md"
+        else:
+            roof["kernel"] = "conv_bn_act_kernel<1> (1x1 with shortcut)"
+            prof = (f"conv1x1_res32_b{s.B}.md" if cfg in ("2", "3")
+                    else f"conv1x1_{cfg}_b{s.B}.md")
         roof["algorithmic_bytes_per_launch"] = nbytes
         roof["algorithmic_ops_per_launch"] = ops
-        prof = f"conv1x1_res32_b{s.B}.md" if cfg in ("2", "3") else f"conv1x1_{cfg}.md"
     else:
         for stg in stages:
             stg["roofline"] = roofline(stg["ops"], stg["bytes"], stg["us"] * 1e-6, hbm, bf16,

@@ -170,6 +170,22 @@ int conv_bn_relu_maxpool_i8(const int8_t *x, const int8_t *w, const int32_t *bia
                             const int32_t *m, int32_t S, int8_t *out, int B, int H, int W, int Ic,
                             int Oc, int R, int stride, void *stream);
 
+/*
+ * The same stem with the image width-folded (the layout step
+ * x1cb_pack_stem): each pixel of the folded tensor carries its filter row's
+ * R taps x Cin channels in its 32-channel block, so the R x R convolution is
+ * an R x 1 convolution with R*Cin useful channels per K step instead of Cin
+ * (21 of 32 for ResNet50's 7x7 over RGB, against 3 of 32 unfolded: 7x fewer
+ * MMAs for the same result).  Stride 2, pad (R-1)/2, 64 outputs, then 3x3
+ * stride-2 max pooling; bit-identical to conv_bn_relu_maxpool_i8 on the
+ * unfolded image.
+ *   folded [B, 1, H, W, 32] (x1cb_pack_stem); wf [1, R, 1, 1, 64, 32]
+ *   (x1cb_pack_stem_weight); bias, m [64]; out [B, 2, Hp, Wp, 32] as above.
+ */
+int stem_conv_bn_relu_maxpool_i8(const int8_t *folded, const int8_t *wf, const int32_t *bias,
+                                 const int32_t *m, int32_t S, int8_t *out, int B, int H, int W,
+                                 int R, void *stream);
+
 /* Bytes of device workspace bottleneck_proj_i8 needs for an H x W input:
  * [B, Cmid/32, H, W, 32] and [B, Cmid/32, Ho, Wo, 32]. */
 size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid);
@@ -255,6 +271,18 @@ int x1cb_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C
  * [Oc/O2, R, R, Ic/32, O2, 32] with O2 = 128 (O2 = 64 for a 64-channel
  * layer); R in {1, 3, 5, 7}. */
 int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R, void *stream);
+
+/* Width-folded stem input: nhwc [B, H, W, Cin] image -> folded [B, 1, H, W, 32]
+ * with channel ds*Cin + ci of pixel (h, u) = channel ci of image pixel
+ * (h, u - (R-1)/2 + ds), zero outside the image and from R*Cin on; needs
+ * R*Cin <= 32. */
+int x1cb_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int Cin, int R,
+                   void *stream);
+
+/* Folded stem weights: oihw [64, Cin, R, R] -> [1, R, 1, 1, 64, 32] with entry
+ * (dr, o, ds*Cin + ci) = w[o, ci, dr, ds], zero from R*Cin on. */
+int x1cb_pack_stem_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Cin, int R,
+                          void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *x1cb_status_string(int status);

@@ -101,3 +101,56 @@ def test_stem_full_size_every_output(oracle):
     ref = oracle.conv_pool(x, w, bias, m, S, stride=2)
     assert torch.equal(got, ref), int((got != ref).sum())
     assert (ref == 0).float().mean() < 0.9
+
+
+def _gpu_folded_stem(x, w, bias, m, S, R):
+    folded = X.x1cb_pack_stem(x.to(DEV).contiguous(), R=R)
+    wf = X.x1cb_pack_stem_weight(w.to(DEV).contiguous())
+    out = X.stem_conv_bn_relu_maxpool_i8(folded, wf, bias.to(DEV), m.to(DEV), S, R=R)
+    torch.cuda.synchronize()
+    st, bits = X.x1cb_last_device_error(clear=True)
+    assert st == 0, hex(bits)
+    return _nhwc(out.cpu())
+
+
+FOLDED = [
+    (2, 224, 224, 3, 7),
+    (1, 37, 29, 3, 7),
+    (3, 20, 18, 4, 7),     # 28 of 32 channels used
+    (2, 15, 17, 10, 3),    # 3x3 over 10 channels: 30 of 32
+    (1, 6, 5, 3, 5),
+]
+
+
+@pytest.mark.parametrize("shape", FOLDED, ids=[str(s) for s in FOLDED])
+def test_folded_stem_parity(oracle, shape):
+    """The width-folded stem (R x 1 over the folded image) against the
+    oracle's R x R stem on the plain image."""
+    B, H, W, Cin, R = shape
+    x, w, bias, m, S = _stem_case(B, H, W, Cin, R, 7 * sum(shape))
+    got = _gpu_folded_stem(x, w, bias, m, S, R)
+    ref = oracle.conv_pool(x, w, bias, m, S, stride=2)
+    assert got.shape == ref.shape
+    assert torch.equal(got, ref), int((got != ref).sum())
+    assert ref.unique().numel() > 10
+
+
+def test_pack_stem_layout():
+    """Folded pixel (h, u), channel ds*Cin + ci = image pixel (h, u - 3 + ds),
+    channel ci (zero outside); channels from R*Cin on are zero."""
+    g = torch.Generator().manual_seed(4)
+    x = torch.randint(-128, 128, (2, 5, 9, 3), generator=g, dtype=torch.int8)
+    got = X.x1cb_pack_stem(x.to(DEV), R=7).cpu().reshape(2, 5, 9, 32)
+    ref = torch.zeros(2, 5, 9, 32, dtype=torch.int8)
+    xp = torch.nn.functional.pad(x, (0, 0, 3, 3))  # pad W by 3 on both sides
+    for ds in range(7):
+        ref[..., ds * 3:ds * 3 + 3] = xp[:, :, ds:ds + 9, :]
+    assert torch.equal(got, ref)
+
+
+def test_folded_stem_full_size_every_output(oracle):
+    """ResNet50's stem at B=64 through the folded path, every output byte."""
+    x, w, bias, m, S = _stem_case(64, 224, 224, 3, 7, 2025)
+    got = _gpu_folded_stem(x, w, bias, m, S, 7)
+    ref = oracle.conv_pool(x, w, bias, m, S, stride=2)
+    assert torch.equal(got, ref), int((got != ref).sum())

@@ -77,6 +77,9 @@ def lib() -> ctypes.CDLL:
         L.conv_bn_relu_maxpool_i8.argtypes = [vp] * 4 + [i32, vp] + [i] * 7 + [vp]
         L.x1cb_describe_chain.argtypes = [i] * 5 + [ctypes.c_char_p, sz]
         L.conv3x3_conv1x1_bn_add_relu_i8.argtypes = [vp] * 7 + [i32, i32, vp, vp] + [i] * 5 + [vp]
+        L.stem_conv_bn_relu_maxpool_i8.argtypes = [vp] * 4 + [i32, vp] + [i] * 4 + [vp]
+        L.x1cb_pack_stem.argtypes = [vp, vp] + [i] * 5 + [vp]
+        L.x1cb_pack_stem_weight.argtypes = [vp, vp] + [i] * 3 + [vp]
         _lib = L
     return _lib
 
@@ -293,6 +296,50 @@ def conv_bn_relu_maxpool_i8(x, w, bias, m, S: int, R: int = 7, stride: int = 2, 
             _dev(m, torch.int32, "m"), int(S), _dev(out, torch.int8, "out"), B, H, W, Ic, Oc,
             int(R), int(stride), _stream(stream, x.device))
     _check(st, "conv_bn_relu_maxpool_i8")
+    return out
+
+
+def x1cb_pack_stem(nhwc, R: int = 7, out=None, stream=None):
+    """Image [B, H, W, Cin] -> width-folded [B, 1, H, W, 32] (R*Cin <= 32)."""
+    B, H, W, Cin = nhwc.shape
+    if out is None:
+        out = torch.empty((B, 1, H, W, 32), dtype=torch.int8, device=nhwc.device)
+    with _same_device(nhwc, out):
+        st = lib().x1cb_pack_stem(_dev(nhwc, torch.int8, "nhwc"), _dev(out, torch.int8, "out"),
+                                  B, H, W, Cin, int(R), _stream(stream, nhwc.device))
+    _check(st, "x1cb_pack_stem")
+    return out
+
+
+def x1cb_pack_stem_weight(oihw, out=None, stream=None):
+    """[64, Cin, R, R] -> folded [1, R, 1, 1, 64, 32]."""
+    Oc, Cin, R, _ = oihw.shape
+    if out is None:
+        out = torch.empty((1, R, 1, 1, Oc, 32), dtype=torch.int8, device=oihw.device)
+    with _same_device(oihw, out):
+        st = lib().x1cb_pack_stem_weight(_dev(oihw, torch.int8, "oihw"),
+                                         _dev(out, torch.int8, "out"), Oc, Cin, R,
+                                         _stream(stream, oihw.device))
+    _check(st, "x1cb_pack_stem_weight")
+    return out
+
+
+def stem_conv_bn_relu_maxpool_i8(folded, wf, bias, m, S: int, R: int = 7, out=None,
+                                 stream=None):
+    """The stem on a width-folded image: R x R stride-2 conv + BN + ReLU +
+    3x3 stride-2 max pooling, 64 outputs.  folded [B, 1, H, W, 32]."""
+    B, C, H, W = _act_shape(folded, "folded")
+    pad = (R - 1) // 2
+    Hc, Wc = (H + 2 * pad - R) // 2 + 1, (W - 1) // 2 + 1
+    if out is None:
+        out = torch.empty((B, 2, _half(Hc), _half(Wc), 32), dtype=torch.int8,
+                          device=folded.device)
+    with _same_device(folded, wf, bias, m, out):
+        st = lib().stem_conv_bn_relu_maxpool_i8(
+            _dev(folded, torch.int8, "folded"), _dev(wf, torch.int8, "wf"),
+            _dev(bias, torch.int32, "bias"), _dev(m, torch.int32, "m"), int(S),
+            _dev(out, torch.int8, "out"), B, H, W, int(R), _stream(stream, folded.device))
+    _check(st, "stem_conv_bn_relu_maxpool_i8")
     return out
 
 

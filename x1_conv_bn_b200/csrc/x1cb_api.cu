@@ -52,7 +52,7 @@ int device_info(int &sms)
 // a B=1 call is latency-bound).
 struct PlanKey {
     int B, H, W, Ic, Oc, R, has_res, sms;
-    int stride, Hin, Win, Ic2, stride2, Hin2, Win2, pool;
+    int stride, Hin, Win, Ic2, stride2, Hin2, Win2, pool, Rw;
     bool operator==(const PlanKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
 
@@ -66,7 +66,7 @@ int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_re
     PlanKey k;
     std::memset(&k, 0, sizeof(k));
     k = PlanKey{B, H, W, Ic, Oc, R, has_res, sms,
-                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2, g.pool};
+                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2, g.pool, g.Rw};
     {
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < used; ++i)
@@ -185,13 +185,14 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
                      int32_t S, int8_t *out, int B, int Hin, int Win, int Ic, int Oc, int R,
                      int stride, const int8_t *x2, const int8_t *w2, int Ic2, int Hin2,
                      int Win2, int stride2, void *stream, bool check_ptrs = true,
-                     bool pool = false)
+                     bool pool = false, int Rw = 0)
 {
     const int pad = (R - 1) / 2;
+    const int Rw_ = Rw > 0 ? Rw : R, padw = (Rw_ - 1) / 2;
     if (Hin < 0 || Win < 0 || stride < 1 || stride > 8 || stride2 < 1 || stride2 > 8)
         return X1CB_ERR_SHAPE;
     const int H = Hin + 2 * pad >= R ? (Hin + 2 * pad - R) / stride + 1 : 0;
-    const int W = Win + 2 * pad >= R ? (Win + 2 * pad - R) / stride + 1 : 0;
+    const int W = Win + 2 * padw >= Rw_ ? (Win + 2 * padw - Rw_) / stride + 1 : 0;
     // (a pooled layer has 64 output channels: checked as 128 here, exactly below)
     if (int e = check_conv_shape(B, Hin, Win, Ic, pool ? 128 : Oc, S))
         return e;
@@ -222,7 +223,7 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
     const size_t in_bytes = static_cast<size_t>(B) * Hin * Win * Ic;
     const size_t in2_bytes = static_cast<size_t>(B) * Hin2 * Win2 * Ic2;
     if (overlap(out, out_bytes, x, in_bytes) || overlap(out, out_bytes, x2, in2_bytes) ||
-        overlap(out, out_bytes, w, static_cast<size_t>(Oc) * Ic * R * R) ||
+        overlap(out, out_bytes, w, static_cast<size_t>(Oc) * Ic * R * Rw_) ||
         overlap(out, out_bytes, w2, static_cast<size_t>(Oc) * Ic2) ||
         overlap(out, out_bytes, bias, Oc * 4u) || overlap(out, out_bytes, m, Oc * 4u))
         return X1CB_ERR_OVERLAP;
@@ -241,6 +242,7 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
     g.Hin2 = Hin2;
     g.Win2 = Win2;
     g.pool = pool ? 1 : 0;
+    g.Rw = Rw;
     ConvPlan p;
     if (int e = get_plan(p, B, H, W, Ic, Oc, R, 0, S, 0, sms, g))
         return e;
@@ -394,6 +396,18 @@ int conv_bn_relu_maxpool_i8(const int8_t *x, const int8_t *w, const int32_t *bia
                             0, 0, 0, 1, stream, true, true);
 }
 
+int stem_conv_bn_relu_maxpool_i8(const int8_t *folded, const int8_t *wf, const int32_t *bias,
+                                 const int32_t *m, int32_t S, int8_t *out, int B, int H, int W,
+                                 int R, void *stream)
+{
+    // R x R stride-2 convolution of the image as an R x 1 convolution of its
+    // width-folded form (one 32-channel block per pixel), then pooling.
+    if (R != 1 && R != 3 && R != 5 && R != 7)
+        return X1CB_ERR_SHAPE;
+    return conv_geom_common(folded, wf, bias, m, S, out, B, H, W, 32, 64, R, 2, nullptr, nullptr,
+                            0, 0, 0, 1, stream, true, true, 1);
+}
+
 size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid)
 {
     if (B < 0 || H < 0 || W < 0 || Cmid < 0)
@@ -511,6 +525,41 @@ int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R,
     if (int e = check_resident({oihw, blocked}))
         return e;
     return launch_pack_weight(oihw, blocked, Oc, Ic, R, static_cast<cudaStream_t>(stream));
+}
+
+int x1cb_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int Cin, int R,
+                   void *stream)
+{
+    if (B < 0 || H < 0 || W < 0 || Cin < 1 || (R != 1 && R != 3 && R != 5 && R != 7) ||
+        R * Cin > 32)
+        return X1CB_ERR_SHAPE;
+    if (static_cast<size_t>(B) * H * W == 0)
+        return X1CB_OK;
+    if (!nhwc || !folded)
+        return X1CB_ERR_NULL;
+    if (!aligned16(folded))
+        return X1CB_ERR_ALIGN;
+    const size_t px = static_cast<size_t>(B) * H * W;
+    if (overlap(nhwc, px * Cin, folded, px * 32))
+        return X1CB_ERR_OVERLAP;
+    if (int e = check_resident({nhwc, folded}))
+        return e;
+    return launch_pack_stem(nhwc, folded, B, H, W, Cin, R, static_cast<cudaStream_t>(stream));
+}
+
+int x1cb_pack_stem_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Cin, int R,
+                          void *stream)
+{
+    if (!oihw || !blocked)
+        return X1CB_ERR_NULL;
+    if (Oc != 64 || Cin < 1 || (R != 1 && R != 3 && R != 5 && R != 7) || R * Cin > 32)
+        return X1CB_ERR_SHAPE;
+    if (overlap(oihw, static_cast<size_t>(Oc) * Cin * R * R, blocked,
+                static_cast<size_t>(R) * Oc * 32))
+        return X1CB_ERR_OVERLAP;
+    if (int e = check_resident({oihw, blocked}))
+        return e;
+    return launch_pack_stem_weight(oihw, blocked, Oc, Cin, R, static_cast<cudaStream_t>(stream));
 }
 
 const char *x1cb_status_string(int s)

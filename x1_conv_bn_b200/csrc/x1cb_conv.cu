@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // blocks; counters instead of divisions keep the issue cheap.
                 // Output pixel (w0, h0) reads input (w0*stride + ds - pad, ...);
                 // a strided map steps `stride` input pixels per loaded pixel.
-                const int wi0 = w0 * p.stride - p.pad, hi0 = h0 * p.stride - p.pad;
+                const int wi0 = w0 * p.stride - p.padw, hi0 = h0 * p.stride - p.pad;
                 int c1 = 0, ds = 0, dr = 0;
                 bool second = false;
                 for (int bx = 0; bx < boxes; ++bx) {
@@ -562,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          h0 * p.stride2, b0, c1, pol);
                     if (wpart) {  // the box's K blocks' weights
                         const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
-                        const int kb0 = second ? c1 : (dr * p.R + ds) * p.C1 + c1;
+                        const int kb0 = second ? c1 : (dr * p.Rw + ds) * p.C1 + c1;
                         for (int i = 0; i < p.a_kc; ++i) {
                             if (!second)
                                 tma_load_4d(wdst + i * wkb, &tmW, bars.a_full(stage), 0, 0,
@@ -583,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     c1 += p.a_kc;
                     if (!second && c1 == p.C1) {
                         c1 = 0;
-                        if (++ds == p.R) {
+                        if (++ds == p.Rw) {
                             ds = 0;
                             if (++dr == p.R)
                                 second = true;  // only reached when C1b > 0
@@ -996,6 +996,10 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     p.Oc = Oc;
     p.R = R;
     p.pad = (R - 1) / 2;
+    // Filter width: R (square), or 1 for a column filter over a width-folded
+    // image (each pixel already holds its row's taps in its channels).
+    p.Rw = g.Rw > 0 ? g.Rw : R;
+    p.padw = (p.Rw - 1) / 2;
     p.C1 = Ic / 32;
     p.O1 = Oc / 32;
     p.has_res = has_res;
@@ -1012,7 +1016,8 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         return X1CB_ERR_SHAPE;  // the TMA's traversal step is at most 8
     // Every tapped input pixel must exist for some output: (H-1)*stride + R - 1
     // - pad < Hin + pad, and the output extent is the convolution's.
-    if ((p.Hin + 2 * p.pad - R) / p.stride + 1 != H || (p.Win + 2 * p.pad - R) / p.stride + 1 != W)
+    if ((p.Hin + 2 * p.pad - R) / p.stride + 1 != H ||
+        (p.Win + 2 * p.padw - p.Rw) / p.stride + 1 != W)
         return X1CB_ERR_SHAPE;
     if (p.C1b && ((H - 1) * p.stride2 >= p.Hin2 || (W - 1) * p.stride2 >= p.Win2))
         return X1CB_ERR_SHAPE;
@@ -1037,7 +1042,7 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     }
     // The 3x3 convolution uses the halo form whenever one framed image row fits
     // in the 128 GEMM rows (stride 1).
-    p.halo = (R == 3 && p.pad == 1 && p.stride == 1 && p.C1b == 0 && !p.pool &&
+    p.halo = (R == 3 && p.Rw == 3 && p.stride == 1 && p.C1b == 0 && !p.pool &&
               W + 2 <= kTileRows) ? 1 : 0;
     if (p.halo) {
         choose_halo_tile(B, H, W, p.th, p.tg);
@@ -1082,7 +1087,7 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     if (mtiles > INT_MAX / 2)
         return X1CB_ERR_SHAPE;
     p.num_m_tiles = static_cast<int>(mtiles);
-    p.kb_a = R * R * p.C1;
+    p.kb_a = R * p.Rw * p.C1;
     p.kb_per_tile = p.kb_a + p.C1b;
 
     const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 12) * 8 + 64;

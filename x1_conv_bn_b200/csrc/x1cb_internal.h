@@ -27,6 +27,7 @@ struct ConvGeom {
     int stride = 1, Hin = 0, Win = 0;
     int Ic2 = 0, stride2 = 1, Hin2 = 0, Win2 = 0;
     int pool = 0;  // 3x3 stride-2 max pooling after the ReLU (64-channel layers)
+    int Rw = 0;    // filter width when it differs from the height (0: square)
 };
 int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
                  int m_r, int num_sms, const ConvGeom &g);
@@ -59,5 +60,9 @@ int launch_pack_act(const int8_t *nhwc, int8_t *nc32, int B, int H, int W, int C
 int launch_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C,
                       cudaStream_t s);
 int launch_pack_weight(const int8_t *oihw, int8_t *blk, int Oc, int Ic, int R, cudaStream_t s);
+int launch_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int Cin, int R,
+                     cudaStream_t s);
+int launch_pack_stem_weight(const int8_t *oihw, int8_t *blk, int Oc, int Cin, int R,
+                            cudaStream_t s);
 
 }  // namespace x1cb

@@ -78,6 +78,58 @@ __global__ void pack_weight_kernel(const int8_t *__restrict__ oihw, int8_t *__re
     }
 }
 
+// The stem's width-folded image: pixel (h, u) of the folded tensor
+// [B, 1, H, W, 32] holds, in channel ds*Cin + ci, channel ci of image pixel
+// (h, u - pad + ds) for the R taps ds of a filter row (zero outside the image;
+// channels from R*Cin on are zero).  An R x R convolution of the image then is
+// an R x 1 convolution of the folded tensor.  One thread per folded pixel.
+__global__ void pack_stem_kernel(const int8_t *__restrict__ nhwc, int8_t *__restrict__ folded,
+                                 int B, int H, int W, int Cin, int R)
+{
+    const long long n = static_cast<long long>(B) * H * W;
+    const int pad = (R - 1) / 2;
+    for (long long q = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; q < n;
+         q += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int u = static_cast<int>(q % W);
+        const long long bh = q / W;  // b * H + h
+        uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int ds = 0; ds < R; ++ds) {
+            const int w = u - pad + ds;
+            if (w < 0 || w >= W)
+                continue;
+            const int8_t *src = nhwc + (bh * W + w) * Cin;
+            for (int ci = 0; ci < Cin; ++ci) {
+                const int c = ds * Cin + ci;
+                words[c >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(src[ci]))
+                                  << (8 * (c & 3));
+            }
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(folded + q * 32);
+        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+        dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    }
+}
+
+// Folded stem weights: [1, R, 1, 1, Oc, 32] with entry (dr, o, ds*Cin + ci) =
+// w[o, ci, dr, ds] of the OIHW weight [Oc, Cin, R, R] (zero from R*Cin on).
+__global__ void pack_stem_weight_kernel(const int8_t *__restrict__ oihw,
+                                        int8_t *__restrict__ blk, int Oc, int Cin, int R)
+{
+    const long long n = static_cast<long long>(R) * Oc * 32;
+    for (long long d = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; d < n;
+         d += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(d % 32);
+        const int o = static_cast<int>((d / 32) % Oc);
+        const int dr = static_cast<int>(d / (32LL * Oc));
+        int8_t v = 0;
+        if (c < R * Cin) {
+            const int ds = c / Cin, ci = c % Cin;
+            v = oihw[((static_cast<long long>(o) * Cin + ci) * R + dr) * R + ds];
+        }
+        blk[d] = v;
+    }
+}
+
 int grid_for(long long n, int threads)
 {
     long long g = (n + threads - 1) / threads;
@@ -114,6 +166,26 @@ int launch_pack_weight(const int8_t *oihw, int8_t *blk, int Oc, int Ic, int R, c
     if (n == 0)
         return X1CB_OK;
     pack_weight_kernel<<<grid_for(n, 256), 256, 0, s>>>(oihw, blk, Oc, Ic, R);
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+}  // namespace x1cb
+
+namespace x1cb {
+
+int launch_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int Cin, int R,
+                     cudaStream_t s)
+{
+    const long long n = static_cast<long long>(B) * H * W;
+    pack_stem_kernel<<<grid_for(n, 256), 256, 0, s>>>(nhwc, folded, B, H, W, Cin, R);
+    return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+int launch_pack_stem_weight(const int8_t *oihw, int8_t *blk, int Oc, int Cin, int R,
+                            cudaStream_t s)
+{
+    const long long n = static_cast<long long>(R) * Oc * 32;
+    pack_stem_weight_kernel<<<grid_for(n, 256), 256, 0, s>>>(oihw, blk, Oc, Cin, R);
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 

@@ -25,7 +25,8 @@ constexpr unsigned kDevDrainFailed = 8u;
 
 struct ConvPlan {
     // problem
-    int B, H, W, Ic, Oc, R, pad;
+    int B, H, W, Ic, Oc, R, pad;  // R, pad: filter height and its padding
+    int Rw, padw;                  // filter width and its padding (R, pad unless folded)
     int C1, O1;       // Ic/32, Oc/32
     int Wp, Hp;       // output spatial dims seen by the tensor maps (1x1: H*W and 1)
     // Convolution stride and the input image the activation map covers

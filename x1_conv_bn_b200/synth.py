@@ -182,6 +182,59 @@ def proj_block_inputs(s: ProjBlockShape, seed: int, device="cpu",
     return out
 
 
+@dataclass(frozen=True)
+class StemShape:
+    """The network's stem: R x R convolution (pad (R-1)/2, stride) of an image
+    of Cin channels (carried in one 32-channel block), BN, ReLU, then 3x3
+    stride-2 max pooling; Oc = 64 output channels."""
+
+    B: int
+    H: int
+    W: int
+    Cin: int = 3
+    Oc: int = 64
+    R: int = 7
+    stride: int = 2
+
+    @property
+    def Hc(self) -> int:
+        return (self.H + 2 * ((self.R - 1) // 2) - self.R) // self.stride + 1
+
+    @property
+    def Wc(self) -> int:
+        return (self.W + 2 * ((self.R - 1) // 2) - self.R) // self.stride + 1
+
+    @property
+    def Hp(self) -> int:
+        return (self.Hc - 1) // 2 + 1
+
+    @property
+    def Wp(self) -> int:
+        return (self.Wc - 1) // 2 + 1
+
+    def ops(self) -> int:
+        """2 x MACs of the convolution over the image's real channels."""
+        return 2 * self.B * self.Hc * self.Wc * self.Oc * self.R * self.R * self.Cin
+
+    def bytes_moved(self) -> int:
+        """Image in (one 32-channel block per pixel, as stored), pooled output
+        out, weights."""
+        C = (self.Cin + 31) // 32 * 32
+        return (self.B * self.H * self.W * C + self.B * self.Hp * self.Wp * self.Oc
+                + self.Oc * C * self.R * self.R + 8 * self.Oc)
+
+
+def stem_inputs(s: StemShape, seed: int, device="cpu", S: int = S_DEFAULT) -> ConvInputs:
+    """Image x in [0, 127] (Cin channels), weights, bias, multiplier (fan-in
+    R*R*Cin)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = _randint(g, X_LO, X_HI, (s.B, s.H, s.W, s.Cin), torch.int8, device)
+    w, bias, m = _draw_layer(g, ConvShape(s.B, s.H, s.W, s.Cin, s.Oc, s.R, False), S, device)
+    return ConvInputs(ConvShape(s.B, s.H, s.W, s.Cin, s.Oc, s.R, False), x, w, bias, m, None, 0,
+                      S)
+
+
 # Named workloads.  Index 1..5 as in the benchmark plan; "4a".."4c" are the
 # three expand convolutions of the sweep.
 CONFIGS: Dict[str, object] = {
@@ -194,9 +247,13 @@ CONFIGS: Dict[str, object] = {
     "5": BlockShape(1024, 28, 28, 512, 128),
     # Res3.1 (the stage's projection block), 56x56x256 in, 28x28x512 out.
     "p31": ProjBlockShape(256, 56, 56, 256, 128, 512),
+    # Res4.x conv2: 3x3 256 -> 256 at 14x14 (weights streamed).
+    "r4c2": ConvShape(512, 14, 14, 256, 256, 3, False),
+    # The stem: 7x7 stride 2 of a 224x224 RGB image, BN, ReLU, 3x3/2 max pool.
+    "stem": StemShape(256, 224, 224),
 }
 CONFIG_SEEDS = {"1": 1001, "2": 1002, "3": 1003, "4a": 1004, "4b": 1004, "4c": 1004, "5": 1005,
-                "p31": 1031}
+                "p31": 1031, "r4c2": 1042, "stem": 1050}
 WORKLOAD_NAMES = {
     "1": "res3.2-conv3 1x1 128->512 +bn+sum+relu, 28x28, B=1",
     "2": "res3.2-conv3 1x1 128->512 +bn+sum+relu, 28x28, B=256",
@@ -207,6 +264,8 @@ WORKLOAD_NAMES = {
     "5": "res3.2 bottleneck block 512->128->128->512, 28x28, B=1024",
     "p31": "res3.1 projection block 256->128->128(s2)->512 + proj 256->512(s2), 56x56->28x28, "
            "B=256",
+    "r4c2": "res4.x conv2 3x3 256->256 +bn+relu, 14x14, B=512",
+    "stem": "stem 7x7/2 3->64 +bn+relu+maxpool 3x3/2, 224x224->56x56, B=256",
 }
 
 
