@@ -148,8 +148,8 @@ def test_wide_images_take_the_per_tap_form(L):
     ((2048, 28, 28, 128, 512, 1, 1), "1"),    # tw 16, row length 784
     ((512, 56, 56, 64, 256, 1, 1), "1"),
     ((1024, 28, 28, 128, 128, 3, 0), "1"),    # halo tile 28 wide
-    ((512, 14, 14, 256, 1024, 1, 1), "0"),    # 14-pixel tiles: not whole 4-pixel groups
-    ((512, 7, 7, 512, 2048, 1, 1), "0"),
+    ((512, 14, 14, 256, 1024, 1, 1), "1"),    # 16-pixel tiles of the 196-pixel image rows
+    ((512, 7, 7, 512, 2048, 1, 1), "0"),      # 49-pixel rows: not whole 4-pixel groups
     ((17, 2, 3, 32, 384, 1, 1), "0"),
 ])
 def test_swizzled_io_stages_only_for_whole_pixel_groups(L, shape, swz):

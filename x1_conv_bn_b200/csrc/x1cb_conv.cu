@@ -920,9 +920,13 @@ int opt_in_smem(const void *kern, int which)
 
 
 // Choose the pixel tile: tw x th pixels of tg images, at most 128 GEMM rows.
-// Cost = MMA rows issued over the whole problem, with a mild penalty for
-// contiguous global runs shorter than 512 bytes; ties go to more rows, then
-// to longer runs.
+// Cost = MMA rows issued over the whole problem, with a penalty for
+// contiguous global runs shorter than 512 bytes (up to 47 % for single
+// 32-byte pixels), and 10 % each for a row
+// count that is not a multiple of 8 (activation boxes then carry one K block
+// each instead of up to four) and for shortcut/output stages that cannot use
+// the 128-byte swizzle (tw or the row not whole 4-pixel groups: bank
+// conflicts in the epilogue); ties go to more rows, then to longer runs.
 void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg)
 {
     double best = 1e300;
@@ -938,8 +942,12 @@ void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg)
             const int seg = (w == Wp) ? w * h * 32 : w * 32;
             double cost = tiles * kTileRows;
             if (seg < 512)
-                cost *= 1.0 + (512 - seg) / 4096.0;
+                cost *= 1.0 + (512 - seg) / 1024.0;
             const int rows = w * h * g;
+            if (rows % 8 != 0)
+                cost *= 1.1;
+            if (w % 4 != 0 || Wp % 4 != 0)
+                cost *= 1.1;
             const bool tie = cost <= best * (1 + 1e-12) && cost >= best * (1 - 1e-12);
             if (cost < best * (1 - 1e-12) ||
                 (tie && (rows > best_rows || (rows == best_rows && seg > best_seg)))) {
@@ -1094,7 +1102,13 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     const int min_slot = p.halo ? 2 * p.a_half : kASlotBytes;
     int chosen = 0;
     long long chosen_work = -1;
-    // A 64-channel layer (the stem) is one CTA group of N = 64.
+    // A 64-channel layer (the stem) is one CTA group of N = 64.  Largest NC
+    // first (the activation is read once per group); but a 1x1 whose tile's K
+    // blocks would not fit the activation ring beside NC's weights takes a
+    // smaller NC when that one does: with the ring shorter than a tile the
+    // producer cannot run a tile ahead and the L2 latency of every box is
+    // exposed (a deep fan-in, e.g. 512 input channels at 7x7).
+    bool chosen_deep = false;
     for (int NC = std::min(Oc, 512); NC >= 64; NC -= (NC > 128 ? 128 : 64)) {
         if (Oc % NC || (NC == 64 && Oc != 64))
             continue;
@@ -1102,17 +1116,22 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         const int n_subs = NC / nmma;
         const int a_min = n_subs > 1 ? (p.halo ? p.C1 : p.kb_per_tile) + 2 : (p.halo ? 2 : 4);
         const int r_min = has_res ? 4 : 2;
-        const long long need = static_cast<long long>(p.kb_per_tile) * NC * 32 + NC * 12 +
-                               static_cast<long long>(a_min) * min_slot + r_min * kRSlotBytes +
-                               fixed;
+        const long long wres = static_cast<long long>(p.kb_per_tile) * NC * 32 + NC * 12;
+        const long long need = wres + static_cast<long long>(a_min) * min_slot +
+                               r_min * kRSlotBytes + fixed;
         if (need > kSmemLimit || a_min > 48)
             continue;
+        const bool deep = p.halo || R != 1 ||
+                          wres + static_cast<long long>(p.kb_per_tile + 2) * kASlotBytes +
+                                  r_min * kRSlotBytes + fixed <= kSmemLimit;
         const long long work = mtiles * (Oc / NC);
-        if (chosen == 0 || (chosen_work < num_sms && work > chosen_work)) {
+        if (chosen == 0 || (chosen_work < num_sms && work > chosen_work) ||
+            (deep && !chosen_deep && work >= num_sms)) {
             chosen = NC;
             chosen_work = work;
+            chosen_deep = deep;
         }
-        if (work >= num_sms)
+        if (work >= num_sms && chosen_deep)
             break;
     }
     // When no resident copy fits (large fan-in), the weights are streamed:
@@ -1136,9 +1155,12 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // of the traffic and get up to 128 KB in flight while the I/O stages only
     // stage results.  The bias-fold tiles are reserved when the rings still
     // reach their minimum beside them.
-    const int a_bytes_want = p.wstream ? 4 * 4 * kASlotBytes
-                             : has_res ? std::min(p.kb_per_tile + 2, 8) * kASlotBytes
-                                       : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
+    // (a deep fan-in with a shortcut -- 8 or more K blocks per tile -- also
+    // gets two tiles of K blocks, so the producer runs a tile ahead)
+    const int a_bytes_want =
+        p.wstream ? 4 * 4 * kASlotBytes
+        : (has_res && p.kb_per_tile < 8) ? std::min(p.kb_per_tile + 2, 8) * kASlotBytes
+                                         : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
     // Several K blocks per activation box (fewer, larger copies) when each
     // K-block tile starts on a 256-byte swizzle atom (row count a multiple of
     // 8) and the ring's minimum still fits the budget.  With two accumulator
