@@ -1,4 +1,5 @@
-"""GPU parity of the projection-block path (Res3.1): the stride-2 3x3, the
+"""GPU parity of the projection-block path (Res3.1): the stride-2 3x3 (phase
+planes of the input, or one strided box per tap for very wide images), the
 Conv3 + projection shortcut in one accumulator, and the three-layer block,
 each through the C ABI against the CPU oracle, byte for byte.
 
@@ -50,6 +51,7 @@ S2_SHAPES = [
     (1, 5, 5, 32, 128),
     (5, 30, 20, 96, 384),
     (1, 2, 3, 32, 256),
+    (1, 3, 260, 32, 128),   # 130 output columns: one box per tap instead of phase planes
 ]
 
 

@@ -494,8 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
             // one filter tap), each a 128-row x 32-byte tile, back to back.
             const uint32_t abytes =
-                p.halo ? static_cast<uint32_t>(2 * 16 * p.plane_m * p.tg)  // two K halves
-                       : static_cast<uint32_t>(p.a_kc * p.rows * 32);
+                p.halo ? static_cast<uint32_t>((p.halo == 2 ? 8 : 2) * 16 * p.plane_m * p.tg)
+                       : static_cast<uint32_t>(p.a_kc * p.rows * 32);  // K halves / blocks
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
             const int boxes = p.kb_per_tile / p.a_kc;  // unused in the halo form
@@ -518,11 +518,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
-                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
-                                         h0 - p.pad, c1, b0, pol);
-                        tma_load_5d_hint(slot + static_cast<uint32_t>(p.a_half), &tmA,
-                                         bars.a_full(stage), 16, w0 - p.pad, h0 - p.pad, c1, b0,
-                                         pol);
+                        if (p.halo == 2) {
+                            // plane (pr, pc) from input (pc - 1, 2*h0 - 1 + pr), step 2
+                            for (int pl = 0; pl < 4; ++pl)
+                                for (int hf = 0; hf < 2; ++hf)
+                                    tma_load_5d_hint(
+                                        slot + static_cast<uint32_t>((2 * pl + hf) * p.a_half),
+                                        &tmA, bars.a_full(stage), 16 * hf, (pl & 1) - 1,
+                                        2 * h0 - 1 + (pl >> 1), c1, b0, pol);
+                        } else {
+                            tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
+                                             h0 - p.pad, c1, b0, pol);
+                            tma_load_5d_hint(slot + static_cast<uint32_t>(p.a_half), &tmA,
+                                             bars.a_full(stage), 16, w0 - p.pad, h0 - p.pad, c1,
+                                             b0, pol);
+                        }
                         if (wpart) {  // the nine taps' weights of channel block c1
                             const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
                             for (int t = 0; t < 9; ++t)
@@ -727,6 +737,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Halo form: tap (dr, ds) reads the slot dr*row_pitch + ds rows on and
             // the weights of K block (dr*3 + ds)*C1 + c1.
             const uint32_t hp = static_cast<uint32_t>(p.row_pitch);
+            // Descriptor offset of tap t (units of 16 bytes): the row shift of the
+            // framed tile; in the stride-2 form also the tap's plane.
+            uint32_t tap_off[9];
+#pragma unroll
+            for (int t = 0; t < 9; ++t) {
+                const uint32_t dr = t / 3, ds = t % 3;
+                tap_off[t] = p.halo == 2
+                                 ? ((dr & 1) * 2 + (ds & 1)) * (2 * p.a_half >> 4) +
+                                       (dr >> 1) * hp + (ds >> 1)
+                                 : dr * hp + ds;
+            }
             // (streamed: the nine taps of one channel block are consecutive)
             const uint64_t b_tap_step =
                 p.wstream ? b_kb_step : static_cast<uint64_t>(p.C1) * b_kb_step;
@@ -774,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (p.halo) {
 #pragma unroll
                             for (int t = 0; t < 9; ++t)
-                                mma_i8(d_tmem, ad + (t / 3) * hp + (t % 3),
+                                mma_i8(d_tmem, ad + tap_off[t],
                                        bd + static_cast<uint64_t>(t) * b_tap_step, idesc,
                                        t == 0 ? accumulate : 1u);
                             bd += b_kb_step;
@@ -1049,10 +1070,40 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.Hpi = p.Hin;
     }
     // The 3x3 convolution uses the halo form whenever one framed image row fits
-    // in the 128 GEMM rows (stride 1).
-    p.halo = (R == 3 && p.Rw == 3 && p.stride == 1 && p.C1b == 0 && !p.pool &&
-              W + 2 <= kTileRows) ? 1 : 0;
-    if (p.halo) {
+    // in the 128 GEMM rows: at stride 1 one framed tile (halo = 1); at stride 2
+    // four phase planes of the input region (halo = 2): plane (pr, pc) holds
+    // the input pixels of row parity pr and column parity pc, so output pixel
+    // (y, x) reads tap (dr, ds) at plane (dr & 1, ds & 1), position
+    // (y + dr / 2, x + ds / 2) -- again a row shift of one framed tile.
+    p.halo = (R == 3 && p.Rw == 3 && p.C1b == 0 && !p.pool &&
+              ((p.stride == 1 && W + 2 <= kTileRows) || (p.stride == 2 && W + 1 <= 126)))
+                 ? p.stride
+                 : 0;
+    if (p.halo == 2) {
+        // th output rows of tg images per tile; a plane is (th+1) x (W+1)
+        // pixels (row pitch W+1); GEMM row m = (g*(th+1) + y)*(W+1) + x.
+        const int pitch = W + 1;
+        long long best = -1;
+        p.th = p.tg = 1;
+        for (int h = 1; h <= H; ++h)
+            for (int g = 1; g <= B; ++g) {
+                const long long last = static_cast<long long>(g - 1) * (h + 1) * pitch +
+                                       static_cast<long long>(h - 1) * pitch + (W - 1);
+                if (last >= kTileRows)
+                    break;
+                const long long tiles = static_cast<long long>((H + h - 1) / h) * ((B + g - 1) / g);
+                if (best < 0 || tiles < best || (tiles == best && h > p.th)) {
+                    best = tiles;
+                    p.th = h;
+                    p.tg = g;
+                }
+            }
+        p.tw = W;
+        p.row_pitch = pitch;
+        p.plane_m = (p.th + 1) * pitch;
+        const int need_rows = std::max(p.tg * p.plane_m, kTileRows + pitch + 1);
+        p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+    } else if (p.halo) {
         choose_halo_tile(B, H, W, p.th, p.tg);
         p.tw = W;
         p.row_pitch = W + 2;
@@ -1099,7 +1150,7 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     p.kb_per_tile = p.kb_a + p.C1b;
 
     const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 12) * 8 + 64;
-    const int min_slot = p.halo ? 2 * p.a_half : kASlotBytes;
+    const int min_slot = p.halo ? (p.halo == 2 ? 8 : 2) * p.a_half : kASlotBytes;
     int chosen = 0;
     long long chosen_work = -1;
     // A 64-channel layer (the stem) is one CTA group of N = 64.  Largest NC
@@ -1177,7 +1228,9 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
             }
     // Halo form: one slot per channel block, all of a tile's blocks in the ring
     // when two accumulator slots share them; slots stay 1024-byte aligned.
-    p.a_part = p.halo ? (2 * p.a_half + 1023) / 1024 * 1024 : p.a_kc * kASlotBytes;
+    // (the stride-2 halo form: four planes of two K halves)
+    p.a_part = p.halo ? ((p.halo == 2 ? 8 : 2) * p.a_half + 1023) / 1024 * 1024
+                      : p.a_kc * kASlotBytes;
     p.w_part = p.wstream ? (p.halo ? 9 : p.a_kc) * p.NC * 32 : 0;
     p.a_slot = p.a_part + p.w_part;
     const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
@@ -1234,7 +1287,20 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
     // box (32, tw, th, tg, a_kc) lands as a_kc K-block tiles one after another.
     // Halo form: dims (32 ch, W, H, C1, B), box (16, tw+2, th+2, 1, tg) -- one K
     // half of the framed tile as 16-byte rows, zeros outside the image.
-    if (p.halo) {
+    if (p.halo == 2) {
+        // Stride-2 planes: dims (32 ch, Win, Hin, C1, B) at traversal step 2;
+        // a box of (2(W+1), 2(th+1)) elements lands one (W+1) x (th+1) plane.
+        const uint64_t dims[5] = {32, (uint64_t)p.Win, (uint64_t)p.Hin, (uint64_t)p.C1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {32, (uint64_t)p.Win * 32, (uint64_t)p.Hin * p.Win * 32,
+                                 (uint64_t)p.C1 * p.Hin * p.Win * 32};
+        const uint32_t box[5] = {16, (uint32_t)(2 * p.row_pitch), (uint32_t)(2 * (p.th + 1)), 1,
+                                 (uint32_t)p.tg};
+        const uint32_t es[5] = {1, 2, 2, 1, 1};
+        if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT8, es))
+            return e;
+    } else if (p.halo) {
         const uint64_t dims[5] = {32, (uint64_t)p.W, (uint64_t)p.H, (uint64_t)p.C1,
                                   (uint64_t)p.B};
         const uint64_t str[4] = {32, (uint64_t)p.W * 32, (uint64_t)p.H * p.W * 32,
