@@ -163,6 +163,175 @@ __device__ __forceinline__ int shortcut_operands(int mode, int m_r, int S, uint3
     return mr2;
 }
 
+// Epilogue of one warp over the accumulator ring: the MMA issuer fills the
+// four slots in issue order with Conv2 tiles and Conv3 chunks (item k in slot
+// k % 4), and turn g takes items g, g+4, ... (it owns slot g, so it sees every
+// phase of its slot in order).  kM2 / kM3: the exact form of each layer when
+// it is the all-32-bit one (2), or -1 for the form chosen at run time
+// (generic, 64-bit or all-32-bit); kK1: the shortcut scale is 1.
+struct ChainEpi {
+    const ChainPlan *p;
+    ChainBars bars;
+    WaitCtl ctl;
+    uint32_t tmem_base;
+    uint8_t *smem;
+    volatile int *io_ticket;
+    const int32_t *cm2;
+    const long long *cc2;
+    const int32_t *cm3;
+    const long long *cc3;
+    int n_my, mode2, mode3;
+};
+
+template <int kM, bool kRes, bool kK1>
+__device__ __forceinline__ void requant_chain(int mode, const uint32_t *v, const int32_t *cm,
+                                          const long long *cC, int ch, const uint32_t *rw,
+                                          int m_r, int S, int mr2, const uint32_t (&rsel)[4],
+                                          uint32_t *ow)
+{
+    if (kM == 2)
+    requant_hi32<kRes, true, kK1, 8>(v, cm + ch, reinterpret_cast<const int32_t *>(cC) + ch,
+                                     rw, mr2, rsel, ow);
+    else
+    requant_any<kRes>(mode, v, cm, cC, ch, rw, m_r, S, mr2, rsel, ow);
+}
+
+template <int kM2, int kM3, bool kK1>
+__device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int lane)
+{
+    const ChainPlan &p = *ce.p;
+    const ChainBars &bars = ce.bars;
+    const WaitCtl &ctl = ce.ctl;
+    const uint32_t tmem_base = ce.tmem_base;
+    uint8_t *smem = ce.smem;
+    volatile int *io_ticket = ce.io_ticket;
+    const int32_t *cm2 = ce.cm2;
+    const long long *cc2 = ce.cc2;
+    const int32_t *cm3 = ce.cm3;
+    const long long *cc3 = ce.cc3;
+    const int n_my = ce.n_my;
+    const int mode2 = ce.mode2, mode3 = ce.mode3;
+    // Item order is the MMA issuer's: Conv2 of tile i, then Conv3 of tile
+    // i - 1 in n_chunks chunks.  Each turn owns slot `turn` (items k with
+    // k % 4 == turn), so it sees every phase of its slot in order.
+    const int q = warp & 3;
+    const int turn = (warp - kEpiWarp0) >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tslot = tmem_base + lane_addr + static_cast<uint32_t>(turn * 128);
+    const uint32_t empty0 = mapa_shared(bars.acc_empty(turn), 0);
+    // Conv3 output rows: this row's place in an output stage (halo rows
+    // outside the image are computed and not stored).
+    const int plane_t = p.tw * p.th;
+    const int xi = row % p.row_pitch;
+    const int yi = (row % p.plane_m) / p.row_pitch;
+    const int gi = row / p.plane_m;
+    const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
+    const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
+    const int chunk_stride = plane_t * 32;
+    const int swz_mask = p.io_swz ? 0x70 : 0;
+    uint32_t rsel3[4];
+    const int mr2 = shortcut_operands(mode3, p.m_r, p.S, rsel3);
+    const uint32_t rsel2[4] = {0, 0, 0, 0};
+    int k = 0;             // item index in issue order
+    uint32_t kph = 0;      // parity of this turn's slot at its next item
+    bool ok = true;
+    for (int i = 0; ok && i <= n_my; ++i) {
+        if (i < n_my) {
+            if ((k & 3) == turn) {
+                // Conv2 of tile i -> int8 -> A buffer i % 2 of this CTA.
+                const int b = i & 1;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
+                    !__all_sync(0xffffffffu,
+                                mbar_wait(bars.a3_empty(b),
+                                          static_cast<uint32_t>((i >> 1) & 1) ^ 1u, ctl,
+                                          kDevTimeoutEpilogue))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint8_t *a3 = smem + p.off_a3 + b * kA3Bytes;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32], ow[8];
+                    __syncwarp();
+                    tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(c * 32), v);
+                    requant_chain<kM2, false, false>(mode2, v, cm2, cc2, c * 32, nullptr, 0, p.S, 0,
+                                                 rsel2, ow);
+                    // K block c of the A buffer: two 16-byte halves, rows 16 bytes apart.
+                    uint4 *dst = reinterpret_cast<uint4 *>(a3 + c * (kA3Bytes / 4) + row * 16);
+                    dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    dst[(kA3Bytes / 8) / 16] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                }
+                fence_proxy_async_smem();  // read by the MMA (async proxy, rank 0's issue)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_cluster(empty0);
+                    mbar_arrive_cluster(mapa_shared(bars.a3_full(b), 0));
+                }
+                kph ^= 1u;
+            }
+            ++k;
+        }
+        if (i >= 1) {
+            const int j = i - 1;
+            for (int c = 0; c < p.n_chunks; ++c, ++k) {
+                if ((k & 3) != turn)
+                    continue;
+                // Conv3 of tile j, output chunk c: shortcut stage n = j*n_chunks + c.
+                const long long n = static_cast<long long>(j) * p.n_chunks + c;
+                const int st = static_cast<int>(n % p.r_stages);
+                const uint32_t st_phase = static_cast<uint32_t>((n / p.r_stages) & 1);
+                // Stages are taken in order (the ticket), so each stage's
+                // previous phase is complete before its arrival is awaited.
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
+                    !__all_sync(0xffffffffu, ticket_wait(io_ticket, static_cast<int>(n), ctl,
+                                                         kDevTimeoutEpilogue)) ||
+                    !__all_sync(0xffffffffu, mbar_wait(bars.io_full(st), st_phase, ctl,
+                                                       kDevTimeoutEpilogue))) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0)
+                    atomicMax(const_cast<int *>(io_ticket), static_cast<int>(n + 1));
+                tc_fence_after();
+                uint8_t *stage = smem + p.off_r + st * kRSlotBytes;
+#pragma unroll 1
+                for (int cs = 0; cs < kRChunks; ++cs) {
+                    const int ch = c * 128 + cs * 32;
+                    uint32_t v[32];
+                    __syncwarp();
+                    tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(cs * 32), v);
+                    const int o = row_off + cs * chunk_stride;
+                    const int sw = swz_mask & (o >> 3);
+                    uint4 *pa = reinterpret_cast<uint4 *>(stage + (o ^ sw));
+                    uint4 *pb = reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw));
+                    const uint4 ra = *pa, rb = *pb;
+                    const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+                    uint32_t ow[8];
+                    requant_chain<kM3, true, kK1>(mode3, v, cm3, cc3, ch, rw, p.m_r, p.S, mr2,
+                                                 rsel3, ow);
+                    if (in_box) {
+                        *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bars.out_ready(st));
+                    mbar_arrive_cluster(empty0);
+                }
+                kph ^= 1u;
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     chain23_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW2,
                    const __grid_constant__ CUtensorMap tmW3,
@@ -469,125 +638,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- epilogue: items of the accumulator ring, turn g takes items g, g+4, ... --
-        // Item order is the MMA issuer's: Conv2 of tile i, then Conv3 of tile
-        // i - 1 in n_chunks chunks.  Each turn owns slot `turn` (items k with
-        // k % 4 == turn), so it sees every phase of its slot in order.
-        const int q = warp & 3;
-        const int turn = (warp - kEpiWarp0) >> 2;
-        const int row = q * 32 + lane;
-        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        const uint32_t tslot = tmem_base + lane_addr + static_cast<uint32_t>(turn * 128);
-        const uint32_t empty0 = mapa_shared(bars.acc_empty(turn), 0);
-        // Conv3 output rows: this row's place in an output stage (halo rows
-        // outside the image are computed and not stored).
-        const int plane_t = p.tw * p.th;
-        const int xi = row % p.row_pitch;
-        const int yi = (row % p.plane_m) / p.row_pitch;
-        const int gi = row / p.plane_m;
-        const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
-        const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
-        const int chunk_stride = plane_t * 32;
-        const int swz_mask = p.io_swz ? 0x70 : 0;
-        uint32_t rsel3[4];
-        const int mr2 = shortcut_operands(mode3, p.m_r, p.S, rsel3);
-        const uint32_t rsel2[4] = {0, 0, 0, 0};
-        int k = 0;             // item index in issue order
-        uint32_t kph = 0;      // parity of this turn's slot at its next item
-        bool ok = true;
-        for (int i = 0; ok && i <= n_my; ++i) {
-            if (i < n_my) {
-                if ((k & 3) == turn) {
-                    // Conv2 of tile i -> int8 -> A buffer i % 2 of this CTA.
-                    const int b = i & 1;
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
-                        !__all_sync(0xffffffffu,
-                                    mbar_wait(bars.a3_empty(b),
-                                              static_cast<uint32_t>((i >> 1) & 1) ^ 1u, ctl,
-                                              kDevTimeoutEpilogue))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    uint8_t *a3 = smem + p.off_a3 + b * kA3Bytes;
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t v[32], ow[8];
-                        __syncwarp();
-                        tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(c * 32), v);
-                        requant_any<false>(mode2, v, cm2, cc2, c * 32, nullptr, 0, p.S, 0, rsel2,
-                                           ow);
-                        // K block c of the A buffer: two 16-byte halves, rows 16 bytes apart.
-                        uint4 *dst = reinterpret_cast<uint4 *>(a3 + c * (kA3Bytes / 4) + row * 16);
-                        dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                        dst[(kA3Bytes / 8) / 16] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-                    }
-                    fence_proxy_async_smem();  // read by the MMA (async proxy, rank 0's issue)
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive_cluster(empty0);
-                        mbar_arrive_cluster(mapa_shared(bars.a3_full(b), 0));
-                    }
-                    kph ^= 1u;
-                }
-                ++k;
-            }
-            if (i >= 1) {
-                const int j = i - 1;
-                for (int c = 0; c < p.n_chunks; ++c, ++k) {
-                    if ((k & 3) != turn)
-                        continue;
-                    // Conv3 of tile j, output chunk c: shortcut stage n = j*n_chunks + c.
-                    const long long n = static_cast<long long>(j) * p.n_chunks + c;
-                    const int st = static_cast<int>(n % p.r_stages);
-                    const uint32_t st_phase = static_cast<uint32_t>((n / p.r_stages) & 1);
-                    // Stages are taken in order (the ticket), so each stage's
-                    // previous phase is complete before its arrival is awaited.
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
-                        !__all_sync(0xffffffffu, ticket_wait(io_ticket, static_cast<int>(n), ctl,
-                                                             kDevTimeoutEpilogue)) ||
-                        !__all_sync(0xffffffffu, mbar_wait(bars.io_full(st), st_phase, ctl,
-                                                           kDevTimeoutEpilogue))) {
-                        ok = false;
-                        break;
-                    }
-                    if (lane == 0)
-                        atomicMax(const_cast<int *>(io_ticket), static_cast<int>(n + 1));
-                    tc_fence_after();
-                    uint8_t *stage = smem + p.off_r + st * kRSlotBytes;
-#pragma unroll 1
-                    for (int cs = 0; cs < kRChunks; ++cs) {
-                        const int ch = c * 128 + cs * 32;
-                        uint32_t v[32];
-                        __syncwarp();
-                        tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(cs * 32), v);
-                        const int o = row_off + cs * chunk_stride;
-                        const int sw = swz_mask & (o >> 3);
-                        uint4 *pa = reinterpret_cast<uint4 *>(stage + (o ^ sw));
-                        uint4 *pb = reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw));
-                        const uint4 ra = *pa, rb = *pb;
-                        const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-                        uint32_t ow[8];
-                        requant_any<true>(mode3, v, cm3, cc3, ch, rw, p.m_r, p.S, mr2, rsel3, ow);
-                        if (in_box) {
-                            *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                            *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(bars.out_ready(st));
-                        mbar_arrive_cluster(empty0);
-                    }
-                    kph ^= 1u;
-                }
-            }
-        }
+        // ---- epilogue: items of the accumulator ring (see chain_epilogue) ---------------
+        // One instantiation per pair of exact forms in use: the fast path keeps
+        // its operands in registers (a form chosen at run time would share
+        // arrays across forms and push them to local memory).
+        const ChainEpi ce{&p, bars, ctl, tmem_base, smem, io_ticket, cm2, cc2, cm3, cc3, n_my,
+                          mode2, mode3};
+        const bool k1 = static_cast<long long>(p.m_r) == (1ll << (p.S - 1));
+        if (mode2 == 2 && mode3 == 2 && k1)
+            chain_epilogue<2, 2, true>(ce, warp, lane);
+        else if (mode2 == 2 && mode3 == 2)
+            chain_epilogue<2, 2, false>(ce, warp, lane);
+        else
+            chain_epilogue<-1, -1, false>(ce, warp, lane);
     }
 
     // ---- tear-down: neither CTA leaves while the other may still reach it ----------

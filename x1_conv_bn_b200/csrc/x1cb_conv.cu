@@ -1154,12 +1154,11 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     int chosen = 0;
     long long chosen_work = -1;
     // A 64-channel layer (the stem) is one CTA group of N = 64.  Largest NC
-    // first (the activation is read once per group); but a 1x1 whose tile's K
-    // blocks would not fit the activation ring beside NC's weights takes a
-    // smaller NC when that one does: with the ring shorter than a tile the
-    // producer cannot run a tile ahead and the L2 latency of every box is
-    // exposed (a deep fan-in, e.g. 512 input channels at 7x7).
-    bool chosen_deep = false;
+    // first: the activation is read once per group, and N = 256 MMAs do twice
+    // the work of N = 128 ones per instruction.  (Measured: the 7x7, 512 ->
+    // 2048 expand conv ran 75 us with NC = 256 and a 5-slot ring, 136 us with
+    // NC = 128 and a 22-slot ring -- the ring depth does not pay for the
+    // halved MMAs and doubled re-reads.)
     for (int NC = std::min(Oc, 512); NC >= 64; NC -= (NC > 128 ? 128 : 64)) {
         if (Oc % NC || (NC == 64 && Oc != 64))
             continue;
@@ -1167,22 +1166,17 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         const int n_subs = NC / nmma;
         const int a_min = n_subs > 1 ? (p.halo ? p.C1 : p.kb_per_tile) + 2 : (p.halo ? 2 : 4);
         const int r_min = has_res ? 4 : 2;
-        const long long wres = static_cast<long long>(p.kb_per_tile) * NC * 32 + NC * 12;
-        const long long need = wres + static_cast<long long>(a_min) * min_slot +
-                               r_min * kRSlotBytes + fixed;
+        const long long need = static_cast<long long>(p.kb_per_tile) * NC * 32 + NC * 12 +
+                               static_cast<long long>(a_min) * min_slot + r_min * kRSlotBytes +
+                               fixed;
         if (need > kSmemLimit || a_min > 48)
             continue;
-        const bool deep = p.halo || R != 1 ||
-                          wres + static_cast<long long>(p.kb_per_tile + 2) * kASlotBytes +
-                                  r_min * kRSlotBytes + fixed <= kSmemLimit;
         const long long work = mtiles * (Oc / NC);
-        if (chosen == 0 || (chosen_work < num_sms && work > chosen_work) ||
-            (deep && !chosen_deep && work >= num_sms)) {
+        if (chosen == 0 || (chosen_work < num_sms && work > chosen_work)) {
             chosen = NC;
             chosen_work = work;
-            chosen_deep = deep;
         }
-        if (work >= num_sms && chosen_deep)
+        if (work >= num_sms)
             break;
     }
     // When no resident copy fits (large fan-in), the weights are streamed:
