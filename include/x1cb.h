@@ -302,6 +302,15 @@ int x1cb_last_device_error(unsigned int *bits, int clear);
  * error. */
 int x1cb_last_epilogue_forms(unsigned int *bits, int clear);
 
+/* Timeline trace of the kernels' pipeline roles, present only in a library
+ * built with -DX1CB_TRACE (the default build returns 0 and copies nothing).
+ * Synchronises the current device, copies up to `words` 64-bit entries of the
+ * trace table to host memory `host` and, with clear != 0, zeroes the table.
+ * Layout: [cta 0..3][event 0..15][n 0..1023] of SM clock values (0: not
+ * recorded); the events of each kernel are listed where it records them.
+ * Returns the number of entries copied, or a negative X1CB_ERR_* code. */
+long long x1cb_trace_copy(unsigned long long *host, long long words, int clear);
+
 /* enable = 0 makes bottleneck_i8 (and bottleneck_i8_noalloc) run conv2 and
  * conv3 as two separate launches even where the fused form applies (for
  * comparisons); 1 (the default) restores the fused form.  Same results

@@ -192,3 +192,90 @@ def test_model_catches_more_turns_than_tmem_stages():
     with pytest.raises((Early, AssertionError)):
         for seed in range(200):
             run(seed, tiles=12, turns=5, stages_per_tile=4, r=8, n_slots=2, stages_per_sub=2)
+
+
+# ---- the activation ring with several issuing lanes --------------------------------
+# The producer warp issues activation boxes in rounds: in round j lane l takes
+# box n = j*lanes + l; the lanes wait for their slots' a_empty parity together
+# (a warp-wide vote), then their copies go out together.  The MMA warp takes
+# the boxes in order (a_full) and commits each slot back (a_empty) after a
+# delay.  Copies land in any order; commits, each covering every earlier MMA
+# of the issuing thread, land in issue order.  Round j's waits follow round
+# j-1's, which saw box j*lanes - 1 - S consumed; a box n of round j needs box
+# n - 2S consumed for its parity to name the right phase, i.e. lanes <= S.
+
+def run_a_ring(seed, S, lanes, boxes=60):
+    rng = random.Random(seed)
+    a_full = [Barrier(1) for _ in range(S)]
+    a_empty = [Barrier(1) for _ in range(S)]
+    events = []
+    last_commit = [0]
+
+    def later(bar, in_order=False):
+        d = rng.randint(1, 8)
+        if in_order:  # not before the previous commit
+            d = max(d, last_commit[0])
+            last_commit[0] = d
+        events.append([d, bar])
+
+    def producer():
+        for base in range(0, boxes, lanes):
+            mine = [n for n in range(base, min(base + lanes, boxes))]
+            # every lane polls its slot; the round proceeds when all are ready
+            while not all(a_empty[n % S].try_wait(n // S - 1 if n >= S else -1) for n in mine):
+                yield
+            for n in mine:
+                later(a_full[n % S])  # expect_tx + copy; lands later
+            yield
+
+    def mma():
+        for n in range(boxes):
+            s, k = n % S, n // S
+            while not a_full[s].try_wait(k):
+                yield
+            later(a_empty[s], in_order=True)  # commit lands after the MMAs
+            yield
+
+    live = [producer(), mma()]
+    steps = 0
+    while live or events:
+        steps += 1
+        assert steps < 200000, "schedule did not finish"
+        for e in events:
+            e[0] -= 1
+        last_commit[0] = max(0, last_commit[0] - 1)
+        for e in [e for e in events if e[0] <= 0]:
+            events.remove(e)
+            e[1].arrive()
+        if live:
+            ag = rng.choice(live)
+            try:
+                next(ag)
+            except StopIteration:
+                live.remove(ag)
+
+
+@pytest.mark.parametrize("S,lanes", [(2, 1), (3, 1), (4, 2), (5, 2), (6, 3), (8, 4), (14, 4)])
+def test_issuing_rounds_within_half_the_ring_are_exact(S, lanes):
+    """The kernels' choice: lanes = min(4, S // 2)."""
+    for seed in range(60):
+        run_a_ring(seed, S, lanes)
+
+
+@pytest.mark.parametrize("S,lanes", [(3, 3), (4, 4)])
+def test_issuing_rounds_up_to_the_ring_depth_are_exact(S, lanes):
+    for seed in range(60):
+        run_a_ring(seed, S, lanes)
+
+
+@pytest.mark.parametrize("S", [2, 3])
+def test_model_catches_more_issuing_lanes_than_slots(S):
+    """Four lanes on a 2- or 3-slot ring: one round holds two boxes of the same
+    slot, and the second one's wait can never be met (or passes early)."""
+    failures = 0
+    for seed in range(20):
+        try:
+            run_a_ring(seed, S, 4)
+        except (Early, AssertionError):
+            failures += 1
+    assert failures == 20

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.x1cb_status_string.restype = ctypes.c_char_p
         L.x1cb_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
         L.x1cb_last_epilogue_forms.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+        L.x1cb_trace_copy.argtypes = [vp, ctypes.c_longlong, i]
+        L.x1cb_trace_copy.restype = ctypes.c_longlong
         L.x1cb_set_block_fusion.argtypes = [i]
         L.x1cb_set_block_fusion.restype = None
         L.x1cb_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -428,6 +430,24 @@ def x1cb_last_epilogue_forms(clear: bool = True) -> int:
     _check(lib().x1cb_last_epilogue_forms(ctypes.byref(bits), int(clear)),
            "x1cb_last_epilogue_forms")
     return bits.value
+
+
+TRACE_SHAPE = (4, 16, 1024)  # [cta][event][n] of SM clock values
+
+
+def x1cb_trace_copy(clear: bool = True):
+    """Timeline table of a trace build as an int64 tensor of TRACE_SHAPE
+    (None when the library was built without the trace)."""
+    import numpy as np
+
+    words = TRACE_SHAPE[0] * TRACE_SHAPE[1] * TRACE_SHAPE[2]
+    buf = np.zeros(words, dtype=np.uint64)
+    n = lib().x1cb_trace_copy(buf.ctypes.data, words, int(clear))
+    if n < 0:
+        raise X1cbError(int(n), "x1cb_trace_copy")
+    if n == 0:
+        return None
+    return torch.from_numpy(buf.view(np.int64).reshape(TRACE_SHAPE).copy())
 
 
 def x1cb_set_block_fusion(enable: bool):

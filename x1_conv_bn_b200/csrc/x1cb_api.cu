@@ -601,6 +601,16 @@ int x1cb_last_epilogue_forms(unsigned int *bits, int clear)
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 
+long long x1cb_trace_copy(unsigned long long *host, long long words, int clear)
+{
+    if (!host && words > 0)
+        return X1CB_ERR_NULL;
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return X1CB_ERR_CUDA;
+    const long long n = copy_trace(host, words, clear != 0);
+    return n < 0 ? X1CB_ERR_CUDA : n;
+}
+
 void x1cb_set_block_fusion(int enable) { g_block_fusion.store(enable ? 1 : 0); }
 
 void x1cb_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns); }

@@ -44,11 +44,9 @@
 #include "x1cb_epi.cuh"
 #include "x1cb_internal.h"
 #include "x1cb_ptx.cuh"
+#include "x1cb_trace.cuh"
 
 namespace x1cb {
-
-extern __device__ unsigned int g_dev_status;
-extern __device__ unsigned int g_dev_forms;
 
 namespace {
 
@@ -236,6 +234,7 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
     int k = 0;             // item index in issue order
     uint32_t kph = 0;      // parity of this turn's slot at its next item
     bool ok = true;
+    const bool tr = q == 0 && lane == 0;  // one trace writer per turn
     for (int i = 0; ok && i <= n_my; ++i) {
         if (i < n_my) {
             if ((k & 3) == turn) {
@@ -250,6 +249,8 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
                     ok = false;
                     break;
                 }
+                if (tr)
+                    X1CB_TRACE_AT(p.trace, 6, i);
                 tc_fence_after();
                 uint8_t *a3 = smem + p.off_a3 + b * kA3Bytes;
 #pragma unroll 1
@@ -267,6 +268,8 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
                 fence_proxy_async_smem();  // read by the MMA (async proxy, rank 0's issue)
                 tc_fence_before();
                 __syncwarp();
+                if (tr)
+                    X1CB_TRACE_AT(p.trace, 7, i);
                 if (lane == 0) {
                     mbar_arrive_cluster(empty0);
                     mbar_arrive_cluster(mapa_shared(bars.a3_full(b), 0));
@@ -287,14 +290,21 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
                 // Stages are taken in order (the ticket), so each stage's
                 // previous phase is complete before its arrival is awaited.
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)) ||
-                    !__all_sync(0xffffffffu, ticket_wait(io_ticket, static_cast<int>(n), ctl,
+                                mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue))) {
+                    ok = false;
+                    break;
+                }
+                if (tr)
+                    X1CB_TRACE_AT(p.trace, 8, n);
+                if (!__all_sync(0xffffffffu, ticket_wait(io_ticket, static_cast<int>(n), ctl,
                                                          kDevTimeoutEpilogue)) ||
                     !__all_sync(0xffffffffu, mbar_wait(bars.io_full(st), st_phase, ctl,
                                                        kDevTimeoutEpilogue))) {
                     ok = false;
                     break;
                 }
+                if (tr)
+                    X1CB_TRACE_AT(p.trace, 9, n);
                 if (lane == 0)
                     atomicMax(const_cast<int *>(io_ticket), static_cast<int>(n + 1));
                 tc_fence_after();
@@ -322,6 +332,8 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
+                if (tr)
+                    X1CB_TRACE_AT(p.trace, 10, n);
                 if (lane == 0) {
                     mbar_arrive(bars.out_ready(st));
                     mbar_arrive_cluster(empty0);
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmO,
                    const int32_t *__restrict__ b2, const int32_t *__restrict__ m2,
                    const int32_t *__restrict__ b3, const int32_t *__restrict__ m3,
-                   const ChainPlan p)
+                   unsigned int *dev_status, unsigned int *dev_forms, const ChainPlan p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -354,13 +366,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Conv3 items take the shortcut stages' arrivals in stage order (ticket).
     volatile int *io_ticket = reinterpret_cast<volatile int *>(smem + p.off_misc + 8);
     ChainBars bars{sbase + static_cast<uint32_t>(p.off_bar), p.a_stages, p.r_stages};
-    const WaitCtl ctl{abort_flag, &g_dev_status, p.wait_limit_ns};
+    const WaitCtl ctl{abort_flag, dev_status, p.wait_limit_ns};
     const uint64_t drain_ns = 200000000ull;
     const int pair0 = blockIdx.x / 2;
     const int pair_step = gridDim.x / 2;
     const int n_my = pair0 < p.n_pairs ? (p.n_pairs - pair0 + pair_step - 1) / pair_step : 0;
 
     // ---- set-up -----------------------------------------------------------------
+    // Trace events (trace builds): 0 producer box n may load; 1 MMA sees tile
+    // n's first box; 2 MMA has a slot for tile n's Conv2; 3 ... committed it;
+    // 4 MMA sees tile n's Conv2 result; 5 MMA committed Conv3 chunk n; 6/7
+    // epilogue starts/ends tile n's Conv2; 8/9/10 epilogue sees the
+    // accumulator / shortcut of chunk n, is done; 11/12 store warp sees chunk
+    // n / has read it; 13 shortcut chunk n issued; 14 weights seen; 15 start, end.
+    if (threadIdx.x == 0)
+        X1CB_TRACE_AT(p.trace, 15, 0);
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *io_ticket = 0;
@@ -406,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fill_consts(mode2, b2, m2, p.Cm, p.S, cm2, cc2);
     fill_consts(mode3, b3, m3, p.Cout, p.S, cm3, cc3);
     if (threadIdx.x == 0)
-        atomicOr(&g_dev_forms, (1u << mode2) | (1u << mode3));
+        atomicOr(dev_forms, (1u << mode2) | (1u << mode3));
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish_pair();
@@ -421,6 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ---- producer: weight halves, then halo tiles --------------------------------
+        // Slots of the halo ring are issued in rounds by n_iss lanes, which wait
+        // for their slots together and issue as one (see the convolution
+        // kernel's producer: one thread issues a tensor copy only every several
+        // hundred cycles; n_iss <= a_stages / 2 keeps each slot barrier's
+        // parity unambiguous).
+        const int n_iss = max(1, min(kAIssuers, p.a_stages / 2));
         if (lane == 0) {
             const uint32_t wfull0 = mapa_shared(bars.w_full(), 0);
             const int half = static_cast<int>(rank) * kHalfRows;
@@ -435,31 +461,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < p.C1; ++kb)
                     tma2_load_4d(sbase + p.off_w3 + (c * p.C1 + kb) * kHalfRows * 32, &tmW3,
                                  wfull0, 0, half, kb, c);
+        }
+        __syncwarp();
+        if (lane < kAIssuers) {
             const uint32_t abytes = static_cast<uint32_t>(2 * 16 * p.plane_m * p.tg);
             const uint64_t pol = policy_evict_first();
-            int stage = 0;
+            const long long total = static_cast<long long>(n_my) * p.C1;
+            long long issued = 0;
+            // this lane's slot n = base + lane: ring stage/phase, pair tile i,
+            // channel block c1 (counters, at most one ring wrap per round)
+            int stage = lane < n_iss ? lane : 0, i = lane / p.C1, c1 = lane % p.C1;
             uint32_t phase = 0;
-            bool ok = true;
-            for (int i = 0; ok && i < n_my; ++i) {
-                const int mt = 2 * (pair0 + i * pair_step) + static_cast<int>(rank);
-                int h0, b0;
-                chain_origin(p, mt, h0, b0);
-                for (int c1 = 0; c1 < p.C1; ++c1) {
-                    if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
-                        ok = false;
-                        break;
-                    }
+            for (long long base = 0; base < total; base += n_iss) {
+                const long long n = base + lane;
+                const bool have = lane < n_iss && n < total;
+                if (!mbar_wait_lanes(kAIssuerMask, have, bars.a_empty(stage), phase ^ 1u, ctl,
+                                     kDevTimeoutProducer))
+                    break;
+                if (have) {
+                    X1CB_TRACE_AT(p.trace, 0, n);
+                    const int mt = 2 * (pair0 + i * pair_step) + static_cast<int>(rank);
+                    int h0, b0;
+                    chain_origin(p, mt, h0, b0);
                     if (leader)
                         mbar_arrive_expect_tx(bars.a_full(stage), 2 * abytes);
                     const uint32_t slot = sbase + p.off_a + stage * p.a_slot;
                     const uint32_t full0 = mapa_shared(bars.a_full(stage), 0);
                     tma2_load_5d_hint(slot, &tmA, full0, 0, -1, h0 - 1, c1, b0, pol);
                     tma2_load_5d_hint(slot + p.a_half, &tmA, full0, 16, -1, h0 - 1, c1, b0, pol);
-                    if (++stage == p.a_stages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
                 }
+                issued = base + n_iss < total ? base + n_iss : total;
+                stage += n_iss;
+                if (stage >= p.a_stages) {
+                    stage -= p.a_stages;
+                    phase ^= 1u;
+                }
+                for (c1 += n_iss; c1 >= p.C1; c1 -= p.C1)
+                    ++i;
+            }
+            // Both CTAs' copies complete on rank 0's barriers: rank 0 lets every
+            // copy still in flight land (the MMA has normally seen them all)
+            // before the exit handshake releases either CTA.
+            __syncwarp(kAIssuerMask);
+            if (leader && lane == 0) {
+                if (!mbar_drain(bars.w_full(), 0, drain_ns))
+                    atomicOr(dev_status, kDevDrainFailed);
+                const long long last = issued < p.a_stages ? issued : p.a_stages;
+                for (long long k = issued - last; k < issued; ++k)
+                    if (!mbar_drain(bars.a_full(static_cast<int>(k % p.a_stages)),
+                                    static_cast<uint32_t>((k / p.a_stages) & 1), drain_ns))
+                        atomicOr(dev_status, kDevDrainFailed);
             }
         }
         __syncwarp();
@@ -481,6 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    X1CB_TRACE_AT(p.trace, 13, issued);
                     mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
                     const uint32_t dst = sbase + p.off_r + stage * kRSlotBytes;
                     if (p.io_swz)
@@ -500,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (long long k = issued - last; k < issued; ++k)
                 if (!mbar_drain(bars.io_full(static_cast<int>(k % p.r_stages)),
                                 static_cast<uint32_t>((k / p.r_stages) & 1), drain_ns))
-                    atomicOr(&g_dev_status, kDevDrainFailed);
+                    atomicOr(dev_status, kDevDrainFailed);
         }
         __syncwarp();
     } else if (warp == 3) {
@@ -519,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    X1CB_TRACE_AT(p.trace, 11, static_cast<long long>(i) * p.n_chunks + c);
                     const uint32_t src = sbase + p.off_r + stage * kRSlotBytes;
                     if (mt < p.num_m_tiles) {
                         if (p.io_swz)
@@ -528,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bulk_commit();
                         bulk_wait_read<0>();
                     }
+                    X1CB_TRACE_AT(p.trace, 12, static_cast<long long>(i) * p.n_chunks + c);
                     mbar_arrive(bars.io_empty(stage));
                     if (++stage == p.r_stages) {
                         stage = 0;
@@ -558,6 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int slot = 0;        // accumulator slot of the next item (Conv2 tile or Conv3 chunk)
             uint32_t sph = 0;    // and its use parity
             bool ok = __all_sync(0xffffffffu, mbar_wait_cl(bars.w_full(), 0, ctl, kDevTimeoutMma));
+            if (lane == 0)
+                X1CB_TRACE_AT(p.trace, 14, 0);
             for (int i = 0; ok && i <= n_my; ++i) {
                 if (i < n_my) {
                     // Conv2 of pair tile i: 4 channel blocks x 9 taps into the next slot.
@@ -566,6 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (lane == 0)
+                        X1CB_TRACE_AT(p.trace, 2, i);
                     tc_fence_after();
                     const uint32_t d = tmem_base + static_cast<uint32_t>(slot * 128);
                     for (int c1 = 0; c1 < p.C1; ++c1) {
@@ -574,6 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
+                        if (c1 == 0 && lane == 0)
+                            X1CB_TRACE_AT(p.trace, 1, i);
                         tc_fence_after();
 #pragma unroll
                         for (int t = 0; t < 9; ++t)
@@ -592,6 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok)
                         break;
                     mma_commit_pair(bars.acc_full(slot));
+                    if (lane == 0)
+                        X1CB_TRACE_AT(p.trace, 3, i);
                     if (++slot == kSlots) {
                         slot = 0;
                         sph ^= 1u;
@@ -606,6 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (lane == 0)
+                        X1CB_TRACE_AT(p.trace, 4, j);
                     tc_fence_after();
                     const uint64_t ad = a3_desc0 + static_cast<uint64_t>(b) * a3_buf_step;
                     for (int c = 0; c < p.n_chunks; ++c) {
@@ -622,6 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             static_cast<uint64_t>(c * p.C1 + kb) * kb_step,
                                         idesc, kb ? 1u : 0u);
                         mma_commit_pair(bars.acc_full(slot));
+                        if (lane == 0)
+                            X1CB_TRACE_AT(p.trace, 5, static_cast<long long>(j) * p.n_chunks + c);
                         if (++slot == kSlots) {
                             slot = 0;
                             sph ^= 1u;
@@ -634,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit_pair(bars.mma_done());
             if (lane == 0 && !mbar_drain(bars.mma_done(), 0, drain_ns))
-                atomicOr(&g_dev_status, kDevDrainFailed);
+                atomicOr(dev_status, kDevDrainFailed);
         }
         __syncwarp();
     } else {
@@ -656,10 +722,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- tear-down: neither CTA leaves while the other may still reach it ----------
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0)
+        X1CB_TRACE_AT(p.trace, 15, 1);
     if (threadIdx.x == 0) {
         mbar_arrive_cluster(mapa_shared(bars.exit_bar(), rank ^ 1u));
         if (!mbar_drain(bars.exit_bar(), 0, 2 * p.wait_limit_ns + drain_ns))
-            atomicOr(&g_dev_status, kDevDrainFailed);
+            atomicOr(dev_status, kDevDrainFailed);
     }
     __syncthreads();
     if (warp == 1) {
@@ -855,8 +923,13 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, chain23_kernel, tmA, tmW2, tmW3, tmR, tmO, b2, m2, b3, m3, p) !=
-        cudaSuccess)
+    unsigned int *dev_status = nullptr, *dev_forms = nullptr;
+    if (int e = device_words(&dev_status, &dev_forms))
+        return e;
+    ChainPlan q = p;
+    q.trace = trace_table();
+    if (cudaLaunchKernelEx(&cfg, chain23_kernel, tmA, tmW2, tmW3, tmR, tmO, b2, m2, b3, m3,
+                           dev_status, dev_forms, q) != cudaSuccess)
         return X1CB_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }

@@ -49,6 +49,7 @@
 #include "x1cb_plan.h"
 #include "x1cb_epi.cuh"
 #include "x1cb_ptx.cuh"
+#include "x1cb_trace.cuh"
 
 namespace x1cb {
 
@@ -58,6 +59,9 @@ __device__ unsigned int g_dev_status;
 // (0 generic, 1 64-bit high word, 2 all-32-bit, 3 all-32-bit with the bias in
 // the MMA).  Observability for tests and benchmarks; one atomic per CTA.
 __device__ unsigned int g_dev_forms;
+#ifdef X1CB_TRACE
+__device__ unsigned long long g_trace[kTraceWords];
+#endif
 
 namespace {
 
@@ -204,6 +208,9 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.acc_full(acc), acc_phase, cx.ctl,
                                                kDevTimeoutEpilogue)))
             return;
+        const bool tr = q == 0 && lane == 0;  // one trace writer per turn
+        if (tr)
+            X1CB_TRACE_AT(p.trace, 4, n);
         tc_fence_after();
         // Before the parity wait on the slot's arrival, make sure its previous
         // phase (stage n - r_stages, another turn's) is complete.  Ring of at
@@ -220,6 +227,8 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.io_full(st), st_phase, cx.ctl,
                                                kDevTimeoutEpilogue)))
             return;
+        if (tr)
+            X1CB_TRACE_AT(p.trace, 5, n);
         // The four warps of a turn each pass the ticket on; it only moves forward.
         if (!deep && lane == 0)
             atomicMax(const_cast<int *>(cx.io_ticket), static_cast<int>(n + 1));
@@ -282,6 +291,8 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             if (!__all_sync(0xffffffffu, mbar_wait(cx.bars.pool_bar(turn), pool_phase, cx.ctl,
                                                    kDevTimeoutEpilogue)))
                 return;
+            if (tr)
+                X1CB_TRACE_AT(p.trace, 10, n);
             pool_phase ^= 1u;
             const int tid = q * 32 + lane;
             const int np = p.pw * p.ph;
@@ -311,6 +322,8 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
+        if (tr)
+            X1CB_TRACE_AT(p.trace, 6, n);
         if (lane == 0) {
             mbar_arrive(cx.bars.out_ready(st));
             mbar_arrive(cx.bars.acc_empty(acc));  // one arrival per stage of the slot
@@ -370,6 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int stages_per_tile = p.NC / (32 * p.stage_ch);
 
     // ---- set-up ---------------------------------------------------------------
+    // Trace events (trace builds): 0 producer box n may load; 1 MMA sees box n;
+    // 2 MMA has slot for sub-tile n; 3 MMA committed sub-tile n; 4 epilogue
+    // sees the accumulator of I/O stage n; 5 ... its shortcut; 6 ... is done;
+    // 7 store warp sees stage n; 8 stage n's store has read it; 9 I/O
+    // producer issues stage n; 10 pool turn met for stage n; 15: start, end.
+    if (threadIdx.x == 0)
+        X1CB_TRACE_AT(p.trace, 15, 0);
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *io_ticket = 0;
@@ -471,6 +491,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ---- producer: resident weights, then activation K blocks ---------------
+        // One thread issues a tensor copy only every several hundred cycles, so
+        // n_iss lanes issue in rounds: in round j lane l takes box
+        // n = j*n_iss + l (boxes counted over the CTA's tiles); the lanes wait
+        // for their slots together (mbar_wait_lanes) and issue as one.  A
+        // round waits for n_iss consecutive slots, so n_iss is at most half
+        // the ring; and each slot barrier's parity stays unambiguous because
+        // a lane's wait for box n follows the round that saw box n - 1 - S
+        // consumed, with the MMA consuming in order.
+        const int n_iss = max(1, min(kAIssuers, p.a_stages / 2));
         if (lane == 0) {
             const uint32_t sw = sbase + p.off_w;
             const int o1 = group * (p.NC / p.O2);  // weight block of this CTA's channels
@@ -488,6 +517,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 mbar_arrive(bars.w_full());  // weights travel with the activation stages
             }
+        }
+        __syncwarp();
+        if (lane < kAIssuers) {
+            const int o1 = group * (p.NC / p.O2);
             // Streamed weights: bytes per stage, each K block NC rows x 32 bytes.
             const uint32_t wpart = static_cast<uint32_t>(p.w_part);
             const uint32_t wkb = static_cast<uint32_t>(p.NC * 32);
@@ -498,118 +531,104 @@ __global__ void __launch_bounds__(kThreads, 1)
                        : static_cast<uint32_t>(p.a_kc * p.rows * 32);  // K halves / blocks
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
-            const int boxes = p.kb_per_tile / p.a_kc;  // unused in the halo form
-            const uint32_t a_slot = static_cast<uint32_t>(p.a_slot);
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t slot = sa;
+            // Boxes per tile: halo form one per channel block; else K blocks run
+            // channel block fastest, then filter column, then filter row, then
+            // (if present) the second source's channel blocks.
+            const int cb = p.C1 / p.a_kc;
+            const int first_boxes = p.halo ? p.C1 : p.R * p.Rw * cb;
+            const int bpt = p.halo ? p.C1 : p.kb_per_tile / p.a_kc;
+            const long long my_tiles =
+                mt_first < p.num_m_tiles ? (p.num_m_tiles - mt_first + mt_step - 1) / mt_step : 0;
+            const long long total = my_tiles * bpt;
             long long issued = 0;
-            bool ok = true;
-            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
-                int w0, h0, b0;
-                tile_origin(p, mt, w0, h0, b0);
-                if (p.halo) {
-                    // One slot per channel block: the tile's pixels plus a one-pixel
-                    // frame (zeros outside the image), each K half as one box.
-                    for (int c1 = 0; c1 < p.C1; ++c1) {
-                        if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl,
-                                       kDevTimeoutProducer)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
-                        if (p.halo == 2) {
-                            // plane (pr, pc) from input (pc - 1, 2*h0 - 1 + pr), step 2
-                            for (int pl = 0; pl < 4; ++pl)
-                                for (int hf = 0; hf < 2; ++hf)
-                                    tma_load_5d_hint(
-                                        slot + static_cast<uint32_t>((2 * pl + hf) * p.a_half),
-                                        &tmA, bars.a_full(stage), 16 * hf, (pl & 1) - 1,
-                                        2 * h0 - 1 + (pl >> 1), c1, b0, pol);
-                        } else {
-                            tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
-                                             h0 - p.pad, c1, b0, pol);
-                            tma_load_5d_hint(slot + static_cast<uint32_t>(p.a_half), &tmA,
-                                             bars.a_full(stage), 16, w0 - p.pad, h0 - p.pad, c1,
-                                             b0, pol);
-                        }
-                        if (wpart) {  // the nine taps' weights of channel block c1
-                            const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
-                            for (int t = 0; t < 9; ++t)
-                                tma_load_4d(wdst + t * wkb, &tmW, bars.a_full(stage), 0, 0,
-                                            t * p.C1 + c1, o1);
-                        }
-                        ++issued;
-                        if (++stage == p.a_stages) {
-                            stage = 0;
-                            phase ^= 1u;
-                            slot = sa;
-                        } else {
-                            slot += a_slot;
-                        }
-                    }
-                    continue;
-                }
-                // K blocks run channel block fastest, then filter column, then
-                // filter row, then (if present) the second source's channel
-                // blocks; counters instead of divisions keep the issue cheap.
-                // Output pixel (w0, h0) reads input (w0*stride + ds - pad, ...);
-                // a strided map steps `stride` input pixels per loaded pixel.
-                const int wi0 = w0 * p.stride - p.padw, hi0 = h0 * p.stride - p.pad;
-                int c1 = 0, ds = 0, dr = 0;
-                bool second = false;
-                for (int bx = 0; bx < boxes; ++bx) {
-                    if (!mbar_wait(bars.a_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
-                        ok = false;
-                        break;
-                    }
+            // This lane's box n = base + lane as ring stage/phase and as (tile i,
+            // box b of the tile), advanced by counters (n_iss <= a_stages / 2:
+            // at most one wrap of the ring per round).
+            int stage = lane < n_iss ? lane : 0, i = lane / bpt, b = lane % bpt;
+            uint32_t phase = 0;
+            for (long long base = 0; base < total; base += n_iss) {
+                const long long n = base + lane;
+                const bool have = lane < n_iss && n < total;
+                if (!mbar_wait_lanes(kAIssuerMask, have, bars.a_empty(stage), phase ^ 1u, ctl,
+                                     kDevTimeoutProducer))
+                    break;
+                if (have) {
+                    X1CB_TRACE_AT(p.trace, 0, n);
+                    const int mt = mt_first + i * mt_step;
+                    int w0, h0, b0;
+                    tile_origin(p, mt, w0, h0, b0);
+                    const uint32_t slot = sa + static_cast<uint32_t>(stage) * p.a_slot;
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
-                    if (!second)
-                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, wi0 + ds, hi0 + dr,
+                    if (p.halo == 2) {
+                        // one slot per channel block c1 = b: plane (pr, pc) from
+                        // input (pc - 1, 2*h0 - 1 + pr), step 2
+                        for (int pl = 0; pl < 4; ++pl)
+                            for (int hf = 0; hf < 2; ++hf)
+                                tma_load_5d_hint(
+                                    slot + static_cast<uint32_t>((2 * pl + hf) * p.a_half), &tmA,
+                                    bars.a_full(stage), 16 * hf, (pl & 1) - 1,
+                                    2 * h0 - 1 + (pl >> 1), b, b0, pol);
+                    } else if (p.halo) {
+                        // the tile's pixels plus a one-pixel frame (zeros outside the
+                        // image), each K half as one box
+                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
+                                         h0 - p.pad, b, b0, pol);
+                        tma_load_5d_hint(slot + static_cast<uint32_t>(p.a_half), &tmA,
+                                         bars.a_full(stage), 16, w0 - p.pad, h0 - p.pad, b, b0,
+                                         pol);
+                    } else if (b < first_boxes) {
+                        // output pixel (w0, h0) reads input (w0*stride + ds - pad, ...);
+                        // a strided map steps `stride` input pixels per loaded pixel
+                        const int c1 = (b % cb) * p.a_kc;
+                        const int tap = b / cb;
+                        const int ds = tap % p.Rw, dr = tap / p.Rw;
+                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0,
+                                         w0 * p.stride - p.padw + ds, h0 * p.stride - p.pad + dr,
                                          b0, c1, pol);
-                    else
+                    } else {
                         tma_load_5d_hint(slot, &tmA2, bars.a_full(stage), 0, w0 * p.stride2,
-                                         h0 * p.stride2, b0, c1, pol);
+                                         h0 * p.stride2, b0, (b - first_boxes) * p.a_kc, pol);
+                    }
                     if (wpart) {  // the box's K blocks' weights
                         const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
-                        const int kb0 = second ? c1 : (dr * p.Rw + ds) * p.C1 + c1;
-                        for (int i = 0; i < p.a_kc; ++i) {
-                            if (!second)
+                        if (p.halo) {  // the nine taps of channel block b
+                            for (int t = 0; t < 9; ++t)
+                                tma_load_4d(wdst + t * wkb, &tmW, bars.a_full(stage), 0, 0,
+                                            t * p.C1 + b, o1);
+                        } else if (b < first_boxes) {
+                            const int kb0 = (b / cb) * p.C1 + (b % cb) * p.a_kc;
+                            for (int i = 0; i < p.a_kc; ++i)
                                 tma_load_4d(wdst + i * wkb, &tmW, bars.a_full(stage), 0, 0,
                                             kb0 + i, o1);
-                            else
+                        } else {
+                            const int kb0 = (b - first_boxes) * p.a_kc;
+                            for (int i = 0; i < p.a_kc; ++i)
                                 tma_load_4d(wdst + i * wkb, &tmW2, bars.a_full(stage), 0, 0,
                                             kb0 + i, o1);
                         }
                     }
-                    ++issued;
-                    if (++stage == p.a_stages) {
-                        stage = 0;
-                        phase ^= 1u;
-                        slot = sa;
-                    } else {
-                        slot += a_slot;
-                    }
-                    c1 += p.a_kc;
-                    if (!second && c1 == p.C1) {
-                        c1 = 0;
-                        if (++ds == p.Rw) {
-                            ds = 0;
-                            if (++dr == p.R)
-                                second = true;  // only reached when C1b > 0
-                        }
-                    }
                 }
+                issued = base + n_iss < total ? base + n_iss : total;
+                stage += n_iss;
+                if (stage >= p.a_stages) {
+                    stage -= p.a_stages;
+                    phase ^= 1u;
+                }
+                for (b += n_iss; b >= bpt; b -= bpt)
+                    ++i;
             }
             // Let every copy still in flight land before shared memory goes away.
-            if (!mbar_drain(bars.w_full(), 0, drain_ns))
-                atomicOr(&g_dev_status, kDevDrainFailed);
-            const long long last = issued < p.a_stages ? issued : p.a_stages;
-            for (long long i = issued - last; i < issued; ++i) {
-                const int s = static_cast<int>(i % p.a_stages);
-                const uint32_t ph = static_cast<uint32_t>((i / p.a_stages) & 1);
-                if (!mbar_drain(bars.a_full(s), ph, drain_ns))
+            __syncwarp(kAIssuerMask);
+            if (lane == 0) {
+                if (!mbar_drain(bars.w_full(), 0, drain_ns))
                     atomicOr(&g_dev_status, kDevDrainFailed);
+                const long long last = issued < p.a_stages ? issued : p.a_stages;
+                for (long long i = issued - last; i < issued; ++i) {
+                    const int s = static_cast<int>(i % p.a_stages);
+                    const uint32_t ph = static_cast<uint32_t>((i / p.a_stages) & 1);
+                    if (!mbar_drain(bars.a_full(s), ph, drain_ns))
+                        atomicOr(&g_dev_status, kDevDrainFailed);
+                }
             }
         }
         __syncwarp();
@@ -623,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
+            [[maybe_unused]] long long n_io = 0;  // stages handed out (trace index)
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
@@ -632,6 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    X1CB_TRACE_AT(p.trace, 9, n_io);
+                    ++n_io;
                     if (kRes) {
                         mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
                         const int o1 = group * (p.NC / 32) + rs * p.stage_ch;
@@ -672,6 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
+            [[maybe_unused]] long long n_st = 0;  // stages stored (trace index)
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
@@ -681,6 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    X1CB_TRACE_AT(p.trace, 7, n_st);
                     const int o1 = group * (p.NC / 32) + rs * p.stage_ch;
                     if (p.pool)  // pooled tile at pooled coordinates ((w0 + 1) / 2, ...)
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes + kRSlotBytes / 2, 0,
@@ -694,6 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0, h0, o1, b0, pol);
                     bulk_commit();
                     bulk_wait_read<0>();
+                    X1CB_TRACE_AT(p.trace, 8, n_st);
+                    ++n_st;
                     mbar_arrive(bars.io_empty(stage));
                     if (++stage == p.r_stages) {
                         stage = 0;
@@ -757,6 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t a_slot_desc = a_desc0;
             int acc = 0;
             uint32_t acc_phase = 0;
+            [[maybe_unused]] long long n_box = 0, n_sub = 0;  // trace indices
             bool ok = __all_sync(0xffffffffu, mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma));
             if (ok && p.inject == 1) {
                 const WaitCtl planted{abort_flag, &g_dev_status, p.wait_limit_ns};
@@ -773,6 +800,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (lane == 0)
+                        X1CB_TRACE_AT(p.trace, 2, n_sub);
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * p.nmma);
                     const bool last_sub = j == p.n_subs - 1;
@@ -788,6 +817,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                          kDevTimeoutMma))) {
                             ok = false;
                             break;
+                        }
+                        if (j == 0) {
+                            if (lane == 0)
+                                X1CB_TRACE_AT(p.trace, 1, n_box);
+                            ++n_box;
                         }
                         uint64_t ad = sd;
                         if (p.wstream)  // this stage's own weights (one N slice: j == 0)
@@ -830,6 +864,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_i8(d_tmem, fold_a, fold_b0 + static_cast<uint64_t>(j) * b_sub_step,
                                idesc, 1u);
                     mma_commit(bars.acc_full(acc));
+                    if (lane == 0)
+                        X1CB_TRACE_AT(p.trace, 3, n_sub);
+                    ++n_sub;
                     if (++acc == n_slots) {
                         acc = 0;
                         acc_phase ^= 1u;
@@ -868,6 +905,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- tear-down ---------------------------------------------------------------
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0)
+        X1CB_TRACE_AT(p.trace, 15, 1);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
@@ -1416,9 +1455,54 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
     auto kern = p.has_res ? conv_bn_act_kernel<true> : conv_bn_act_kernel<false>;
     if (int e = opt_in_smem(reinterpret_cast<const void *>(kern), p.has_res))
         return e;
-    kern<<<p.grid, kThreads, p.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, tmA2, tmW2, bias, mult,
-                                                      p);
+    ConvPlan q = p;
+    q.trace = trace_table();
+    kern<<<q.grid, kThreads, q.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, tmA2, tmW2, bias, mult,
+                                                      q);
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+}
+
+// The library's kernels live in separate translation units compiled without
+// relocatable device code, where a device variable cannot be shared by
+// declaration: the other kernels receive these addresses as parameters.
+int device_words(unsigned int **status, unsigned int **forms)
+{
+    void *ps = nullptr, *pf = nullptr;
+    if (cudaGetSymbolAddress(&ps, g_dev_status) != cudaSuccess ||
+        cudaGetSymbolAddress(&pf, g_dev_forms) != cudaSuccess)
+        return X1CB_ERR_CUDA;
+    *status = static_cast<unsigned int *>(ps);
+    *forms = static_cast<unsigned int *>(pf);
+    return X1CB_OK;
+}
+
+unsigned long long *trace_table()
+{
+#ifdef X1CB_TRACE
+    void *t = nullptr;
+    return cudaGetSymbolAddress(&t, g_trace) == cudaSuccess
+               ? static_cast<unsigned long long *>(t)
+               : nullptr;
+#else
+    return nullptr;
+#endif
+}
+
+long long copy_trace(unsigned long long *host, long long words, bool clear)
+{
+#ifdef X1CB_TRACE
+    const long long n = words < kTraceWords ? words : kTraceWords;
+    if (n > 0 && cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)) != cudaSuccess)
+        return -1;
+    if (clear && cudaMemset(trace_table(), 0, sizeof(g_trace)) != cudaSuccess)
+        return -1;
+    return n;
+#else
+    (void)host;
+    (void)words;
+    (void)clear;
+    return 0;
+#endif
 }
 
 unsigned int read_and_clear_dev_status(bool clear)

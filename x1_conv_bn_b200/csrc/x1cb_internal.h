@@ -43,7 +43,14 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
                  const int32_t *m2, const int8_t *w3, const int32_t *b3, const int32_t *m3,
                  const int8_t *x, int8_t *out, cudaStream_t stream);
 
+// Device addresses of the sticky status word and the epilogue-forms word of
+// the current device (for kernels outside the convolution's translation unit).
+int device_words(unsigned int **status, unsigned int **forms);
 unsigned int read_and_clear_dev_status(bool clear);
+// Timeline table of trace builds (null in the default build); copy_trace
+// copies up to `words` of it to the host (returns the words copied).
+unsigned long long *trace_table();
+long long copy_trace(unsigned long long *host, long long words, bool clear);
 unsigned int read_and_clear_dev_forms(bool clear);
 
 // The bottleneck chain behind bottleneck_i8 and bottleneck_i8_noalloc.

@@ -8,6 +8,8 @@ namespace x1cb {
 constexpr int kEpiWarp0 = 4;        // warps 0-3: producers, MMA issuer, store
 constexpr int kEpiWarps = 16;       // 4 per TMEM lane quarter
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr int kAIssuers = 4;            // lanes of the producer warp issuing activation copies
+constexpr unsigned kAIssuerMask = (1u << kAIssuers) - 1;
 static_assert(kEpiWarp0 % 4 == 0 && kEpiWarps % 4 == 0, "roles must be whole warpgroups");
 constexpr int kTileRows = 128;      // MMA M
 constexpr int kKBlock = 32;         // int8 channels per K block (one MMA K step)
@@ -94,6 +96,7 @@ struct ConvPlan {
     int inject;  // test hook: 1 = the MMA warp waits on a barrier nobody arrives on
     unsigned long long wait_limit_ns;
     int grid;
+    unsigned long long *trace;  // timeline table (trace builds only; else null)
 };
 
 // Launch plan of the fused Conv2 -> Conv3 kernel (pairs of CTAs; see
@@ -111,6 +114,7 @@ struct ChainPlan {
     int io_swz;  // output/shortcut stages in the 128-byte swizzle (else 8-byte-element rows)
     int grid;    // CTAs (two per cluster)
     unsigned long long wait_limit_ns;
+    unsigned long long *trace;  // timeline table (trace builds only; else null)
 };
 
 }  // namespace x1cb

@@ -105,6 +105,53 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
 }
 
+// Non-blocking probe of phase `parity` (mbarrier.test_wait never suspends
+// the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Warp-synchronous bounded wait of the lanes in `mask`: each lane with
+// want = true waits for phase `parity` of its own barrier, and all return
+// together once every lane's phase is complete, so the lanes stay converged
+// and issue their next instructions (tensor copies) as one.  Lanes poll
+// without suspending: a suspended lane would hold up the warp's others.
+// Returns false for all lanes when the CTA was told to abort or the limit
+// passed (then one lane raises the abort flag and records `code`).
+__device__ __forceinline__ bool mbar_wait_lanes(unsigned mask, bool want, uint32_t bar,
+                                                uint32_t parity, const WaitCtl &ctl,
+                                                unsigned int code)
+{
+    bool ready = !want || mbar_test_wait(bar, parity);
+    if (__all_sync(mask, ready))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        ready = ready || mbar_test_wait(bar, parity);
+        if (__all_sync(mask, ready))
+            return true;
+        if ((it & 63u) == 0) {
+            const bool stop = *ctl.abort_flag || globaltimer_ns() - t0 > ctl.limit_ns;
+            if (__any_sync(mask, stop)) {
+                if (stop && !*ctl.abort_flag) {
+                    *ctl.abort_flag = 1;
+                    atomicOr(ctl.status, code);
+                }
+                return false;
+            }
+        }
+    }
+}
+
 // Bounded wait until a monotonic shared-memory counter reaches at least
 // `want` (napping between polls); same abort and limit rules as mbar_wait.
 __device__ __forceinline__ bool ticket_wait(const volatile int *ticket, int want,
@@ -272,8 +319,12 @@ __device__ __forceinline__ uint32_t requant4_fast(uint32_t a0, uint32_t a1, uint
 // kAddBias = false: the accumulator already holds acc + bias (folded into the
 // MMA), so the four additions are skipped and b is ignored.  kK1: k == 1.
 // The high word is a plain multiply-high and the small addend a separate add
-// (hi32(u*m) + c is what a fused multiply-high-add computes, but written apart
-// the add of r + 1 is one three-input add when k == 1).
+// (with k == 1, h + r + 1 is one three-input add).  The clamp to [0, 255] and
+// the packing are one saturating convert-and-pack per two outputs
+// (cvt.pack.sat.u8.s32: d = c << 16 | sat(a) << 8 | sat(b)), and the halving
+// is done on the packed word: each byte is at most 255, so a shift of the
+// whole word by one and a mask of the bits that crossed a byte boundary
+// halve the four bytes exactly.
 template <bool kRes, bool kAddBias = true, bool kK1 = false>
 __device__ __forceinline__ uint32_t requant4_hi32(uint32_t a0, uint32_t a1, uint32_t a2,
                                                   uint32_t a3, int4 m, int4 b, uint32_t rword,
@@ -294,20 +345,11 @@ __device__ __forceinline__ uint32_t requant4_hi32(uint32_t a0, uint32_t a1, uint
             c = kK1 ? r + 1 : r * k + 1;
         }
         y[e] = h + c;
-        asm("min.relu.s32 %0, %0, 255;" : "+r"(y[e]));
     }
-    uint32_t d;
-    asm("{\n\t"
-        ".reg .b32 p, q;\n\t"
-        "mad.lo.u32 p, %2, 256, %1;\n\t"
-        "mad.lo.u32 q, %4, 256, %3;\n\t"
-        "mad.lo.u32 p, q, 65536, p;\n\t"
-        "shr.b32 p, p, 1;\n\t"
-        "and.b32 %0, p, 0x7f7f7f7f;\n\t"
-        "}"
-        : "=r"(d)
-        : "r"(y[0]), "r"(y[1]), "r"(y[2]), "r"(y[3]));
-    return d;
+    uint32_t hi, d;
+    asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(hi) : "r"(y[3]), "r"(y[2]), "r"(0));
+    asm("cvt.pack.sat.u8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(y[1]), "r"(y[0]), "r"(hi));
+    return (d >> 1) & 0x7f7f7f7fu;
 }
 
 // L2 policy for data read or written once: evict it first.
