@@ -172,15 +172,18 @@ int conv_bn_relu_maxpool_i8(const int8_t *x, const int8_t *w, const int32_t *bia
 
 /*
  * The same stem with the image width-folded (the layout step
- * x1cb_pack_stem): each pixel of the folded tensor carries its filter row's
- * R taps x Cin channels in its 32-channel block, so the R x R convolution is
- * an R x 1 convolution with R*Cin useful channels per K step instead of Cin
+ * x1cb_pack_stem): each pixel of the folded tensor carries, for one output
+ * column, its filter row's R taps x Cin channels in its 32-channel block, so
+ * the R x R stride-2 convolution is an R x 1 convolution (rows at stride 2,
+ * columns at stride 1) with R*Cin useful channels per K step instead of Cin
  * (21 of 32 for ResNet50's 7x7 over RGB, against 3 of 32 unfolded: 7x fewer
- * MMAs for the same result).  Stride 2, pad (R-1)/2, 64 outputs, then 3x3
- * stride-2 max pooling; bit-identical to conv_bn_relu_maxpool_i8 on the
- * unfolded image.
- *   folded [B, 1, H, W, 32] (x1cb_pack_stem); wf [1, R, 1, 1, 64, 32]
+ * MMAs for the same result).  Pad (R-1)/2, 64 outputs, then 3x3 stride-2 max
+ * pooling; bit-identical to conv_bn_relu_maxpool_i8 on the unfolded image.
+ * H, W are the image's dims; Wc = (W + 2*((R-1)/2) - R)/2 + 1.
+ *   folded [B, 1, H, Wc, 32] (x1cb_pack_stem); wf [1, R, 1, 1, 64, 32]
  *   (x1cb_pack_stem_weight); bias, m [64]; out [B, 2, Hp, Wp, 32] as above.
+ * Each CTA tile loads one box of 2*16 + R - 2 folded rows x 8 columns and
+ * computes 8 x 16 conv pixels, pooled to 3 x 7.
  */
 int stem_conv_bn_relu_maxpool_i8(const int8_t *folded, const int8_t *wf, const int32_t *bias,
                                  const int32_t *m, int32_t S, int8_t *out, int B, int H, int W,
@@ -272,10 +275,11 @@ int x1cb_unpack_act(const int8_t *nc32, int8_t *nhwc, int B, int H, int W, int C
  * layer); R in {1, 3, 5, 7}. */
 int x1cb_pack_weight(const int8_t *oihw, int8_t *blocked, int Oc, int Ic, int R, void *stream);
 
-/* Width-folded stem input: nhwc [B, H, W, Cin] image -> folded [B, 1, H, W, 32]
- * with channel ds*Cin + ci of pixel (h, u) = channel ci of image pixel
- * (h, u - (R-1)/2 + ds), zero outside the image and from R*Cin on; needs
- * R*Cin <= 32. */
+/* Width-folded stem input: nhwc [B, H, W, Cin] image -> folded
+ * [B, 1, H, Wc, 32], Wc = (W + 2*((R-1)/2) - R)/2 + 1 (the stride-2 output
+ * columns), with channel ds*Cin + ci of pixel (h, c) = channel ci of image
+ * pixel (h, 2c - (R-1)/2 + ds), zero outside the image and from R*Cin on;
+ * needs R*Cin <= 32. */
 int x1cb_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int Cin, int R,
                    void *stream);
 

@@ -106,7 +106,8 @@ def test_stem_full_size_every_output(oracle):
 def _gpu_folded_stem(x, w, bias, m, S, R):
     folded = X.x1cb_pack_stem(x.to(DEV).contiguous(), R=R)
     wf = X.x1cb_pack_stem_weight(w.to(DEV).contiguous())
-    out = X.stem_conv_bn_relu_maxpool_i8(folded, wf, bias.to(DEV), m.to(DEV), S, R=R)
+    out = X.stem_conv_bn_relu_maxpool_i8(folded, wf, bias.to(DEV), m.to(DEV), S, R=R,
+                                         W=x.shape[2])
     torch.cuda.synchronize()
     st, bits = X.x1cb_last_device_error(clear=True)
     assert st == 0, hex(bits)
@@ -135,16 +136,21 @@ def test_folded_stem_parity(oracle, shape):
     assert ref.unique().numel() > 10
 
 
-def test_pack_stem_layout():
-    """Folded pixel (h, u), channel ds*Cin + ci = image pixel (h, u - 3 + ds),
-    channel ci (zero outside); channels from R*Cin on are zero."""
-    g = torch.Generator().manual_seed(4)
-    x = torch.randint(-128, 128, (2, 5, 9, 3), generator=g, dtype=torch.int8)
-    got = X.x1cb_pack_stem(x.to(DEV), R=7).cpu().reshape(2, 5, 9, 32)
-    ref = torch.zeros(2, 5, 9, 32, dtype=torch.int8)
-    xp = torch.nn.functional.pad(x, (0, 0, 3, 3))  # pad W by 3 on both sides
+@pytest.mark.parametrize("W", [9, 10])
+def test_pack_stem_layout(W):
+    """Folded pixel (h, c), channel ds*Cin + ci = image pixel (h, 2c - 3 + ds),
+    channel ci (zero outside); channels from R*Cin on are zero; Wc = the
+    stride-2 convolution's output columns."""
+    g = torch.Generator().manual_seed(4 + W)
+    x = torch.randint(-128, 128, (2, 5, W, 3), generator=g, dtype=torch.int8)
+    Wc = (W + 6 - 7) // 2 + 1
+    got = X.x1cb_pack_stem(x.to(DEV), R=7).cpu()
+    assert got.shape == (2, 1, 5, Wc, 32)
+    got = got.reshape(2, 5, Wc, 32)
+    ref = torch.zeros(2, 5, Wc, 32, dtype=torch.int8)
+    xp = torch.nn.functional.pad(x, (0, 0, 3, 3 + 2))  # pad W by 3 (and 2 for the last column)
     for ds in range(7):
-        ref[..., ds * 3:ds * 3 + 3] = xp[:, :, ds:ds + 9, :]
+        ref[..., ds * 3:ds * 3 + 3] = xp[:, :, ds:ds + 2 * Wc:2, :]
     assert torch.equal(got, ref)
 
 

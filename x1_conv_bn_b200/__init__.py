@@ -301,11 +301,19 @@ def conv_bn_relu_maxpool_i8(x, w, bias, m, S: int, R: int = 7, stride: int = 2, 
     return out
 
 
+def stem_fold_width(W: int, R: int = 7) -> int:
+    """Columns of the folded stem tensor: the stride-2 convolution's outputs."""
+    pad = (R - 1) // 2
+    return (W + 2 * pad - R) // 2 + 1 if W + 2 * pad >= R else 0
+
+
 def x1cb_pack_stem(nhwc, R: int = 7, out=None, stream=None):
-    """Image [B, H, W, Cin] -> width-folded [B, 1, H, W, 32] (R*Cin <= 32)."""
+    """Image [B, H, W, Cin] -> width-folded [B, 1, H, Wc, 32] (R*Cin <= 32),
+    Wc = stem_fold_width(W, R)."""
     B, H, W, Cin = nhwc.shape
     if out is None:
-        out = torch.empty((B, 1, H, W, 32), dtype=torch.int8, device=nhwc.device)
+        out = torch.empty((B, 1, H, stem_fold_width(W, R), 32), dtype=torch.int8,
+                          device=nhwc.device)
     with _same_device(nhwc, out):
         st = lib().x1cb_pack_stem(_dev(nhwc, torch.int8, "nhwc"), _dev(out, torch.int8, "out"),
                                   B, H, W, Cin, int(R), _stream(stream, nhwc.device))
@@ -327,12 +335,18 @@ def x1cb_pack_stem_weight(oihw, out=None, stream=None):
 
 
 def stem_conv_bn_relu_maxpool_i8(folded, wf, bias, m, S: int, R: int = 7, out=None,
-                                 stream=None):
+                                 stream=None, W: Optional[int] = None):
     """The stem on a width-folded image: R x R stride-2 conv + BN + ReLU +
-    3x3 stride-2 max pooling, 64 outputs.  folded [B, 1, H, W, 32]."""
-    B, C, H, W = _act_shape(folded, "folded")
+    3x3 stride-2 max pooling, 64 outputs.  folded [B, 1, H, Wc, 32] from
+    x1cb_pack_stem; W is the image width (any width whose folded width is Wc
+    gives the same result; default 2*Wc)."""
+    B, C, H, Wc = _act_shape(folded, "folded")
     pad = (R - 1) // 2
-    Hc, Wc = (H + 2 * pad - R) // 2 + 1, (W - 1) // 2 + 1
+    if W is None:
+        W = 2 * Wc
+    if stem_fold_width(W, R) != Wc:
+        raise X1cbError(X1CB_ERR_SHAPE, "stem_conv_bn_relu_maxpool_i8: W does not fold to Wc")
+    Hc = (H + 2 * pad - R) // 2 + 1
     if out is None:
         out = torch.empty((B, 2, _half(Hc), _half(Wc), 32), dtype=torch.int8,
                           device=folded.device)

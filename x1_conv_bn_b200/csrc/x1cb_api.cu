@@ -52,7 +52,7 @@ int device_info(int &sms)
 // a B=1 call is latency-bound).
 struct PlanKey {
     int B, H, W, Ic, Oc, R, has_res, sms;
-    int stride, Hin, Win, Ic2, stride2, Hin2, Win2, pool, Rw;
+    int stride, Hin, Win, Ic2, stride2, Hin2, Win2, pool, Rw, stride_w;
     bool operator==(const PlanKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
 
@@ -66,7 +66,8 @@ int get_plan(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_re
     PlanKey k;
     std::memset(&k, 0, sizeof(k));
     k = PlanKey{B, H, W, Ic, Oc, R, has_res, sms,
-                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2, g.pool, g.Rw};
+                g.stride, g.Hin, g.Win, g.Ic2, g.stride2, g.Hin2, g.Win2, g.pool, g.Rw,
+                g.stride_w};
     {
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < used; ++i)
@@ -185,14 +186,15 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
                      int32_t S, int8_t *out, int B, int Hin, int Win, int Ic, int Oc, int R,
                      int stride, const int8_t *x2, const int8_t *w2, int Ic2, int Hin2,
                      int Win2, int stride2, void *stream, bool check_ptrs = true,
-                     bool pool = false, int Rw = 0)
+                     bool pool = false, int Rw = 0, int stride_w = 0)
 {
     const int pad = (R - 1) / 2;
     const int Rw_ = Rw > 0 ? Rw : R, padw = (Rw_ - 1) / 2;
+    const int sw = stride_w > 0 ? stride_w : stride;
     if (Hin < 0 || Win < 0 || stride < 1 || stride > 8 || stride2 < 1 || stride2 > 8)
         return X1CB_ERR_SHAPE;
     const int H = Hin + 2 * pad >= R ? (Hin + 2 * pad - R) / stride + 1 : 0;
-    const int W = Win + 2 * padw >= Rw_ ? (Win + 2 * padw - Rw_) / stride + 1 : 0;
+    const int W = Win + 2 * padw >= Rw_ ? (Win + 2 * padw - Rw_) / sw + 1 : 0;
     // (a pooled layer has 64 output channels: checked as 128 here, exactly below)
     if (int e = check_conv_shape(B, Hin, Win, Ic, pool ? 128 : Oc, S))
         return e;
@@ -243,6 +245,7 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
     g.Win2 = Win2;
     g.pool = pool ? 1 : 0;
     g.Rw = Rw;
+    g.stride_w = stride_w;
     ConvPlan p;
     if (int e = get_plan(p, B, H, W, Ic, Oc, R, 0, S, 0, sms, g))
         return e;
@@ -401,11 +404,14 @@ int stem_conv_bn_relu_maxpool_i8(const int8_t *folded, const int8_t *wf, const i
                                  int R, void *stream)
 {
     // R x R stride-2 convolution of the image as an R x 1 convolution of its
-    // width-folded form (one 32-channel block per pixel), then pooling.
-    if (R != 1 && R != 3 && R != 5 && R != 7)
+    // width-folded form (one 32-channel block per output column: the fold
+    // applied the column stride), then pooling.
+    if ((R != 1 && R != 3 && R != 5 && R != 7) || W < 0)
         return X1CB_ERR_SHAPE;
-    return conv_geom_common(folded, wf, bias, m, S, out, B, H, W, 32, 64, R, 2, nullptr, nullptr,
-                            0, 0, 0, 1, stream, true, true, 1);
+    const int pad = (R - 1) / 2;
+    const int Wc = W + 2 * pad >= R ? (W + 2 * pad - R) / 2 + 1 : 0;
+    return conv_geom_common(folded, wf, bias, m, S, out, B, H, Wc, 32, 64, R, 2, nullptr, nullptr,
+                            0, 0, 0, 1, stream, true, true, 1, 1);
 }
 
 size_t bottleneck_proj_i8_workspace_size(int B, int H, int W, int Cmid)
@@ -533,14 +539,16 @@ int x1cb_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int 
     if (B < 0 || H < 0 || W < 0 || Cin < 1 || (R != 1 && R != 3 && R != 5 && R != 7) ||
         R * Cin > 32)
         return X1CB_ERR_SHAPE;
-    if (static_cast<size_t>(B) * H * W == 0)
+    const int pad = (R - 1) / 2;
+    const int Wc = W + 2 * pad >= R ? (W + 2 * pad - R) / 2 + 1 : 0;
+    if (static_cast<size_t>(B) * H * Wc == 0)
         return X1CB_OK;
     if (!nhwc || !folded)
         return X1CB_ERR_NULL;
     if (!aligned16(folded))
         return X1CB_ERR_ALIGN;
     const size_t px = static_cast<size_t>(B) * H * W;
-    if (overlap(nhwc, px * Cin, folded, px * 32))
+    if (overlap(nhwc, px * Cin, folded, static_cast<size_t>(B) * H * Wc * 32))
         return X1CB_ERR_OVERLAP;
     if (int e = check_resident({nhwc, folded}))
         return e;

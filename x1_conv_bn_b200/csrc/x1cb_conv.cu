@@ -527,8 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
             // one filter tap), each a 128-row x 32-byte tile, back to back.
             const uint32_t abytes =
-                p.halo ? static_cast<uint32_t>((p.halo == 2 ? 8 : 2) * 16 * p.plane_m * p.tg)
-                       : static_cast<uint32_t>(p.a_kc * p.rows * 32);  // K halves / blocks
+                p.halo == 3 ? static_cast<uint32_t>((2 * p.th + p.R - 2) * p.tw * 32)
+                : p.halo    ? static_cast<uint32_t>((p.halo == 2 ? 8 : 2) * 16 * p.plane_m * p.tg)
+                            : static_cast<uint32_t>(p.a_kc * p.rows * 32);  // K halves / blocks
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
             // Boxes per tile: halo form one per channel block; else K blocks run
@@ -568,6 +569,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     slot + static_cast<uint32_t>((2 * pl + hf) * p.a_half), &tmA,
                                     bars.a_full(stage), 16 * hf, (pl & 1) - 1,
                                     2 * h0 - 1 + (pl >> 1), b, b0, pol);
+                    } else if (p.halo == 3) {
+                        // the tile's columns, input rows from 2*h0 - pad on (output
+                        // row y, tap dr reads input row 2y - pad + dr)
+                        tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0, 2 * h0 - p.pad,
+                                         b0, 0, pol);
                     } else if (p.halo) {
                         // the tile's pixels plus a one-pixel frame (zeros outside the
                         // image), each K half as one box
@@ -743,9 +749,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // lies below 256 KB, so moving an operand by `b` bytes is adding
             // b / 16 to its descriptor.
             const uint32_t idesc = idesc_i8(kTileRows, p.nmma);
+            // (folded stem: output row y reads input row 2y + dr, two input rows
+            // of tw 32-byte pixels per GEMM row group)
             const uint64_t a_desc0 =
-                p.halo ? smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half))
-                       : smem_desc_sw32(sbase + p.off_a);
+                p.halo == 3 ? smem_desc_sw32(sbase + p.off_a, static_cast<uint32_t>(2 * p.tw * 32))
+                : p.halo    ? smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half))
+                            : smem_desc_sw32(sbase + p.off_a);
+            const uint32_t h3_row_step = static_cast<uint32_t>(p.tw * 32) >> 4;  // next tap
             const uint64_t b_desc0 = smem_desc_sw32(sbase + p.off_w);
             // Streamed weights: each ring stage carries its K blocks' weights
             // right after its activation part (same 32-byte swizzle layout as the
@@ -826,7 +836,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint64_t ad = sd;
                         if (p.wstream)  // this stage's own weights (one N slice: j == 0)
                             bd = w_desc0 + (sd - a_desc0);
-                        if (p.halo) {
+                        if (p.halo == 3) {
+                            // filter row dr: the slot dr input rows on, weight K block dr
+                            for (int dr = 0; dr < p.R; ++dr)
+                                mma_i8(d_tmem, ad + static_cast<uint64_t>(dr) * h3_row_step,
+                                       bd + static_cast<uint64_t>(dr) * b_kb_step, idesc,
+                                       dr == 0 ? accumulate : 1u);
+                            bd += static_cast<uint64_t>(p.R) * b_kb_step;
+                        } else if (p.halo) {
 #pragma unroll
                             for (int t = 0; t < 9; ++t)
                                 mma_i8(d_tmem, ad + tap_off[t],
@@ -1074,18 +1091,22 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     p.S = S;
     p.m_r = m_r;
     p.stride = g.stride < 1 ? 1 : g.stride;
+    p.stride_w = g.stride_w > 0 ? g.stride_w : p.stride;
     p.Hin = g.Hin ? g.Hin : H;
     p.Win = g.Win ? g.Win : W;
     p.C1b = g.Ic2 / 32;
     p.stride2 = g.stride2 < 1 ? 1 : g.stride2;
     p.Hin2 = g.Hin2;
     p.Win2 = g.Win2;
-    if (p.stride > 8 || p.stride2 > 8 || g.Ic2 % 32 || g.Ic2 < 0)
+    if (p.stride > 8 || p.stride_w > 8 || p.stride2 > 8 || g.Ic2 % 32 || g.Ic2 < 0)
         return X1CB_ERR_SHAPE;  // the TMA's traversal step is at most 8
     // Every tapped input pixel must exist for some output: (H-1)*stride + R - 1
     // - pad < Hin + pad, and the output extent is the convolution's.
     if ((p.Hin + 2 * p.pad - R) / p.stride + 1 != H ||
-        (p.Win + 2 * p.padw - p.Rw) / p.stride + 1 != W)
+        (p.Win + 2 * p.padw - p.Rw) / p.stride_w + 1 != W)
+        return X1CB_ERR_SHAPE;
+    // Column strides other than the row stride exist only for the folded stem.
+    if (p.stride_w != p.stride && !(g.pool && p.Rw == 1 && p.stride_w == 1 && p.stride == 2))
         return X1CB_ERR_SHAPE;
     if (p.C1b && ((H - 1) * p.stride2 >= p.Hin2 || (W - 1) * p.stride2 >= p.Win2))
         return X1CB_ERR_SHAPE;
@@ -1118,6 +1139,10 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
               ((p.stride == 1 && W + 2 <= kTileRows) || (p.stride == 2 && W + 1 <= 126)))
                  ? p.stride
                  : 0;
+    // The folded stem (column filter, rows at stride 2, columns at stride 1,
+    // one channel block, pooled): one slot of input rows per tile (halo = 3).
+    if (p.pool && p.Rw == 1 && p.stride == 2 && p.stride_w == 1 && p.C1 == 1 && p.C1b == 0)
+        p.halo = 3;
     if (p.halo == 2) {
         // th output rows of tg images per tile; a plane is (th+1) x (W+1)
         // pixels (row pitch W+1); GEMM row m = (g*(th+1) + y)*(W+1) + x.
@@ -1142,6 +1167,17 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.plane_m = (p.th + 1) * pitch;
         const int need_rows = std::max(p.tg * p.plane_m, kTileRows + pitch + 1);
         p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+    } else if (p.halo == 3) {
+        // 8 x 16 conv pixels (GEMM row m = y*8 + x) pooled to 3 x 7: conv
+        // columns 0-6 and rows 0-14 of the tile feed the pooled pixels.
+        p.tw = 8;
+        p.th = 16;
+        p.tg = 1;
+        p.pw = 3;
+        p.ph = 7;
+        p.row_pitch = p.tw;
+        p.plane_m = p.tw * p.th;
+        p.a_half = 0;
     } else if (p.halo) {
         choose_halo_tile(B, H, W, p.th, p.tg);
         p.tw = W;
@@ -1189,7 +1225,11 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     p.kb_per_tile = p.kb_a + p.C1b;
 
     const int fixed = 1024 /*alignment slack*/ + 64 /*misc*/ + Bars::count(48, 12) * 8 + 64;
-    const int min_slot = p.halo ? (p.halo == 2 ? 8 : 2) * p.a_half : kASlotBytes;
+    // (halo = 3: 2*th + R - 2 input rows of tw 32-byte pixels)
+    const int h3_bytes = (2 * p.th + R - 2) * p.tw * 32;
+    const int min_slot = p.halo == 3   ? (h3_bytes + 1023) / 1024 * 1024
+                         : p.halo      ? (p.halo == 2 ? 8 : 2) * p.a_half
+                                       : kASlotBytes;
     int chosen = 0;
     long long chosen_work = -1;
     // A 64-channel layer (the stem) is one CTA group of N = 64.  Largest NC
@@ -1222,6 +1262,8 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // 128 output channels per CTA, each ring stage bringing its K blocks'
     // weights from L2 next to its activations.
     p.wstream = chosen == 0 ? 1 : 0;
+    if (p.wstream && p.halo == 3)
+        return X1CB_ERR_SHAPE;
     if (p.wstream)
         chosen = Oc == 64 ? 64 : 128;
     p.NC = chosen;
@@ -1262,12 +1304,15 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // Halo form: one slot per channel block, all of a tile's blocks in the ring
     // when two accumulator slots share them; slots stay 1024-byte aligned.
     // (the stride-2 halo form: four planes of two K halves)
-    p.a_part = p.halo ? ((p.halo == 2 ? 8 : 2) * p.a_half + 1023) / 1024 * 1024
-                      : p.a_kc * kASlotBytes;
+    p.a_part = p.halo == 3 ? (h3_bytes + 1023) / 1024 * 1024
+               : p.halo    ? ((p.halo == 2 ? 8 : 2) * p.a_half + 1023) / 1024 * 1024
+                           : p.a_kc * kASlotBytes;
     p.w_part = p.wstream ? (p.halo ? 9 : p.a_kc) * p.NC * 32 : 0;
     p.a_slot = p.a_part + p.w_part;
     const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
-    const int a_want = std::max(a_min, p.wstream ? 4 : a_bytes_want / p.a_slot);
+    const int a_want = std::max(a_min, p.wstream      ? 4
+                                       : p.halo == 3 ? 12  // one slot per tile: a deep ring
+                                                     : a_bytes_want / p.a_slot);
     const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 4;
     auto layout = [&](int fold, int a, int r) {
         p.fold_room = fold;
@@ -1332,6 +1377,15 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         const uint32_t es[5] = {1, 2, 2, 1, 1};
         if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
                                CU_TENSOR_MAP_DATA_TYPE_UINT8, es))
+            return e;
+    } else if (p.halo == 3) {
+        // Folded stem: dims (32 ch, Win, Hin, B, 1); a box of the tile's tw
+        // columns and all 2*th + R - 2 input rows it needs, 32-byte swizzle.
+        const uint64_t dims[5] = {32, (uint64_t)p.Wpi, (uint64_t)p.Hpi, (uint64_t)p.B, 1};
+        const uint64_t str[4] = {32, (uint64_t)p.Wpi * 32, (uint64_t)p.Hpi * p.Wpi * 32,
+                                 (uint64_t)p.B * p.Hpi * p.Wpi * 32};
+        const uint32_t box[5] = {32, (uint32_t)p.tw, (uint32_t)(2 * p.th + p.R - 2), 1, 1};
+        if (int e = encode_map(&tmA, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     } else if (p.halo) {
         const uint64_t dims[5] = {32, (uint64_t)p.W, (uint64_t)p.H, (uint64_t)p.C1,

@@ -28,6 +28,7 @@ struct ConvGeom {
     int Ic2 = 0, stride2 = 1, Hin2 = 0, Win2 = 0;
     int pool = 0;  // 3x3 stride-2 max pooling after the ReLU (64-channel layers)
     int Rw = 0;    // filter width when it differs from the height (0: square)
+    int stride_w = 0;  // column stride when it differs from the row stride (0: same)
 };
 int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int has_res, int S,
                  int m_r, int num_sms, const ConvGeom &g);

@@ -78,30 +78,32 @@ __global__ void pack_weight_kernel(const int8_t *__restrict__ oihw, int8_t *__re
     }
 }
 
-// The stem's width-folded image: pixel (h, u) of the folded tensor
-// [B, 1, H, W, 32] holds, in channel ds*Cin + ci, channel ci of image pixel
-// (h, u - pad + ds) for the R taps ds of a filter row (zero outside the image;
-// channels from R*Cin on are zero).  An R x R convolution of the image then is
-// an R x 1 convolution of the folded tensor.  One thread per folded pixel.
+// The stem's width-folded image: pixel (h, c) of the folded tensor
+// [B, 1, H, Wc, 32] (Wc output columns of the stride-2 convolution) holds, in
+// channel ds*Cin + ci, channel ci of image pixel (h, 2c - pad + ds) for the R
+// taps ds of a filter row (zero outside the image; channels from R*Cin on are
+// zero).  The R x R stride-2 convolution of the image then is an R x 1
+// convolution of the folded tensor, stride 2 along rows and 1 along columns.
+// One thread per folded pixel.
 __global__ void pack_stem_kernel(const int8_t *__restrict__ nhwc, int8_t *__restrict__ folded,
-                                 int B, int H, int W, int Cin, int R)
+                                 int B, int H, int W, int Wc, int Cin, int R)
 {
-    const long long n = static_cast<long long>(B) * H * W;
+    const long long n = static_cast<long long>(B) * H * Wc;
     const int pad = (R - 1) / 2;
     for (long long q = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; q < n;
          q += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const int u = static_cast<int>(q % W);
-        const long long bh = q / W;  // b * H + h
+        const int c = static_cast<int>(q % Wc);
+        const long long bh = q / Wc;  // b * H + h
         uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         for (int ds = 0; ds < R; ++ds) {
-            const int w = u - pad + ds;
+            const int w = 2 * c - pad + ds;
             if (w < 0 || w >= W)
                 continue;
             const int8_t *src = nhwc + (bh * W + w) * Cin;
             for (int ci = 0; ci < Cin; ++ci) {
-                const int c = ds * Cin + ci;
-                words[c >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(src[ci]))
-                                  << (8 * (c & 3));
+                const int k = ds * Cin + ci;
+                words[k >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(src[ci]))
+                                  << (8 * (k & 3));
             }
         }
         uint4 *dst = reinterpret_cast<uint4 *>(folded + q * 32);
@@ -176,8 +178,10 @@ namespace x1cb {
 int launch_pack_stem(const int8_t *nhwc, int8_t *folded, int B, int H, int W, int Cin, int R,
                      cudaStream_t s)
 {
-    const long long n = static_cast<long long>(B) * H * W;
-    pack_stem_kernel<<<grid_for(n, 256), 256, 0, s>>>(nhwc, folded, B, H, W, Cin, R);
+    const int pad = (R - 1) / 2;
+    const int Wc = W + 2 * pad >= R ? (W + 2 * pad - R) / 2 + 1 : 0;
+    const long long n = static_cast<long long>(B) * H * Wc;
+    pack_stem_kernel<<<grid_for(n, 256), 256, 0, s>>>(nhwc, folded, B, H, W, Wc, Cin, R);
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 

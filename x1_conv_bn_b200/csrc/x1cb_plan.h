@@ -35,6 +35,7 @@ struct ConvPlan {
     // (Wpi, Hpi: the input's dims as the map sees them; H*W and 1 for a
     // stride-1 1x1).  Output pixel (h, w) reads input rows h*stride + dr - pad.
     int stride, Hin, Win, Wpi, Hpi;
+    int stride_w;  // column stride (the folded stem: 1, its fold applied the 2)
     // Optional second activation source whose K blocks follow the first's in
     // the same accumulator (the projection shortcut of a downsampling block):
     // a 1x1 at stride `stride2` over a Hin2 x Win2 image of C1b channel blocks.
@@ -81,6 +82,12 @@ struct ConvPlan {
     // swizzle, the two 16-byte K halves `a_half` bytes apart), and every
     // filter tap reads it shifted by dr*(tw+2)+ds rows.  GEMM row m of the
     // tile is pixel (g, y, x) with m = (g*(th+2) + y)*row_pitch + x.
+    // halo = 2: the stride-2 3x3 over four phase planes.  halo = 3: a column
+    // filter (R x 1, row stride 2, column stride 1) over a width-folded image
+    // with one channel block, pooled: one slot holds the 2*th + R - 2 input
+    // rows of the tile's tw = 8 columns (32-byte swizzle, one 256-byte atom
+    // per input row), and tap dr reads it dr rows on with 512 bytes between
+    // GEMM row groups (output row y reads input row 2y + dr).
     int halo;
     int row_pitch;  // GEMM rows per image row: tw, or tw+2 in the halo form
     int plane_m;    // GEMM rows per image of the tile: tw*th, or (th+2)*(tw+2)

@@ -437,15 +437,16 @@ __device__ __forceinline__ void tc_fence_after()
 
 // Shared-memory matrix descriptor for a K-major operand stored with the
 // 32-byte swizzle: rows of 32 bytes (= 32 int8 = one MMA K step), 8-row
-// groups 256 bytes apart.
-__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr)
+// groups `group_bytes` apart (256: back to back).  The swizzle follows the
+// address, so a start moved by a multiple of 256 bytes keeps its pattern.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr, uint32_t group_bytes = 256)
 {
     uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
-    d |= static_cast<uint64_t>(1) << 16;                  // leading offset (unused here)
-    d |= static_cast<uint64_t>(256 >> 4) << 32;           // stride between 8-row groups
-    d |= static_cast<uint64_t>(1) << 46;                  // descriptor version
-    d |= static_cast<uint64_t>(6) << 61;                  // 32-byte swizzle
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);          // start address
+    d |= static_cast<uint64_t>(1) << 16;                          // leading offset (unused here)
+    d |= static_cast<uint64_t>((group_bytes >> 4) & 0x3FFFu) << 32;  // between 8-row groups
+    d |= static_cast<uint64_t>(1) << 46;                          // descriptor version
+    d |= static_cast<uint64_t>(6) << 61;                          // 32-byte swizzle
     return d;
 }
 

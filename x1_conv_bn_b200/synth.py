@@ -217,11 +217,12 @@ class StemShape:
         return 2 * self.B * self.Hc * self.Wc * self.Oc * self.R * self.R * self.Cin
 
     def bytes_moved(self) -> int:
-        """Image in (one 32-channel block per pixel, as stored), pooled output
-        out, weights."""
-        C = (self.Cin + 31) // 32 * 32
-        return (self.B * self.H * self.W * C + self.B * self.Hp * self.Wp * self.Oc
-                + self.Oc * C * self.R * self.R + 8 * self.Oc)
+        """The stem's input as the kernel reads it -- the width-folded image,
+        one 32-byte block per image row and output column (H x Wc) -- plus the
+        pooled output, the folded weights (R K blocks of 64 x 32) and the
+        per-channel constants."""
+        return (self.B * self.H * self.Wc * 32 + self.B * self.Hp * self.Wp * self.Oc
+                + self.Oc * 32 * self.R + 8 * self.Oc)
 
 
 def stem_inputs(s: StemShape, seed: int, device="cpu", S: int = S_DEFAULT) -> ConvInputs:
