@@ -120,6 +120,18 @@ def _plan(shape):
     return dict(kv.split("=") for kv in X.x1cb_describe_plan(*shape).split())
 
 
+@pytest.mark.parametrize("B,Ic,R,res", [(1, 128, 1, 1), (1024, 128, 1, 1), (2048, 256, 1, 0),
+                                        (512, 128, 3, 0), (64, 512, 1, 1)])
+def test_channel_groups_are_whole_mmas(L, B, Ic, R, res):
+    """Every output width (multiples of 128): a CTA's NC channels are n_subs
+    whole MMAs of nmma columns, and the groups tile Oc exactly (a 384-channel
+    group of one 256-column MMA would leave a third uncomputed)."""
+    for Oc in range(128, 2049, 128):
+        p = _plan((B, 28, 28, Ic, Oc, R, res))
+        NC, nmma, subs, groups = (int(p[k]) for k in ("NC", "nmma", "subs", "groups"))
+        assert nmma * subs == NC and NC * groups == Oc, (Oc, p)
+
+
 @pytest.mark.parametrize("shape,tile", [
     ((1024, 28, 28, 128, 128, 3, 0), "28x4x1"),   # Res3.2 conv2: 4 rows + frame = 120 GEMM rows
     ((2, 30, 28, 128, 128, 3, 0), "28x4x1"),      # ragged in H: 8 tiles per image, last one 2 rows

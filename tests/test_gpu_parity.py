@@ -106,6 +106,21 @@ def test_conv1x1_parity(oracle, shape, has_res):
     _assert_spread(ref)
 
 
+# Shapes whose plans once went wrong: 384- and 768-channel layers large enough
+# for wide channel groups (a group must be whole N = 256 MMAs), and a 512 -> 256
+# layer with a shortcut whose 4-K-block boxes did not fit beside its weights.
+WIDE_GROUPS = [(96, 16, 16, 128, 384), (48, 16, 16, 128, 768), (26, 28, 28, 512, 256)]
+
+
+@pytest.mark.parametrize("shape", WIDE_GROUPS, ids=[str(s) for s in WIDE_GROUPS])
+def test_conv1x1_channel_groups(oracle, shape):
+    s = synth.ConvShape(*shape, R=1, has_res=True)
+    inp = synth.conv_inputs(s, 77 + shape[4])
+    got = _nhwc(_gpu_conv(inp))
+    ref = _oracle_conv(oracle, inp)
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
+
+
 @pytest.mark.parametrize("S", [12, 24, 31, 40])
 def test_conv1x1_full_int8_range(oracle, S):
     """x, w, r over [-128, 127], negative multipliers, wide bias, several shifts."""

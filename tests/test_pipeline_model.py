@@ -279,3 +279,4 @@ def test_model_catches_more_issuing_lanes_than_slots(S):
         except (Early, AssertionError):
             failures += 1
     assert failures == 20
+

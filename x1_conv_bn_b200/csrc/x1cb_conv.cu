@@ -1239,9 +1239,10 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // NC = 128 and a 22-slot ring -- the ring depth does not pay for the
     // halved MMAs and doubled re-reads.)
     for (int NC = std::min(Oc, 512); NC >= 64; NC -= (NC > 128 ? 128 : 64)) {
-        if (Oc % NC || (NC == 64 && Oc != 64))
-            continue;
         const int nmma = NC >= 256 ? 256 : (NC >= 128 ? 128 : 64);
+        // (a group must be whole MMAs: no 384-channel groups of one N = 256 MMA)
+        if (Oc % NC || (NC == 64 && Oc != 64) || NC % nmma)
+            continue;
         const int n_subs = NC / nmma;
         const int a_min = n_subs > 1 ? (p.halo ? p.C1 : p.kb_per_tile) + 2 : (p.halo ? 2 : 4);
         const int r_min = has_res ? 4 : 2;
@@ -1293,26 +1294,14 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // slots per tile the whole tile's K blocks stay in the ring until the
     // second slot's MMAs are done.
     auto ring_min = [&](int kc) { return p.n_subs > 1 ? p.kb_per_tile / kc + 1 : 2; };
-    p.a_kc = 1;
+    int kc_first = 1;
     if (!p.halo)
         for (int kc = 4; kc > 1; kc /= 2)
             if (p.C1 % kc == 0 && p.C1b % kc == 0 && p.rows % 8 == 0 &&
                 ring_min(kc) * kc * kASlotBytes <= a_bytes_want) {
-                p.a_kc = kc;
+                kc_first = kc;
                 break;
             }
-    // Halo form: one slot per channel block, all of a tile's blocks in the ring
-    // when two accumulator slots share them; slots stay 1024-byte aligned.
-    // (the stride-2 halo form: four planes of two K halves)
-    p.a_part = p.halo == 3 ? (h3_bytes + 1023) / 1024 * 1024
-               : p.halo    ? ((p.halo == 2 ? 8 : 2) * p.a_half + 1023) / 1024 * 1024
-                           : p.a_kc * kASlotBytes;
-    p.w_part = p.wstream ? (p.halo ? 9 : p.a_kc) * p.NC * 32 : 0;
-    p.a_slot = p.a_part + p.w_part;
-    const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
-    const int a_want = std::max(a_min, p.wstream      ? 4
-                                       : p.halo == 3 ? 12  // one slot per tile: a deep ring
-                                                     : a_bytes_want / p.a_slot);
     const int r_lo = has_res ? 4 : 2, r_hi = has_res ? 12 : 4;
     auto layout = [&](int fold, int a, int r) {
         p.fold_room = fold;
@@ -1333,11 +1322,28 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.smem_bytes = p.off_misc + 16 + 1024;  // + alignment slack of the base
         return p.smem_bytes <= kSmemLimit;
     };
+    // Largest box first; fewer K blocks per box when its ring does not fit
+    // beside the weights and the I/O ring.
     bool placed = false;
-    for (int fold = 1; fold >= 0 && !placed; --fold)
-        for (int a = a_want; a >= a_min && !placed; --a)
-            for (int r = r_hi; r >= r_lo && !placed; --r)
-                placed = layout(fold, a, r);
+    for (int kc = kc_first; kc >= 1 && !placed; kc /= 2) {
+        p.a_kc = kc;
+        // Halo form: one slot per channel block, all of a tile's blocks in the
+        // ring when two accumulator slots share them; slots stay 1024-byte
+        // aligned.  (the stride-2 halo form: four planes of two K halves)
+        p.a_part = p.halo == 3 ? (h3_bytes + 1023) / 1024 * 1024
+                   : p.halo    ? ((p.halo == 2 ? 8 : 2) * p.a_half + 1023) / 1024 * 1024
+                               : p.a_kc * kASlotBytes;
+        p.w_part = p.wstream ? (p.halo ? 9 : p.a_kc) * p.NC * 32 : 0;
+        p.a_slot = p.a_part + p.w_part;
+        const int a_min = p.halo ? (p.n_subs > 1 ? p.C1 + 1 : 2) : ring_min(p.a_kc);
+        const int a_want = std::max(a_min, p.wstream      ? 4
+                                           : p.halo == 3 ? 12  // one slot per tile: a deep ring
+                                                         : a_bytes_want / p.a_slot);
+        for (int fold = 1; fold >= 0 && !placed; --fold)
+            for (int a = a_want; a >= a_min && !placed; --a)
+                for (int r = r_hi; r >= r_lo && !placed; --r)
+                    placed = layout(fold, a, r);
+    }
     if (!placed)
         return X1CB_ERR_SHAPE;
     p.io_wide = p.tw * 4 <= 256 && !p.pool ? 1 : 0;  // TMA boxes span at most 256 elements
