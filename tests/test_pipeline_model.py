@@ -280,3 +280,97 @@ def test_model_catches_more_issuing_lanes_than_slots(S):
             failures += 1
     assert failures == 20
 
+
+
+# ---- two MMA warps on one activation ring -------------------------------------------
+# Without a shortcut, the convolution kernel's warp 2 issues MMAs too: warp 1
+# takes the CTA's even tiles, warp 2 the odd ones, each box by box.  With both
+# consuming one ring, a warp can wait on a slot whose previous box (the other
+# warp's) has not landed, and its parity wait passes on the box before.  Each
+# warp therefore owns half of the ring (even tiles' boxes in slots 0..S/2-1,
+# odd tiles' in S/2..S-1), taken in order; the producer still issues boxes in
+# tile order, in rounds.
+
+def ring_pos(n, S, bpt, split):
+    if not split:
+        return n % S, n // S
+    half = S // 2
+    t, b = divmod(n, bpt)
+    li = (t // 2) * bpt + b
+    return (t % 2) * half + li % half, li // half
+
+
+def run_two_mma_warps(seed, S, lanes, bpt, split, tiles=16):
+    rng = random.Random(seed)
+    a_full = [Barrier(1) for _ in range(S)]
+    a_empty = [Barrier(1) for _ in range(S)]
+    events = []
+    last_commit = [0, 0]
+    boxes = tiles * bpt
+
+    def later(bar, who=None):
+        d = rng.randint(1, 8)
+        if who is not None:  # a warp's commits land in its issue order
+            d = max(d, last_commit[who])
+            last_commit[who] = d
+        events.append([d, bar])
+
+    def producer():
+        for base in range(0, boxes, lanes):
+            mine = list(range(base, min(base + lanes, boxes)))
+            pos = [ring_pos(n, S, bpt, split) for n in mine]
+            while not all(a_empty[s].try_wait(k - 1 if k else -1) for s, k in pos):
+                yield
+            for s, _ in pos:
+                later(a_full[s])
+            yield
+
+    def mma(w):
+        for t in range(w, tiles, 2):
+            for b in range(bpt):
+                s, k = ring_pos(t * bpt + b, S, bpt, split)
+                while not a_full[s].try_wait(k):
+                    yield
+                later(a_empty[s], who=w)
+                yield
+
+    live = [producer(), mma(0), mma(1)]
+    steps = 0
+    while live or events:
+        steps += 1
+        assert steps < 100000, "schedule did not finish"
+        for e in events:
+            e[0] -= 1
+        last_commit[0] = max(0, last_commit[0] - 1)
+        last_commit[1] = max(0, last_commit[1] - 1)
+        for e in [e for e in events if e[0] <= 0]:
+            events.remove(e)
+            e[1].arrive()
+        if live:
+            ag = rng.choice(live)
+            try:
+                next(ag)
+            except StopIteration:
+                live.remove(ag)
+
+
+# (S, lanes, bpt): conv1 and the 3x3 (6, 3, 4), the folded stem (12, 4, 1),
+# small even rings
+SPLIT_CASES = [(6, 3, 4), (12, 4, 1), (4, 2, 1), (4, 2, 3), (8, 4, 2)]
+
+
+@pytest.mark.parametrize("S,lanes,bpt", SPLIT_CASES, ids=[str(c) for c in SPLIT_CASES])
+def test_two_mma_warps_on_split_ring_are_exact(S, lanes, bpt):
+    for seed in range(40):
+        run_two_mma_warps(seed, S, lanes, bpt, split=True)
+
+
+def test_model_catches_two_mma_warps_sharing_the_ring():
+    """The shared ring: a warp's wait passes on the other warp's older box."""
+    failures = 0
+    for seed in range(40):
+        try:
+            run_two_mma_warps(seed, 6, 3, 4, split=False)
+        except (Early, AssertionError):
+            failures += 1
+    assert failures > 0

@@ -109,6 +109,28 @@ __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, 
     b0 = ig * p.tg;
 }
 
+// Ring position of activation box n (boxes counted over the CTA's tiles, bpt
+// per tile).  One MMA warp: slot n % a_stages.  Two: the even tiles' boxes
+// take the first half of the ring and the odd tiles' the second, each half in
+// order, so each half has one consumer that takes its boxes in order (a
+// parity wait on a slot is exact only then).
+__device__ __forceinline__ void a_ring_pos(const ConvPlan &p, bool split, int n, int bpt,
+                                           int &stage, uint32_t &phase)
+{
+    if (split) {
+        const int half = p.a_stages / 2;
+        const int t = n / bpt, b = n - t * bpt;
+        const int li = (t >> 1) * bpt + b;  // the box's place in its half
+        const int q = li / half;
+        stage = (t & 1) * half + (li - q * half);
+        phase = static_cast<uint32_t>(q & 1);
+    } else {
+        const int q = n / p.a_stages;
+        stage = n - q * p.a_stages;
+        phase = static_cast<uint32_t>(q & 1);
+    }
+}
+
 // Epilogue of one warp.  For every tile of this CTA and every accumulator
 // slot it reads its 32 TMEM lanes (= 32 pixels of the tile), two adjacent
 // 32-channel chunks per I/O stage, requantises them (with the shortcut bytes
@@ -346,7 +368,9 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     }
 }
 
-template <bool kRes>
+// kSplit: two MMA warps (warp 2 issues MMAs; no shortcut), a separate
+// instantiation so that the one-issuer kernels keep their code as it was.
+template <bool kRes, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_bn_act_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmW,
@@ -394,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         *io_ticket = 0;
         mbar_init(bars.w_full(), 1);
-        mbar_init(bars.mma_done(), 1);
+        mbar_init(bars.mma_done(), kSplit ? 2 : 1);  // each MMA warp's final commit
         mbar_init(bars.never(), 1);
         for (int s = 0; s < p.a_stages; ++s) {
             mbar_init(bars.a_full(s), 1);
@@ -545,11 +569,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             // This lane's box n = base + lane as ring stage/phase and as (tile i,
             // box b of the tile), advanced by counters (n_iss <= a_stages / 2:
             // at most one wrap of the ring per round).
-            int stage = lane < n_iss ? lane : 0, i = lane / bpt, b = lane % bpt;
-            uint32_t phase = 0;
+            // This lane's box n = base + lane: tile i, box b of the tile, and the
+            // ring position of the next box of each half (one half: the whole
+            // ring), all advanced by counters over the n_iss boxes of a round
+            // (see a_ring_pos; no divisions on the issue path).
+            constexpr bool split = kSplit;
+            const int half = split ? p.a_stages / 2 : p.a_stages;
+            int i = 0, b = 0, pos0 = 0, pos1 = 0;
+            uint32_t ph0 = 0u, ph1 = 0u;
+            if (!split) {
+                pos0 = lane < n_iss ? lane : 0;
+                i = lane / bpt;
+                b = lane % bpt;
+            } else {
+                for (int k = 0; k < lane && k < n_iss; ++k) {  // past box (i, b)
+                    if (i & 1) {
+                        if (++pos1 == half) {
+                            pos1 = 0;
+                            ph1 ^= 1u;
+                        }
+                    } else if (++pos0 == half) {
+                        pos0 = 0;
+                        ph0 ^= 1u;
+                    }
+                    if (++b == bpt) {
+                        b = 0;
+                        ++i;
+                    }
+                }
+            }
             for (long long base = 0; base < total; base += n_iss) {
                 const long long n = base + lane;
                 const bool have = lane < n_iss && n < total;
+                const bool odd = split && (i & 1);
+                const int stage = odd ? half + pos1 : pos0;
+                const uint32_t phase = odd ? ph1 : ph0;
                 if (!mbar_wait_lanes(kAIssuerMask, have, bars.a_empty(stage), phase ^ 1u, ctl,
                                      kDevTimeoutProducer))
                     break;
@@ -615,30 +669,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 issued = base + n_iss < total ? base + n_iss : total;
-                stage += n_iss;
-                if (stage >= p.a_stages) {
-                    stage -= p.a_stages;
-                    phase ^= 1u;
+                if (!split) {  // (n_iss <= a_stages / 2: at most one wrap)
+                    pos0 += n_iss;
+                    if (pos0 >= half) {
+                        pos0 -= half;
+                        ph0 ^= 1u;
+                    }
+                    for (b += n_iss; b >= bpt; b -= bpt)
+                        ++i;
+                } else {
+                    for (int k = 0; k < n_iss; ++k) {  // past box (i, b)
+                        if (i & 1) {
+                            if (++pos1 == half) {
+                                pos1 = 0;
+                                ph1 ^= 1u;
+                            }
+                        } else if (++pos0 == half) {
+                            pos0 = 0;
+                            ph0 ^= 1u;
+                        }
+                        if (++b == bpt) {
+                            b = 0;
+                            ++i;
+                        }
+                    }
                 }
-                for (b += n_iss; b >= bpt; b -= bpt)
-                    ++i;
             }
             // Let every copy still in flight land before shared memory goes away.
             __syncwarp(kAIssuerMask);
             if (lane == 0) {
                 if (!mbar_drain(bars.w_full(), 0, drain_ns))
                     atomicOr(&g_dev_status, kDevDrainFailed);
-                const long long last = issued < p.a_stages ? issued : p.a_stages;
-                for (long long i = issued - last; i < issued; ++i) {
-                    const int s = static_cast<int>(i % p.a_stages);
-                    const uint32_t ph = static_cast<uint32_t>((i / p.a_stages) & 1);
+                // The latest box of every slot: the last a_stages boxes of one
+                // ring; for a split ring, walking back until every slot was seen
+                // (the walk and its divisions run once, on the way out).
+                const unsigned long long all_slots = (1ull << p.a_stages) - 1;
+                unsigned long long seen = 0;
+                const int n_issued = static_cast<int>(issued);
+                const int stop = split ? 0 : (n_issued > p.a_stages ? n_issued - p.a_stages : 0);
+                for (int i = n_issued - 1; i >= stop && seen != all_slots; --i) {
+                    int s;
+                    uint32_t ph;
+                    a_ring_pos(p, split, i, bpt, s, ph);
+                    if (seen >> s & 1ull)
+                        continue;
+                    seen |= 1ull << s;
                     if (!mbar_drain(bars.a_full(s), ph, drain_ns))
                         atomicOr(&g_dev_status, kDevDrainFailed);
                 }
             }
         }
         __syncwarp();
-    } else if (warp == 2) {
+    } else if (warp == 2 && !kSplit) {
         // ---- producer of I/O stages: shortcut tiles, issued as early as the ring
         // allows; without a shortcut it only hands out free stages ----------------
         if (lane == 0) {
@@ -694,12 +776,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 3) {
         // ---- TMA store of finished I/O stages ----------------------------------------
         // Each stage goes back to the producer as soon as its store has read it
-        // (the global writes complete in the background).
+        // (the global writes complete in the background).  With warp 2 issuing
+        // MMAs (no shortcut), this warp also hands the stages out: a stage's
+        // next use may start (io_full) once its store has read it, and every
+        // stage's first use at once.
+        constexpr bool hand_out = kSplit;
         if (lane == 0) {
             const uint32_t sio = sbase + p.off_r;
             const uint64_t pol = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
+            if (hand_out)
+                for (int s = 0; s < p.r_stages; ++s)
+                    mbar_arrive(bars.io_full(s));
             [[maybe_unused]] long long n_st = 0;  // stages stored (trace index)
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
@@ -727,6 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     X1CB_TRACE_AT(p.trace, 8, n_st);
                     ++n_st;
                     mbar_arrive(bars.io_empty(stage));
+                    if (hand_out)
+                        mbar_arrive(bars.io_full(stage));
                     if (++stage == p.r_stages) {
                         stage = 0;
                         phase ^= 1u;
@@ -737,10 +828,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_wait_all();
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---- MMA issuer -----------------------------------------------------------
+    } else if (warp == 1 || (kSplit && warp == 2)) {
+        // ---- MMA issuers (warp 2 only when it has no shortcut to load) -------------
         // The whole warp runs the loop (waits are warp votes, so it stays
-        // converged) and one elected lane issues each MMA and commit.
+        // converged) and one elected lane issues each MMA and commit.  With two
+        // issuing warps, warp 1 takes the CTA's even tiles and warp 2 the odd
+        // ones, each stepping its ring and slot counters over the other's tiles.
+        const int mw = warp == 1 ? 0 : 1;
         {
             // The issue loop is kept free of divisions and descriptor rebuilds:
             // the dependent integer work between two MMAs would otherwise cost
@@ -788,19 +882,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t b_tap_step =
                 p.wstream ? b_kb_step : static_cast<uint64_t>(p.C1) * b_kb_step;
             const int n_slots = p.n_slots;
-            int a_stage = 0;
+            // This warp's part of the activation ring: all of it, or with two MMA
+            // warps its half (see a_ring_pos), taken in order.
+            const int ring_len = kSplit ? p.a_stages / 2 : p.a_stages;
+            const int ring_begin = mw * ring_len, ring_end = ring_begin + ring_len;
+            const uint64_t ring_desc0 = a_desc0 + static_cast<uint64_t>(ring_begin) * a_slot_step;
+            int a_stage = ring_begin;
             uint32_t a_phase = 0;
-            uint64_t a_slot_desc = a_desc0;
+            uint64_t a_slot_desc = ring_desc0;
             int acc = 0;
             uint32_t acc_phase = 0;
             [[maybe_unused]] long long n_box = 0, n_sub = 0;  // trace indices
             bool ok = __all_sync(0xffffffffu, mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma));
-            if (ok && p.inject == 1) {
+            if (ok && p.inject == 1 && mw == 0) {
                 const WaitCtl planted{abort_flag, &g_dev_status, p.wait_limit_ns};
                 ok = __all_sync(0xffffffffu,  // test hook
                                 mbar_wait(bars.never(), 0, planted, kDevTimeoutMma));
             }
-            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
+            int tile = 0;  // the CTA's tile count
+            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step, ++tile) {
+                if (kSplit && (tile & 1) != mw) {
+                    // the other issuer's tile (its boxes are in the other half of
+                    // the ring): its accumulator slots
+                    for (acc += p.n_subs; acc >= n_slots; acc -= n_slots)
+                        acc_phase ^= 1u;
+                    n_box += boxes;
+                    n_sub += p.n_subs;
+                    continue;
+                }
                 int st = a_stage;
                 uint32_t ph = a_phase;
                 uint64_t sd = a_slot_desc;
@@ -867,10 +976,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         accumulate = 1u;
                         if (last_sub)
                             mma_commit(bars.a_empty(st));  // slot free once these MMAs finish
-                        if (++st == p.a_stages) {
-                            st = 0;
+                        if (++st == ring_end) {
+                            st = ring_begin;
                             ph ^= 1u;
-                            sd = a_desc0;
+                            sd = ring_desc0;
                         } else {
                             sd += a_slot_step;
                         }
@@ -1346,6 +1455,16 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     }
     if (!placed)
         return X1CB_ERR_SHAPE;
+    // Two MMA warps (see the plan field) on an even ring of at least 4 slots:
+    // each takes half of it.
+    // (Measured: the folded stem, whose one box per tile feeds R MMAs, ran 17 %
+    // faster with a second issuer; the 3x3 halo form, bound by its six-slot
+    // activation ring behind 144 KB of weights, gained nothing, and a 1x1 with
+    // 4 K blocks per box lost 35 % to the half ring's exposed load latency.)
+    p.n_mma_warps = (p.halo == 3 && !has_res && !p.wstream && p.nmma <= 128 && p.n_subs == 1 &&
+                     p.n_slots % 2 == 0 && p.a_stages % 2 == 0 && p.a_stages >= 4)
+                        ? 2
+                        : 1;
     p.io_wide = p.tw * 4 <= 256 && !p.pool ? 1 : 0;  // TMA boxes span at most 256 elements
     // The swizzled stages need whole 4-pixel groups and 1024-byte aligned stages.
     p.io_swz = (p.tw % 4 == 0 && p.Wp % 4 == 0 && p.off_r % 1024 == 0 && !p.pool) ? 1 : 0;
@@ -1512,8 +1631,11 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
             tmR = tmO;  // unused
         }
     }
-    auto kern = p.has_res ? conv_bn_act_kernel<true> : conv_bn_act_kernel<false>;
-    if (int e = opt_in_smem(reinterpret_cast<const void *>(kern), p.has_res))
+    auto kern = p.has_res ? conv_bn_act_kernel<true, false>
+                : p.n_mma_warps > 1 ? conv_bn_act_kernel<false, true>
+                                    : conv_bn_act_kernel<false, false>;
+    if (int e = opt_in_smem(reinterpret_cast<const void *>(kern),
+                            p.has_res ? 1 : (p.n_mma_warps > 1 ? 3 : 0)))
         return e;
     ConvPlan q = p;
     q.trace = trace_table();

@@ -53,6 +53,14 @@ struct ConvPlan {
     int O2;        // output channels per weight block: 128, or Oc for a 64-channel layer
     int stage_ch;  // 32-channel chunks per I/O stage: 4, or 2 for a 64-channel layer
     int n_slots;   // accumulator slots in TMEM (512 columns / nmma)
+    // MMA issuing warps, 1 or 2.  One thread issues a tcgen05.mma only every
+    // ~90 cycles, while an N <= 128 MMA takes 64 tensor cycles or less; a
+    // layer without a shortcut has no shortcut loads for warp 2, so warp 2
+    // can be a second MMA issuer (warp 1 takes the CTA's even tiles, warp 2
+    // the odd ones; each owns half of the activation ring and the accumulator
+    // slots of its tiles, n_slots even) while the store warp hands the I/O
+    // stages back out.  Used where it measured faster: the folded stem.
+    int n_mma_warps;
     int kb_per_tile;  // R*R*C1
     int a_kc;         // K blocks per activation TMA box (divides C1)
     int a_slot;       // bytes per ring stage: activation part + streamed weights
