@@ -94,12 +94,35 @@ struct Bars {
     static int count(int a, int r) { return 3 + 2 * a + 3 * r + 16 + 4; }
 };
 
+// A layer with a shortcut is always a plain stride-1 1x1 (the planner and the
+// API admit no other): its instantiation reads these plan fields as
+// constants, so it carries none of the halo, pooling, narrow-stage or
+// second-source code (which cost the shortcut layers up to 4 % when it was
+// compiled into them).
+template <bool kRes> __device__ __forceinline__ int plan_halo(const ConvPlan &p)
+{
+    return kRes ? 0 : p.halo;
+}
+template <bool kRes> __device__ __forceinline__ bool plan_pool(const ConvPlan &p)
+{
+    return !kRes && p.pool;
+}
+template <bool kRes> __device__ __forceinline__ int plan_stage_ch(const ConvPlan &p)
+{
+    return kRes ? kRChunks : p.stage_ch;
+}
+template <bool kRes> __device__ __forceinline__ int plan_c1b(const ConvPlan &p)
+{
+    return kRes ? 0 : p.C1b;
+}
+
+template <bool kRes>
 __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, int &h0, int &b0)
 {
     const int iw = mt % p.nTw;
     const int ih = (mt / p.nTw) % p.nTh;
     const int ig = mt / (p.nTw * p.nTh);
-    if (p.pool) {  // conv origin of pooled tile (iw, ih): one pixel before 2 * pooled origin
+    if (plan_pool<kRes>(p)) {  // conv origin of pooled tile (iw, ih): one pixel before 2 * pooled origin
         w0 = 2 * iw * p.pw - 1;
         h0 = 2 * ih * p.ph - 1;
     } else {
@@ -182,13 +205,13 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
     // This row's 32 bytes inside chunk 0 of an I/O stage ([tg][4][th][tw][32]);
     // rows outside the box read row 0's bytes and write nothing.
-    const int row_off = in_box ? ((gi * p.stage_ch) * plane_t + yi * p.tw + xi) * 32 : 0;
+    const int row_off = in_box ? ((gi * plan_stage_ch<kRes>(p)) * plane_t + yi * p.tw + xi) * 32 : 0;
     const int chunk_stride = plane_t * 32;
     // (o >> 3) & 0x70 is bits 7-9 of o moved to bits 4-6: the 128-byte swizzle.
     const int swz_mask = p.io_swz ? 0x70 : 0;
     const int n_slots = p.n_slots;
     const int chunks_per_sub = p.nmma / 32;
-    const int stages_per_sub = chunks_per_sub / p.stage_ch;
+    const int stages_per_sub = chunks_per_sub / plan_stage_ch<kRes>(p);
     const long long my_tiles =
         cx.mt_first < p.num_m_tiles ? (p.num_m_tiles - cx.mt_first + cx.mt_step - 1) / cx.mt_step
                                     : 0;
@@ -257,16 +280,16 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
         uint8_t *stage = cx.io + st * kRSlotBytes;
         bool conv_px = true;  // pool mode: this row is a pixel of the conv output
-        if (p.pool) {
+        if (plan_pool<kRes>(p)) {
             const int mt = cx.mt_first + static_cast<int>(n / (p.n_subs * stages_per_sub)) *
                                              cx.mt_step;
             int w0, h0, b0;
-            tile_origin(p, mt, w0, h0, b0);
+            tile_origin<kRes>(p, mt, w0, h0, b0);
             conv_px = w0 + xi >= 0 && w0 + xi < p.W && h0 + yi >= 0 && h0 + yi < p.H;
         }
 #pragma unroll 1
-        for (int c = 0; c < p.stage_ch; ++c) {
-            const int cs = rl * p.stage_ch + c;        // chunk within the TMEM slot
+        for (int c = 0; c < plan_stage_ch<kRes>(p); ++c) {
+            const int cs = rl * plan_stage_ch<kRes>(p) + c;        // chunk within the TMEM slot
             const int gch = j * chunks_per_sub + cs;   // chunk within the CTA's channels
             uint32_t v[32];
             __syncwarp();
@@ -294,13 +317,13 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
                 requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
             }
             if (in_box) {
-                if (p.pool && !conv_px)  // outside the conv output: never the maximum
+                if (plan_pool<kRes>(p) && !conv_px)  // outside the conv output: never the maximum
                     ow[0] = ow[1] = ow[2] = ow[3] = ow[4] = ow[5] = ow[6] = ow[7] = 0u;
                 *pa = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 *pb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
             }
         }
-        if (p.pool) {
+        if (plan_pool<kRes>(p)) {
             // Every conv pixel of the tile is in the stage once the turn's four
             // warps are here; then each thread pools 16-byte pieces (16 channels)
             // of pooled pixels into the upper half of the stage.
@@ -319,7 +342,7 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             const int tid = q * 32 + lane;
             const int np = p.pw * p.ph;
             uint8_t *pooled = stage + kRSlotBytes / 2;
-            for (int k = tid; k < np * p.stage_ch * 2; k += 128) {
+            for (int k = tid; k < np * plan_stage_ch<kRes>(p) * 2; k += 128) {
                 const int half = k & 1;
                 const int c = (k >> 1) / np;
                 const int pix = (k >> 1) % np;
@@ -404,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int group = blockIdx.x % p.n_groups;
     const int mt_first = blockIdx.x / p.n_groups;
     const int mt_step = gridDim.x / p.n_groups;
-    const int stages_per_tile = p.NC / (32 * p.stage_ch);
+    const int stages_per_tile = p.NC / (32 * plan_stage_ch<kRes>(p));
 
     // ---- set-up ---------------------------------------------------------------
     // Trace events (trace builds): 0 producer box n may load; 1 MMA sees box n;
@@ -434,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 8; ++s) {
             mbar_init(bars.acc_full(s), 1);
             // every stage of the slot, each from one warp per lane quarter
-            mbar_init(bars.acc_empty(s), 4 * (p.nmma / (32 * p.stage_ch)));
+            mbar_init(bars.acc_empty(s), 4 * (p.nmma / (32 * plan_stage_ch<kRes>(p))));
         }
         fence_mbar_init();
     }
@@ -444,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmO);
         if (kRes)
             tma_prefetch_desc(&tmR);
-        if (p.C1b) {
+        if (plan_c1b<kRes>(p)) {
             tma_prefetch_desc(&tmA2);
             tma_prefetch_desc(&tmW2);
         }
@@ -543,7 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-        if (lane < kAIssuers) {
+        const unsigned iss_mask = (1u << n_iss) - 1;  // the issuing lanes
+        if (lane < n_iss) {
             const int o1 = group * (p.NC / p.O2);
             // Streamed weights: bytes per stage, each K block NC rows x 32 bytes.
             const uint32_t wpart = static_cast<uint32_t>(p.w_part);
@@ -551,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // One box = a_kc consecutive K blocks (channel blocks c1..c1+a_kc-1 of
             // one filter tap), each a 128-row x 32-byte tile, back to back.
             const uint32_t abytes =
-                p.halo == 3 ? static_cast<uint32_t>((2 * p.th + p.R - 2) * p.tw * 32)
-                : p.halo    ? static_cast<uint32_t>((p.halo == 2 ? 8 : 2) * 16 * p.plane_m * p.tg)
+                plan_halo<kRes>(p) == 3 ? static_cast<uint32_t>((2 * p.th + p.R - 2) * p.tw * 32)
+                : plan_halo<kRes>(p)    ? static_cast<uint32_t>((plan_halo<kRes>(p) == 2 ? 8 : 2) * 16 * p.plane_m * p.tg)
                             : static_cast<uint32_t>(p.a_kc * p.rows * 32);  // K halves / blocks
             const uint32_t sa = sbase + p.off_a;
             const uint64_t pol = policy_evict_first();
@@ -560,8 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // channel block fastest, then filter column, then filter row, then
             // (if present) the second source's channel blocks.
             const int cb = p.C1 / p.a_kc;
-            const int first_boxes = p.halo ? p.C1 : p.R * p.Rw * cb;
-            const int bpt = p.halo ? p.C1 : p.kb_per_tile / p.a_kc;
+            const int first_boxes = plan_halo<kRes>(p) ? p.C1 : p.R * p.Rw * cb;
+            const int bpt = plan_halo<kRes>(p) ? p.C1 : p.kb_per_tile / p.a_kc;
             const long long my_tiles =
                 mt_first < p.num_m_tiles ? (p.num_m_tiles - mt_first + mt_step - 1) / mt_step : 0;
             const long long total = my_tiles * bpt;
@@ -604,17 +628,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool odd = split && (i & 1);
                 const int stage = odd ? half + pos1 : pos0;
                 const uint32_t phase = odd ? ph1 : ph0;
-                if (!mbar_wait_lanes(kAIssuerMask, have, bars.a_empty(stage), phase ^ 1u, ctl,
+                if (!mbar_wait_lanes(iss_mask, have, bars.a_empty(stage), phase ^ 1u, ctl,
                                      kDevTimeoutProducer))
                     break;
                 if (have) {
                     X1CB_TRACE_AT(p.trace, 0, n);
                     const int mt = mt_first + i * mt_step;
                     int w0, h0, b0;
-                    tile_origin(p, mt, w0, h0, b0);
+                    tile_origin<kRes>(p, mt, w0, h0, b0);
                     const uint32_t slot = sa + static_cast<uint32_t>(stage) * p.a_slot;
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
-                    if (p.halo == 2) {
+                    if (plan_halo<kRes>(p) == 2) {
                         // one slot per channel block c1 = b: plane (pr, pc) from
                         // input (pc - 1, 2*h0 - 1 + pr), step 2
                         for (int pl = 0; pl < 4; ++pl)
@@ -623,12 +647,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     slot + static_cast<uint32_t>((2 * pl + hf) * p.a_half), &tmA,
                                     bars.a_full(stage), 16 * hf, (pl & 1) - 1,
                                     2 * h0 - 1 + (pl >> 1), b, b0, pol);
-                    } else if (p.halo == 3) {
+                    } else if (plan_halo<kRes>(p) == 3) {
                         // the tile's columns, input rows from 2*h0 - pad on (output
                         // row y, tap dr reads input row 2y - pad + dr)
                         tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0, 2 * h0 - p.pad,
                                          b0, 0, pol);
-                    } else if (p.halo) {
+                    } else if (plan_halo<kRes>(p)) {
                         // the tile's pixels plus a one-pixel frame (zeros outside the
                         // image), each K half as one box
                         tma_load_5d_hint(slot, &tmA, bars.a_full(stage), 0, w0 - p.pad,
@@ -651,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (wpart) {  // the box's K blocks' weights
                         const uint32_t wdst = slot + static_cast<uint32_t>(p.a_part);
-                        if (p.halo) {  // the nine taps of channel block b
+                        if (plan_halo<kRes>(p)) {  // the nine taps of channel block b
                             for (int t = 0; t < 9; ++t)
                                 tma_load_4d(wdst + t * wkb, &tmW, bars.a_full(stage), 0, 0,
                                             t * p.C1 + b, o1);
@@ -696,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // Let every copy still in flight land before shared memory goes away.
-            __syncwarp(kAIssuerMask);
+            __syncwarp(iss_mask);
             if (lane == 0) {
                 if (!mbar_drain(bars.w_full(), 0, drain_ns))
                     atomicOr(&g_dev_status, kDevDrainFailed);
@@ -724,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- producer of I/O stages: shortcut tiles, issued as early as the ring
         // allows; without a shortcut it only hands out free stages ----------------
         if (lane == 0) {
-            const uint32_t rbytes = static_cast<uint32_t>(p.stage_ch * p.rows * 32);
+            const uint32_t rbytes = static_cast<uint32_t>(plan_stage_ch<kRes>(p) * p.rows * 32);
             const uint32_t sio = sbase + p.off_r;
             const uint64_t pol = policy_evict_first();
             int stage = 0;
@@ -734,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
-                tile_origin(p, mt, w0, h0, b0);
+                tile_origin<kRes>(p, mt, w0, h0, b0);
                 for (int rs = 0; rs < stages_per_tile; ++rs) {
                     if (!mbar_wait(bars.io_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer)) {
                         ok = false;
@@ -744,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++n_io;
                     if (kRes) {
                         mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
-                        const int o1 = group * (p.NC / 32) + rs * p.stage_ch;
+                        const int o1 = group * (p.NC / 32) + rs * plan_stage_ch<kRes>(p);
                         if (p.io_swz)
                             tma_load_5d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
                                              0, w0 / 4, h0, o1, b0, pol);
@@ -793,15 +817,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
                 int w0, h0, b0;
-                tile_origin(p, mt, w0, h0, b0);
+                tile_origin<kRes>(p, mt, w0, h0, b0);
                 for (int rs = 0; rs < stages_per_tile; ++rs) {
                     if (!mbar_wait(bars.out_ready(stage), phase, ctl, kDevTimeoutProducer)) {
                         ok = false;
                         break;
                     }
                     X1CB_TRACE_AT(p.trace, 7, n_st);
-                    const int o1 = group * (p.NC / 32) + rs * p.stage_ch;
-                    if (p.pool)  // pooled tile at pooled coordinates ((w0 + 1) / 2, ...)
+                    const int o1 = group * (p.NC / 32) + rs * plan_stage_ch<kRes>(p);
+                    if (plan_pool<kRes>(p))  // pooled tile at pooled coordinates ((w0 + 1) / 2, ...)
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes + kRSlotBytes / 2, 0,
                                           (w0 + 1) / 2, (h0 + 1) / 2, o1, b0, pol);
                     else if (p.io_swz)
@@ -846,8 +870,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (folded stem: output row y reads input row 2y + dr, two input rows
             // of tw 32-byte pixels per GEMM row group)
             const uint64_t a_desc0 =
-                p.halo == 3 ? smem_desc_sw32(sbase + p.off_a, static_cast<uint32_t>(2 * p.tw * 32))
-                : p.halo    ? smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half))
+                plan_halo<kRes>(p) == 3 ? smem_desc_sw32(sbase + p.off_a, static_cast<uint32_t>(2 * p.tw * 32))
+                : plan_halo<kRes>(p)    ? smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half))
                             : smem_desc_sw32(sbase + p.off_a);
             const uint32_t h3_row_step = static_cast<uint32_t>(p.tw * 32) >> 4;  // next tap
             const uint64_t b_desc0 = smem_desc_sw32(sbase + p.off_w);
@@ -862,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
             const uint32_t b_kb_step = static_cast<uint32_t>(p.NC * 32) >> 4;     // next K block of weights
             const uint32_t b_sub_step = static_cast<uint32_t>(p.nmma * 32) >> 4;  // next N slice
-            const int boxes = p.halo ? p.C1 : p.kb_per_tile / p.a_kc;
+            const int boxes = plan_halo<kRes>(p) ? p.C1 : p.kb_per_tile / p.a_kc;
             const int kc = p.a_kc;
             // Halo form: tap (dr, ds) reads the slot dr*row_pitch + ds rows on and
             // the weights of K block (dr*3 + ds)*C1 + c1.
@@ -873,7 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int t = 0; t < 9; ++t) {
                 const uint32_t dr = t / 3, ds = t % 3;
-                tap_off[t] = p.halo == 2
+                tap_off[t] = plan_halo<kRes>(p) == 2
                                  ? ((dr & 1) * 2 + (ds & 1)) * (2 * p.a_half >> 4) +
                                        (dr >> 1) * hp + (ds >> 1)
                                  : dr * hp + ds;
@@ -945,14 +969,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint64_t ad = sd;
                         if (p.wstream)  // this stage's own weights (one N slice: j == 0)
                             bd = w_desc0 + (sd - a_desc0);
-                        if (p.halo == 3) {
+                        if (plan_halo<kRes>(p) == 3) {
                             // filter row dr: the slot dr input rows on, weight K block dr
                             for (int dr = 0; dr < p.R; ++dr)
                                 mma_i8(d_tmem, ad + static_cast<uint64_t>(dr) * h3_row_step,
                                        bd + static_cast<uint64_t>(dr) * b_kb_step, idesc,
                                        dr == 0 ? accumulate : 1u);
                             bd += static_cast<uint64_t>(p.R) * b_kb_step;
-                        } else if (p.halo) {
+                        } else if (plan_halo<kRes>(p)) {
 #pragma unroll
                             for (int t = 0; t < 9; ++t)
                                 mma_i8(d_tmem, ad + tap_off[t],

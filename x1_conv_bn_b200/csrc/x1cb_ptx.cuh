@@ -120,36 +120,33 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Warp-synchronous bounded wait of the lanes in `mask`: each lane with
-// want = true waits for phase `parity` of its own barrier, and all return
-// together once every lane's phase is complete, so the lanes stay converged
-// and issue their next instructions (tensor copies) as one.  Lanes poll
-// without suspending: a suspended lane would hold up the warp's others.
-// Returns false for all lanes when the CTA was told to abort or the limit
-// passed (then one lane raises the abort flag and records `code`).
+// Warp-synchronous bounded wait of the lanes in `mask` (lanes 0..n-1 of a
+// converged warp): each lane with want = true waits for phase `parity` of its
+// own barrier, and all return together once every lane's phase is complete,
+// so the lanes stay converged and issue their next instructions (tensor
+// copies) as one.  A first non-blocking probe of all of them; then the whole
+// warp takes the lanes' barriers in turn with the sleeping wait, which wakes
+// when the phase completes and leaves the issue slots to the other warps
+// meanwhile (a warp spinning on the probe measured 10 % off the epilogue's
+// pace).  Returns false for all lanes when the CTA was told to abort or a
+// wait ran out of time (then that wait raised the abort flag and recorded
+// `code`).
 __device__ __forceinline__ bool mbar_wait_lanes(unsigned mask, bool want, uint32_t bar,
                                                 uint32_t parity, const WaitCtl &ctl,
                                                 unsigned int code)
 {
-    bool ready = !want || mbar_test_wait(bar, parity);
+    const bool ready = !want || mbar_test_wait(bar, parity);
     if (__all_sync(mask, ready))
         return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        ready = ready || mbar_test_wait(bar, parity);
-        if (__all_sync(mask, ready))
-            return true;
-        if ((it & 63u) == 0) {
-            const bool stop = *ctl.abort_flag || globaltimer_ns() - t0 > ctl.limit_ns;
-            if (__any_sync(mask, stop)) {
-                if (stop && !*ctl.abort_flag) {
-                    *ctl.abort_flag = 1;
-                    atomicOr(ctl.status, code);
-                }
-                return false;
-            }
-        }
+    const int n = 32 - __clz(mask);
+    for (int l = 0; l < n; ++l) {
+        const uint32_t b = __shfl_sync(mask, bar, l);
+        const uint32_t ph = __shfl_sync(mask, parity, l);
+        const bool w = __shfl_sync(mask, (want && !ready) ? 1 : 0, l) != 0;
+        if (w && !__all_sync(mask, mbar_wait(b, ph, ctl, code)))
+            return false;
     }
+    return true;
 }
 
 // Bounded wait until a monotonic shared-memory counter reaches at least
