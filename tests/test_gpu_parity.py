@@ -121,6 +121,24 @@ def test_conv1x1_channel_groups(oracle, shape):
     assert torch.equal(got, ref), _first_mismatch(got, ref)
 
 
+# Shortcut layers whose resident weights take more than 96 KB stage the
+# shortcut and result in 8 KB pieces (two 32-channel chunks): N = 256 groups
+# with 4-K-block boxes and a batch tail, and N = 128 groups (four accumulator
+# slots) with one K block per box on 125-row tiles.
+NARROW_IO = [(43, 7, 7, 512, 2048), (9, 7, 7, 1024, 256)]
+
+
+@pytest.mark.parametrize("shape", NARROW_IO, ids=[str(s) for s in NARROW_IO])
+def test_conv1x1_narrow_io_stages(oracle, shape):
+    assert "stage_ch=2" in X.x1cb_describe_plan(*shape, 1, True)
+    s = synth.ConvShape(*shape, R=1, has_res=True)
+    inp = synth.conv_inputs(s, 91 + shape[0])
+    got = _nhwc(_gpu_conv(inp))
+    ref = _oracle_conv(oracle, inp)
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
+    _assert_spread(oracle.pack_act(ref))
+
+
 @pytest.mark.parametrize("S", [12, 24, 31, 40])
 def test_conv1x1_full_int8_range(oracle, S):
     """x, w, r over [-128, 127], negative multipliers, wide bias, several shifts."""

@@ -161,6 +161,14 @@ CASES = [
     dict(stages_per_tile=1, r=3, n_slots=4, stages_per_sub=1),
     dict(stages_per_tile=1, r=2, n_slots=4, stages_per_sub=1),
     dict(stages_per_tile=2, r=12, n_slots=4, stages_per_sub=1),
+    # shallow I/O rings beside large resident weights or deeper activation rings
+    dict(stages_per_tile=4, r=6, n_slots=2, stages_per_sub=2),
+    dict(stages_per_tile=4, r=5, n_slots=2, stages_per_sub=2),
+    dict(stages_per_tile=2, r=2, n_slots=2, stages_per_sub=2),
+    dict(stages_per_tile=2, r=3, n_slots=2, stages_per_sub=2),
+    # 8 KB stages: two 32-channel chunks, four stages per N = 256 accumulator
+    dict(stages_per_tile=4, r=4, n_slots=2, stages_per_sub=4),
+    dict(stages_per_tile=4, r=3, n_slots=2, stages_per_sub=4),
 ]
 
 

@@ -645,10 +645,10 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
                   "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
-                  "wstream=%d mwarps=%d",
+                  "wstream=%d mwarps=%d stage_ch=%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo, p.io_swz, p.wstream, p.n_mma_warps);
+                  p.halo, p.io_swz, p.wstream, p.n_mma_warps, p.stage_ch);
     return X1CB_OK;
 }
 
@@ -688,10 +688,11 @@ int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int st
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
                   "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
-                  "out=%dx%d stride=%d kb2=%d wstream=%d pool=%dx%d mwarps=%d",
+                  "out=%dx%d stride=%d kb2=%d wstream=%d pool=%dx%d mwarps=%d stage_ch=%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream, p.pw, p.ph, p.n_mma_warps);
+                  p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream, p.pw, p.ph, p.n_mma_warps,
+                  p.stage_ch);
     return X1CB_OK;
 }
 

@@ -95,28 +95,36 @@ struct Bars {
 };
 
 // A layer with a shortcut is always a plain stride-1 1x1 (the planner and the
-// API admit no other): its instantiation reads these plan fields as
-// constants, so it carries none of the halo, pooling, narrow-stage or
-// second-source code (which cost the shortcut layers up to 4 % when it was
-// compiled into them).
-template <bool kRes> __device__ __forceinline__ int plan_halo(const ConvPlan &p)
+// API admit no other): its instantiations (kRes = 1: I/O stages of four
+// 32-channel chunks; kRes = 2: of two, for layers whose resident weights leave
+// little room for the rings) read these plan fields as constants, so they
+// carry none of the halo, pooling or second-source code (which cost the
+// shortcut layers up to 4 % when it was compiled into them).  kRes = 0: no
+// shortcut, every form.
+template <int kRes> __device__ __forceinline__ int plan_halo(const ConvPlan &p)
 {
     return kRes ? 0 : p.halo;
 }
-template <bool kRes> __device__ __forceinline__ bool plan_pool(const ConvPlan &p)
+template <int kRes> __device__ __forceinline__ bool plan_pool(const ConvPlan &p)
 {
     return !kRes && p.pool;
 }
-template <bool kRes> __device__ __forceinline__ int plan_stage_ch(const ConvPlan &p)
+template <int kRes> __device__ __forceinline__ int plan_stage_ch(const ConvPlan &p)
 {
-    return kRes ? kRChunks : p.stage_ch;
+    return kRes == 1 ? kRChunks : (kRes == 2 ? kRChunks / 2 : p.stage_ch);
 }
-template <bool kRes> __device__ __forceinline__ int plan_c1b(const ConvPlan &p)
+template <int kRes> __device__ __forceinline__ int plan_c1b(const ConvPlan &p)
 {
     return kRes ? 0 : p.C1b;
 }
+// Bytes between I/O ring slots: a shortcut layer's stages are packed at their
+// own size; the others keep 16 KB slots (pooled tiles use the upper half).
+template <int kRes> __device__ __forceinline__ int plan_r_slot(const ConvPlan &p)
+{
+    return kRes ? plan_stage_ch<kRes>(p) * kTileRows * 32 : kRSlotBytes;
+}
 
-template <bool kRes>
+template <int kRes>
 __device__ __forceinline__ void tile_origin(const ConvPlan &p, int mt, int &w0, int &h0, int &b0)
 {
     const int iw = mt % p.nTw;
@@ -185,7 +193,7 @@ struct EpiCtx {
 // every phase of it.  I/O slots: before awaiting a stage's arrival a turn
 // makes sure the slot's previous stage is complete (see below), so each
 // slot's phases are observed in order whatever the ring depth.
-template <bool kRes, int kMode, bool kK1 = false>
+template <int kRes, int kMode, bool kK1 = false>
 __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int lane)
 {
     constexpr int kTurns = kEpiWarps / 4;                 // warps per TMEM lane quarter
@@ -278,7 +286,7 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         if (!deep && lane == 0)
             atomicMax(const_cast<int *>(cx.io_ticket), static_cast<int>(n + 1));
         const uint32_t tbase = cx.tmem_base + lane_addr + static_cast<uint32_t>(acc * p.nmma);
-        uint8_t *stage = cx.io + st * kRSlotBytes;
+        uint8_t *stage = cx.io + st * plan_r_slot<kRes>(p);
         bool conv_px = true;  // pool mode: this row is a pixel of the conv output
         if (plan_pool<kRes>(p)) {
             const int mt = cx.mt_first + static_cast<int>(n / (p.n_subs * stages_per_sub)) *
@@ -308,13 +316,13 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             }
             uint32_t ow[8];
             if (kMode >= 2) {
-                requant_hi32<kRes, kMode == 2, kK1, 8>(
+                requant_hi32<(kRes != 0), kMode == 2, kK1, 8>(
                     v, cx.cm + gch * 32, reinterpret_cast<const int32_t *>(cx.cC) + gch * 32, rw,
                     mr2, rsel, ow);
             } else if (kMode == 1) {
-                requant_fast<kRes, 8>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2, rsel, ow);
+                requant_fast<(kRes != 0), 8>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, mr2, rsel, ow);
             } else {
-                requant32<kRes>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
+                requant32<(kRes != 0)>(v, cx.cm + gch * 32, cx.cC + gch * 32, rw, p.m_r, p.S, ow);
             }
             if (in_box) {
                 if (plan_pool<kRes>(p) && !conv_px)  // outside the conv output: never the maximum
@@ -393,7 +401,7 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
 
 // kSplit: two MMA warps (warp 2 issues MMAs; no shortcut), a separate
 // instantiation so that the one-issuer kernels keep their code as it was.
-template <bool kRes, bool kSplit>
+template <int kRes, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_bn_act_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmW,
@@ -770,13 +778,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive_expect_tx(bars.io_full(stage), rbytes);
                         const int o1 = group * (p.NC / 32) + rs * plan_stage_ch<kRes>(p);
                         if (p.io_swz)
-                            tma_load_5d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
+                            tma_load_5d_hint(sio + stage * plan_r_slot<kRes>(p), &tmR, bars.io_full(stage),
                                              0, w0 / 4, h0, o1, b0, pol);
                         else if (p.io_wide)
-                            tma_load_4d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
+                            tma_load_4d_hint(sio + stage * plan_r_slot<kRes>(p), &tmR, bars.io_full(stage),
                                              w0 * 4, h0, o1, b0, pol);
                         else
-                            tma_load_5d_hint(sio + stage * kRSlotBytes, &tmR, bars.io_full(stage),
+                            tma_load_5d_hint(sio + stage * plan_r_slot<kRes>(p), &tmR, bars.io_full(stage),
                                              0, w0, h0, o1, b0, pol);
                         ++issued;
                     } else {
@@ -829,12 +837,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes + kRSlotBytes / 2, 0,
                                           (w0 + 1) / 2, (h0 + 1) / 2, o1, b0, pol);
                     else if (p.io_swz)
-                        tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0 / 4, h0, o1, b0,
+                        tma_store_5d_hint(&tmO, sio + stage * plan_r_slot<kRes>(p), 0, w0 / 4, h0, o1, b0,
                                           pol);
                     else if (p.io_wide)
-                        tma_store_4d_hint(&tmO, sio + stage * kRSlotBytes, w0 * 4, h0, o1, b0, pol);
+                        tma_store_4d_hint(&tmO, sio + stage * plan_r_slot<kRes>(p), w0 * 4, h0, o1, b0, pol);
                     else
-                        tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes, 0, w0, h0, o1, b0, pol);
+                        tma_store_5d_hint(&tmO, sio + stage * plan_r_slot<kRes>(p), 0, w0, h0, o1, b0, pol);
                     bulk_commit();
                     bulk_wait_read<0>();
                     X1CB_TRACE_AT(p.trace, 8, n_st);
@@ -1038,11 +1046,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         group, mt_first, mt_step};
         const bool k1 = kRes && static_cast<long long>(p.m_r) == (1ll << (p.S - 1));
         if (mode == 3 && k1)
-            epilogue_warp<kRes, 3, kRes>(cx, warp, lane);
+            epilogue_warp<kRes, 3, (kRes != 0)>(cx, warp, lane);
         else if (mode == 3)
             epilogue_warp<kRes, 3>(cx, warp, lane);
         else if (mode == 2 && k1)
-            epilogue_warp<kRes, 2, kRes>(cx, warp, lane);
+            epilogue_warp<kRes, 2, (kRes != 0)>(cx, warp, lane);
         else if (mode == 2)
             epilogue_warp<kRes, 2>(cx, warp, lane);
         else if (mode == 1)
@@ -1129,15 +1137,18 @@ int opt_in_smem(const void *kern, int which)
 }
 
 
-// Choose the pixel tile: tw x th pixels of tg images, at most 128 GEMM rows.
+// Choose the pixel tile: tw x th pixels of tg images, at most 128 GEMM rows,
+// for a layer of kb K blocks per tile.
 // Cost = MMA rows issued over the whole problem, with a penalty for
 // contiguous global runs shorter than 512 bytes (up to 47 % for single
-// 32-byte pixels), and 10 % each for a row
-// count that is not a multiple of 8 (activation boxes then carry one K block
-// each instead of up to four) and for shortcut/output stages that cannot use
-// the 128-byte swizzle (tw or the row not whole 4-pixel groups: bank
-// conflicts in the epilogue); ties go to more rows, then to longer runs.
-void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg)
+// 32-byte pixels); for a row count that is not a multiple of 8 (activation
+// boxes then carry one K block each instead of up to four: 10 %, or 35 % for
+// more than 4 K blocks per tile, where the box count sets the pace -- measured
+// on the 7x7 512 -> 2048 expand conv: 88 us with 125-row tiles of 16 boxes,
+// 58 us with 120-row tiles of 4); and 10 % for shortcut/output stages that
+// cannot use the 128-byte swizzle (tw or the row not whole 4-pixel groups:
+// bank conflicts in the epilogue); ties go to more rows, then to longer runs.
+void choose_tile(int B, int Wp, int Hp, int kb, int &tw, int &th, int &tg)
 {
     double best = 1e300;
     int best_rows = 0, best_seg = 0;
@@ -1155,7 +1166,7 @@ void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg)
                 cost *= 1.0 + (512 - seg) / 1024.0;
             const int rows = w * h * g;
             if (rows % 8 != 0)
-                cost *= 1.1;
+                cost *= kb > 4 ? 1.35 : 1.1;
             if (w % 4 != 0 || Wp % 4 != 0)
                 cost *= 1.1;
             const bool tie = cost <= best * (1 + 1e-12) && cost >= best * (1 - 1e-12);
@@ -1341,7 +1352,7 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.plane_m = p.tw * p.th;
         p.a_half = 0;
     } else {
-        choose_tile(B, p.Wp, p.Hp, p.tw, p.th, p.tg);
+        choose_tile(B, p.Wp, p.Hp, R * p.Rw * p.C1 + p.C1b, p.tw, p.th, p.tg);
         p.row_pitch = p.tw;
         p.plane_m = p.tw * p.th;
         p.a_half = 0;
@@ -1409,29 +1420,41 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     p.n_slots = kTmemCols / p.nmma;
 
     const int wbytes = p.wstream ? 0 : p.kb_per_tile * p.NC * 32;
+    // A shortcut layer whose resident weights take more than 96 KB stages its
+    // shortcut and result in 8 KB pieces (two 32-channel chunks): its I/O ring
+    // then keeps four stages in flight beside an activation ring of whole
+    // 16 KB boxes.  (Measured on the 7x7 512 -> 2048 expand conv, 128 KB of
+    // weights: with 16 KB stages only two fit beside the activation boxes.)
+    if (has_res && wbytes > 96 * 1024)
+        p.stage_ch = kRChunks / 2;
+    const int r_slot = has_res ? p.stage_ch * kTileRows * 32 : kRSlotBytes;
     // The activation ring budget: with a shortcut the I/O ring (shortcut in,
     // result out) needs the space -- its depth sets the bytes in flight -- so
-    // about a tile's K blocks plus two; without one the activations are most
+    // about two tiles' K blocks plus two; without one the activations are most
     // of the traffic and get up to 128 KB in flight while the I/O stages only
     // stage results.  The bias-fold tiles are reserved when the rings still
     // reach their minimum beside them.
-    // (a deep fan-in with a shortcut -- 8 or more K blocks per tile -- also
-    // gets two tiles of K blocks, so the producer runs a tile ahead)
+    // (Measured on the 1x1 128 -> 512 with shortcut, B = 2048: 326 us with
+    // 24 KB of activation ring and seven I/O stages, 314 us with 40 KB and
+    // six, 329 us with 40 KB and five.  A deep fan-in with a shortcut -- 8 or
+    // more K blocks per tile -- gets two tiles of K blocks.)
     const int a_bytes_want =
         p.wstream ? 4 * 4 * kASlotBytes
-        : (has_res && p.kb_per_tile < 8) ? std::min(p.kb_per_tile + 2, 8) * kASlotBytes
+        : (has_res && p.kb_per_tile < 8) ? std::min(2 * p.kb_per_tile + 2, 10) * kASlotBytes
                                          : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
     // Several K blocks per activation box (fewer, larger copies) when each
     // K-block tile starts on a 256-byte swizzle atom (row count a multiple of
-    // 8) and the ring's minimum still fits the budget.  With two accumulator
-    // slots per tile the whole tile's K blocks stay in the ring until the
-    // second slot's MMAs are done.
+    // 8) and the budget holds one box more than the ring's minimum.  With two
+    // accumulator slots per tile the whole tile's K blocks stay in the ring
+    // until the second slot's MMAs are done.  (Measured on the 1x1 128 -> 512
+    // with shortcut: two 16 KB boxes, each a whole tile, 380 us against 314
+    // with five 8 KB boxes.)
     auto ring_min = [&](int kc) { return p.n_subs > 1 ? p.kb_per_tile / kc + 1 : 2; };
     int kc_first = 1;
     if (!p.halo)
         for (int kc = 4; kc > 1; kc /= 2)
             if (p.C1 % kc == 0 && p.C1b % kc == 0 && p.rows % 8 == 0 &&
-                ring_min(kc) * kc * kASlotBytes <= a_bytes_want) {
+                (ring_min(kc) + 1) * kc * kASlotBytes <= a_bytes_want) {
                 kc_first = kc;
                 break;
             }
@@ -1448,8 +1471,8 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         // The per-channel bias/offset table (modes 0-2) and the fold digit rows
         // (mode 3) are never used together, so they share space when folding
         // is possible.
-        p.off_cc = fold ? p.off_bb : p.off_r + r * kRSlotBytes;
-        p.off_cm = (fold ? p.off_r + r * kRSlotBytes : p.off_cc + p.NC * 8);
+        p.off_cc = fold ? p.off_bb : p.off_r + r * r_slot;
+        p.off_cm = (fold ? p.off_r + r * r_slot : p.off_cc + p.NC * 8);
         p.off_bar = (p.off_cm + p.NC * 4 + 7) & ~7;
         p.off_misc = p.off_bar + Bars::count(a, r) * 8;
         p.smem_bytes = p.off_misc + 16 + 1024;  // + alignment slack of the base
@@ -1655,11 +1678,13 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
             tmR = tmO;  // unused
         }
     }
-    auto kern = p.has_res ? conv_bn_act_kernel<true, false>
-                : p.n_mma_warps > 1 ? conv_bn_act_kernel<false, true>
-                                    : conv_bn_act_kernel<false, false>;
+    const bool narrow = p.has_res && p.stage_ch == kRChunks / 2;
+    auto kern = narrow                ? conv_bn_act_kernel<2, false>
+                : p.has_res           ? conv_bn_act_kernel<1, false>
+                : p.n_mma_warps > 1   ? conv_bn_act_kernel<0, true>
+                                      : conv_bn_act_kernel<0, false>;
     if (int e = opt_in_smem(reinterpret_cast<const void *>(kern),
-                            p.has_res ? 1 : (p.n_mma_warps > 1 ? 3 : 0)))
+                            narrow ? 4 : p.has_res ? 1 : (p.n_mma_warps > 1 ? 3 : 0)))
         return e;
     ConvPlan q = p;
     q.trace = trace_table();

@@ -10,7 +10,7 @@
 
 namespace x1cb {
 
-void choose_tile(int B, int Wp, int Hp, int &tw, int &th, int &tg);
+void choose_tile(int B, int Wp, int Hp, int kb, int &tw, int &th, int &tg);
 void choose_halo_tile(int B, int H, int W, int &th, int &tg);
 int encode_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
                const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swz,
