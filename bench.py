@@ -782,17 +782,19 @@ def main(argv=None):
     if stages is None:
         roof = roofline(ops, nbytes, ms_max * 1e-3, hbm, bf16, peak_kind)
         if isinstance(s, synth.StemShape):
-            roof["kernel"] = ("conv_bn_act_kernel<false, true> (folded stem: seven filter-row "
+            roof["kernel"] = ("conv_bn_act_kernel<0, true> (folded stem: seven filter-row "
                               "MMAs of K=32 over the width-folded image, two MMA-issuing "
                               "warps, + BN + ReLU + 3x3/2 max pool)")
             roof["note"] = ("ops count the image's 3 real channels; the kernel multiplies the "
                             "folded 32-channel block (21 used)")
             prof = f"stem_b{s.B}.md"
         elif s.R == 3:
-            roof["kernel"] = "conv_bn_act_kernel<false, false> (3x3, halo form)"
+            roof["kernel"] = "conv_bn_act_kernel<0, false> (3x3, halo form)"
             prof = f"conv3x3_{cfg}_b{s.B}.md"
         else:
-            roof["kernel"] = "conv_bn_act_kernel<true, false> (1x1 with shortcut)"
+            narrow = "stage_ch=2" in X.x1cb_describe_plan(s.B, s.H, s.W, s.Ic, s.Oc, 1, True)
+            roof["kernel"] = (f"conv_bn_act_kernel<{2 if narrow else 1}, false> (1x1 with shortcut, "
+                              f"{'8' if narrow else '16'} KB shortcut/result stages)")
             prof = (f"conv1x1_res32_b{s.B}.md" if cfg in ("2", "3")
                     else f"conv1x1_{cfg}_b{s.B}.md")
         roof["algorithmic_bytes_per_launch"] = nbytes
