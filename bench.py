@@ -68,8 +68,9 @@ def parse(argv=None):
     ap.add_argument("--cpu-1thread", action="store_true",
                     help="also time the oracle sample on one host thread")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-fusion", action="store_true",
-                    help="block workloads: run conv2 and conv3 as separate launches")
+    ap.add_argument("--fusion", action="store_true",
+                    help="block workloads: run conv2 and conv3 as one fused launch "
+                         "(the library's default is two launches)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--dry-run", action="store_true",
@@ -160,16 +161,17 @@ def is_block(s):
     return isinstance(s, (synth.BlockShape, synth.ProjBlockShape))
 
 
-def block_fused(s, fused=True):
+def block_fused(s, fused=False):
     """Whether the library runs this bottleneck's conv2 and conv3 as one
-    launch (its fused form: Cmid = 128, Cout up to 1024, whole-row I/O)."""
+    launch: fusion enabled and the fused form applies (Cmid = 128, Cout up
+    to 1024, whole-row I/O)."""
     return (fused and isinstance(s, synth.BlockShape) and s.Cmid == 128 and s.Cin % 128 == 0
             and s.Cin <= 1024 and s.W + 2 <= 128 and (s.W % 4 == 0 or 4 * s.W <= 256))
 
 
-def launches_per_step(cfg, fused=True):
-    """Kernel launches of one step: the Res3.2 block fuses conv2 and conv3 into
-    one launch (Cmid = 128); the projection block takes three."""
+def launches_per_step(cfg, fused=False):
+    """Kernel launches of one step: three per block, two when the Res3.2
+    block's conv2 and conv3 run fused (Cmid = 128)."""
     s = synth.CONFIGS[cfg]
     if isinstance(s, synth.BlockShape):
         return 2 if block_fused(s, fused) else 3
@@ -497,7 +499,7 @@ def dry_run(a, rank, world):
                           "dry_run": True, "scaling": "weak"}), flush=True)
 
 
-def block_stage_calls(cfg, dev, seed, fusion=True):
+def block_stage_calls(cfg, dev, seed, fusion=False):
     """For the block workloads: the three stages as separate calls on the same
     buffers (conv1 x -> y1, conv2 y1 -> y2, conv3 y2 (+x) -> out), for
     per-stage timing.  Returns (label, ops, bytes, call) per stage."""
@@ -643,7 +645,7 @@ def main(argv=None):
     if not os.path.exists(X.LIB_PATH):
         _build.build()
     X.lib()
-    X.x1cb_set_block_fusion(not a.no_fusion)
+    X.x1cb_set_block_fusion(a.fusion)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = None
@@ -696,7 +698,7 @@ def main(argv=None):
         stages = []
         with torch.cuda.stream(stream):
             for lab, s_ops, s_bytes, fn in block_stage_calls(
-                    cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank), not a.no_fusion):
+                    cfg, dev, shard_seed(synth.CONFIG_SEEDS[cfg], rank), a.fusion):
                 t = time_launches(fn, stream, max(20, min(200, a.steps)))
                 stages.append({"stage": lab, "us": t * 1e3, "ops": s_ops, "bytes": s_bytes})
         torch.cuda.synchronize()
@@ -777,7 +779,7 @@ def main(argv=None):
         return 0
 
     hbm, bf16, peak_kind = peaks()
-    launches = launches_per_step(cfg, not a.no_fusion)
+    launches = launches_per_step(cfg, a.fusion)
     gbs = nbytes / (ms_max * 1e-3) / 1e9
     if stages is None:
         roof = roofline(ops, nbytes, ms_max * 1e-3, hbm, bf16, peak_kind)

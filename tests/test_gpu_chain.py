@@ -30,7 +30,7 @@ def _need_gpu():
     X.x1cb_set_block_fusion(True)
     X.x1cb_last_device_error(clear=True)
     yield
-    X.x1cb_set_block_fusion(True)
+    X.x1cb_set_block_fusion(False)  # the library's default
 
 
 def _nhwc(t):
@@ -52,7 +52,7 @@ def _run(x, args, inp, fused):
         out = X.bottleneck_i8(x, *args, inp.m_r, inp.S)
         torch.cuda.synchronize()
     finally:
-        X.x1cb_set_block_fusion(True)
+        X.x1cb_set_block_fusion(True)  # this module's setting
     st, bits = X.x1cb_last_device_error(clear=True)
     assert st == 0, hex(bits)
     return out

@@ -18,7 +18,7 @@ namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{0};
 std::atomic<int> g_inject{0};
-std::atomic<int> g_block_fusion{1};
+std::atomic<int> g_block_fusion{0};
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 
 struct DevInfo {
