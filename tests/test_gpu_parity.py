@@ -298,6 +298,35 @@ def test_conv3x3_parity(oracle, shape):
     assert torch.equal(got, ref), (got != ref).sum().item()
 
 
+# The 128 -> 128 3x3 runs on CTA pairs (each CTA holds half the weights):
+# several images per tile, a ragged last row of tiles, an odd tile count (the
+# second CTA of the last pair has no tile), unswizzled output rows (W = 14),
+# wide rows (two image rows per tile) and a single pixel.
+PAIR_3X3 = [(11, 6, 6), (2, 30, 28), (3, 9, 12), (4, 14, 14), (5, 56, 56), (1, 1, 1), (7, 28, 28)]
+
+
+@pytest.mark.parametrize("shape", PAIR_3X3, ids=[str(s) for s in PAIR_3X3])
+def test_conv3x3_on_cta_pairs(oracle, shape):
+    B, H, W = shape
+    assert " pair=1 " in X.x1cb_describe_plan(B, H, W, 128, 128, 3, False)
+    s = synth.ConvShape(B, H, W, 128, 128, R=3, has_res=False)
+    inp = synth.conv_inputs(s, seed=500 + B * H + W)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref), (got != ref).sum().item()
+
+
+@pytest.mark.parametrize("S", [12, 33])
+def test_conv3x3_on_cta_pairs_full_int8_range(oracle, S):
+    """Full-range operands and wide biases and multipliers at two shifts (the
+    pair kernel picks its exact form from them at run time)."""
+    s = synth.ConvShape(3, 9, 12, 128, 128, 3, False)
+    inp = synth.full_range_conv_inputs(s, 17 + S, S=S)
+    ref = oracle.pack_act(_oracle_conv(oracle, inp))
+    got = _gpu_conv(inp)
+    assert torch.equal(got, ref), (got != ref).sum().item()
+
+
 def test_conv3x3_full_int8_range(oracle):
     s = synth.ConvShape(2, 9, 11, 64, 128, 3, False)
     inp = synth.full_range_conv_inputs(s, 7, S=33)
@@ -384,7 +413,8 @@ def test_full_size_1x1_every_output(oracle, cfg):
 STRESS = [
     (256, 28, 28, 128, 512, 1, True),   # Res3.2 Conv3 (I/O ring of 7 stages)
     (96, 28, 28, 512, 128, 1, False),   # Res3.2 conv1 (3 stages)
-    (96, 28, 28, 128, 128, 3, False),   # Res3.2 conv2, halo form (2 stages)
+    (96, 28, 28, 128, 128, 3, False),   # Res3.2 conv2 on CTA pairs (4 stages)
+    (96, 28, 28, 64, 128, 3, False),    # a 3x3 of one CTA, halo form (2 stages)
 ]
 
 

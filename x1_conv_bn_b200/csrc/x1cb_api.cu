@@ -171,6 +171,18 @@ int conv_common(const int8_t *x, const int8_t *w, const int32_t *bias, const int
     if (check_ptrs)
         if (int e = check_resident({x, w, bias, m, r, out}))
             return e;
+    // The 128 -> 128 3x3 (the bottleneck's Conv2) runs on CTA pairs that
+    // share each MMA and hold half the weights each: a deeper halo ring than
+    // one SM can keep beside all 144 KB of them.
+    if (R == 3 && !r && Ic == 128 && Oc == 128 && g_inject.load() == 0) {
+        ChainPlan cp;
+        if (plan_conv2_pair(cp, B, H, W, S) == X1CB_OK) {
+            const unsigned long long lim = g_wait_limit_ns.load();
+            cp.wait_limit_ns = lim ? lim : kDefaultWaitNs;
+            return launch_chain(cp, x, w, bias, m, nullptr, nullptr, nullptr, nullptr, out,
+                                static_cast<cudaStream_t>(stream));
+        }
+    }
     ConvPlan p;
     if (int e = get_plan(p, B, H, W, Ic, Oc, R, r != nullptr, S, m_r, sms))
         return e;
@@ -649,6 +661,15 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
                   p.halo, p.io_swz, p.wstream, p.n_mma_warps, p.stage_ch);
+    // The 128 -> 128 3x3 runs on CTA pairs instead (see conv_common): its
+    // plan follows the single-CTA one.
+    ChainPlan cp;
+    if (R == 3 && !has_res && Ic == 128 && Oc == 128 && plan_conv2_pair(cp, B, H, W, 24) == X1CB_OK) {
+        const size_t n = std::strlen(buf);
+        std::snprintf(buf + n, len - n, " pair=1 pair_tile=%dx%dx%d pair_a_stages=%d "
+                      "pair_r_stages=%d pair_smem=%d", cp.tw, cp.th, cp.tg, cp.a_stages,
+                      cp.r_stages, cp.smem_bytes);
+    }
     return X1CB_OK;
 }
 

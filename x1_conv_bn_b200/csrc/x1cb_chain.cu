@@ -344,6 +344,83 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
     }
 }
 
+// Epilogue of the 3x3 alone on CTA pairs (kC3 = false): the MMA issuer puts
+// pair tile i's accumulator in slot i % 4 and turn g takes tiles g, g+4, ...
+// (it owns slot g, so it sees every phase of it in order).  Each tile is
+// requantised into one output stage (128 channels of the tile's rows) in
+// stage order (the ticket), which the store warp writes back.
+template <int kM2>
+__device__ __forceinline__ void conv2_epilogue(const ChainEpi &ce, int warp, int lane)
+{
+    const ChainPlan &p = *ce.p;
+    const ChainBars &bars = ce.bars;
+    const WaitCtl &ctl = ce.ctl;
+    const int q = warp & 3;
+    const int turn = (warp - kEpiWarp0) >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tslot = ce.tmem_base + lane_addr + static_cast<uint32_t>(turn * 128);
+    const uint32_t empty0 = mapa_shared(bars.acc_empty(turn), 0);
+    // This row's place in an output stage (halo rows outside the image are
+    // computed and not stored).
+    const int plane_t = p.tw * p.th;
+    const int xi = row % p.row_pitch;
+    const int yi = (row % p.plane_m) / p.row_pitch;
+    const int gi = row / p.plane_m;
+    const bool in_box = xi < p.tw && yi < p.th && gi < p.tg;
+    const int row_off = in_box ? ((gi * kRChunks) * plane_t + yi * p.tw + xi) * 32 : 0;
+    const int chunk_stride = plane_t * 32;
+    const int swz_mask = p.io_swz ? 0x70 : 0;
+    const uint32_t rsel[4] = {0, 0, 0, 0};
+    uint32_t kph = 0;
+    const bool tr = q == 0 && lane == 0;
+    for (int i = turn; i < ce.n_my; i += kSlots) {
+        const int st = i % p.r_stages;
+        const uint32_t st_phase = static_cast<uint32_t>((i / p.r_stages) & 1);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)))
+            return;
+        if (tr)
+            X1CB_TRACE_AT(p.trace, 6, i);
+        if (!__all_sync(0xffffffffu, ticket_wait(ce.io_ticket, i, ctl, kDevTimeoutEpilogue)) ||
+            !__all_sync(0xffffffffu,
+                        mbar_wait(bars.io_full(st), st_phase, ctl, kDevTimeoutEpilogue)))
+            return;
+        if (lane == 0)
+            atomicMax(const_cast<int *>(ce.io_ticket), i + 1);
+        tc_fence_after();
+        uint8_t *stage = ce.smem + p.off_r + st * kRSlotBytes;
+#pragma unroll 1
+        for (int cs = 0; cs < kRChunks; ++cs) {
+            uint32_t v[32], ow[8];
+            __syncwarp();
+            tmem_ld_32x32b_x32_sync(tslot + static_cast<uint32_t>(cs * 32), v);
+            requant_chain<kM2, false, false>(ce.mode2, v, ce.cm2, ce.cc2, cs * 32, nullptr, 0,
+                                             p.S, 0, rsel, ow);
+            const int o = row_off + cs * chunk_stride;
+            const int sw = swz_mask & (o >> 3);
+            if (in_box) {
+                *reinterpret_cast<uint4 *>(stage + (o ^ sw)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                *reinterpret_cast<uint4 *>(stage + ((o + 16) ^ sw)) =
+                    make_uint4(ow[4], ow[5], ow[6], ow[7]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (tr)
+            X1CB_TRACE_AT(p.trace, 7, i);
+        if (lane == 0) {
+            mbar_arrive(bars.out_ready(st));
+            mbar_arrive_cluster(empty0);
+        }
+        kph ^= 1u;
+    }
+}
+
+// kC3 = true: Conv2 -> Conv3 fused; false: the 3x3 alone (Conv2's layout,
+// output stored like Conv3's).
+template <bool kC3>
 __global__ void __launch_bounds__(kThreads, 1)
     chain23_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW2,
                    const __grid_constant__ CUtensorMap tmW3,
@@ -412,8 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmW2);
-        tma_prefetch_desc(&tmW3);
-        tma_prefetch_desc(&tmR);
+        if (kC3) {
+            tma_prefetch_desc(&tmW3);
+            tma_prefetch_desc(&tmR);
+        }
         tma_prefetch_desc(&tmO);
     }
     // Exact forms of the two layers (every CTA takes the same decision).
@@ -422,9 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t *cm3 = reinterpret_cast<int32_t *>(smem + p.off_cm3);
     long long *cc3 = reinterpret_cast<long long *>(smem + p.off_cc3);
     const int mode2 = pick_form(b2, m2, p.Cm, 0, p.S, 9 * p.Cm, false);
-    const int mode3 = pick_form(b3, m3, p.Cout, p.m_r, p.S, p.Cm, true);
+    const int mode3 = kC3 ? pick_form(b3, m3, p.Cout, p.m_r, p.S, p.Cm, true) : mode2;
     fill_consts(mode2, b2, m2, p.Cm, p.S, cm2, cc2);
-    fill_consts(mode3, b3, m3, p.Cout, p.S, cm3, cc3);
+    if (kC3)
+        fill_consts(mode3, b3, m3, p.Cout, p.S, cm3, cc3);
     if (threadIdx.x == 0)
         atomicOr(dev_forms, (1u << mode2) | (1u << mode3));
     if (warp == 1) {
@@ -451,16 +531,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t wfull0 = mapa_shared(bars.w_full(), 0);
             const int half = static_cast<int>(rank) * kHalfRows;
             const uint32_t w2_bytes = 9 * p.C1 * kHalfRows * 32;
-            const uint32_t w3_bytes = p.n_chunks * p.C1 * kHalfRows * 32;
+            const uint32_t w3_bytes = kC3 ? p.n_chunks * p.C1 * kHalfRows * 32 : 0;
             if (leader)  // both CTAs' halves complete on rank 0's barrier
                 mbar_arrive_expect_tx(bars.w_full(), 2 * (w2_bytes + w3_bytes));
             for (int kb = 0; kb < 9 * p.C1; ++kb)
                 tma2_load_4d(sbase + p.off_w2 + kb * kHalfRows * 32, &tmW2, wfull0, 0, half, kb,
                              0);
-            for (int c = 0; c < p.n_chunks; ++c)
-                for (int kb = 0; kb < p.C1; ++kb)
-                    tma2_load_4d(sbase + p.off_w3 + (c * p.C1 + kb) * kHalfRows * 32, &tmW3,
-                                 wfull0, 0, half, kb, c);
+            if (kC3)
+                for (int c = 0; c < p.n_chunks; ++c)
+                    for (int kb = 0; kb < p.C1; ++kb)
+                        tma2_load_4d(sbase + p.off_w3 + (c * p.C1 + kb) * kHalfRows * 32, &tmW3,
+                                     wfull0, 0, half, kb, c);
         }
         __syncwarp();
         if (lane < kAIssuers) {
@@ -511,6 +592,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!mbar_drain(bars.a_full(static_cast<int>(k % p.a_stages)),
                                     static_cast<uint32_t>((k / p.a_stages) & 1), drain_ns))
                         atomicOr(dev_status, kDevDrainFailed);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2 && !kC3) {
+        // ---- the 3x3 alone: hand out output stages (nothing to load) -----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int i = 0; i < n_my; ++i) {
+                if (!mbar_wait(bars.io_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer))
+                    break;
+                mbar_arrive(bars.io_full(stage));
+                if (++stage == p.r_stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
         __syncwarp();
@@ -659,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sph ^= 1u;
                     }
                 }
-                if (i >= 1) {
+                if (kC3 && i >= 1) {
                     // Conv3 of pair tile i - 1: A = its Conv2 result (buffer (i-1) % 2),
                     // one 128-channel chunk per slot.
                     const int j = i - 1, b = j & 1;
@@ -711,12 +808,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const ChainEpi ce{&p, bars, ctl, tmem_base, smem, io_ticket, cm2, cc2, cm3, cc3, n_my,
                           mode2, mode3};
         const bool k1 = static_cast<long long>(p.m_r) == (1ll << (p.S - 1));
-        if (mode2 == 2 && mode3 == 2 && k1)
+        if (!kC3) {
+            if (mode2 == 2)
+                conv2_epilogue<2>(ce, warp, lane);
+            else
+                conv2_epilogue<-1>(ce, warp, lane);
+        } else if (mode2 == 2 && mode3 == 2 && k1) {
             chain_epilogue<2, 2, true>(ce, warp, lane);
-        else if (mode2 == 2 && mode3 == 2)
+        } else if (mode2 == 2 && mode3 == 2) {
             chain_epilogue<2, 2, false>(ce, warp, lane);
-        else
+        } else {
             chain_epilogue<-1, -1, false>(ce, warp, lane);
+        }
     }
 
     // ---- tear-down: neither CTA leaves while the other may still reach it ----------
@@ -740,17 +843,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- host side --------------------------------------------------------------
 
-int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r)
+namespace {
+
+// Plan of the CTA-pair kernel: c3 = fused Conv2 -> Conv3, else the 3x3 alone
+// (Cout = Cm).
+int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r, bool c3)
 {
     std::memset(&p, 0, sizeof(p));
-    // The fused form: one 128-channel Conv2 (its output is Conv3's whole K), a
-    // halo tile row that fits the 128 GEMM rows, and output rows that the I/O
-    // maps can move whole (4-pixel groups, or rows of at most 256 8-byte units).
-    if (Cm != 128 || Cout < 128 || Cout % 128 || Cout > 1024 || W + 2 > kTileRows || H < 1 ||
+    // One 128-channel Conv2 (its output is Conv3's whole K), a halo tile row
+    // that fits the 128 GEMM rows, and output rows that the I/O maps can move
+    // whole (4-pixel groups, or rows of at most 256 8-byte units).
+    if ((!c3 && Cout != Cm) || Cm != 128 || Cout < 128 || Cout % 128 || Cout > 1024 || W + 2 > kTileRows || H < 1 ||
         W < 1 || B < 1)
         return X1CB_ERR_SHAPE;
     if (W % 4 != 0 && 4 * W > 256)
         return X1CB_ERR_SHAPE;
+    p.c3 = c3 ? 1 : 0;
     p.B = B;
     p.H = H;
     p.W = W;
@@ -778,14 +886,14 @@ int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m
     p.io_swz = W % 4 == 0 ? 1 : 0;
 
     const int w2_bytes = 9 * p.C1 * kHalfRows * 32;
-    const int w3_bytes = p.n_chunks * p.C1 * kHalfRows * 32;
+    const int w3_bytes = c3 ? p.n_chunks * p.C1 * kHalfRows * 32 : 0;
     auto layout = [&](int a, int r) {
         p.a_stages = a;
         p.r_stages = r;
         p.off_w2 = 0;
         p.off_w3 = w2_bytes;
         p.off_a3 = (p.off_w3 + w3_bytes + 1023) / 1024 * 1024;
-        p.off_a = p.off_a3 + kA3Bufs * kA3Bytes;
+        p.off_a = p.off_a3 + (c3 ? kA3Bufs * kA3Bytes : 0);
         p.off_r = p.off_a + a * p.a_slot;
         p.off_cm2 = p.off_r + r * kRSlotBytes;
         p.off_cc2 = p.off_cm2 + p.Cm * 4;
@@ -796,11 +904,20 @@ int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m
         p.smem_bytes = p.off_misc + 16 + 1024;
         return p.smem_bytes <= kSmemLimit;
     };
-    // Deepest shortcut ring beside at least four halo slots (fewer if needed).
     bool placed = false;
-    for (int a = 4; a >= 2 && !placed; --a)
-        for (int r = 8; r >= 2 && !placed; --r)
-            placed = layout(a, r);
+    if (c3) {
+        // Deepest shortcut ring beside at least four halo slots (fewer if needed).
+        for (int a = 4; a >= 2 && !placed; --a)
+            for (int r = 8; r >= 2 && !placed; --r)
+                placed = layout(a, r);
+    } else {
+        // The 3x3 alone holds half its weights per CTA (72 KB) and no Conv3
+        // operands: a deep halo ring (up to four tiles of channel blocks)
+        // beside output stages for each epilogue turn.
+        for (int r = kSlots; r >= 2 && !placed; --r)
+            for (int a = 16; a >= 4 && !placed; --a)
+                placed = layout(a, r);
+    }
     if (!placed)
         return X1CB_ERR_SHAPE;
     p.grid = 2 * std::max(1, std::min(74, p.n_pairs));
@@ -808,18 +925,32 @@ int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m
     return X1CB_OK;
 }
 
+}  // namespace
+
+int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r)
+{
+    return plan_pair(p, B, H, W, Cm, Cout, S, m_r, true);
+}
+
+int plan_conv2_pair(ChainPlan &p, int B, int H, int W, int S)
+{
+    return plan_pair(p, B, H, W, 128, 128, S, 0, false);
+}
+
 // Clusters of two CTAs of chain23_kernel that fit on the current device at
 // once with `smem` bytes of shared memory each (cached per device and size).
-int resident_clusters(int smem, int &clusters)
+int resident_clusters(int smem, int &clusters, bool c3)
 {
     static std::mutex mu;
-    static int cached[64] = {}, cached_smem[64] = {};
+    static int cached[2][64] = {}, cached_smem[2][64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return X1CB_ERR_CUDA;
+    const int k = c3 ? 1 : 0;
+    auto kern = c3 ? chain23_kernel<true> : chain23_kernel<false>;
     std::lock_guard<std::mutex> lk(mu);
-    if (cached[dev] == 0 || cached_smem[dev] != smem) {
-        if (int e = opt_in_smem(reinterpret_cast<const void *>(chain23_kernel), 2))
+    if (cached[k][dev] == 0 || cached_smem[k][dev] != smem) {
+        if (int e = opt_in_smem(reinterpret_cast<const void *>(kern), c3 ? 2 : 5))
             return e;
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
@@ -834,14 +965,14 @@ int resident_clusters(int smem, int &clusters)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, chain23_kernel, &cfg) != cudaSuccess || n < 1) {
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
             cudaGetLastError();
             return X1CB_ERR_CUDA;
         }
-        cached[dev] = n;
-        cached_smem[dev] = smem;
+        cached[k][dev] = n;
+        cached_smem[k][dev] = smem;
     }
-    clusters = cached[dev];
+    clusters = cached[k][dev];
     return X1CB_OK;
 }
 
@@ -867,12 +998,14 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
         if (int e = encode_map(&tmW2, w2, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }
-    {  // Conv3 weights [Cout/128][C1][128][32]
+    if (p.c3) {  // Conv3 weights [Cout/128][C1][128][32]
         const uint64_t dims[4] = {32, 128, (uint64_t)p.C1, (uint64_t)p.n_chunks};
         const uint64_t str[3] = {32, 4096, (uint64_t)p.C1 * 4096};
         const uint32_t box[4] = {32, kHalfRows, 1, 1};
         if (int e = encode_map(&tmW3, w3, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
+    } else {
+        tmW3 = tmW2;  // unused
     }
     const uint64_t O1 = p.Cout / 32;
     if (p.io_swz) {  // 128-byte rows of 4 pixels: (16 x 8 B, W/4, H, O1, B)
@@ -884,8 +1017,10 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
         if (int e = encode_map(&tmO, out, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_DATA_TYPE_UINT64))
             return e;
-        if (int e = encode_map(&tmR, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
-                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+        if (!p.c3)
+            tmR = tmO;  // unused
+        else if (int e = encode_map(&tmR, x, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                                    CU_TENSOR_MAP_DATA_TYPE_UINT64))
             return e;
     } else {  // whole rows of W*32 bytes as 8-byte units: (4W, H, O1, B)
         const uint64_t dims[4] = {(uint64_t)p.W * 4, (uint64_t)p.H, O1, (uint64_t)p.B};
@@ -896,18 +1031,21 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
         if (int e = encode_map(&tmO, out, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
                                CU_TENSOR_MAP_DATA_TYPE_UINT64))
             return e;
-        if (int e = encode_map(&tmR, x, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
-                               CU_TENSOR_MAP_DATA_TYPE_UINT64))
+        if (!p.c3)
+            tmR = tmO;  // unused
+        else if (int e = encode_map(&tmR, x, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_DATA_TYPE_UINT64))
             return e;
     }
-    if (int e = opt_in_smem(reinterpret_cast<const void *>(chain23_kernel), 2))
+    auto kern = p.c3 ? chain23_kernel<true> : chain23_kernel<false>;
+    if (int e = opt_in_smem(reinterpret_cast<const void *>(kern), p.c3 ? 2 : 5))
         return e;
     // The kernel is persistent with a static assignment of pair tiles, so it
     // must not launch more clusters than can be resident at once: a cluster
     // needs two SMs of one GPC, and a GPC with an odd number of free SMs
     // leaves one over.
     int clusters = 0;
-    if (int e = resident_clusters(p.smem_bytes, clusters))
+    if (int e = resident_clusters(p.smem_bytes, clusters, p.c3 != 0))
         return e;
     const int grid = 2 * std::max(1, std::min(clusters, p.n_pairs));
     cudaLaunchConfig_t cfg;
@@ -928,7 +1066,7 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
         return e;
     ChainPlan q = p;
     q.trace = trace_table();
-    if (cudaLaunchKernelEx(&cfg, chain23_kernel, tmA, tmW2, tmW3, tmR, tmO, b2, m2, b3, m3,
+    if (cudaLaunchKernelEx(&cfg, kern, tmA, tmW2, tmW3, tmR, tmO, b2, m2, b3, m3,
                            dev_status, dev_forms, q) != cudaSuccess)
         return X1CB_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;

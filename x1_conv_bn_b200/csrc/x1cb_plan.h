@@ -118,6 +118,7 @@ struct ConvPlan {
 // x1cb_chain.cu).  Conv2 is the 3x3 (pad 1, halo tiles of th rows x tg
 // images, full width); Conv3 the 1x1 with the shortcut.
 struct ChainPlan {
+    int c3;  // 1: Conv2 -> Conv3 fused; 0: the 3x3 alone (Cout = Cm, stored like Conv3)
     int B, H, W, Cm, Cout, S, m_r;
     int C1, n_chunks;  // Cm/32 channel blocks, Cout/128 output chunks
     int th, tg, tw, row_pitch, plane_m, a_half, rows;
