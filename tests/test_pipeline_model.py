@@ -363,8 +363,8 @@ def run_two_mma_warps(seed, S, lanes, bpt, split, tiles=16):
 
 
 # (S, lanes, bpt): conv1 and the 3x3 (6, 3, 4), the folded stem (12, 4, 1),
-# small even rings
-SPLIT_CASES = [(6, 3, 4), (12, 4, 1), (4, 2, 1), (4, 2, 3), (8, 4, 2)]
+# the 3x3 on CTA pairs (14, 4, 4), small even rings
+SPLIT_CASES = [(6, 3, 4), (12, 4, 1), (14, 4, 4), (16, 4, 4), (4, 2, 1), (4, 2, 3), (8, 4, 2)]
 
 
 @pytest.mark.parametrize("S,lanes,bpt", SPLIT_CASES, ids=[str(c) for c in SPLIT_CASES])

@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         *io_ticket = 0;
         mbar_init(bars.w_full(), 1);
-        mbar_init(bars.mma_done(), 1);
+        mbar_init(bars.mma_done(), kC3 ? 1 : 2);  // each MMA issuer's final commit
         mbar_init(bars.exit_bar(), 1);
         for (int s = 0; s < p.a_stages; ++s) {
             mbar_init(bars.a_full(s), 1);
@@ -549,13 +549,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_first();
             const long long total = static_cast<long long>(n_my) * p.C1;
             long long issued = 0;
-            // this lane's slot n = base + lane: ring stage/phase, pair tile i,
-            // channel block c1 (counters, at most one ring wrap per round)
-            int stage = lane < n_iss ? lane : 0, i = lane / p.C1, c1 = lane % p.C1;
-            uint32_t phase = 0;
+            // This lane's slot n = base + lane: pair tile i, channel block c1
+            // and the ring position of the next box of each half, advanced by
+            // counters.  Fused: one ring (pos0).  The 3x3 alone: two MMA
+            // warps, even pair tiles in slots [0, a/2), odd ones in [a/2, a),
+            // each half consumed in order by its warp.
+            constexpr bool split = !kC3;
+            const int half = split ? p.a_stages / 2 : p.a_stages;
+            int i = 0, c1 = 0, pos0 = 0, pos1 = 0;
+            uint32_t ph0 = 0u, ph1 = 0u;
+            auto step = [&]() {  // past box (i, c1)
+                if (split && (i & 1)) {
+                    if (++pos1 == half) {
+                        pos1 = 0;
+                        ph1 ^= 1u;
+                    }
+                } else if (++pos0 == half) {
+                    pos0 = 0;
+                    ph0 ^= 1u;
+                }
+                if (++c1 == p.C1) {
+                    c1 = 0;
+                    ++i;
+                }
+            };
+            for (int k = 0; k < lane && k < n_iss; ++k)
+                step();
             for (long long base = 0; base < total; base += n_iss) {
                 const long long n = base + lane;
                 const bool have = lane < n_iss && n < total;
+                const bool odd = split && (i & 1);
+                const int stage = odd ? half + pos1 : pos0;
+                const uint32_t phase = odd ? ph1 : ph0;
                 if (!mbar_wait_lanes(kAIssuerMask, have, bars.a_empty(stage), phase ^ 1u, ctl,
                                      kDevTimeoutProducer))
                     break;
@@ -572,13 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma2_load_5d_hint(slot + p.a_half, &tmA, full0, 16, -1, h0 - 1, c1, b0, pol);
                 }
                 issued = base + n_iss < total ? base + n_iss : total;
-                stage += n_iss;
-                if (stage >= p.a_stages) {
-                    stage -= p.a_stages;
-                    phase ^= 1u;
-                }
-                for (c1 += n_iss; c1 >= p.C1; c1 -= p.C1)
-                    ++i;
+                for (int k = 0; k < n_iss; ++k)
+                    step();
             }
             // Both CTAs' copies complete on rank 0's barriers: rank 0 lets every
             // copy still in flight land (the MMA has normally seen them all)
@@ -587,31 +607,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader && lane == 0) {
                 if (!mbar_drain(bars.w_full(), 0, drain_ns))
                     atomicOr(dev_status, kDevDrainFailed);
-                const long long last = issued < p.a_stages ? issued : p.a_stages;
-                for (long long k = issued - last; k < issued; ++k)
-                    if (!mbar_drain(bars.a_full(static_cast<int>(k % p.a_stages)),
-                                    static_cast<uint32_t>((k / p.a_stages) & 1), drain_ns))
+                // the latest box of every slot (split ring: walk back until
+                // both halves' slots are seen)
+                unsigned int seen = 0;
+                const unsigned int all = (1u << p.a_stages) - 1u;
+                for (long long k = issued - 1; k >= 0 && seen != all && k >= issued - 4 * p.a_stages;
+                     --k) {
+                    int st;
+                    uint32_t ph;
+                    if (split) {
+                        const long long t = k / p.C1, li = (t >> 1) * p.C1 + (k - t * p.C1);
+                        st = static_cast<int>((t & 1) * half + li % half);
+                        ph = static_cast<uint32_t>((li / half) & 1);
+                    } else {
+                        st = static_cast<int>(k % p.a_stages);
+                        ph = static_cast<uint32_t>((k / p.a_stages) & 1);
+                    }
+                    if (seen & (1u << st))
+                        continue;
+                    seen |= 1u << st;
+                    if (!mbar_drain(bars.a_full(st), ph, drain_ns))
                         atomicOr(dev_status, kDevDrainFailed);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 2 && !kC3) {
-        // ---- the 3x3 alone: hand out output stages (nothing to load) -----------------
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int i = 0; i < n_my; ++i) {
-                if (!mbar_wait(bars.io_empty(stage), phase ^ 1u, ctl, kDevTimeoutProducer))
-                    break;
-                mbar_arrive(bars.io_full(stage));
-                if (++stage == p.r_stages) {
-                    stage = 0;
-                    phase ^= 1u;
                 }
             }
         }
         __syncwarp();
-    } else if (warp == 2) {
+    } else if (warp == 2 && kC3) {
         // ---- shortcut stages (own rows) ------------------------------------------------
         if (lane == 0) {
             const uint32_t rbytes = static_cast<uint32_t>(kRChunks * p.rows * 32);
@@ -654,11 +675,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 3) {
         // ---- stores of finished output stages (own rows) -------------------------------
+        // The 3x3 alone has no shortcut to load: this warp hands the stages
+        // out, each one's first use at once and its next use as soon as its
+        // store has read it.
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            if (!kC3)
+                for (int s = 0; s < p.r_stages; ++s)
+                    mbar_arrive(bars.io_full(s));
             for (int i = 0; ok && i < n_my; ++i) {
                 const int mt = 2 * (pair0 + i * pair_step) + static_cast<int>(rank);
                 int h0, b0;
@@ -679,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bulk_wait_read<0>();
                     }
                     X1CB_TRACE_AT(p.trace, 12, static_cast<long long>(i) * p.n_chunks + c);
-                    mbar_arrive(bars.io_empty(stage));
+                    mbar_arrive(kC3 ? bars.io_empty(stage) : bars.io_full(stage));
                     if (++stage == p.r_stages) {
                         stage = 0;
                         phase ^= 1u;
@@ -689,9 +716,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_wait_all();
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---- MMA issuer (rank 0) -------------------------------------------------------
-        if (leader) {
+    } else if (warp == 1 || (!kC3 && warp == 2)) {
+        // ---- MMA issuers (rank 0) ------------------------------------------------------
+        if (leader && !kC3) {
+            // The 3x3 alone: warp 1 issues the even pair tiles and warp 2 the odd
+            // ones (one thread issues an MMA only every ~92 cycles, an M = 256,
+            // N = 128 one takes 64 on the tensor pipe), each from its half of
+            // the halo ring and into slots i % 4 (two per warp).
+            const int mw = warp - 1;
+            const int half = p.a_stages / 2;
+            const uint32_t idesc = idesc_i8(256, 128);
+            const uint64_t a_desc0 =
+                smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half));
+            const uint64_t w2_desc0 = smem_desc_sw32(sbase + p.off_w2);
+            const uint32_t kb_step = (kHalfRows * 32) >> 4;
+            const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
+            const uint32_t hp = static_cast<uint32_t>(p.row_pitch);
+            const uint64_t ring_desc0 = a_desc0 + static_cast<uint64_t>(mw * half) * a_slot_step;
+            int pos = 0;
+            uint32_t ph = 0;
+            uint64_t sd = ring_desc0;
+            bool ok = __all_sync(0xffffffffu, mbar_wait_cl(bars.w_full(), 0, ctl, kDevTimeoutMma));
+            for (int i = mw; ok && i < n_my; i += 2) {
+                const int slot = i & 3;
+                const uint32_t sph = static_cast<uint32_t>((i >> 2) & 1);
+                if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.acc_empty(slot), sph ^ 1u, ctl,
+                                                          kDevTimeoutMma)))
+                    break;
+                if (lane == 0)
+                    X1CB_TRACE_AT(p.trace, 2, i);
+                tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(slot * 128);
+                for (int c1 = 0; c1 < p.C1; ++c1) {
+                    const int st = mw * half + pos;
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait_cl(bars.a_full(st), ph, ctl, kDevTimeoutMma))) {
+                        ok = false;
+                        break;
+                    }
+                    if (c1 == 0 && lane == 0)
+                        X1CB_TRACE_AT(p.trace, 1, i);
+                    tc_fence_after();
+#pragma unroll
+                    for (int t = 0; t < 9; ++t)
+                        mma_i8_pair(d, sd + (t / 3) * hp + (t % 3),
+                                    w2_desc0 + static_cast<uint64_t>(t * p.C1 + c1) * kb_step,
+                                    idesc, (c1 | t) ? 1u : 0u);
+                    mma_commit_pair(bars.a_empty(st));
+                    if (++pos == half) {
+                        pos = 0;
+                        ph ^= 1u;
+                        sd = ring_desc0;
+                    } else {
+                        sd += a_slot_step;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit_pair(bars.acc_full(slot));
+                if (lane == 0)
+                    X1CB_TRACE_AT(p.trace, 3, i);
+            }
+            mma_commit_pair(bars.mma_done());
+            if (lane == 0 && !mbar_drain(bars.mma_done(), 0, drain_ns))
+                atomicOr(dev_status, kDevDrainFailed);
+        } else if (leader) {
             const uint32_t idesc = idesc_i8(256, 128);
             const uint64_t a_desc0 =
                 smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half));
@@ -912,10 +1001,11 @@ int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_
                 placed = layout(a, r);
     } else {
         // The 3x3 alone holds half its weights per CTA (72 KB) and no Conv3
-        // operands: a deep halo ring (up to four tiles of channel blocks)
-        // beside output stages for each epilogue turn.
+        // operands: a deep halo ring (up to four tiles of channel blocks, an
+        // even number: half for each MMA warp) beside output stages for each
+        // epilogue turn.
         for (int r = kSlots; r >= 2 && !placed; --r)
-            for (int a = 16; a >= 4 && !placed; --a)
+            for (int a = 16; a >= 4 && !placed; a -= 2)
                 placed = layout(a, r);
     }
     if (!placed)
