@@ -810,7 +810,7 @@ def main(argv=None):
         roof["kernel"] = "stage " + top["stage"] + " (the block's slowest launch)"
         roof["algorithmic_bytes_per_launch"] = top["bytes"]
         roof["algorithmic_ops_per_launch"] = top["ops"]
-        prof = f"bottleneck_{cfg}_b{s.B}.md"
+        prof = f"bottleneck_{cfg}_b{s.B}" + ("_fused" if block_fused(s, a.fusion) else "") + ".md"
     roof["traffic"] = read_traffic(prof, kernel_source_sha("chain" if stages and
                                                            "fused" in roof["kernel"] else "conv"))
     roof["traffic_source"] = (f"ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
