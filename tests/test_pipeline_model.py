@@ -263,7 +263,8 @@ def run_a_ring(seed, S, lanes, boxes=60):
                 live.remove(ag)
 
 
-@pytest.mark.parametrize("S,lanes", [(2, 1), (3, 1), (4, 2), (5, 2), (6, 3), (8, 4), (14, 4)])
+@pytest.mark.parametrize("S,lanes", [(2, 1), (3, 1), (4, 2), (5, 2), (6, 3), (7, 3), (8, 4), (14, 4),
+                                     (28, 4)])
 def test_issuing_rounds_within_half_the_ring_are_exact(S, lanes):
     """The kernels' choice: lanes = min(4, S // 2)."""
     for seed in range(60):

@@ -1431,17 +1431,21 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // The activation ring budget: with a shortcut the I/O ring (shortcut in,
     // result out) needs the space -- its depth sets the bytes in flight -- so
     // about two tiles' K blocks plus two; without one the activations are most
-    // of the traffic and get up to 128 KB in flight while the I/O stages only
+    // of the traffic and get up to 112 KB in flight while the I/O stages only
     // stage results.  The bias-fold tiles are reserved when the rings still
     // reach their minimum beside them.
     // (Measured on the 1x1 128 -> 512 with shortcut, B = 2048: 326 us with
     // 24 KB of activation ring and seven I/O stages, 314 us with 40 KB and
     // six, 329 us with 40 KB and five.  A deep fan-in with a shortcut -- 8 or
-    // more K blocks per tile -- gets two tiles of K blocks.)
+    // more K blocks per tile -- gets two tiles of K blocks.  Without a
+    // shortcut, 1x1 512 -> 128 at B = 1024: 107.4 us with six 16 KB boxes,
+    // 104.4 with seven; 256 -> 128 at 56x56, B = 256: 72.1 us with four,
+    // 65.7 with seven.)
     const int a_bytes_want =
         p.wstream ? 4 * 4 * kASlotBytes
-        : (has_res && p.kb_per_tile < 8) ? std::min(2 * p.kb_per_tile + 2, 10) * kASlotBytes
-                                         : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
+        : !has_res ? 28 * kASlotBytes
+        : p.kb_per_tile < 8 ? std::min(2 * p.kb_per_tile + 2, 10) * kASlotBytes
+                            : std::min(2 * p.kb_per_tile, 24) * kASlotBytes;
     // Several K blocks per activation box (fewer, larger copies) when each
     // K-block tile starts on a 256-byte swizzle atom (row count a multiple of
     // 8) and the budget holds one box more than the ring's minimum.  With two
