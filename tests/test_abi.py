@@ -132,14 +132,19 @@ def test_channel_groups_are_whole_mmas(L, B, Ic, R, res):
         assert nmma * subs == NC and NC * groups == Oc, (Oc, p)
 
 
-def test_large_resident_weights_take_whole_boxes_and_narrow_stages(L):
-    """7x7 512 -> 2048 expand conv with shortcut (B = 512): 128 KB of resident
-    weights per CTA.  The tile's rows are a multiple of 8 so that each
-    activation box carries four K blocks, and the shortcut/result stages are
-    8 KB so that four fit beside the activation ring."""
+def test_large_resident_weights_take_whole_boxes_and_cta_pairs(L):
+    """7x7 512 -> 2048 expand conv with shortcut (B = 512): 128 KB of weights
+    per 256-channel group.  The tile's rows are a multiple of 8 so that each
+    activation box carries four K blocks, and the layer runs on CTA pairs
+    (64 KB of weights each) with four 16 KB shortcut/result stages; a layer
+    whose group is not one N = 256 MMA (1024 -> 256: N = 128 groups) stages
+    the shortcut in 8 KB pieces instead."""
     p = _plan((512, 7, 7, 512, 2048, 1, 1))
     assert int(p["rows"]) % 8 == 0 and p["kc"] == "4", p
-    assert p["stage_ch"] == "2" and int(p["r_stages"]) >= 4 and int(p["a_stages"]) >= 3, p
+    assert p["cta_pair"] == "1" and int(p["grid"]) % 2 == 0, p
+    assert p["stage_ch"] == "4" and int(p["r_stages"]) >= 4 and int(p["a_stages"]) >= 5, p
+    q = _plan((9, 7, 7, 1024, 256, 1, 1))
+    assert q["cta_pair"] == "0" and q["stage_ch"] == "2" and int(q["r_stages"]) >= 4, q
     # the Res3.2 conv3 (64 KB of weights) keeps 16 KB stages, six of them
     q = _plan((2048, 28, 28, 128, 512, 1, 1))
     assert q["stage_ch"] == "4" and int(q["r_stages"]) >= 6, q

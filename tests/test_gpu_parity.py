@@ -121,11 +121,11 @@ def test_conv1x1_channel_groups(oracle, shape):
     assert torch.equal(got, ref), _first_mismatch(got, ref)
 
 
-# Shortcut layers whose resident weights take more than 96 KB stage the
-# shortcut and result in 8 KB pieces (two 32-channel chunks): N = 256 groups
-# with 4-K-block boxes and a batch tail, and N = 128 groups (four accumulator
-# slots) with one K block per box on 125-row tiles.
-NARROW_IO = [(43, 7, 7, 512, 2048), (9, 7, 7, 1024, 256)]
+# Shortcut layers whose resident weights take more than 96 KB and whose
+# channel group is not one N = 256 MMA stage the shortcut and result in 8 KB
+# pieces (two 32-channel chunks): N = 128 groups (four accumulator slots)
+# with one K block per box on 125-row tiles.
+NARROW_IO = [(9, 7, 7, 1024, 256)]
 
 
 @pytest.mark.parametrize("shape", NARROW_IO, ids=[str(s) for s in NARROW_IO])
@@ -137,6 +137,35 @@ def test_conv1x1_narrow_io_stages(oracle, shape):
     ref = _oracle_conv(oracle, inp)
     assert torch.equal(got, ref), _first_mismatch(got, ref)
     _assert_spread(oracle.pack_act(ref))
+
+
+# Shortcut layers whose 256-channel groups take more than 96 KB of weights run
+# on CTA pairs sharing each MMA (M = 256): an even and an odd tile count (the
+# second CTA of the last pair has no tile), a batch tail, and one channel group
+# over many pairs.
+PAIR_1X1 = [(43, 7, 7, 512, 2048), (41, 7, 7, 512, 2048), (26, 28, 28, 512, 256)]
+
+
+@pytest.mark.parametrize("shape", PAIR_1X1, ids=[str(s) for s in PAIR_1X1])
+def test_conv1x1_on_cta_pairs(oracle, shape):
+    assert "cta_pair=1" in X.x1cb_describe_plan(*shape, 1, True)
+    s = synth.ConvShape(*shape, R=1, has_res=True)
+    inp = synth.conv_inputs(s, 71 + shape[0])
+    got = _nhwc(_gpu_conv(inp))
+    ref = _oracle_conv(oracle, inp)
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
+    _assert_spread(oracle.pack_act(ref))
+
+
+@pytest.mark.parametrize("S", [12, 24, 40])
+def test_conv1x1_on_cta_pairs_full_int8_range(oracle, S):
+    """Full-range operands at three shifts: the epilogue forms with and
+    without the bias folded into the pair's MMAs."""
+    s = synth.ConvShape(41, 7, 7, 512, 2048, R=1, has_res=True)
+    inp = synth.full_range_conv_inputs(s, 300 + S, S=S)
+    got = _nhwc(_gpu_conv(inp))
+    ref = _oracle_conv(oracle, inp)
+    assert torch.equal(got, ref), _first_mismatch(got, ref)
 
 
 @pytest.mark.parametrize("S", [12, 24, 31, 40])

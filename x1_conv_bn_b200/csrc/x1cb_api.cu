@@ -657,10 +657,10 @@ int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, 
     std::snprintf(buf, len,
                   "tile=%dx%dx%d rows=%d m_tiles=%d NC=%d groups=%d nmma=%d subs=%d kb=%d "
                   "kc=%d a_stages=%d r_stages=%d fold=%d smem=%d grid=%d halo=%d swz=%d "
-                  "wstream=%d mwarps=%d stage_ch=%d",
+                  "wstream=%d mwarps=%d stage_ch=%d cta_pair=%d",
                   p.tw, p.th, p.tg, p.rows, p.num_m_tiles, p.NC, p.n_groups, p.nmma, p.n_subs,
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
-                  p.halo, p.io_swz, p.wstream, p.n_mma_warps, p.stage_ch);
+                  p.halo, p.io_swz, p.wstream, p.n_mma_warps, p.stage_ch, p.pair);
     // The 128 -> 128 3x3 runs on CTA pairs instead (see conv_common): its
     // plan follows the single-CTA one.
     ChainPlan cp;

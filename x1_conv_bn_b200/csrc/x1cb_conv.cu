@@ -91,14 +91,17 @@ struct Bars {
     {
         return at(3 + 2 * a_stages + 3 * r_stages + 16 + turn);
     }
-    static int count(int a, int r) { return 3 + 2 * a + 3 * r + 16 + 4; }
+    // CTA pairs: each CTA arrives on the other's before leaving.
+    __device__ uint32_t exit_bar() const { return at(3 + 2 * a_stages + 3 * r_stages + 20); }
+    static int count(int a, int r) { return 3 + 2 * a + 3 * r + 16 + 4 + 1; }
 };
 
 // A layer with a shortcut is always a plain stride-1 1x1 (the planner and the
 // API admit no other): its instantiations (kRes = 1: I/O stages of four
 // 32-channel chunks; kRes = 2: of two, for layers whose resident weights leave
-// little room for the rings) read these plan fields as constants, so they
-// carry none of the halo, pooling or second-source code (which cost the
+// little room for the rings; kRes = 3: four, on pairs of CTAs that share each
+// MMA and hold half the weights each) read these plan fields as constants, so
+// they carry none of the halo, pooling or second-source code (which cost the
 // shortcut layers up to 4 % when it was compiled into them).  kRes = 0: no
 // shortcut, every form.
 template <int kRes> __device__ __forceinline__ int plan_halo(const ConvPlan &p)
@@ -111,7 +114,7 @@ template <int kRes> __device__ __forceinline__ bool plan_pool(const ConvPlan &p)
 }
 template <int kRes> __device__ __forceinline__ int plan_stage_ch(const ConvPlan &p)
 {
-    return kRes == 1 ? kRChunks : (kRes == 2 ? kRChunks / 2 : p.stage_ch);
+    return kRes == 1 || kRes == 3 ? kRChunks : (kRes == 2 ? kRChunks / 2 : p.stage_ch);
 }
 template <int kRes> __device__ __forceinline__ int plan_c1b(const ConvPlan &p)
 {
@@ -175,7 +178,7 @@ struct EpiCtx {
     volatile int *io_ticket;  // I/O stages before this one have been seen to arrive
     const int32_t *cm;
     const long long *cC;
-    int group, mt_first, mt_step;
+    int group, mt_first, mt_step, mt_end;
 };
 
 // kMode: 3 = all-32-bit form with the bias folded into the MMA, 2 = all-32-bit
@@ -221,7 +224,7 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
     const int chunks_per_sub = p.nmma / 32;
     const int stages_per_sub = chunks_per_sub / plan_stage_ch<kRes>(p);
     const long long my_tiles =
-        cx.mt_first < p.num_m_tiles ? (p.num_m_tiles - cx.mt_first + cx.mt_step - 1) / cx.mt_step
+        cx.mt_first < cx.mt_end ? (cx.mt_end - cx.mt_first + cx.mt_step - 1) / cx.mt_step
                                     : 0;
     const long long total = my_tiles * p.n_subs * stages_per_sub;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
@@ -379,7 +382,12 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             X1CB_TRACE_AT(p.trace, 6, n);
         if (lane == 0) {
             mbar_arrive(cx.bars.out_ready(st));
-            mbar_arrive(cx.bars.acc_empty(acc));  // one arrival per stage of the slot
+            // one arrival per stage of the slot (CTA pairs: from both CTAs, on
+            // rank 0's barrier, which its MMA warp waits on)
+            if (kRes == 3)
+                mbar_arrive_cluster(mapa_shared(cx.bars.acc_empty(acc), 0));
+            else
+                mbar_arrive(cx.bars.acc_empty(acc));
         }
         st += kTurns;
         while (st >= p.r_stages) {
@@ -397,6 +405,32 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             }
         }
     }
+}
+
+// MMA-side operations of one CTA or of a CTA pair (rank 0 issues M = 256
+// MMAs over both CTAs' operands; its waits see the other CTA's arrivals with
+// cluster scope, its commits arrive on both CTAs' barriers).
+template <bool kPair>
+__device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t parity, const WaitCtl &ctl,
+                                         unsigned int code)
+{
+    return kPair ? mbar_wait_cl(bar, parity, ctl, code) : mbar_wait(bar, parity, ctl, code);
+}
+template <bool kPair>
+__device__ __forceinline__ void mma_issue(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    if (kPair)
+        mma_i8_pair(d, a, b, idesc, accumulate);
+    else
+        mma_i8(d, a, b, idesc, accumulate);
+}
+template <bool kPair> __device__ __forceinline__ void mma_commit_to(uint32_t bar)
+{
+    if (kPair)
+        mma_commit_pair(bar);
+    else
+        mma_commit(bar);
 }
 
 // kSplit: two MMA warps (warp 2 issues MMAs; no shortcut), a separate
@@ -432,9 +466,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                       p.inject == 1 ? 4 * p.wait_limit_ns : p.wait_limit_ns};
     const uint64_t drain_ns = 200000000ull;  // 0.2 s for copies/MMAs already issued
 
-    const int group = blockIdx.x % p.n_groups;
-    const int mt_first = blockIdx.x / p.n_groups;
-    const int mt_step = gridDim.x / p.n_groups;
+    // CTA pairs (kRes = 3): cluster c = blockIdx.x / 2 takes channel group
+    // c % n_groups and pair tiles pt = c / n_groups + k * (clusters per group);
+    // rank r of the pair takes m-tile 2 pt + r (past the last tile: zeros
+    // loaded, nothing stored), so both ranks run the same number of tiles.
+    constexpr bool kPair = kRes == 3;
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = kPair ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
+    const int units = kPair ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
+    const int group = unit % p.n_groups;
+    const int mt_first = kPair ? 2 * (unit / p.n_groups) + static_cast<int>(rank)
+                               : unit / p.n_groups;
+    const int mt_step = kPair ? 2 * (units / p.n_groups) : units / p.n_groups;
+    const int mt_end = kPair ? (p.num_m_tiles + 1) & ~1 : p.num_m_tiles;
     const int stages_per_tile = p.NC / (32 * plan_stage_ch<kRes>(p));
 
     // ---- set-up ---------------------------------------------------------------
@@ -464,9 +509,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bars.pool_bar(t), 4);
         for (int s = 0; s < 8; ++s) {
             mbar_init(bars.acc_full(s), 1);
-            // every stage of the slot, each from one warp per lane quarter
-            mbar_init(bars.acc_empty(s), 4 * (p.nmma / (32 * plan_stage_ch<kRes>(p))));
+            // every stage of the slot, each from one warp per lane quarter (of
+            // both CTAs of a pair)
+            mbar_init(bars.acc_empty(s),
+                      (kPair ? 8 : 4) * (p.nmma / (32 * plan_stage_ch<kRes>(p))));
         }
+        mbar_init(bars.exit_bar(), 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -508,9 +556,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 *ta = reinterpret_cast<uint4 *>(smem + p.off_ba);
         for (int i = threadIdx.x; i < kTileRows * 2; i += blockDim.x)
             ta[i] = make_uint4(0x7F7F7F01u, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        for (int n = threadIdx.x; n < p.NC; n += blockDim.x) {
+        // (CTA pairs: this CTA's half of the B rows, channels rank * NC/2 on)
+        const int nb = kPair ? p.NC / 2 : p.NC;
+        for (int n = threadIdx.x; n < nb; n += blockDim.x) {
             uint32_t w[8];
-            bias_digits(bias[group * p.NC + n], w);
+            bias_digits(bias[group * p.NC + static_cast<int>(rank) * nb + n], w);
             uint4 *tb = reinterpret_cast<uint4 *>(smem + p.off_bb + n * 32);
             tb[0] = make_uint4(w[0], w[1], w[2], w[3]);
             tb[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -536,11 +586,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-        tmem_relinquish();
+        if (kPair) {
+            tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+            tmem_relinquish();
+        }
         tc_fence_before();
     }
     __syncthreads();
+    if (kPair)  // both CTAs' barriers and TMEM exist before traffic crosses
+        cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -558,7 +615,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t sw = sbase + p.off_w;
             const int o1 = group * (p.NC / p.O2);  // weight block of this CTA's channels
-            if (!p.wstream) {
+            if (kPair) {
+                // this CTA's half of each K block (output channels rank * NC/2
+                // on), both halves completing on rank 0's barrier
+                const int half_nc = p.NC / 2;
+                const uint32_t wbytes = static_cast<uint32_t>(p.kb_per_tile * half_nc * 32);
+                if (leader)
+                    mbar_arrive_expect_tx(bars.w_full(), 2 * wbytes);
+                const uint32_t wfull0 = mapa_shared(bars.w_full(), 0);
+                for (int kb = 0; kb < p.kb_per_tile; ++kb)
+                    tma2_load_4d(sw + kb * half_nc * 32, &tmW, wfull0, 0, 0, kb,
+                                 o1 + static_cast<int>(rank));
+            } else if (!p.wstream) {
                 const uint32_t wbytes = static_cast<uint32_t>(p.kb_per_tile * p.NC * 32);
                 mbar_arrive_expect_tx(bars.w_full(), wbytes);
                 // The second source's weights (if any) follow the first's K blocks.
@@ -595,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int first_boxes = plan_halo<kRes>(p) ? p.C1 : p.R * p.Rw * cb;
             const int bpt = plan_halo<kRes>(p) ? p.C1 : p.kb_per_tile / p.a_kc;
             const long long my_tiles =
-                mt_first < p.num_m_tiles ? (p.num_m_tiles - mt_first + mt_step - 1) / mt_step : 0;
+                mt_first < mt_end ? (mt_end - mt_first + mt_step - 1) / mt_step : 0;
             const long long total = my_tiles * bpt;
             long long issued = 0;
             // This lane's box n = base + lane as ring stage/phase and as (tile i,
@@ -645,6 +713,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     int w0, h0, b0;
                     tile_origin<kRes>(p, mt, w0, h0, b0);
                     const uint32_t slot = sa + static_cast<uint32_t>(stage) * p.a_slot;
+                    if (kPair) {
+                        // this CTA's tile, completing on rank 0's barrier (which
+                        // expects both CTAs' boxes)
+                        if (leader)
+                            mbar_arrive_expect_tx(bars.a_full(stage), 2 * abytes);
+                        tma2_load_5d_hint(slot, &tmA, mapa_shared(bars.a_full(stage), 0), 0, w0,
+                                          h0, b0, b * p.a_kc, pol);
+                    } else {
                     mbar_arrive_expect_tx(bars.a_full(stage), abytes + wpart);
                     if (plan_halo<kRes>(p) == 2) {
                         // one slot per channel block c1 = b: plane (pr, pc) from
@@ -699,6 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             kb0 + i, o1);
                         }
                     }
+                    }  // (not a pair)
                 }
                 issued = base + n_iss < total ? base + n_iss : total;
                 if (!split) {  // (n_iss <= a_stages / 2: at most one wrap)
@@ -728,8 +805,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // Let every copy still in flight land before shared memory goes away.
+            // (CTA pairs: both CTAs' copies complete on rank 0's barriers, and the
+            // exit handshake holds rank 1 until rank 0 has drained them.)
             __syncwarp(iss_mask);
-            if (lane == 0) {
+            if (lane == 0 && leader) {
                 if (!mbar_drain(bars.w_full(), 0, drain_ns))
                     atomicOr(&g_dev_status, kDevDrainFailed);
                 // The latest box of every slot: the last a_stages boxes of one
@@ -764,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long issued = 0;
             [[maybe_unused]] long long n_io = 0;  // stages handed out (trace index)
             bool ok = true;
-            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
+            for (int mt = mt_first; ok && mt < mt_end; mt += mt_step) {
                 int w0, h0, b0;
                 tile_origin<kRes>(p, mt, w0, h0, b0);
                 for (int rs = 0; rs < stages_per_tile; ++rs) {
@@ -823,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(bars.io_full(s));
             [[maybe_unused]] long long n_st = 0;  // stages stored (trace index)
             bool ok = true;
-            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step) {
+            for (int mt = mt_first; ok && mt < mt_end; mt += mt_step) {
                 int w0, h0, b0;
                 tile_origin<kRes>(p, mt, w0, h0, b0);
                 for (int rs = 0; rs < stages_per_tile; ++rs) {
@@ -833,7 +912,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     X1CB_TRACE_AT(p.trace, 7, n_st);
                     const int o1 = group * (p.NC / 32) + rs * plan_stage_ch<kRes>(p);
-                    if (plan_pool<kRes>(p))  // pooled tile at pooled coordinates ((w0 + 1) / 2, ...)
+                    if (kPair && mt >= p.num_m_tiles) {
+                        // (a pair's tile past the last one: nothing to store)
+                    } else if (plan_pool<kRes>(p))  // pooled tile at pooled coordinates ((w0 + 1) / 2, ...)
                         tma_store_5d_hint(&tmO, sio + stage * kRSlotBytes + kRSlotBytes / 2, 0,
                                           (w0 + 1) / 2, (h0 + 1) / 2, o1, b0, pol);
                     else if (p.io_swz)
@@ -843,8 +924,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_store_4d_hint(&tmO, sio + stage * plan_r_slot<kRes>(p), w0 * 4, h0, o1, b0, pol);
                     else
                         tma_store_5d_hint(&tmO, sio + stage * plan_r_slot<kRes>(p), 0, w0, h0, o1, b0, pol);
-                    bulk_commit();
-                    bulk_wait_read<0>();
+                    if (!kPair || mt < p.num_m_tiles) {
+                        bulk_commit();
+                        bulk_wait_read<0>();
+                    }
                     X1CB_TRACE_AT(p.trace, 8, n_st);
                     ++n_st;
                     mbar_arrive(bars.io_empty(stage));
@@ -867,14 +950,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // issuing warps, warp 1 takes the CTA's even tiles and warp 2 the odd
         // ones, each stepping its ring and slot counters over the other's tiles.
         const int mw = warp == 1 ? 0 : 1;
-        {
+        if (!kPair || leader) {  // (CTA pairs: rank 0 issues every MMA, M = 256)
             // The issue loop is kept free of divisions and descriptor rebuilds:
             // the dependent integer work between two MMAs would otherwise cost
             // more than the MMA itself (64-128 tensor cycles).  A descriptor's
             // start-address field is the byte address / 16 and every operand
             // lies below 256 KB, so moving an operand by `b` bytes is adding
             // b / 16 to its descriptor.
-            const uint32_t idesc = idesc_i8(kTileRows, p.nmma);
+            const uint32_t idesc = idesc_i8(kPair ? 2 * kTileRows : kTileRows, p.nmma);
             // (folded stem: output row y reads input row 2y + dr, two input rows
             // of tw 32-byte pixels per GEMM row group)
             const uint64_t a_desc0 =
@@ -892,7 +975,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t fold_b0 = smem_desc_sw32(sbase + p.off_bb);
             const uint32_t a_sub_step = static_cast<uint32_t>(p.rows * 32) >> 4;  // next K block in a box
             const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
-            const uint32_t b_kb_step = static_cast<uint32_t>(p.NC * 32) >> 4;     // next K block of weights
+            // next K block of weights (CTA pairs: each CTA holds NC/2 rows of it)
+            const uint32_t b_kb_step = static_cast<uint32_t>((kPair ? p.NC / 2 : p.NC) * 32) >> 4;
             const uint32_t b_sub_step = static_cast<uint32_t>(p.nmma * 32) >> 4;  // next N slice
             const int boxes = plan_halo<kRes>(p) ? p.C1 : p.kb_per_tile / p.a_kc;
             const int kc = p.a_kc;
@@ -925,14 +1009,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             [[maybe_unused]] long long n_box = 0, n_sub = 0;  // trace indices
-            bool ok = __all_sync(0xffffffffu, mbar_wait(bars.w_full(), 0, ctl, kDevTimeoutMma));
+            bool ok = __all_sync(0xffffffffu, mma_wait<kPair>(bars.w_full(), 0, ctl, kDevTimeoutMma));
             if (ok && p.inject == 1 && mw == 0) {
                 const WaitCtl planted{abort_flag, &g_dev_status, p.wait_limit_ns};
                 ok = __all_sync(0xffffffffu,  // test hook
                                 mbar_wait(bars.never(), 0, planted, kDevTimeoutMma));
             }
             int tile = 0;  // the CTA's tile count
-            for (int mt = mt_first; ok && mt < p.num_m_tiles; mt += mt_step, ++tile) {
+            for (int mt = mt_first; ok && mt < mt_end; mt += mt_step, ++tile) {
                 if (kSplit && (tile & 1) != mw) {
                     // the other issuer's tile (its boxes are in the other half of
                     // the ring): its accumulator slots
@@ -946,7 +1030,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t ph = a_phase;
                 uint64_t sd = a_slot_desc;
                 for (int j = 0; ok && j < p.n_subs; ++j) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(bars.acc_empty(acc), acc_phase ^ 1u,
+                    if (!__all_sync(0xffffffffu, mma_wait<kPair>(bars.acc_empty(acc), acc_phase ^ 1u,
                                                            ctl, kDevTimeoutMma))) {
                         ok = false;
                         break;
@@ -964,7 +1048,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int box = 0; box < boxes; ++box) {
                         // The slot was written by TMA and is read by the MMA, both in the
                         // async proxy; the barrier's transaction count orders them.
-                        if (j == 0 && !__all_sync(0xffffffffu, mbar_wait(bars.a_full(st), ph, ctl,
+                        if (j == 0 && !__all_sync(0xffffffffu, mma_wait<kPair>(bars.a_full(st), ph, ctl,
                                                                          kDevTimeoutMma))) {
                             ok = false;
                             break;
@@ -980,34 +1064,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (plan_halo<kRes>(p) == 3) {
                             // filter row dr: the slot dr input rows on, weight K block dr
                             for (int dr = 0; dr < p.R; ++dr)
-                                mma_i8(d_tmem, ad + static_cast<uint64_t>(dr) * h3_row_step,
+                                mma_issue<kPair>(d_tmem, ad + static_cast<uint64_t>(dr) * h3_row_step,
                                        bd + static_cast<uint64_t>(dr) * b_kb_step, idesc,
                                        dr == 0 ? accumulate : 1u);
                             bd += static_cast<uint64_t>(p.R) * b_kb_step;
                         } else if (plan_halo<kRes>(p)) {
 #pragma unroll
                             for (int t = 0; t < 9; ++t)
-                                mma_i8(d_tmem, ad + tap_off[t],
+                                mma_issue<kPair>(d_tmem, ad + tap_off[t],
                                        bd + static_cast<uint64_t>(t) * b_tap_step, idesc,
                                        t == 0 ? accumulate : 1u);
                             bd += b_kb_step;
                         } else if (kc == 4) {
-                            mma_i8(d_tmem, ad, bd, idesc, accumulate);
-                            mma_i8(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
-                            mma_i8(d_tmem, ad + 2 * a_sub_step, bd + 2 * b_kb_step, idesc, 1u);
-                            mma_i8(d_tmem, ad + 3 * a_sub_step, bd + 3 * b_kb_step, idesc, 1u);
+                            mma_issue<kPair>(d_tmem, ad, bd, idesc, accumulate);
+                            mma_issue<kPair>(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
+                            mma_issue<kPair>(d_tmem, ad + 2 * a_sub_step, bd + 2 * b_kb_step, idesc, 1u);
+                            mma_issue<kPair>(d_tmem, ad + 3 * a_sub_step, bd + 3 * b_kb_step, idesc, 1u);
                             bd += 4 * b_kb_step;
                         } else if (kc == 2) {
-                            mma_i8(d_tmem, ad, bd, idesc, accumulate);
-                            mma_i8(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
+                            mma_issue<kPair>(d_tmem, ad, bd, idesc, accumulate);
+                            mma_issue<kPair>(d_tmem, ad + a_sub_step, bd + b_kb_step, idesc, 1u);
                             bd += 2 * b_kb_step;
                         } else {
-                            mma_i8(d_tmem, ad, bd, idesc, accumulate);
+                            mma_issue<kPair>(d_tmem, ad, bd, idesc, accumulate);
                             bd += b_kb_step;
                         }
                         accumulate = 1u;
                         if (last_sub)
-                            mma_commit(bars.a_empty(st));  // slot free once these MMAs finish
+                            mma_commit_to<kPair>(bars.a_empty(st));  // slot free once these MMAs finish
                         if (++st == ring_end) {
                             st = ring_begin;
                             ph ^= 1u;
@@ -1019,9 +1103,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok)
                         break;
                     if (fold)  // + bias: constant A tile x digit rows of this slot's channels
-                        mma_i8(d_tmem, fold_a, fold_b0 + static_cast<uint64_t>(j) * b_sub_step,
+                        mma_issue<kPair>(d_tmem, fold_a, fold_b0 + static_cast<uint64_t>(j) * b_sub_step,
                                idesc, 1u);
-                    mma_commit(bars.acc_full(acc));
+                    mma_commit_to<kPair>(bars.acc_full(acc));
                     if (lane == 0)
                         X1CB_TRACE_AT(p.trace, 3, n_sub);
                     ++n_sub;
@@ -1035,7 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a_slot_desc = sd;
             }
             // Make sure no MMA is still reading shared memory or writing TMEM.
-            mma_commit(bars.mma_done());
+            mma_commit_to<kPair>(bars.mma_done());
             if (lane == 0 && !mbar_drain(bars.mma_done(), 0, drain_ns))
                 atomicOr(&g_dev_status, kDevDrainFailed);
         }
@@ -1043,7 +1127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---- epilogue ---------------------------------------------------------------
         const EpiCtx cx{&p, bars, ctl, tmem_base, smem + p.off_r, io_ticket, cm, cC,
-                        group, mt_first, mt_step};
+                        group, mt_first, mt_step, mt_end};
         const bool k1 = kRes && static_cast<long long>(p.m_r) == (1ll << (p.S - 1));
         if (mode == 3 && k1)
             epilogue_warp<kRes, 3, (kRes != 0)>(cx, warp, lane);
@@ -1065,9 +1149,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (threadIdx.x == 0)
         X1CB_TRACE_AT(p.trace, 15, 1);
+    if (kPair) {
+        // neither CTA of a pair leaves while the other may still reach it (its
+        // copies complete on rank 0's barriers, its arrivals cross over)
+        if (threadIdx.x == 0) {
+            mbar_arrive_cluster(mapa_shared(bars.exit_bar(), rank ^ 1u));
+            if (!mbar_drain(bars.exit_bar(), 0, 2 * p.wait_limit_ns + drain_ns))
+                atomicOr(&g_dev_status, kDevDrainFailed);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        if (kPair)
+            tmem_dealloc_pair(tmem_base, kTmemCols);
+        else
+            tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
@@ -1419,13 +1516,19 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     p.stage_ch = p.NC >= 128 ? kRChunks : p.NC / 32;
     p.n_slots = kTmemCols / p.nmma;
 
-    const int wbytes = p.wstream ? 0 : p.kb_per_tile * p.NC * 32;
-    // A shortcut layer whose resident weights take more than 96 KB stages its
-    // shortcut and result in 8 KB pieces (two 32-channel chunks): its I/O ring
-    // then keeps four stages in flight beside an activation ring of whole
-    // 16 KB boxes.  (Measured on the 7x7 512 -> 2048 expand conv, 128 KB of
-    // weights: with 16 KB stages only two fit beside the activation boxes.)
-    if (has_res && wbytes > 96 * 1024)
+    // A shortcut layer whose resident weights take more than 96 KB runs on CTA
+    // pairs when its group is one N = 256 MMA (each CTA then holds half the
+    // weights); otherwise it stages its shortcut and result in 8 KB pieces
+    // (two 32-channel chunks), so that four stages stay in flight beside an
+    // activation ring of whole 16 KB boxes.  (Measured on the 7x7 512 -> 2048
+    // expand conv, 128 KB of weights: with 16 KB stages only two fit beside
+    // the activation boxes.)
+    const int full_wbytes = p.wstream ? 0 : p.kb_per_tile * p.NC * 32;
+    p.pair = (has_res && full_wbytes > 96 * 1024 && p.NC == 256 && p.n_subs == 1)
+                 ? 1
+                 : 0;
+    const int wbytes = p.pair ? full_wbytes / 2 : full_wbytes;
+    if (has_res && !p.pair && wbytes > 96 * 1024)
         p.stage_ch = kRChunks / 2;
     const int r_slot = has_res ? p.stage_ch * kTileRows * 32 : kRSlotBytes;
     // The activation ring budget: with a shortcut the I/O ring (shortcut in,
@@ -1470,7 +1573,7 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.off_w = 0;
         p.off_ba = p.off_w + wbytes;
         p.off_bb = p.off_ba + (fold ? kTileRows * 32 : 0);
-        p.off_a = p.off_bb + (fold ? p.NC * 32 : 0);
+        p.off_a = p.off_bb + (fold ? (p.pair ? p.NC / 2 : p.NC) * 32 : 0);
         p.off_r = p.off_a + a * p.a_slot;
         // The per-channel bias/offset table (modes 0-2) and the fold digit rows
         // (mode 3) are never used together, so they share space when folding
@@ -1520,12 +1623,14 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
     // The swizzled stages need whole 4-pixel groups and 1024-byte aligned stages.
     p.io_swz = (p.tw % 4 == 0 && p.Wp % 4 == 0 && p.off_r % 1024 == 0 && !p.pool) ? 1 : 0;
 
-    const long long work = mtiles * p.n_groups;
-    long long grid = std::min<long long>(num_sms, work);
+    // Pairs: units are clusters of two CTAs, each taking pair tiles.
+    const int per_unit = p.pair ? 2 : 1;
+    const long long work = (mtiles + per_unit - 1) / per_unit * p.n_groups;
+    long long grid = std::min<long long>(num_sms / per_unit, work);
     grid = (grid / p.n_groups) * p.n_groups;
     if (grid < p.n_groups)
         grid = p.n_groups;
-    p.grid = static_cast<int>(grid);
+    p.grid = static_cast<int>(grid) * per_unit;
     p.wait_limit_ns = 2000000000ull;
     return X1CB_OK;
 }
@@ -1602,11 +1707,13 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
                                CU_TENSOR_MAP_DATA_TYPE_UINT8, es))
             return e;
     }
-    // Weights [Oc/128][KB][128][32]: dims (32, 128, KB, Oc/128); box (32,128,1,NC/128).
+    // Weights [Oc/128][KB][128][32]: dims (32, 128, KB, Oc/128); box (32,128,1,NC/128)
+    // (CTA pairs: one 128-row block, each CTA's half of a 256-channel group).
     {
         const uint64_t dims[4] = {32, (uint64_t)p.O2, (uint64_t)p.kb_a, (uint64_t)(p.Oc / p.O2)};
         const uint64_t str[3] = {32, (uint64_t)p.O2 * 32, (uint64_t)p.kb_a * p.O2 * 32};
-        const uint32_t box[4] = {32, (uint32_t)p.O2, 1, (uint32_t)(p.NC / p.O2)};
+        const uint32_t box[4] = {32, (uint32_t)p.O2, 1,
+                                 (uint32_t)(p.pair ? 1 : p.NC / p.O2)};
         if (int e = encode_map(&tmW, w, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return e;
     }
@@ -1683,17 +1790,51 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         }
     }
     const bool narrow = p.has_res && p.stage_ch == kRChunks / 2;
-    auto kern = narrow                ? conv_bn_act_kernel<2, false>
+    auto kern = p.pair                ? conv_bn_act_kernel<3, false>
+                : narrow              ? conv_bn_act_kernel<2, false>
                 : p.has_res           ? conv_bn_act_kernel<1, false>
                 : p.n_mma_warps > 1   ? conv_bn_act_kernel<0, true>
                                       : conv_bn_act_kernel<0, false>;
     if (int e = opt_in_smem(reinterpret_cast<const void *>(kern),
-                            narrow ? 4 : p.has_res ? 1 : (p.n_mma_warps > 1 ? 3 : 0)))
+                            p.pair ? 6 : narrow ? 4 : p.has_res ? 1 : (p.n_mma_warps > 1 ? 3 : 0)))
         return e;
     ConvPlan q = p;
     q.trace = trace_table();
-    kern<<<q.grid, kThreads, q.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, tmA2, tmW2, bias, mult,
-                                                      q);
+    if (!p.pair) {
+        kern<<<q.grid, kThreads, q.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, tmA2, tmW2, bias,
+                                                          mult, q);
+        return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
+    }
+    // CTA pairs: clusters of two, no more than can be resident at once (the
+    // kernel is persistent with a static assignment of pair tiles), a whole
+    // number of clusters per channel group.
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = q.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int resident = 0;
+    if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident < 1) {
+        cudaGetLastError();
+        return X1CB_ERR_CUDA;
+    }
+    int clusters = std::min(q.grid / 2, resident);
+    clusters = std::max(q.n_groups, clusters / q.n_groups * q.n_groups);
+    if (clusters > resident)
+        return X1CB_ERR_SHAPE;  // fewer resident pairs than channel groups
+    q.grid = 2 * clusters;
+    cfg.gridDim = dim3(q.grid, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, tmA, tmW, tmR, tmO, tmA2, tmW2, bias, mult, q) !=
+        cudaSuccess)
+        return X1CB_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
 }
 

@@ -61,6 +61,11 @@ struct ConvPlan {
     // slots of its tiles, n_slots even) while the store warp hands the I/O
     // stages back out.  Used where it measured faster: the folded stem.
     int n_mma_warps;
+    // CTA pairs (shortcut layers whose NC = 256 weights take more than 96 KB):
+    // clusters of two CTAs of one channel group share each MMA (M = 256, each
+    // CTA's 128 rows), each holding half of every K block's weights; grid
+    // counts CTAs (two per cluster).
+    int pair;
     int kb_per_tile;  // R*R*C1
     int a_kc;         // K blocks per activation TMA box (divides C1)
     int a_slot;       // bytes per ring stage: activation part + streamed weights
