@@ -70,6 +70,37 @@ def test_conv3x3_stride2_parity(oracle, shape):
     _spread(ref)
 
 
+# The 128 -> 128 3x3 at stride 2 runs on CTA pairs (phase planes as above):
+# several images per tile, odd input extents, an odd tile count, one pixel.
+PAIR_S2 = [(2, 56, 56), (3, 9, 13), (5, 8, 8), (2, 57, 57), (1, 1, 1), (7, 28, 20)]
+
+
+@pytest.mark.parametrize("shape", PAIR_S2, ids=[str(s) for s in PAIR_S2])
+def test_conv3x3_stride2_on_cta_pairs(oracle, shape):
+    B, H, W = shape
+    assert " pair=1 " in X.x1cb_describe_plan_ex(B, H, W, 128, 128, 3, 2)
+    inp = synth.conv_inputs(synth.ConvShape(B, H, W, 128, 128, 3, False), 900 + sum(shape))
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    w = X.x1cb_pack_weight(inp.w.to(DEV))
+    out = X.conv3x3s2_bn_relu_i8(x, w, inp.bias.to(DEV), inp.m.to(DEV), inp.S)
+    _status_ok()
+    ref = oracle.conv_strided(inp.x, inp.w, inp.bias, inp.m, inp.S, 2)
+    got = _nhwc(out.cpu())
+    assert got.shape == ref.shape
+    assert torch.equal(got, ref), int((got != ref).sum())
+
+
+def test_conv3x3_stride2_on_cta_pairs_full_int8_range(oracle):
+    s = synth.ConvShape(3, 13, 11, 128, 128, 3, False)
+    inp = synth.full_range_conv_inputs(s, 23, S=33)
+    x = X.x1cb_pack_act(inp.x.to(DEV))
+    w = X.x1cb_pack_weight(inp.w.to(DEV))
+    out = X.conv3x3s2_bn_relu_i8(x, w, inp.bias.to(DEV), inp.m.to(DEV), inp.S)
+    _status_ok()
+    ref = oracle.conv_strided(inp.x, inp.w, inp.bias, inp.m, inp.S, 2)
+    assert torch.equal(_nhwc(out.cpu()), ref)
+
+
 def test_conv3x3_stride2_full_int8_range(oracle):
     s = synth.ConvShape(2, 13, 11, 64, 128, 3, False)
     inp = synth.full_range_conv_inputs(s, 17, S=33)

@@ -247,6 +247,18 @@ int conv_geom_common(const int8_t *x, const int8_t *w, const int32_t *bias, cons
     if (check_ptrs)
         if (int e = check_resident({x, w, bias, m, out, x2, w2}))
             return e;
+    // The 128 -> 128 3x3 at stride 2 (the projection block's Conv2) runs on
+    // CTA pairs, as at stride 1 (see conv_common).
+    if (R == 3 && Rw_ == 3 && stride == 2 && sw == 2 && Ic == 128 && Oc == 128 && !pool &&
+        !Ic2 && g_inject.load() == 0) {
+        ChainPlan cp;
+        if (plan_conv2_pair(cp, B, H, W, S, 2, Hin, Win) == X1CB_OK) {
+            const unsigned long long lim = g_wait_limit_ns.load();
+            cp.wait_limit_ns = lim ? lim : kDefaultWaitNs;
+            return launch_chain(cp, x, w, bias, m, nullptr, nullptr, nullptr, nullptr, out,
+                                static_cast<cudaStream_t>(stream));
+        }
+    }
     ConvGeom g;
     g.stride = stride;
     g.Hin = Hin;
@@ -714,6 +726,15 @@ int x1cb_describe_plan_ex(int B, int Hin, int Win, int Ic, int Oc, int R, int st
                   p.kb_per_tile, p.a_kc, p.a_stages, p.r_stages, p.fold_room, p.smem_bytes, p.grid,
                   p.halo, p.io_swz, H, W, p.stride, p.C1b, p.wstream, p.pw, p.ph, p.n_mma_warps,
                   p.stage_ch);
+    // The 128 -> 128 3x3 at stride 1 or 2 runs on CTA pairs instead.
+    ChainPlan cp;
+    if (R == 3 && Ic == 128 && Oc == 128 && !Ic2 && !has_res && !pool && stride <= 2 &&
+        plan_conv2_pair(cp, B, H, W, 24, stride, Hin, Win) == X1CB_OK) {
+        const size_t n = std::strlen(buf);
+        std::snprintf(buf + n, len - n, " pair=1 pair_tile=%dx%dx%d pair_a_stages=%d "
+                      "pair_r_stages=%d pair_smem=%d", cp.tw, cp.th, cp.tg, cp.a_stages,
+                      cp.r_stages, cp.smem_bytes);
+    }
     return X1CB_OK;
 }
 

@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         *io_ticket = 0;
         mbar_init(bars.w_full(), 1);
-        mbar_init(bars.mma_done(), kC3 ? 1 : 2);  // each MMA issuer's final commit
+        mbar_init(bars.mma_done(), kC3 ? 1 : p.issuers);  // each MMA issuer's final commit
         mbar_init(bars.exit_bar(), 1);
         for (int s = 0; s < p.a_stages; ++s) {
             mbar_init(bars.a_full(s), 1);
@@ -545,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         if (lane < kAIssuers) {
-            const uint32_t abytes = static_cast<uint32_t>(2 * 16 * p.plane_m * p.tg);
+            const uint32_t abytes =
+                static_cast<uint32_t>((p.stride == 2 ? 8 : 2) * 16 * p.plane_m * p.tg);
             const uint64_t pol = policy_evict_first();
             const long long total = static_cast<long long>(n_my) * p.C1;
             long long issued = 0;
@@ -554,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // counters.  Fused: one ring (pos0).  The 3x3 alone: two MMA
             // warps, even pair tiles in slots [0, a/2), odd ones in [a/2, a),
             // each half consumed in order by its warp.
-            constexpr bool split = !kC3;
+            const bool split = !kC3 && p.issuers == 2;
             const int half = split ? p.a_stages / 2 : p.a_stages;
             int i = 0, c1 = 0, pos0 = 0, pos1 = 0;
             uint32_t ph0 = 0u, ph1 = 0u;
@@ -593,8 +594,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive_expect_tx(bars.a_full(stage), 2 * abytes);
                     const uint32_t slot = sbase + p.off_a + stage * p.a_slot;
                     const uint32_t full0 = mapa_shared(bars.a_full(stage), 0);
-                    tma2_load_5d_hint(slot, &tmA, full0, 0, -1, h0 - 1, c1, b0, pol);
-                    tma2_load_5d_hint(slot + p.a_half, &tmA, full0, 16, -1, h0 - 1, c1, b0, pol);
+                    if (!kC3 && p.stride == 2) {
+                        // plane (pr, pc) from input (pc - 1, 2*h0 - 1 + pr), step 2,
+                        // each K half a box
+                        for (int pl = 0; pl < 4; ++pl)
+                            for (int hf = 0; hf < 2; ++hf)
+                                tma2_load_5d_hint(slot + static_cast<uint32_t>((2 * pl + hf) *
+                                                                               p.a_half),
+                                                  &tmA, full0, 16 * hf, (pl & 1) - 1,
+                                                  2 * h0 - 1 + (pl >> 1), c1, b0, pol);
+                    } else {
+                        tma2_load_5d_hint(slot, &tmA, full0, 0, -1, h0 - 1, c1, b0, pol);
+                        tma2_load_5d_hint(slot + p.a_half, &tmA, full0, 16, -1, h0 - 1, c1, b0,
+                                          pol);
+                    }
                 }
                 issued = base + n_iss < total ? base + n_iss : total;
                 for (int k = 0; k < n_iss; ++k)
@@ -718,13 +731,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 1 || (!kC3 && warp == 2)) {
         // ---- MMA issuers (rank 0) ------------------------------------------------------
-        if (leader && !kC3) {
+        if (leader && !kC3 && warp - 1 < p.issuers) {
             // The 3x3 alone: warp 1 issues the even pair tiles and warp 2 the odd
             // ones (one thread issues an MMA only every ~92 cycles, an M = 256,
             // N = 128 one takes 64 on the tensor pipe), each from its half of
             // the halo ring and into slots i % 4 (two per warp).
             const int mw = warp - 1;
-            const int half = p.a_stages / 2;
+            const int nw = p.issuers;                 // issuing warps: ring parts, tile step
+            const int half = p.a_stages / nw;
             const uint32_t idesc = idesc_i8(256, 128);
             const uint64_t a_desc0 =
                 smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half));
@@ -732,12 +746,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t kb_step = (kHalfRows * 32) >> 4;
             const uint32_t a_slot_step = static_cast<uint32_t>(p.a_slot) >> 4;
             const uint32_t hp = static_cast<uint32_t>(p.row_pitch);
+            // Descriptor offset of tap (dr, ds), units of 16 bytes: the row shift of
+            // the framed tile; at stride 2 also the tap's phase plane.
+            uint32_t tap_off[9];
+#pragma unroll
+            for (int t = 0; t < 9; ++t) {
+                const uint32_t dr = t / 3, ds = t % 3;
+                tap_off[t] = p.stride == 2 ? ((dr & 1) * 2 + (ds & 1)) * (2 * p.a_half >> 4) +
+                                                 (dr >> 1) * hp + (ds >> 1)
+                                           : dr * hp + ds;
+            }
             const uint64_t ring_desc0 = a_desc0 + static_cast<uint64_t>(mw * half) * a_slot_step;
             int pos = 0;
             uint32_t ph = 0;
             uint64_t sd = ring_desc0;
             bool ok = __all_sync(0xffffffffu, mbar_wait_cl(bars.w_full(), 0, ctl, kDevTimeoutMma));
-            for (int i = mw; ok && i < n_my; i += 2) {
+            for (int i = mw; ok && i < n_my; i += nw) {
                 const int slot = i & 3;
                 const uint32_t sph = static_cast<uint32_t>((i >> 2) & 1);
                 if (!__all_sync(0xffffffffu, mbar_wait_cl(bars.acc_empty(slot), sph ^ 1u, ctl,
@@ -759,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int t = 0; t < 9; ++t)
-                        mma_i8_pair(d, sd + (t / 3) * hp + (t % 3),
+                        mma_i8_pair(d, sd + tap_off[t],
                                     w2_desc0 + static_cast<uint64_t>(t * p.C1 + c1) * kb_step,
                                     idesc, (c1 | t) ? 1u : 0u);
                     mma_commit_pair(bars.a_empty(st));
@@ -780,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit_pair(bars.mma_done());
             if (lane == 0 && !mbar_drain(bars.mma_done(), 0, drain_ns))
                 atomicOr(dev_status, kDevDrainFailed);
-        } else if (leader) {
+        } else if (leader && kC3) {
             const uint32_t idesc = idesc_i8(256, 128);
             const uint64_t a_desc0 =
                 smem_desc_rows16(sbase + p.off_a, static_cast<uint32_t>(p.a_half));
@@ -936,9 +960,15 @@ namespace {
 
 // Plan of the CTA-pair kernel: c3 = fused Conv2 -> Conv3, else the 3x3 alone
 // (Cout = Cm).
-int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r, bool c3)
+int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r, bool c3,
+              int stride = 1, int Hin = 0, int Win = 0)
 {
     std::memset(&p, 0, sizeof(p));
+    // (stride 2: the 3x3 alone, pad 1, output (Hin-1)/2+1 x (Win-1)/2+1, a
+    // plane row of W+1 pixels within the 128 GEMM rows)
+    if (stride != 1 && (c3 || stride != 2 || W + 1 > 126 || H != (Hin - 1) / 2 + 1 ||
+                        W != (Win - 1) / 2 + 1))
+        return X1CB_ERR_SHAPE;
     // One 128-channel Conv2 (its output is Conv3's whole K), a halo tile row
     // that fits the 128 GEMM rows, and output rows that the I/O maps can move
     // whole (4-pixel groups, or rows of at most 256 8-byte units).
@@ -948,6 +978,9 @@ int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_
     if (W % 4 != 0 && 4 * W > 256)
         return X1CB_ERR_SHAPE;
     p.c3 = c3 ? 1 : 0;
+    p.stride = stride;
+    p.Hin = stride == 2 ? Hin : H;
+    p.Win = stride == 2 ? Win : W;
     p.B = B;
     p.H = H;
     p.W = W;
@@ -957,13 +990,40 @@ int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_
     p.m_r = m_r;
     p.C1 = Cm / 32;
     p.n_chunks = Cout / 128;
-    choose_halo_tile(B, H, W, p.th, p.tg);
-    p.tw = W;
-    p.row_pitch = W + 2;
-    p.plane_m = (p.th + 2) * (W + 2);
-    const int need_rows = std::max(p.tg * p.plane_m, kTileRows + 2 * p.row_pitch + 2);
-    p.a_half = ((need_rows + 7) / 8) * 8 * 16;
-    p.a_slot = (2 * p.a_half + 1023) / 1024 * 1024;
+    if (stride == 2) {
+        // th output rows of tg images; a plane is (th+1) x (W+1) pixels, GEMM
+        // row m = (g*(th+1) + y)*(W+1) + x; fewest tiles, ties to taller ones
+        const int pitch = W + 1;
+        long long best = -1;
+        p.th = p.tg = 1;
+        for (int h = 1; h <= H; ++h)
+            for (int g = 1; g <= B; ++g) {
+                const long long last = static_cast<long long>(g - 1) * (h + 1) * pitch +
+                                       static_cast<long long>(h - 1) * pitch + (W - 1);
+                if (last >= kTileRows)
+                    break;
+                const long long t = static_cast<long long>((H + h - 1) / h) * ((B + g - 1) / g);
+                if (best < 0 || t < best || (t == best && h > p.th)) {
+                    best = t;
+                    p.th = h;
+                    p.tg = g;
+                }
+            }
+        p.tw = W;
+        p.row_pitch = pitch;
+        p.plane_m = (p.th + 1) * pitch;
+        const int need_rows = std::max(p.tg * p.plane_m, kTileRows + pitch + 1);
+        p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+        p.a_slot = (8 * p.a_half + 1023) / 1024 * 1024;  // four planes of two K halves
+    } else {
+        choose_halo_tile(B, H, W, p.th, p.tg);
+        p.tw = W;
+        p.row_pitch = W + 2;
+        p.plane_m = (p.th + 2) * (W + 2);
+        const int need_rows = std::max(p.tg * p.plane_m, kTileRows + 2 * p.row_pitch + 2);
+        p.a_half = ((need_rows + 7) / 8) * 8 * 16;
+        p.a_slot = (2 * p.a_half + 1023) / 1024 * 1024;
+    }
     p.rows = p.tw * p.th * p.tg;
     p.nTh = (H + p.th - 1) / p.th;
     p.nTg = (B + p.tg - 1) / p.tg;
@@ -1003,7 +1063,17 @@ int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_
         // The 3x3 alone holds half its weights per CTA (72 KB) and no Conv3
         // operands: a deep halo ring (up to four tiles of channel blocks, an
         // even number: half for each MMA warp) beside output stages for each
-        // epilogue turn.
+        // epilogue turn.  At stride 2 a channel block's four planes take
+        // 20 KB: the ring first (at least six slots), then the stages.
+        // At stride 2 a channel block's four planes take 20 KB: one issuing
+        // warp over the whole ring, the ring first (measured: two issuers with
+        // two 20 KB slots each ran the Res3.1 conv2 at 69.2 us against 64.7 on
+        // one SM per tile).
+        p.issuers = stride == 2 ? 1 : 2;
+        if (stride == 2)
+            for (int a = 16; a >= 4 && !placed; --a)
+                for (int r = kSlots - 1; r >= 2 && !placed; --r)
+                    placed = layout(a, r);
         for (int r = kSlots; r >= 2 && !placed; --r)
             for (int a = 16; a >= 4 && !placed; a -= 2)
                 placed = layout(a, r);
@@ -1022,9 +1092,9 @@ int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m
     return plan_pair(p, B, H, W, Cm, Cout, S, m_r, true);
 }
 
-int plan_conv2_pair(ChainPlan &p, int B, int H, int W, int S)
+int plan_conv2_pair(ChainPlan &p, int B, int H, int W, int S, int stride, int Hin, int Win)
 {
-    return plan_pair(p, B, H, W, 128, 128, S, 0, false);
+    return plan_pair(p, B, H, W, 128, 128, S, 0, false, stride, Hin, Win);
 }
 
 // Clusters of two CTAs of chain23_kernel that fit on the current device at
@@ -1071,7 +1141,20 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
                  const int8_t *x, int8_t *out, cudaStream_t stream)
 {
     CUtensorMap tmA, tmW2, tmW3, tmR, tmO;
-    {  // Conv2 input, halo form: dims (32, W, H, C1, B), box (16, W+2, th+2, 1, tg)
+    if (p.stride == 2) {
+        // Stride-2 planes: dims (32, Win, Hin, C1, B) at traversal step 2; a box
+        // of (2(W+1), 2(th+1)) elements lands one (W+1) x (th+1) plane.
+        const uint64_t dims[5] = {32, (uint64_t)p.Win, (uint64_t)p.Hin, (uint64_t)p.C1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {32, (uint64_t)p.Win * 32, (uint64_t)p.Hin * p.Win * 32,
+                                 (uint64_t)p.C1 * p.Hin * p.Win * 32};
+        const uint32_t box[5] = {16, (uint32_t)(2 * p.row_pitch), (uint32_t)(2 * (p.th + 1)), 1,
+                                 (uint32_t)p.tg};
+        const uint32_t es[5] = {1, 2, 2, 1, 1};
+        if (int e = encode_map(&tmA, y1, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                               CU_TENSOR_MAP_DATA_TYPE_UINT8, es))
+            return e;
+    } else {  // Conv2 input, halo form: dims (32, W, H, C1, B), box (16, W+2, th+2, 1, tg)
         const uint64_t dims[5] = {32, (uint64_t)p.W, (uint64_t)p.H, (uint64_t)p.C1,
                                   (uint64_t)p.B};
         const uint64_t str[4] = {32, (uint64_t)p.W * 32, (uint64_t)p.H * p.W * 32,

@@ -39,7 +39,8 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
 // form) and launch.  y1 [B, Cm/32, H, W, 32] is Conv1's output, x the block
 // input (the shortcut), out the block output.
 int plan_chain(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_r);
-int plan_conv2_pair(ChainPlan &p, int B, int H, int W, int S);
+int plan_conv2_pair(ChainPlan &p, int B, int H, int W, int S, int stride = 1, int Hin = 0,
+                    int Win = 0);
 int resident_clusters(int smem, int &clusters, bool c3 = true);
 int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const int32_t *b2,
                  const int32_t *m2, const int8_t *w3, const int32_t *b3, const int32_t *m3,

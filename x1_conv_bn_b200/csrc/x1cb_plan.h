@@ -124,6 +124,11 @@ struct ConvPlan {
 // images, full width); Conv3 the 1x1 with the shortcut.
 struct ChainPlan {
     int c3;  // 1: Conv2 -> Conv3 fused; 0: the 3x3 alone (Cout = Cm, stored like Conv3)
+    // The 3x3 alone at stride 2 (stride = 2): input Hin x Win, the halo tile
+    // as four phase planes of (th+1) x (W+1) pixels (see the convolution
+    // kernel's stride-2 halo form).
+    int stride, Hin, Win;
+    int issuers;  // the 3x3 alone: MMA-issuing warps (2: even / odd pair tiles, half a ring each)
     int B, H, W, Cm, Cout, S, m_r;
     int C1, n_chunks;  // Cm/32 channel blocks, Cout/128 output chunks
     int th, tg, tw, row_pitch, plane_m, a_half, rows;
