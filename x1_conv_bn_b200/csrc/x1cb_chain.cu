@@ -495,6 +495,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tma_prefetch_desc(&tmO);
     }
+    // Global memory only after the preceding grid (programmatic dependent
+    // launch: this CTA may have started while it drained).
+    griddep_wait();
     // Exact forms of the two layers (every CTA takes the same decision).
     int32_t *cm2 = reinterpret_cast<int32_t *>(smem + p.off_cm2);
     long long *cc2 = reinterpret_cast<long long *>(smem + p.off_cc2);
@@ -1227,13 +1230,17 @@ int launch_chain(const ChainPlan &p, const int8_t *y1, const int8_t *w2, const i
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = p.smem_bytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // a programmatic dependent of the preceding kernel (see the kernel's
+    // griddep_wait)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     unsigned int *dev_status = nullptr, *dev_forms = nullptr;
     if (int e = device_words(&dev_status, &dev_forms))
         return e;

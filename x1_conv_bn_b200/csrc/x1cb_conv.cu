@@ -528,6 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmW2);
         }
     }
+    // Launched as a dependent of the preceding kernel (programmatic dependent
+    // launch), this CTA may start while that kernel drains: everything above
+    // touches only shared memory and the kernel parameters; from here on the
+    // kernel reads and writes global memory, so it waits for the preceding
+    // grid to complete.
+    griddep_wait();
     // Folded-BN constants of this CTA's channels.  Generic form:
     // C = bias*m + 2^(S-1), so that t = acc*m + C (+ r*m_r) is one wide
     // multiply-add per term.  Fast form (when exact for every channel of the
@@ -1800,27 +1806,36 @@ int launch_conv(const ConvPlan &p, const int8_t *x, const int8_t *w, const int32
         return e;
     ConvPlan q = p;
     q.trace = trace_table();
+    // Every launch is a programmatic dependent of the preceding kernel on the
+    // stream: its CTAs may start (shared-memory set-up, TMEM allocation) as
+    // that kernel's CTAs leave, and wait for it to complete before touching
+    // global memory (griddep_wait in the kernel).
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(q.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = q.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (!p.pair) {
-        kern<<<q.grid, kThreads, q.smem_bytes, stream>>>(tmA, tmW, tmR, tmO, tmA2, tmW2, bias,
-                                                          mult, q);
+        if (cudaLaunchKernelEx(&cfg, kern, tmA, tmW, tmR, tmO, tmA2, tmW2, bias, mult, q) !=
+            cudaSuccess)
+            return X1CB_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? X1CB_OK : X1CB_ERR_CUDA;
     }
     // CTA pairs: clusters of two, no more than can be resident at once (the
     // kernel is persistent with a static assignment of pair tiles), a whole
     // number of clusters per channel group.
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = q.smem_bytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
     int resident = 0;
     if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident < 1) {
         cudaGetLastError();

@@ -528,6 +528,14 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32_sync(uint32_t taddr, uint32_t
 // the result.  Rank 0 issues the MMAs; both CTAs load their operands and
 // drain their accumulators.
 
+// Programmatic dependent launch: wait until the grids this one depends on
+// (the preceding kernel on the stream) have completed and their memory is
+// visible; a no-op when the kernel was launched without the attribute.
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
     uint32_t r;
