@@ -248,6 +248,21 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         }
         rsel[b] = sel;
     }
+    // Pool mode: this thread's 16-byte piece of the pooled stage -- piece k
+    // (pooled pixel k/2 mod np of chunk k/2/np, K half k&1) of the tile's
+    // np * stage_ch * 2, all within the turn's 128 threads (the planner
+    // checks) -- as offsets into the stage, the same for every tile.
+    int pool_src = -1, pool_dst = 0;
+    const int pool_row = p.tw * 32;
+    if (plan_pool<kRes>(p)) {
+        const int k = q * 32 + lane, np = p.pw * p.ph;
+        if (k < np * plan_stage_ch<kRes>(p) * 2) {
+            const int half = k & 1, c = (k >> 1) / np, pix = (k >> 1) % np;
+            const int pi = pix / p.pw, pj = pix % p.pw;
+            pool_src = c * chunk_stride + half * 16 + (2 * pi * p.tw + 2 * pj) * 32;
+            pool_dst = kRSlotBytes / 2 + (c * np + pix) * 32 + half * 16;
+        }
+    }
     // Position of stage n = turn: I/O ring slot and phase, stage within its
     // accumulator slot (rl), N slice (j), accumulator slot and phase.
     int st = turn % p.r_stages;
@@ -350,28 +365,21 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
             if (tr)
                 X1CB_TRACE_AT(p.trace, 10, n);
             pool_phase ^= 1u;
-            const int tid = q * 32 + lane;
-            const int np = p.pw * p.ph;
-            uint8_t *pooled = stage + kRSlotBytes / 2;
-            for (int k = tid; k < np * plan_stage_ch<kRes>(p) * 2; k += 128) {
-                const int half = k & 1;
-                const int c = (k >> 1) / np;
-                const int pix = (k >> 1) % np;
-                const int pi = pix / p.pw, pj = pix % p.pw;
-                const uint8_t *src = stage + c * chunk_stride + half * 16;
+            if (pool_src >= 0) {  // this thread's piece (offsets fixed per layer)
+                const uint8_t *src = stage + pool_src;
                 uint4 mx = make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int r = 0; r < 3; ++r)
 #pragma unroll
                     for (int t = 0; t < 3; ++t) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(
-                            src + ((2 * pi + r) * p.tw + 2 * pj + t) * 32);
+                        const uint4 v =
+                            *reinterpret_cast<const uint4 *>(src + r * pool_row + t * 32);
                         mx.x = __vmaxu4(mx.x, v.x);
                         mx.y = __vmaxu4(mx.y, v.y);
                         mx.z = __vmaxu4(mx.z, v.z);
                         mx.w = __vmaxu4(mx.w, v.w);
                     }
-                *reinterpret_cast<uint4 *>(pooled + (c * np + pix) * 32 + half * 16) = mx;
+                *reinterpret_cast<uint4 *>(stage + pool_dst) = mx;
             }
         }
         // Results must be visible to the TMA store (async proxy).
@@ -1461,6 +1469,10 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         p.a_half = 0;
     }
     p.rows = p.tw * p.th * p.tg;
+    // pooled tiles (64 channels: stages of two chunks): every 16-byte piece of
+    // the pooled stage is one epilogue thread's (a turn has 128)
+    if (p.pool && p.pw * p.ph * (Oc / 32) * 2 > 128)
+        return X1CB_ERR_SHAPE;
     p.nTw = p.pool ? (p.Wpo + p.pw - 1) / p.pw : (p.Wp + p.tw - 1) / p.tw;
     p.nTh = p.pool ? (p.Hpo + p.ph - 1) / p.ph : (p.Hp + p.th - 1) / p.th;
     p.nTg = (B + p.tg - 1) / p.tg;
