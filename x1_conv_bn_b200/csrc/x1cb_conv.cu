@@ -248,6 +248,18 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         }
         rsel[b] = sel;
     }
+    // Pool mode (64 channels: one stage per tile, so turn g takes tiles g,
+    // g + kTurns, ...): the tile coordinates (iw, ih) of this turn's next
+    // tile and their step, tracked with carries (image index unused).
+    int pool_iw = 0, pool_ih = 0, pool_dw = 0, pool_dh = 0;
+    if (plan_pool<kRes>(p)) {
+        const int mt0 = cx.mt_first + turn * cx.mt_step;
+        pool_iw = mt0 % p.nTw;
+        pool_ih = (mt0 / p.nTw) % p.nTh;
+        const int d = kTurns * cx.mt_step;
+        pool_dw = d % p.nTw;
+        pool_dh = (d / p.nTw) % p.nTh;
+    }
     // Pool mode: this thread's 16-byte piece of the pooled stage -- piece k
     // (pooled pixel k/2 mod np of chunk k/2/np, K half k&1) of the tile's
     // np * stage_ch * 2, all within the turn's 128 threads (the planner
@@ -307,11 +319,19 @@ __device__ __forceinline__ void epilogue_warp(const EpiCtx &cx, int warp, int la
         uint8_t *stage = cx.io + st * plan_r_slot<kRes>(p);
         bool conv_px = true;  // pool mode: this row is a pixel of the conv output
         if (plan_pool<kRes>(p)) {
-            const int mt = cx.mt_first + static_cast<int>(n / (p.n_subs * stages_per_sub)) *
-                                             cx.mt_step;
-            int w0, h0, b0;
-            tile_origin<kRes>(p, mt, w0, h0, b0);
+            // the tile's conv origin: one pixel before twice its pooled origin
+            const int w0 = 2 * pool_iw * p.pw - 1, h0 = 2 * pool_ih * p.ph - 1;
             conv_px = w0 + xi >= 0 && w0 + xi < p.W && h0 + yi >= 0 && h0 + yi < p.H;
+            // next stage of this turn: kTurns tiles on (one stage per pooled
+            // tile), tile coordinates advanced with carries, no divisions
+            pool_iw += pool_dw;
+            if (pool_iw >= p.nTw) {
+                pool_iw -= p.nTw;
+                ++pool_ih;
+            }
+            pool_ih += pool_dh;
+            if (pool_ih >= p.nTh)
+                pool_ih -= p.nTh;
         }
 #pragma unroll 1
         for (int c = 0; c < plan_stage_ch<kRes>(p); ++c) {
