@@ -332,7 +332,11 @@ void x1cb_set_wait_limit_ns(unsigned long long ns);
 void x1cb_debug_inject(int mode);
 
 /* Describes the launch plan chosen for a convolution shape into buf (a
- * short text), for tests and benchmarks.  Returns X1CB_OK or an error. */
+ * short text of key=value fields), for tests and benchmarks: cta_pair=1
+ * marks a shortcut layer that runs on clusters of two CTAs sharing each MMA,
+ * and a trailing "pair=1 pair_..." group gives the plan of a 128 -> 128 3x3
+ * (stride 1 or 2), which runs on CTA pairs instead of the single-CTA plan
+ * before it.  Returns X1CB_OK or an error. */
 int x1cb_describe_plan(int B, int H, int W, int Ic, int Oc, int R, int has_res, char *buf,
                        size_t len);
 
