@@ -233,6 +233,8 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
     const uint32_t rsel2[4] = {0, 0, 0, 0};
     int k = 0;             // item index in issue order
     uint32_t kph = 0;      // parity of this turn's slot at its next item
+    int c3_st = 0;         // shortcut ring slot and phase of the next Conv3 chunk
+    uint32_t c3_ph = 0;
     bool ok = true;
     const bool tr = q == 0 && lane == 0;  // one trace writer per turn
     for (int i = 0; ok && i <= n_my; ++i) {
@@ -281,12 +283,18 @@ __device__ __forceinline__ void chain_epilogue(const ChainEpi &ce, int warp, int
         if (i >= 1) {
             const int j = i - 1;
             for (int c = 0; c < p.n_chunks; ++c, ++k) {
+                // Conv3 of tile j, output chunk c: shortcut stage n = j*n_chunks + c,
+                // ring slot n % r_stages and phase (n / r_stages) & 1, counted
+                // over every chunk (this turn's or not)
+                const int n = j * p.n_chunks + c;
+                const int st = c3_st;
+                const uint32_t st_phase = c3_ph;
+                if (++c3_st == p.r_stages) {
+                    c3_st = 0;
+                    c3_ph ^= 1u;
+                }
                 if ((k & 3) != turn)
                     continue;
-                // Conv3 of tile j, output chunk c: shortcut stage n = j*n_chunks + c.
-                const long long n = static_cast<long long>(j) * p.n_chunks + c;
-                const int st = static_cast<int>(n % p.r_stages);
-                const uint32_t st_phase = static_cast<uint32_t>((n / p.r_stages) & 1);
                 // Stages are taken in order (the ticket), so each stage's
                 // previous phase is complete before its arrival is awaited.
                 if (!__all_sync(0xffffffffu,
@@ -374,9 +382,11 @@ __device__ __forceinline__ void conv2_epilogue(const ChainEpi &ce, int warp, int
     const uint32_t rsel[4] = {0, 0, 0, 0};
     uint32_t kph = 0;
     const bool tr = q == 0 && lane == 0;
+    // output stage of tile i: ring slot i % r_stages, phase (i / r_stages) & 1,
+    // advanced by counters (kSlots tiles per step)
+    int st = turn % p.r_stages;
+    uint32_t st_phase = static_cast<uint32_t>((turn / p.r_stages) & 1);
     for (int i = turn; i < ce.n_my; i += kSlots) {
-        const int st = i % p.r_stages;
-        const uint32_t st_phase = static_cast<uint32_t>((i / p.r_stages) & 1);
         if (!__all_sync(0xffffffffu,
                         mbar_wait(bars.acc_full(turn), kph, ctl, kDevTimeoutEpilogue)))
             return;
@@ -415,6 +425,11 @@ __device__ __forceinline__ void conv2_epilogue(const ChainEpi &ce, int warp, int
             mbar_arrive_cluster(empty0);
         }
         kph ^= 1u;
+        for (int a = 0; a < kSlots; ++a)
+            if (++st == p.r_stages) {
+                st = 0;
+                st_phase ^= 1u;
+            }
     }
 }
 
