@@ -1640,10 +1640,16 @@ int plan_conv_ex(ConvPlan &p, int B, int H, int W, int Ic, int Oc, int R, int ha
         const int a_want = std::max(a_min, p.wstream      ? 4
                                            : p.halo == 3 ? 12  // one slot per tile: a deep ring
                                                          : a_bytes_want / p.a_slot);
-        for (int fold = 1; fold >= 0 && !placed; --fold)
-            for (int a = a_want; a >= a_min && !placed; --a)
-                for (int r = r_hi; r >= r_lo && !placed; --r)
-                    placed = layout(fold, a, r);
+        // A projection layer whose boxes hold several K blocks takes a deeper
+        // floor of output stages before its activation ring may grow.
+        // (Measured on the Res3.1 Conv3 with its stride-2 projection,
+        // B = 256: 69.8 us with four 16 KB boxes and three output stages,
+        // 73.1 with five and two, 72.0 with three and four.)
+        for (int r_floor = p.C1b && kc > 1 ? std::max(r_lo, 3) : r_lo; r_floor >= r_lo && !placed; --r_floor)
+            for (int fold = 1; fold >= 0 && !placed; --fold)
+                for (int a = a_want; a >= a_min && !placed; --a)
+                    for (int r = r_hi; r >= r_floor && !placed; --r)
+                        placed = layout(fold, a, r);
     }
     if (!placed)
         return X1CB_ERR_SHAPE;
