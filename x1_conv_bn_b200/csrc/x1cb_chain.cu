@@ -1082,11 +1082,11 @@ int plan_pair(ChainPlan &p, int B, int H, int W, int Cm, int Cout, int S, int m_
         // operands: a deep halo ring (up to four tiles of channel blocks, an
         // even number: half for each MMA warp) beside output stages for each
         // epilogue turn.  At stride 2 a channel block's four planes take
-        // 20 KB: the ring first (at least six slots), then the stages.
-        // At stride 2 a channel block's four planes take 20 KB: one issuing
-        // warp over the whole ring, the ring first (measured: two issuers with
-        // two 20 KB slots each ran the Res3.1 conv2 at 69.2 us against 64.7 on
-        // one SM per tile).
+        // 20 KB: one issuing warp over the whole ring, the ring first, then
+        // the stages (measured on the Res3.1 conv2, B = 256: two issuers with
+        // two 20 KB slots each 69.2 us against 64.7 on one SM per tile; one
+        // issuer with five slots and three stages 47.5 us, 47.5 with two
+        // stages, 48.8-48.9 with four slots).
         p.issuers = stride == 2 ? 1 : 2;
         if (stride == 2)
             for (int a = 16; a >= 4 && !placed; --a)
